@@ -1,0 +1,426 @@
+"""CPU oracle for the fused MoE expert layer.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this module. The CUDA
+library never calls it, and it shares no code with the library: no kernels, no
+headers, no tables, no helpers. Its inputs come from ``workloads.py``.
+
+It is written to be read against the pages, not to be fast:
+
+* fp64 everywhere, with a BLAS matmul as the only library step;
+* intermediates are never rounded to bf16;
+* the one place where floating point decides an integer (the dynamic NVFP4
+  activation codes) takes that decision in fp32 with IEEE division, the
+  precision the CUDA kernels use.
+
+Page citations name the page's module and the class, method or docstring:
+
+* [moonep]   vllm.model_executor.layers.fused_moe.experts.moonep_experts
+* [fi_ep]    vllm.model_executor.layers.fused_moe.experts.flashinfer_moe_ep
+* [dsv4_fi]  vllm.models.deepseek_v4.nvidia.fi_moe (DeepseekV4MegaMoEExpertsFI)
+* [trtllm]   vllm.model_executor.layers.fused_moe.experts.trtllm_mxfp4_moe
+
+Readings taken where the pages are silent are listed in the design doc and repeated
+at the function that takes them.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+# --------------------------------------------------------------------------------------
+# FP4 / FP8 codecs. The pages name the formats (MXFP4: e2m1 values with an e8m0 scale per
+# 32 along K [trtllm: _supports_quant_scheme, kMxfp4Static]; NVFP4: e2m1 values with an
+# fp8-e4m3 scale per 16 along K plus an fp32 weight_scale_2 [dsv4_fi: _realloc_nvfp4_params])
+# but not the bit-level codes. Those are the public OCP Microscaling (MX) v1.0 element
+# formats, written out here from their definitions.
+# --------------------------------------------------------------------------------------
+
+# e2m1: 1 sign bit (bit 3), 2 exponent bits (bias 1), 1 mantissa bit; no inf/NaN.
+# Exponent field 0 is subnormal: value = m * 0.5. Otherwise 2^(e-1) * (1 + m/2).
+def _e2m1_magnitudes() -> np.ndarray:
+    mags = []
+    for code in range(8):
+        e, m = code >> 1, code & 1
+        mags.append(m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0))
+    return np.array(mags, dtype=np.float64)
+
+
+E2M1_MAG = _e2m1_magnitudes()          # [0, .5, 1, 1.5, 2, 3, 4, 6]
+E2M1_MAX = 6.0
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """e2m1 code (0..15) -> value, fp64."""
+    c = np.asarray(codes).astype(np.int64)
+    mag = E2M1_MAG[c & 7]
+    return np.where(c & 8, -mag, mag)
+
+
+def unpack_e2m1(packed) -> np.ndarray:
+    """Packed bytes ``[..., K/2]`` -> codes ``[..., K]``; the even-K value sits in the low nibble."""
+    p = np.asarray(packed).astype(np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = p & 0x0F
+    out[..., 1::2] = p >> 4
+    return out
+
+
+# e4m3 (the "fn" variant): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no inf;
+# exponent 15 with mantissa 7 is NaN, so the largest finite value is 448.
+def e4m3_decode(codes) -> np.ndarray:
+    c = np.asarray(codes).astype(np.int64)
+    s, e, m = (c >> 7) & 1, (c >> 3) & 0xF, c & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, 2.0 ** (e - 7.0) * (1.0 + m / 8.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(s == 1, -mag, mag)
+
+
+E4M3_MAX = 448.0
+
+
+def e8m0_decode(codes) -> np.ndarray:
+    """e8m0 (MX shared scale): an unsigned biased exponent, value 2^(s-127); 255 is NaN."""
+    s = np.asarray(codes).astype(np.int64)
+    return np.where(s == 255, np.nan, np.ldexp(1.0, s - 127))
+
+
+def _encode_rne_satfinite(v, table_vals: np.ndarray, sign_bit: int) -> np.ndarray:
+    """Round |v| to the nearest entry of ``table_vals`` (non-negative, ascending, index = code),
+    ties to the even code (even mantissa), saturating to the largest entry; the sign of v
+    (including -0) goes to ``sign_bit``. NaN inputs are not expected and not handled."""
+    x = np.asarray(v, dtype=np.float64)
+    neg = np.signbit(x)
+    a = np.minimum(np.abs(x), table_vals[-1])
+    hi = np.clip(np.searchsorted(table_vals, a, side="left"), 0, len(table_vals) - 1)
+    lo = np.clip(hi - 1, 0, len(table_vals) - 1)
+    dlo, dhi = a - table_vals[lo], table_vals[hi] - a
+    pick = np.where(dhi < dlo, hi, np.where(dlo < dhi, lo, np.where(lo % 2 == 0, lo, hi)))
+    return (pick | (neg.astype(np.int64) << sign_bit)).astype(np.uint8)
+
+
+_E4M3_POS = e4m3_decode(np.arange(0, 127))      # codes 0..126: the non-negative finite values
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """Real -> e2m1 code, round to nearest even, saturate to +-6."""
+    return _encode_rne_satfinite(v, E2M1_MAG, 3)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """Real -> e4m3 code, round to nearest even, saturate to +-448."""
+    return _encode_rne_satfinite(v, _E4M3_POS, 7)
+
+
+# --------------------------------------------------------------------------------------
+# Weights
+# --------------------------------------------------------------------------------------
+
+def to_f64(t) -> np.ndarray:
+    """bf16 / fp32 torch tensor (or array) -> fp64 numpy, exactly."""
+    if isinstance(t, torch.Tensor):
+        return t.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def weight_rows(ws, g: int) -> np.ndarray:
+    """Dequantised weights of row ``g`` of a projection, fp64 ``[N,K]``, without its global alpha.
+
+    BF16 as stored. MXFP4: e2m1(q) * 2^(s-127), one e8m0 scale per 32 along K
+    [trtllm: TrtLlmMxfp4ExpertsBase]. NVFP4: e2m1(q) * e4m3(s), one scale per 16 along K;
+    the per-expert fp32 ``weight_scale_2`` stays a separate epilogue alpha
+    [dsv4_fi: _realloc_nvfp4_params; fi_ep: epilogue_from_quant_config].
+    Every product is exact in fp64.
+    """
+    if ws.fmt == "bf16":
+        return to_f64(ws.data[g])
+    q = e2m1_decode(unpack_e2m1(ws.data[g].numpy()))
+    if ws.fmt == "mxfp4":
+        sc = e8m0_decode(ws.scale[g].numpy())
+        return q * np.repeat(sc, 32, axis=-1)
+    if ws.fmt == "nvfp4":
+        sc = e4m3_decode(ws.scale[g].numpy())
+        return q * np.repeat(sc, 16, axis=-1)
+    raise ValueError(ws.fmt)
+
+
+def weight_alpha(ws) -> np.ndarray:
+    """Per-row global scale (fc1/fc2 epilogue alpha): NVFP4 ``weight_scale_2``, else 1.
+
+    [fi_ep: epilogue_from_quant_config] MXFP4 carries no global scale and keeps the default
+    epilogue; NVFP4's per-expert globals become the alphas [dsv4_fi: finalize_weights].
+    """
+    if ws.alpha is None:
+        return np.ones(ws.G, dtype=np.float64)
+    return to_f64(ws.alpha)
+
+
+# --------------------------------------------------------------------------------------
+# S1 routing
+# --------------------------------------------------------------------------------------
+
+def route_topk(logits, topk: int):
+    """Softmax -> top-k -> renormalise ("Renormalize" routing [trtllm: _invoke_kernel,
+    routing_method_type]; int32 ids [fi_ep: FlashInferMoeEpExperts.apply]).
+
+    Selection is on the fp32 logits: experts ordered by (logit descending, id ascending), so
+    ties go to the lower expert id and -0 ties +0. Over the selected k, with l_0 the largest,
+    ``w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)``, which equals the softmax over all E
+    experts restricted to the k and renormalised (the common factor cancels).
+    Returns ``ids [T,k] int32`` (in selection order) and ``w [T,k]`` fp64.
+    """
+    L = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    T, E = L.shape
+    if not (1 <= topk <= E):
+        raise ValueError("need 1 <= topk <= E")
+    if T == 0:
+        return np.zeros((0, topk), np.int32), np.zeros((0, topk), np.float64)
+    eid = np.broadcast_to(np.arange(E), (T, E))
+    order = np.lexsort((eid, -L), axis=-1)          # primary key last: -logit, then id
+    ids = order[:, :topk]
+    sel = np.take_along_axis(L, ids, axis=1)
+    z = np.exp(sel - sel[:, :1])
+    w = z / z.sum(axis=1, keepdims=True)
+    return ids.astype(np.int32), w
+
+
+# --------------------------------------------------------------------------------------
+# S2 permutation into expert-contiguous segments
+# --------------------------------------------------------------------------------------
+
+def assign_rows(ids, E: int, B: int, replica_src):
+    """Expert-contiguous segments over G = E + B weight rows [moonep: module docstring, apply].
+
+    Segment g lists its (token, k) assignments in ascending token order. ``cu_seqlens[g]`` is
+    the inclusive running sum of the segment lengths, as ``torch.cumsum(expert_num_tokens)``
+    [moonep: MoonEPExperts.apply]. Rows [E, E+B) are redundant copies of hot experts; the pages
+    do not say how a replicated expert's tokens are shared out (that lives in the unseen
+    MoonEPPrepareAndFinalize), so this reading is taken: let R(e) be e followed by the slots s
+    with replica_src[s] == e in ascending s; e's n assignments (ascending token order) are cut
+    into |R(e)| contiguous chunks, chunk i holding n // |R| + (i < n % |R|) of them, and chunk i
+    goes to row R(e)[i]. Unused slots (replica_src = -1) stay empty.
+
+    Returns dict with ``row [T,k]`` (weight row of each assignment), ``cu_seqlens [G]``,
+    ``perm_token [NvS]``, ``perm_k [NvS]`` and ``inv_perm [T,k]`` (position of (t,k) in NvS).
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    T, k = ids.shape
+    G = E + B
+    src = np.asarray(replica_src, dtype=np.int64).reshape(-1) if B else np.zeros(0, np.int64)
+    if src.shape[0] != B:
+        raise ValueError("replica_src must have B entries")
+    reps = [[e] for e in range(E)]
+    for s in range(B):
+        if src[s] >= 0:
+            reps[int(src[s])].append(E + s)
+    per_expert = [[] for _ in range(E)]
+    for t in range(T):
+        for j in range(k):
+            per_expert[int(ids[t, j])].append((t, j))
+    segments = [[] for _ in range(G)]
+    for e in range(E):
+        lst, R = per_expert[e], reps[e]
+        q, r = divmod(len(lst), len(R))
+        pos = 0
+        for i, row in enumerate(R):
+            size = q + (1 if i < r else 0)
+            segments[row] = lst[pos:pos + size]
+            pos += size
+    counts = np.array([len(s) for s in segments], dtype=np.int64)
+    cu = np.cumsum(counts).astype(np.int32) if G else np.zeros(0, np.int32)
+    NvS = T * k
+    perm_token = np.empty(NvS, np.int32)
+    perm_k = np.empty(NvS, np.int32)
+    inv_perm = np.empty((T, k), np.int32)
+    row = np.empty((T, k), np.int32)
+    p = 0
+    for g, seg in enumerate(segments):
+        for (t, j) in seg:
+            perm_token[p], perm_k[p], inv_perm[t, j], row[t, j] = t, j, p, g
+            p += 1
+    return dict(row=row, cu_seqlens=cu, perm_token=perm_token, perm_k=perm_k, inv_perm=inv_perm)
+
+
+def segment_bounds(cu_seqlens):
+    """(start, end) of every segment from inclusive end offsets."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    starts = np.concatenate([[0], cu[:-1]]) if len(cu) else cu
+    return list(zip(starts.tolist(), cu.tolist()))
+
+
+# --------------------------------------------------------------------------------------
+# S3 / S5 grouped GEMM
+# --------------------------------------------------------------------------------------
+
+def grouped_gemm(a, ws, cu_seqlens, M_alloc: int | None = None):
+    """``out[seg_g] = alpha_g * a[seg_g] @ W[g].T`` for every segment; rows past the last
+    segment end are zero [moonep: moonep_grouped_gemm]. ``a`` is fp64 ``[M,K]``."""
+    a = np.asarray(a, dtype=np.float64)
+    M = a.shape[0] if M_alloc is None else M_alloc
+    alpha = weight_alpha(ws)
+    out = np.zeros((M, ws.N), dtype=np.float64)
+    for g, (s, e) in enumerate(segment_bounds(cu_seqlens)):
+        if e > s:  # empty segments are skipped
+            out[s:e] = alpha[g] * (a[s:e] @ weight_rows(ws, g).T)
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# S4 activation
+# --------------------------------------------------------------------------------------
+
+def silu_and_mul(gate, up):
+    """silu(gate) * up = gate / (1 + e^-gate) * up [moonep: module docstring, apply]."""
+    with np.errstate(over="ignore"):
+        return gate / (1.0 + np.exp(-gate)) * up
+
+
+def situ_and_mul(gate, up, alpha: float, beta: float):
+    """SITU gated activation [trtllm: TrtLlmMxfp4ExpertsBase.__init__, SITU comment]:
+    left = alpha * tanh(x0/alpha) * sigmoid(x0) on the gate, right = beta * tanh(x1/beta) on the
+    up projection, output left * right; alpha = situ_beta, beta = situ_linear_beta, both > 0.
+    The sigmoid takes the raw gate, as written."""
+    if not (alpha > 0 and beta > 0):
+        raise ValueError("SITU needs alpha > 0 and beta > 0")
+    with np.errstate(over="ignore"):
+        sig = 1.0 / (1.0 + np.exp(-gate))
+    return alpha * np.tanh(gate / alpha) * sig * (beta * np.tanh(up / beta))
+
+
+def act_and_mul(gate, up, act: str = "silu", situ_alpha: float = 1.0, situ_beta: float = 1.0,
+                route_w=None):
+    """Gated activation times the per-row route weight (``act *= route_weight``
+    [moonep: MoonEPExperts.apply])."""
+    h = silu_and_mul(gate, up) if act == "silu" else situ_and_mul(gate, up, situ_alpha, situ_beta)
+    if route_w is not None:
+        h = h * np.asarray(route_w, dtype=np.float64)[:, None]
+    return h
+
+
+# --------------------------------------------------------------------------------------
+# S2q dynamic NVFP4 activation quantisation
+# --------------------------------------------------------------------------------------
+
+NVFP4_ROW_DIV = np.float32(6.0 * 448.0)   # 2688: e2m1 max times e4m3 max
+
+
+def nvfp4_quantize_rows(v):
+    """Dynamic NVFP4 quantisation of activation rows.
+
+    The pages only say the megakernel quantises activations dynamically and drops the
+    checkpoint's input scales [fi_ep: epilogue_from_quant_config; dsv4_fi: forward,
+    stage_inputs(..., quantize_input=True)]. Reading taken: e2m1 codes with one e4m3 scale per
+    16 values and one fp32 scale per row, all decisions in fp32 with IEEE division:
+
+      s_r  = amax_r / 2688
+      sb_b = e4m3_rne_satfinite(amax_b / (6 * s_r))        per 16-value block b
+      q    = e2m1_rne_satfinite(v / (sb_b * s_r))           (sb_b * s_r rounded to fp32)
+      value = e2m1(q) * sb_b * s_r
+
+    A zero row, and any block whose scale rounds to zero, quantises to +0 codes.
+    Returns ``codes [R,K] uint8``, ``sb [R,K/16] uint8`` (e4m3 codes), ``s [R] float32``.
+    """
+    x = np.asarray(v, dtype=np.float32)
+    R, K = x.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    ax = np.abs(x)
+    amax = ax.max(axis=1) if K else np.zeros(R, np.float32)
+    s = (amax / NVFP4_ROW_DIV).astype(np.float32)
+    six_s = (np.float32(6.0) * s).astype(np.float32)
+    bmax = ax.reshape(R, K // 16, 16).max(axis=2)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(six_s[:, None] > 0, bmax / six_s[:, None], np.float32(0)).astype(np.float32)
+    sb = e4m3_encode(ratio)
+    step = (e4m3_decode(sb).astype(np.float32) * s[:, None]).astype(np.float32)
+    step_k = np.repeat(step, 16, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = np.where(step_k > 0, x / step_k, np.float32(0)).astype(np.float32)
+    codes = e2m1_encode(y)
+    codes = np.where(step_k > 0, codes, 0).astype(np.uint8)
+    return codes, sb, s
+
+
+def nvfp4_dequantize_rows(codes, sb, s):
+    """Value of quantised rows: e2m1(q) * e4m3(sb) * s_r, fp64 (exact)."""
+    return (e2m1_decode(codes) * np.repeat(e4m3_decode(sb), 16, axis=1)
+            * np.asarray(s, dtype=np.float64)[:, None])
+
+
+# --------------------------------------------------------------------------------------
+# S6 combine
+# --------------------------------------------------------------------------------------
+
+def combine(y, inv_perm, topk_w=None):
+    """``out[t] = sum_k y[inv_perm[t,k]]`` in k order (times ``topk_w[t,k]`` when the route
+    weight was not already applied in the activation) [trtllm: do_finalize; fi_ep: module
+    docstring, the megakernel combines]."""
+    y = np.asarray(y, dtype=np.float64)
+    inv = np.asarray(inv_perm, dtype=np.int64)
+    T, k = inv.shape
+    out = np.zeros((T, y.shape[1]), dtype=np.float64)
+    for j in range(k):
+        rows = y[inv[:, j]]
+        out += rows if topk_w is None else rows * np.asarray(topk_w, np.float64)[:, j:j + 1]
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# The whole layer
+# --------------------------------------------------------------------------------------
+
+def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
+                tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False):
+    """The fused expert layer: route -> permute -> gate/up grouped GEMMs -> activation times
+    route weight -> down grouped GEMM -> combine [moonep: module docstring and apply;
+    trtllm: _invoke_kernel; fi_ep: apply].
+
+    ``cfg`` supplies E, B, topk, act, situ_alpha, situ_beta and act_quant. With act_quant, x
+    (in token order) and every activation row are NVFP4-quantised (``nvfp4_quantize_rows``)
+    before their GEMM. ``tokens`` restricts the expert maths to the rows those tokens need
+    (routing and permutation are always computed in full). With ``apply_topk_in_fc1`` false
+    the route weight moves from the activation to the combine [fi_ep: apply_topk_in_fc1].
+
+    Returns a dict: ids, w, row, cu_seqlens, perm_token, perm_k, perm_w, inv_perm, tokens and
+    out (fp64 ``[len(tokens), H]``); with ``keep``, also xq (codes/sb/s), h and y rows.
+    """
+    ids, w = route_topk(logits, cfg.topk)
+    perm = assign_rows(ids, cfg.E, cfg.B, replica_src)
+    T, k = ids.shape
+    inv = perm["inv_perm"]
+    perm_w = w[perm["perm_token"], perm["perm_k"]] if T else np.zeros(0)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    need = np.zeros(T * k, dtype=bool)
+    need[inv[tok].reshape(-1)] = True
+
+    x64 = to_f64(x)
+    res = dict(ids=ids, w=w, perm_w=perm_w, tokens=tok, **perm)
+    if cfg.act_quant:
+        codes, sb, s = nvfp4_quantize_rows(np.asarray(x.float().numpy(), np.float32))
+        x64 = nvfp4_dequantize_rows(codes, sb, s)
+        if keep:
+            res.update(xq_codes=codes, xq_sb=sb, xq_s=s)
+
+    a_g, a_u, a_d = weight_alpha(w_gate), weight_alpha(w_up), weight_alpha(w_down)
+    y = np.zeros((T * k, w_down.N), dtype=np.float64)
+    h_keep = np.zeros((T * k, w_gate.N), dtype=np.float64) if keep else None
+    for g, (s0, s1) in enumerate(segment_bounds(perm["cu_seqlens"])):
+        rows = np.nonzero(need[s0:s1])[0] + s0
+        if len(rows) == 0:
+            continue
+        a = x64[perm["perm_token"][rows]]
+        gate = a_g[g] * (a @ weight_rows(w_gate, g).T)
+        up = a_u[g] * (a @ weight_rows(w_up, g).T)
+        h = act_and_mul(gate, up, cfg.act, cfg.situ_alpha, cfg.situ_beta,
+                        perm_w[rows] if apply_topk_in_fc1 else None)
+        if cfg.act_quant:
+            hc, hsb, hs = nvfp4_quantize_rows(h.astype(np.float32))
+            h = nvfp4_dequantize_rows(hc, hsb, hs)
+        if keep:
+            h_keep[rows] = h
+        y[rows] = a_d[g] * (h @ weight_rows(w_down, g).T)
+    out = combine(y, inv[tok], None if apply_topk_in_fc1 else w[tok])
+    res["out"] = out
+    if keep:
+        res.update(h=h_keep, y=y)
+    return res

@@ -1,0 +1,418 @@
+"""Pins for the CPU oracle: each checks it against something other than itself.
+
+Codecs against the OCP MX element tables (tests/golden) and torch's float8 types; routing
+against a brute-force loop written differently (repeated argmax, softmax over all experts);
+the grouped GEMM against pure-Python dot products; activations against closed forms and
+limits; the whole layer against a per-token loop with no permutation and against a dense
+SwiGLU MLP; the NVFP4 activation quantiser against a brute-force nearest-grid-point search.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import moe_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_pairs(name):
+    rows = []
+    with open(os.path.join(GOLD, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                a, b = line.split()
+                rows.append((float(a), float(b)))
+    return rows
+
+
+# ------------------------------------------------------------------ codecs
+
+def test_e2m1_decode_matches_ocp_table():
+    for code, val in _read_pairs("e2m1_ocp_mx_v1.txt"):
+        got = O.e2m1_decode(np.array([int(code)]))[0]
+        assert got == val and math.copysign(1, got) == math.copysign(1, val), (code, got, val)
+
+
+def test_e2m1_encode_ties_and_saturation():
+    for v, expect in _read_pairs("rne_ties.txt"):
+        c = O.e2m1_encode(np.array([v], np.float32))[0]
+        got = O.e2m1_decode(np.array([c]))[0]
+        assert got == expect and math.copysign(1, got) == math.copysign(1, expect), (v, got, expect)
+
+
+def test_e4m3_decode_matches_torch_all_codes():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_decode(np.arange(256))
+    both_nan = np.isnan(ref) & np.isnan(got)
+    assert np.all(both_nan | (ref == got))
+    assert O.e4m3_decode(np.array([0x7E]))[0] == 448.0
+
+
+def test_e8m0_decode_matches_torch():
+    if not hasattr(torch, "float8_e8m0fnu"):
+        pytest.skip("torch without float8_e8m0fnu")
+    codes = torch.arange(255, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    assert np.array_equal(ref, O.e8m0_decode(np.arange(255)))
+    assert np.isnan(O.e8m0_decode(np.array([255]))[0])
+
+
+def test_e4m3_encode_matches_torch_rne():
+    g = torch.Generator().manual_seed(3)
+    v = torch.cat([torch.rand(20000, generator=g) * 448.0,
+                   torch.rand(20000, generator=g) * 0.02,          # subnormal range
+                   torch.tensor([0.0, 2.0 ** -10, 3 * 2.0 ** -11, 448.0, 464.0 - 1e-3])])
+    ref = v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = O.e4m3_encode(v.numpy())
+    assert np.array_equal(ref, got)
+    assert O.e4m3_encode(np.array([1e6], np.float32))[0] == 0x7E       # satfinite
+    assert O.e4m3_encode(np.array([-1e6], np.float32))[0] == 0xFE
+
+
+@pytest.mark.parametrize("enc,dec,n", [(O.e2m1_encode, O.e2m1_decode, 16),
+                                       (O.e4m3_encode, O.e4m3_decode, 256)])
+def test_encode_is_nearest_grid_point(enc, dec, n):
+    grid = dec(np.arange(n))
+    grid = grid[np.isfinite(grid)]
+    vmax = np.max(grid)
+    rng = np.random.default_rng(0)
+    v = (rng.standard_normal(5000) * vmax / 3).astype(np.float32)
+    c = enc(v)
+    got = dec(c)
+    best = np.min(np.abs(np.minimum(np.abs(v), vmax)[:, None] - np.abs(grid)[None, :]), axis=1)
+    assert np.allclose(np.abs(np.minimum(np.abs(v), vmax) - np.abs(got)), best, rtol=0, atol=0)
+    assert np.all(np.signbit(got) == np.signbit(v))
+
+
+def test_unpack_nibble_order():
+    p = np.array([[0x21, 0xF0]], dtype=np.uint8)
+    assert O.unpack_e2m1(p).tolist() == [[1, 2, 0, 15]]
+
+
+# ------------------------------------------------------------------ routing
+
+def _route_brute(logits, k):
+    """Repeated argmax (first maximum = lowest id) and a full softmax, renormalised."""
+    L = np.asarray(logits, np.float32).astype(np.float64)
+    T, E = L.shape
+    ids = np.zeros((T, k), np.int64)
+    w = np.zeros((T, k))
+    for t in range(T):
+        avail = list(range(E))
+        for j in range(k):
+            best = avail[0]
+            for e in avail[1:]:
+                if L[t, e] > L[t, best]:
+                    best = e
+            ids[t, j] = best
+            avail.remove(best)
+        p = [math.exp(L[t, e]) for e in range(E)]
+        tot = sum(p)
+        sel = [p[e] / tot for e in ids[t]]
+        w[t] = [q / sum(sel) for q in sel]
+    return ids, w
+
+
+@pytest.mark.parametrize("T,E,k,int_logits", [(64, 8, 2, False), (64, 8, 2, True),
+                                              (33, 16, 5, True), (20, 64, 8, False), (7, 4, 4, True)])
+def test_route_matches_bruteforce(T, E, k, int_logits):
+    g = torch.Generator().manual_seed(T * E + k)
+    L = torch.randn(T, E, generator=g)
+    if int_logits:
+        L = torch.randint(-2, 3, (T, E), generator=g).float()
+        L[0, :] = 0.0
+        L[1, ::2] = -0.0        # -0 ties +0
+    ids, w = O.route_topk(L.numpy(), k)
+    bids, bw = _route_brute(L.numpy(), k)
+    assert np.array_equal(ids, bids)
+    assert np.allclose(w, bw, rtol=1e-13, atol=1e-15)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-14)
+    for t in range(T):
+        assert len(set(ids[t].tolist())) == k
+        sl = L.numpy()[t, ids[t]]
+        assert np.all(np.diff(sl) <= 0)
+
+
+def test_route_empty_and_full_k():
+    ids, w = O.route_topk(np.zeros((0, 8), np.float32), 2)
+    assert ids.shape == (0, 2)
+    ids, w = O.route_topk(np.zeros((3, 4), np.float32), 4)
+    assert ids.tolist() == [[0, 1, 2, 3]] * 3 and np.allclose(w, 0.25)
+
+
+# ------------------------------------------------------------------ permutation
+
+def _perm_case(T, E, k, B, used, seed):
+    g = torch.Generator().manual_seed(seed)
+    L = torch.randn(T, E, generator=g) * 2
+    ids, w = O.route_topk(L.numpy(), k)
+    src = -np.ones(B, np.int64)
+    if B:
+        src[:used] = torch.randperm(E, generator=g)[:used].numpy()
+    return ids, w, src
+
+
+@pytest.mark.parametrize("T,E,k,B,used", [(16, 8, 2, 0, 0), (50, 8, 3, 4, 2), (64, 16, 4, 6, 6),
+                                          (1, 4, 1, 2, 1), (0, 4, 2, 2, 1)])
+def test_permute_invariants(T, E, k, B, used):
+    ids, w, src = _perm_case(T, E, k, B, used, seed=T + 7 * B)
+    p = O.assign_rows(ids, E, B, src)
+    cu, pt, pk, inv, row = p["cu_seqlens"], p["perm_token"], p["perm_k"], p["inv_perm"], p["row"]
+    G = E + B
+    assert cu.shape == (G,) and (G == 0 or cu[-1] == T * k)
+    assert np.all(np.diff(np.concatenate([[0], cu])) >= 0)
+    # every (t, j) appears exactly once; the permutation inverts
+    assert sorted(zip(pt.tolist(), pk.tolist())) == [(t, j) for t in range(T) for j in range(k)]
+    for t in range(T):
+        for j in range(k):
+            assert pt[inv[t, j]] == t and pk[inv[t, j]] == j
+    # each segment: ascending token ids, rows of a replica serve only their source expert
+    for g, (s0, s1) in enumerate(O.segment_bounds(cu)):
+        toks = pt[s0:s1]
+        assert np.all(np.diff(toks) > 0)
+        expert = g if g < E else src[g - E]
+        if g >= E and src[g - E] < 0:
+            assert s1 == s0                           # unused slot is empty
+        for q in range(s0, s1):
+            assert ids[pt[q], pk[q]] == expert and row[pt[q], pk[q]] == g
+    # replica split is balanced: sizes of an expert's rows differ by at most one, larger first
+    for e in range(E):
+        rows = [e] + [E + s for s in range(B) if src[s] == e]
+        sizes = [cu[r] - (cu[r - 1] if r else 0) for r in rows]
+        assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+    # permute-then-unpermute identity on a payload
+    x = np.arange(T * 3, dtype=np.float64).reshape(T, 3)
+    xp = x[pt]
+    for t in range(T):
+        for j in range(k):
+            assert np.array_equal(xp[inv[t, j]], x[t])
+
+
+# ------------------------------------------------------------------ grouped GEMM
+
+def test_grouped_gemm_matches_python_dots():
+    seg = [3, 0, 4, 1]
+    cu = np.cumsum(seg).astype(np.int32)
+    a, wt, _ = W.gen_grouped_gemm_case(10, seg, 5, 6, seed=1)
+    ws = W.WeightSet("bf16", wt)
+    out = O.grouped_gemm(O.to_f64(a), ws, cu, M_alloc=10)
+    A, Wf = a.double().tolist(), wt.double().tolist()
+    start = 0
+    for g, n in enumerate(seg):
+        for r in range(start, start + n):
+            for c in range(5):
+                ref = sum(A[r][kk] * Wf[g][c][kk] for kk in range(6))
+                assert abs(out[r, c] - ref) <= 1e-15 * max(1.0, abs(ref))
+        start += n
+    assert np.all(out[8:] == 0)                       # padding rows past cu[-1] are zero
+
+
+def test_grouped_gemm_fp4_weights_scale_and_alpha():
+    # NVFP4 codes for +1 (0x2) everywhere, block scales 1.0 (e4m3 0x38), alpha 2 -> a row sum times 2
+    G, N, K = 2, 3, 32
+    data = torch.full((G, N, K // 2), 0x22, dtype=torch.uint8)
+    scale = torch.full((G, N, K // 16), 0x38, dtype=torch.uint8)
+    ws = W.WeightSet("nvfp4", data, scale, torch.tensor([2.0, 0.5]))
+    a = np.arange(4 * K, dtype=np.float64).reshape(4, K) / 7
+    out = O.grouped_gemm(a, ws, np.array([1, 4], np.int32))
+    assert np.allclose(out[0], 2.0 * a[0].sum()) and np.allclose(out[1:], 0.5 * a[1:].sum(1)[:, None])
+    # MXFP4: code 0x7 (6.0) with e8m0 126 (0.5) -> every weight 3.0
+    ws = W.WeightSet("mxfp4", torch.full((1, 2, K // 2), 0x77, dtype=torch.uint8),
+                     torch.full((1, 2, K // 32), 126, dtype=torch.uint8))
+    out = O.grouped_gemm(a[:2], ws, np.array([2], np.int32))
+    assert np.allclose(out, 3.0 * a[:2].sum(1)[:, None])
+
+
+# ------------------------------------------------------------------ activations
+
+def test_silu_closed_forms():
+    x = np.linspace(-30, 30, 601)
+    one = np.ones_like(x)
+    assert O.silu_and_mul(np.zeros(1), np.ones(1))[0] == 0.0
+    # silu(x) - silu(-x) = x * (sigmoid(x) + sigmoid(-x)) = x
+    assert np.allclose(O.silu_and_mul(x, one) - O.silu_and_mul(-x, one), x, atol=1e-12)
+    assert np.allclose(O.silu_and_mul(x, 3 * one), 3 * O.silu_and_mul(x, one))
+    assert np.all(O.silu_and_mul(x, one) >= -0.2785)   # global minimum of x*sigmoid(x)
+
+
+def test_situ_limits_and_symmetries():
+    rng = np.random.default_rng(1)
+    g, u = rng.standard_normal(1000) * 3, rng.standard_normal(1000) * 3
+    # alpha, beta -> infinity: alpha*tanh(x/alpha) -> x, so SITU -> silu(gate) * up
+    big = O.situ_and_mul(g, u, 1e4, 1e4)
+    assert np.allclose(big, O.silu_and_mul(g, u), rtol=1e-6, atol=1e-9)
+    s = O.situ_and_mul(g, u, 1.0, 1.0)
+    assert np.allclose(O.situ_and_mul(g, -u, 1.0, 1.0), -s)        # odd in the up input
+    assert np.all(np.abs(O.situ_and_mul(g, u, 0.7, 1.3)) <= 0.7 * 1.3 + 1e-15)
+    # gate -> +inf: left factor -> alpha; gate -> -inf: -> 0
+    assert np.allclose(O.situ_and_mul(np.full(3, 50.0), np.array([0.1, 1, 9]), 2.0, 1.5),
+                       2.0 * 1.5 * np.tanh(np.array([0.1, 1, 9]) / 1.5))
+    assert np.allclose(O.situ_and_mul(np.full(3, -60.0), np.ones(3), 2.0, 1.5), 0.0, atol=1e-20)
+    with pytest.raises(ValueError):
+        O.situ_and_mul(g, u, 0.0, 1.0)
+
+
+# ------------------------------------------------------------------ NVFP4 activation quant
+
+def _quant_brute(row):
+    """Per element: nearest point of the block's grid e2m1 * step, ties to the even code."""
+    row = np.asarray(row, np.float32)
+    amax = np.float32(np.max(np.abs(row)))
+    s = np.float32(amax / np.float32(2688.0))
+    codes = []
+    for b in range(len(row) // 16):
+        blk = row[16 * b:16 * b + 16]
+        r = np.float32(np.float32(np.max(np.abs(blk))) / np.float32(np.float32(6.0) * s)) if s > 0 else 0.0
+        sb = O.e4m3_encode(np.array([r], np.float32))[0]
+        step = np.float32(np.float32(O.e4m3_decode(np.array([sb]))[0]) * s)
+        for v in blk:
+            if step == 0:
+                codes.append(0)
+                continue
+            y = float(np.float32(v / step))
+            best = min(range(16), key=lambda c: (abs(min(abs(y), 6.0) - O.E2M1_MAG[c & 7]), c & 1)
+                       if (c >> 3) == (1 if math.copysign(1, y) < 0 else 0) else (1e9, 0))
+            codes.append(best)
+    return np.array(codes, np.uint8)
+
+
+def test_nvfp4_quant_matches_bruteforce_and_bounds():
+    x = W.gen_rows(6, 64, seed=5, dtype=torch.float32).numpy()
+    x[2, 16:32] = 0.0                                   # an all-zero block
+    x[3] *= 1e-3
+    x[4, 5] = 40.0                                      # an outlier
+    x[5] = 0.0                                          # an all-zero row
+    codes, sb, s = O.nvfp4_quantize_rows(x)
+    for r in range(6):
+        assert np.array_equal(codes[r], _quant_brute(x[r])), r
+    deq = O.nvfp4_dequantize_rows(codes, sb, s)
+    assert np.all(deq[5] == 0) and s[5] == 0
+    # the largest element of a row lands near the top of its block's range
+    for r in range(5):
+        i = int(np.argmax(np.abs(x[r])))
+        assert abs(deq[r, i] - x[r, i]) <= 0.25 * abs(x[r, i])
+    # values already on the grid quantise to themselves
+    codes2, sb2, s2 = O.nvfp4_quantize_rows(deq.astype(np.float32))
+    assert np.allclose(O.nvfp4_dequantize_rows(codes2, sb2, s2), deq, rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------ the whole layer
+
+def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
+    """Per token, per chosen expert, the expert MLP on that token alone: no permutation,
+    own routing, pure-Python dot products."""
+    ids, w = _route_brute(inp.logits.numpy(), cfg.topk)
+    x = O.to_f64(inp.x)
+    if cfg.act_quant:
+        c, sb, s = O.nvfp4_quantize_rows(inp.x.float().numpy())
+        x = O.nvfp4_dequantize_rows(c, sb, s)
+    ag, au, ad = (O.weight_alpha(inp.w_gate), O.weight_alpha(inp.w_up), O.weight_alpha(inp.w_down))
+    out = np.zeros((cfg.T, cfg.H))
+    Wg = [O.weight_rows(inp.w_gate, e).tolist() for e in range(cfg.E)]
+    Wu = [O.weight_rows(inp.w_up, e).tolist() for e in range(cfg.E)]
+    Wd = [O.weight_rows(inp.w_down, e).tolist() for e in range(cfg.E)]
+    for t in range(cfg.T):
+        xt = x[t].tolist()
+        for j in range(cfg.topk):
+            e = int(ids[t, j])
+            gate = [ag[e] * sum(a * b for a, b in zip(row, xt)) for row in Wg[e]]
+            up = [au[e] * sum(a * b for a, b in zip(row, xt)) for row in Wu[e]]
+            if cfg.act == "silu":
+                h = [gg / (1 + math.exp(-gg)) * uu for gg, uu in zip(gate, up)]
+            else:
+                al, be = cfg.situ_alpha, cfg.situ_beta
+                h = [al * math.tanh(gg / al) / (1 + math.exp(-gg)) * be * math.tanh(uu / be)
+                     for gg, uu in zip(gate, up)]
+            if apply_topk_in_fc1:
+                h = [v * w[t, j] for v in h]
+            if cfg.act_quant:
+                c, sb, s = O.nvfp4_quantize_rows(np.array([h], np.float32))
+                h = O.nvfp4_dequantize_rows(c, sb, s)[0].tolist()
+            y = [ad[e] * sum(a * b for a, b in zip(row, h)) for row in Wd[e]]
+            wt = 1.0 if apply_topk_in_fc1 else w[t, j]
+            out[t] += wt * np.array(y)
+    return out
+
+
+SMALL = {
+    "tiny": W.CONFIGS["tiny"],
+    "replicas": W.MoEConfig("replicas", T=12, H=32, I=48, E=6, topk=3, B=4, B_used=3, logit_std=2.0),
+    "mxfp4_situ": W.MoEConfig("mxfp4_situ", T=8, H=64, I=64, E=4, topk=2, act="situ",
+                              situ_alpha=0.8, situ_beta=1.7, wfmt="mxfp4"),
+    "nvfp4_quant": W.MoEConfig("nvfp4_quant", T=8, H=64, I=32, E=4, topk=2, wfmt="nvfp4",
+                               act_quant=1),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_matches_per_token_loop(name):
+    cfg = SMALL[name]
+    inp = W.gen_inputs(cfg)
+    res = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(),
+                        inp.w_gate, inp.w_up, inp.w_down)
+    ref = _layer_brute(cfg, inp)
+    scale = np.max(np.abs(ref))
+    if cfg.act_quant:
+        # the activation codes are decided in fp32 on values whose fp64 rounding order
+        # differs between the two loops; a flipped code moves one element by one step
+        assert np.linalg.norm(res["out"] - ref) <= 1e-3 * np.linalg.norm(ref)
+    else:
+        assert np.max(np.abs(res["out"] - ref)) <= 1e-12 * scale
+
+
+def test_layer_weight_in_combine_equals_weight_in_activation():
+    cfg = SMALL["replicas"]
+    inp = W.gen_inputs(cfg)
+    args = (cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down)
+    a = O.moe_forward(*args)["out"]
+    b = O.moe_forward(*args, apply_topk_in_fc1=False)["out"]
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_layer_redundant_slots_do_not_change_output():
+    cfg = SMALL["replicas"]
+    inp = W.gen_inputs(cfg)
+    a = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(),
+                      inp.w_gate, inp.w_up, inp.w_down)["out"]
+    cfg0 = cfg.with_(B=0, B_used=0)
+    strip = lambda ws: W.WeightSet(ws.fmt, ws.data[:cfg.E])
+    b = O.moe_forward(cfg0, inp.x, inp.logits.numpy(), np.zeros(0, np.int32),
+                      strip(inp.w_gate), strip(inp.w_up), strip(inp.w_down))["out"]
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_layer_single_expert_is_dense_swiglu():
+    cfg = W.MoEConfig("dense", T=9, H=40, I=24, E=1, topk=1)
+    inp = W.gen_inputs(cfg)
+    res = O.moe_forward(cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32),
+                        inp.w_gate, inp.w_up, inp.w_down)
+    x = inp.x.double()
+    wg, wu, wd = (inp.w_gate.data[0].double(), inp.w_up.data[0].double(), inp.w_down.data[0].double())
+    ref = torch.nn.functional.silu(x @ wg.T) * (x @ wu.T) @ wd.T       # textbook SwiGLU MLP
+    assert np.allclose(res["w"], 1.0)
+    assert np.allclose(res["out"], ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_layer_token_subset_matches_full():
+    cfg = SMALL["replicas"]
+    inp = W.gen_inputs(cfg)
+    args = (cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down)
+    full = O.moe_forward(*args)["out"]
+    sub = O.moe_forward(*args, tokens=[0, 5, 11])["out"]
+    assert np.allclose(sub, full[[0, 5, 11]], rtol=1e-13, atol=1e-16)   # BLAS order may differ
+
+
+def test_workload_generator_is_deterministic_and_replicas_copy():
+    cfg = SMALL["replicas"]
+    a, b = W.gen_inputs(cfg), W.gen_inputs(cfg)
+    assert torch.equal(a.x, b.x) and torch.equal(a.w_down.data, b.w_down.data)
+    src, copy_of = W.gen_replica_src(cfg)
+    for s in range(cfg.B):
+        assert torch.equal(a.w_gate.data[cfg.E + s], a.w_gate.data[int(copy_of[s])])
+    assert (src[cfg.B_used:] == -1).all() and (src[:cfg.B_used] >= 0).all()
