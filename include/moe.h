@@ -1,0 +1,241 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) fused MoE expert layer.
+ *
+ * The layer, as the pages state it (vLLM API pages for the MoonEP experts,
+ * FlashInfer MoE-EP experts, DeepSeek-V4 FlashInfer MoE and TRTLLM MXFP4
+ * experts):
+ *
+ *   top-k routing -> permute into expert-contiguous segments (cu_seqlens over
+ *   E experts plus B redundant slots) -> gate and up grouped GEMMs -> gated
+ *   activation times the route weight -> down grouped GEMM -> top-k combine.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named in a signature are DEVICE pointers unless stated otherwise,
+ *     owned by the caller, 16-byte aligned (TMA operands: 128-byte aligned is
+ *     not needed, 16 is). The library never allocates on these paths.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launches are
+ *     asynchronous; nothing synchronises except moe_get_device_error and
+ *     moe_prepare_weights.
+ *   - Host-side validation returns a status with nothing launched. Nothing
+ *     throws across the ABI. Errors a kernel detects (an out-of-range expert id,
+ *     a pipeline wait that timed out) are written to an error word at the start
+ *     of the caller's workspace and read back with moe_get_device_error.
+ *   - bf16 is IEEE-style bfloat16 stored as uint16; rounding to it is RNE.
+ *   - T = 0 (no tokens) is a no-op that returns MOE_OK.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,         /* a size, pointer or scalar argument is out of range */
+    MOE_ERR_UNSUPPORTED = 2,         /* valid, but this format/activation/shape is not implemented */
+    MOE_ERR_ALIGNMENT = 3,           /* K not a multiple of the block size, or a misaligned pointer */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+    MOE_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+    MOE_ERR_DEVICE = 6,              /* a kernel reported bad data (e.g. an expert id >= E) */
+    MOE_ERR_TIMEOUT = 7,             /* a kernel's bounded pipeline wait ran out */
+    MOE_ERR_NOT_PREPARED = 8         /* FP4 weights used before moe_prepare_weights */
+} moe_status_t;
+
+typedef enum { MOE_ACT_SILU = 0, MOE_ACT_SITU = 1 } moe_act_t;
+
+typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt_t;
+
+/*
+ * One projection's weights, G = E + B rows ([E, E+B) are the redundant slots),
+ * each an [N, K] matrix with K (the reduction axis) contiguous — the
+ * `[G, N, K]` convention of the MoonEP page's moonep_grouped_gemm.
+ *
+ *   data  : BF16  -> bf16 [G,N,K]
+ *           MXFP4 -> uint8 [G,N,K/2] packed e2m1, even k in the low nibble
+ *           NVFP4 -> same packing
+ *   scale : MXFP4 -> uint8 e8m0 [G,N,K/32] (value 2^(s-127)), the MXFP4 format
+ *                    of the TRTLLM MXFP4 page (kMxfp4Static)
+ *           NVFP4 -> uint8 fp8-e4m3 [G,N,K/16], the w13/w2_weight_scale planes of
+ *                    the DeepSeek-V4 FI page (_realloc_nvfp4_params)
+ *           BF16  -> NULL
+ *   alpha : NULL (=1) or fp32 [G], a per-row global scale applied in the GEMM
+ *           epilogue: NVFP4 weight_scale_2 (FlashInfer MoE-EP page,
+ *           epilogue_from_quant_config: finite, > 0, one per expert).
+ *   kdata, kscale, kalpha : the kernel-format copy that moe_prepare_weights
+ *           writes into caller memory; NULL until then. BF16 needs none.
+ */
+typedef struct {
+    int32_t fmt;            /* moe_wfmt_t */
+    int32_t G, N, K;
+    const void* data;
+    const void* scale;
+    const float* alpha;
+    const void* kdata;
+    const void* kscale;
+    const float* kalpha;
+} moe_weight_t;
+
+/* Gated activation. SITU (TRTLLM MXFP4 page, TrtLlmMxfp4ExpertsBase, SITU
+ * comment): left = situ_alpha*tanh(g/situ_alpha)*sigmoid(g),
+ * right = situ_beta*tanh(u/situ_beta); both must be > 0 (else INVALID_ARG).
+ * SILU: silu(g)*u (MoonEP page, module docstring). */
+typedef struct {
+    int32_t act;            /* moe_act_t */
+    float situ_alpha;       /* activation_situ_beta */
+    float situ_beta;        /* activation_situ_linear_beta */
+} moe_act_params_t;
+
+const char* moe_status_string(moe_status_t s);
+
+/* Library version string and the compute capability the kernels target. */
+const char* moe_version(void);
+
+/*
+ * S1 — top-k routing, softmax -> top-k -> renormalise ("Renormalize" routing
+ * of the TRTLLM MXFP4 page, _invoke_kernel; int32 ids as in the FlashInfer
+ * MoE-EP page, apply).
+ *   logits      fp32 [T,E], finite.
+ *   topk_ids    int32 [T,topk] out: experts by descending logit, ties to the
+ *               lower id (selection on the fp32 logits).
+ *   topk_w      fp32 [T,topk] out: exp(l_j - l_0) / sum_i exp(l_i - l_0).
+ * 1 <= topk <= min(E, 32), 1 <= E <= 1024, else INVALID_ARG/UNSUPPORTED.
+ */
+moe_status_t moe_route_topk(const float* logits, int T, int E, int topk,
+                            int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
+/*
+ * S2 — permute into expert-contiguous segments (MoonEP page: module docstring
+ * and MoonEPExperts.apply; cu_seqlens = cumsum of per-row lengths).
+ *   topk_ids/topk_w [T,topk]; replica_src int32 [B] (source expert of each
+ *   redundant slot, -1 = unused; may be NULL when B == 0).
+ *   Outputs, NvS = T*topk:
+ *     cu_seqlens int32 [E+B]: inclusive segment end offsets.
+ *     perm_token int32 [NvS]: token of each segment row (ascending per segment).
+ *     perm_w     fp32 [NvS]:  its route weight.
+ *     inv_perm   int32 [T,topk]: segment row of each (token, k).
+ *     x_perm     bf16 [M_alloc,H] or NULL: x rows gathered into segment order;
+ *                M_alloc >= NvS, rows >= NvS are left untouched.
+ *   A replicated expert's n assignments (ascending token) are cut into
+ *   contiguous chunks over [e, its slots ascending], chunk i holding
+ *   n/R + (i < n%R) rows. Indices are bit-exact with the oracle.
+ *   An expert id outside [0,E) sets MOE_ERR_DEVICE in the workspace error word.
+ *   ws: at least moe_permute_workspace_size(T, topk, E, B) bytes.
+ */
+size_t moe_permute_workspace_size(int T, int topk, int E, int B);
+moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, int topk,
+                         int E, int B, const int32_t* replica_src,
+                         const void* x, int H,
+                         int32_t* cu_seqlens, int32_t* perm_token, float* perm_w,
+                         int32_t* inv_perm, void* x_perm, int M_alloc,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * S3/S5 — grouped GEMM: out[seg_g] = alpha_g * a[seg_g] @ W[g]^T for every
+ * cu_seqlens segment; rows [cu_seqlens[G-1], M_alloc) of out are written as zero
+ * (MoonEP page, moonep_grouped_gemm). Empty segments are skipped.
+ *   a    bf16 [M_alloc, K];   out bf16 [M_alloc, N];   cu_seqlens int32 [G] on device.
+ *   w    BF16 weights, or FP4 weights already prepared (else NOT_PREPARED).
+ *   FP4: each row of a is converted to f16 times a power of two chosen from the
+ *   row's max (exact except below 2^-30 of that max); the products with the
+ *   exactly-dequantised weights accumulate in fp32 on the tensor cores.
+ *   ws: at least moe_grouped_gemm_workspace_size(M_alloc, w) bytes.
+ */
+size_t moe_grouped_gemm_workspace_size(int M_alloc, const moe_weight_t* w);
+moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
+                              const int32_t* cu_seqlens, void* out,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * S4 — gated activation times route weight: out[r,i] = act(gate[r,i], up[r,i]) * perm_w[r]
+ * (MoonEP page, MoonEPExperts.apply). gate/up/out bf16 [M, I]; perm_w fp32 [M]
+ * or NULL (no scaling). Computed in fp32, rounded once to bf16.
+ */
+moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm_w,
+                             int M, int I, moe_act_params_t act, void* out,
+                             moe_stream_t stream);
+
+/*
+ * S6 — combine: out[t] = sum_k w_k * y_perm[inv_perm[t,k]], summed in fp32 in k
+ * order and rounded once to bf16 (TRTLLM MXFP4 page, do_finalize). topk_w fp32
+ * [T,topk], or NULL when the route weight was already applied (w_k = 1).
+ * y_perm bf16 [>= T*topk, H]; out bf16 [T,H].
+ */
+moe_status_t moe_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w,
+                         int T, int topk, int H, void* out, moe_stream_t stream);
+
+/*
+ * S2q — dynamic NVFP4 quantisation of activation rows (FlashInfer MoE-EP page,
+ * epilogue_from_quant_config: activations are quantised inside the kernel and
+ * the checkpoint's input scales drop out). Per row r, in fp32 with IEEE
+ * division: s_r = amax_r/2688; per 16 values sb = e4m3_rne_satfinite(amax_b/(6 s_r));
+ * q = e2m1_rne_satfinite(v/(sb*s_r)). A zero row or a zero block scale gives +0 codes.
+ *   in       bf16 (in_is_f32 = 0) or fp32 (in_is_f32 = 1) [R,K], K % 16 == 0.
+ *   codes    uint8 [R,K/2] packed e2m1 (even k in the low nibble).
+ *   sb       uint8 [R,K/16] e4m3.   s  fp32 [R].
+ *   deq_f16  optional f16 [R,K]: e2m1(q)*sb, the GEMM operand (s_r applied later).
+ */
+moe_status_t moe_quantize_nvfp4(const void* in, int in_is_f32, int R, int K,
+                                uint8_t* codes, uint8_t* sb, float* s, void* deq_f16,
+                                moe_stream_t stream);
+
+/*
+ * S0 — one-time conversion of FP4 weights into the kernel's tile layout
+ * (FlashInfer MoE-EP page, process_weights_after_loading; DeepSeek-V4 FI page,
+ * finalize_weights). Untimed; synchronises `stream`.
+ *   dst: caller device memory of moe_prepared_weight_bytes(w) bytes. On success
+ *   w->kdata/kscale/kalpha point into dst. BF16 weights: no-op, MOE_OK.
+ *   MXFP4 rows whose scales span more than 36 binades cannot be staged exactly
+ *   in f16: MOE_ERR_UNSUPPORTED. Non-finite or non-positive alpha: INVALID_ARG.
+ */
+size_t moe_prepared_weight_bytes(const moe_weight_t* w);
+moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,
+                                 moe_stream_t stream);
+
+/*
+ * The fused layer: S1 -> S2 (-> S2q) -> S3+S4 -> S5 -> S6, launched back to back
+ * on one stream (programmatic dependent launch between kernels), no host sync,
+ * no allocation. The DeepSeek-V4 FI page's forward (MoEEpTensors: hidden states,
+ * ids, weights, fc1/fc2 alpha) and the TRTLLM monolithic apply (router logits in,
+ * finalized output out) are the two shapes this mirrors.
+ *   x bf16 [T,H]; router_logits fp32 [T,E]; weights [E+B, I, H] gate/up and
+ *   [E+B, H, I] down, all in one format; FP4 weights must be prepared.
+ *   act_quant = 1: dynamic NVFP4 activations (NVFP4 weights only).
+ *   apply_topk_in_fc1 = 1 applies the route weight in the activation (default);
+ *   0 applies it in the combine (FlashInfer MoE-EP page, apply_topk_in_fc1).
+ *   topk_ids_out/topk_w_out: optional [T,topk] copies of the routing.
+ *   T <= T_max given to moe_forward_workspace_size, else INVALID_ARG.
+ */
+typedef struct {
+    const void* x;
+    const float* router_logits;
+    int32_t T, H, I, E, B, topk;
+    const int32_t* replica_src;     /* [B] or NULL */
+    moe_weight_t w_gate, w_up, w_down;
+    moe_act_params_t act;
+    int32_t apply_topk_in_fc1;
+    int32_t act_quant;
+    void* out;                      /* bf16 [T,H] */
+    int32_t* topk_ids_out;          /* optional */
+    float* topk_w_out;              /* optional */
+    int32_t T_max;                  /* capacity the workspace was sized for */
+} moe_forward_args_t;
+
+size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,
+                                  int wfmt, int act_quant);
+moe_status_t moe_forward(const moe_forward_args_t* args, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* Synchronises `stream`, returns (and clears) the error word a kernel wrote at
+ * the start of `ws` (any workspace passed to the entry points above). */
+moe_status_t moe_get_device_error(void* ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_MOE_H */

@@ -1,0 +1,439 @@
+// The extern "C" boundary: argument validation, workspace planning and the
+// launch sequences. Host code only; kernels live in the other .cu files.
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace moe {
+size_t prepared_weight_bytes(const moe_weight_t* w);
+moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaStream_t st);
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+inline cudaStream_t S(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+inline size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopk = 32;
+
+bool act_ok(const moe_act_params_t& a) {
+    if (a.act == MOE_ACT_SILU) return true;
+    if (a.act == MOE_ACT_SITU)
+        return std::isfinite(a.situ_alpha) && std::isfinite(a.situ_beta) && a.situ_alpha > 0.f && a.situ_beta > 0.f;
+    return false;
+}
+
+// Checks one projection's descriptor against the expected shape.
+moe_status_t check_weight(const moe_weight_t& w, int G, int N, int K) {
+    if (w.G != G || w.N != N || w.K != K || !w.data) return MOE_ERR_INVALID_ARG;
+    if (w.fmt != MOE_W_BF16 && w.fmt != MOE_W_MXFP4 && w.fmt != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+    if (!aligned16(w.data)) return MOE_ERR_ALIGNMENT;
+    if (w.fmt == MOE_W_BF16) {
+        if (K % 8) return MOE_ERR_ALIGNMENT;
+        return MOE_OK;
+    }
+    if (!w.scale) return MOE_ERR_INVALID_ARG;
+    if (K % (w.fmt == MOE_W_MXFP4 ? 32 : 16)) return MOE_ERR_ALIGNMENT;
+    if (!w.kdata || !w.kscale || !w.kalpha) return MOE_ERR_NOT_PREPARED;
+    return MOE_OK;
+}
+
+const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? w.alpha : w.kalpha; }
+
+// ----------------------------------------------------------------- forward workspace
+struct FwdWs {
+    size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
+        xq_deq, act, act2, act2_scale, act_codes, act_sb, y, bytes;
+};
+
+FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
+    FwdWs L{};
+    const size_t NvS = (size_t)T_max * topk;
+    const int G = E + B;
+    size_t off = kErrBytes;
+    auto take = [&](size_t b) {
+        const size_t o = off;
+        off += up256(b);
+        return o;
+    };
+    const bool fp4 = wfmt != MOE_W_BF16;
+    L.ids = take(4 * NvS);
+    L.w = take(4 * NvS);
+    L.cu = take(4 * (size_t)G);
+    L.perm_token = take(4 * NvS);
+    L.perm_w = take(4 * NvS);
+    L.inv = take(4 * NvS);
+    L.perm_scratch = take(permute_ws_layout(T_max, topk, E, B).bytes);
+    L.xperm = take(2 * NvS * H);
+    L.tscale = take(fp4 ? 4 * NvS : 0);
+    L.xq_codes = take(act_quant ? (size_t)T_max * H / 2 : 0);
+    L.xq_sb = take(act_quant ? (size_t)T_max * H / 16 : 0);
+    L.xq_s = take(act_quant ? 4 * (size_t)T_max : 0);
+    L.xq_deq = take(act_quant ? 2 * (size_t)T_max * H : 0);
+    L.act = take((fp4 ? 4 : 2) * NvS * I);  // fp32 when a row pass follows
+    L.act2 = take(fp4 ? 2 * NvS * I : 0);
+    L.act2_scale = take(fp4 ? 4 * NvS : 0);
+    L.act_codes = take(act_quant ? NvS * I / 2 : 0);
+    L.act_sb = take(act_quant ? NvS * I / 16 : 0);
+    L.y = take(2 * NvS * H);
+    L.bytes = off;
+    return L;
+}
+
+const char* kStatusNames[] = {"MOE_OK",
+                              "MOE_ERR_INVALID_ARG",
+                              "MOE_ERR_UNSUPPORTED",
+                              "MOE_ERR_ALIGNMENT",
+                              "MOE_ERR_WORKSPACE_TOO_SMALL",
+                              "MOE_ERR_CUDA",
+                              "MOE_ERR_DEVICE",
+                              "MOE_ERR_TIMEOUT",
+                              "MOE_ERR_NOT_PREPARED"};
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+    const int i = static_cast<int>(s);
+    if (i < 0 || i >= (int)(sizeof(kStatusNames) / sizeof(kStatusNames[0]))) return "MOE_ERR_UNKNOWN";
+    return kStatusNames[i];
+}
+
+const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
+
+moe_status_t moe_route_topk(const float* logits, int T, int E, int topk, int32_t* topk_ids, float* topk_w,
+                            moe_stream_t stream) {
+    if (T < 0 || E < 1 || topk < 1 || topk > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_route_topk(logits, T, E, topk, topk_ids, topk_w, S(stream), false));
+}
+
+size_t moe_permute_workspace_size(int T, int topk, int E, int B) {
+    if (T < 0 || topk < 1 || E < 1 || B < 0) return 0;
+    return kErrBytes + permute_ws_layout(T, topk, E, B).bytes;
+}
+
+moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, int topk, int E, int B,
+                         const int32_t* replica_src, const void* x, int H, int32_t* cu_seqlens, int32_t* perm_token,
+                         float* perm_w, int32_t* inv_perm, void* x_perm, int M_alloc, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    if (T < 0 || topk < 1 || E < 1 || B < 0 || topk > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts || E + B > 2 * kMaxExperts || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
+    if (B > 0 && !replica_src) return MOE_ERR_INVALID_ARG;
+    if (!cu_seqlens || !ws) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_permute_workspace_size(T, topk, E, B)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (x_perm) {
+        if (!x || H <= 0 || M_alloc < T * topk) return MOE_ERR_INVALID_ARG;
+        if (H % 8 || !aligned16(x) || !aligned16(x_perm)) return MOE_ERR_ALIGNMENT;
+    }
+    if (T > 0 && (!topk_ids || !perm_token || !perm_w || !inv_perm)) return MOE_ERR_INVALID_ARG;
+    char* w = static_cast<char*>(ws);
+    cudaStream_t st = S(stream);
+    cudaError_t e = launch_permute(topk_ids, topk_w, T, topk, E, B, replica_src, cu_seqlens, perm_token, perm_w,
+                                   inv_perm, reinterpret_cast<DevError*>(w), w + kErrBytes, st, false);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (x_perm) e = launch_gather(0, x, H, perm_token, T * topk, x_perm, nullptr, nullptr, st, true);
+    return cuda_status(e);
+}
+
+size_t moe_grouped_gemm_workspace_size(int M_alloc, const moe_weight_t* w) {
+    if (!w || M_alloc < 0) return 0;
+    size_t b = kErrBytes;
+    if (w->fmt != MOE_W_BF16) b += up256(2 * (size_t)M_alloc * w->K) + up256(4 * (size_t)M_alloc);
+    return b;
+}
+
+moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w, const int32_t* cu_seqlens,
+                              void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!w || M_alloc < 0 || w->G < 1 || w->N < 1 || w->K < 1) return MOE_ERR_INVALID_ARG;
+    if (w->G > 1024) return MOE_ERR_UNSUPPORTED;
+    moe_status_t s = check_weight(*w, w->G, w->N, w->K);
+    if (s != MOE_OK) return s;
+    if (M_alloc == 0) return MOE_OK;
+    if (!a || !cu_seqlens || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(out) || w->N % 8) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < moe_grouped_gemm_workspace_size(M_alloc, w)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = S(stream);
+    char* wsb = static_cast<char*>(ws);
+    GemmProblem p{};
+    p.M_alloc = M_alloc;
+    p.cu_seqlens = cu_seqlens;
+    p.G = w->G;
+    p.N = w->N;
+    p.K = w->K;
+    p.wfmt = w->fmt;
+    p.dual = false;
+    p.alpha0 = weight_alpha(*w);
+    p.out_scale = 1.0f;
+    p.out = out;
+    p.out_kind = OUT_BF16;
+    p.zero_pad = true;
+    p.err = reinterpret_cast<DevError*>(wsb);
+    bool pdl = false;
+    if (w->fmt == MOE_W_BF16) {
+        p.x = a;
+        p.w0 = w->data;
+    } else {
+        __half* a16 = reinterpret_cast<__half*>(wsb + kErrBytes);
+        float* sc = reinterpret_cast<float*>(wsb + kErrBytes + up256(2 * (size_t)M_alloc * w->K));
+        cudaError_t e = launch_rows_to_f16(a, false, M_alloc, w->K, a16, sc, st, false);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        p.x = a16;
+        p.tscale = sc;
+        p.kdata0 = w->kdata;
+        p.kscale0 = w->kscale;
+        pdl = true;
+    }
+    return cuda_status(launch_grouped_gemm(p, st, pdl));
+}
+
+moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm_w, int M, int I,
+                             moe_act_params_t act, void* out, moe_stream_t stream) {
+    if (M < 0 || I < 0 || !act_ok(act)) return MOE_ERR_INVALID_ARG;
+    if ((size_t)M * I == 0) return MOE_OK;
+    if (!gate || !up || !out) return MOE_ERR_INVALID_ARG;
+    if (I % 8 || !aligned16(gate) || !aligned16(up) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_act_and_mul(static_cast<const __nv_bfloat16*>(gate),
+                                          static_cast<const __nv_bfloat16*>(up), perm_w, M, I, act.act,
+                                          act.situ_alpha, act.situ_beta, static_cast<__nv_bfloat16*>(out),
+                                          S(stream), false));
+}
+
+moe_status_t moe_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w, int T, int topk, int H,
+                         void* out, moe_stream_t stream) {
+    if (T < 0 || topk < 1 || H < 1) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !inv_perm || !out) return MOE_ERR_INVALID_ARG;
+    if (H % 8 || !aligned16(y_perm) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_combine(static_cast<const __nv_bfloat16*>(y_perm), inv_perm, topk_w, T, topk, H,
+                                      static_cast<__nv_bfloat16*>(out), S(stream), false));
+}
+
+moe_status_t moe_quantize_nvfp4(const void* in, int in_is_f32, int R, int K, uint8_t* codes, uint8_t* sb, float* s,
+                                void* deq_f16, moe_stream_t stream) {
+    if (R < 0 || K < 0) return MOE_ERR_INVALID_ARG;
+    if (K % 16) return MOE_ERR_ALIGNMENT;
+    if ((size_t)R * K == 0) return MOE_OK;
+    if (!in || !codes || !sb || !s) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(in) || !aligned16(codes) || (deq_f16 && !aligned16(deq_f16))) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_quant_nvfp4(in, in_is_f32 != 0, R, K, codes, sb, s, static_cast<__half*>(deq_f16),
+                                          S(stream), false));
+}
+
+size_t moe_prepared_weight_bytes(const moe_weight_t* w) {
+    if (!w) return 0;
+    return prepared_weight_bytes(w);
+}
+
+moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, moe_stream_t stream) {
+    if (!w || w->G < 1 || w->N < 1 || w->K < 1 || !w->data) return MOE_ERR_INVALID_ARG;
+    if (w->fmt == MOE_W_BF16) return MOE_OK;
+    if (w->fmt != MOE_W_MXFP4 && w->fmt != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+    if (!w->scale || !dst) return MOE_ERR_INVALID_ARG;
+    if (w->K % (w->fmt == MOE_W_MXFP4 ? 32 : 16)) return MOE_ERR_ALIGNMENT;
+    if (w->alpha) {
+        // epilogue alphas must be finite and positive (FlashInfer MoE-EP page,
+        // epilogue_from_quant_config -> require_finite_positive_scales)
+        std::vector<float> h(w->G);
+        if (cudaMemcpy(h.data(), w->alpha, sizeof(float) * w->G, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        for (float v : h)
+            if (!std::isfinite(v) || !(v > 0.0f)) return MOE_ERR_INVALID_ARG;
+    }
+    return prepare_weights(w, dst, dst_bytes, S(stream));
+}
+
+size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
+    if (T_max < 0 || H < 1 || I < 1 || E < 1 || B < 0 || topk < 1) return 0;
+    return fwd_layout(T_max, H, I, E, B, topk, wfmt, act_quant).bytes;
+}
+
+moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    const int T = p->T, H = p->H, I = p->I, E = p->E, B = p->B, k = p->topk;
+    if (T < 0 || H < 1 || I < 1 || E < 1 || B < 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+    if (T > p->T_max) return MOE_ERR_INVALID_ARG;  // the workspace was sized for T_max tokens
+    if (E > kMaxExperts || E + B > 1024 || k > kMaxTopk) return MOE_ERR_UNSUPPORTED;
+    if (!act_ok(p->act)) return MOE_ERR_INVALID_ARG;
+    const int G = E + B;
+    const int fmt = p->w_gate.fmt;
+    if (p->w_up.fmt != fmt || p->w_down.fmt != fmt) return MOE_ERR_UNSUPPORTED;
+    moe_status_t s;
+    if ((s = check_weight(p->w_gate, G, I, H)) != MOE_OK) return s;
+    if ((s = check_weight(p->w_up, G, I, H)) != MOE_OK) return s;
+    if ((s = check_weight(p->w_down, G, H, I)) != MOE_OK) return s;
+    if (p->act_quant && fmt != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+    if (H % 16 || I % 16) return MOE_ERR_ALIGNMENT;
+    if (B > 0 && !p->replica_src) return MOE_ERR_INVALID_ARG;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_forward_workspace_size(p->T_max, H, I, E, B, k, fmt, p->act_quant))
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T == 0) return MOE_OK;
+    if (!p->x || !p->router_logits || !p->out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(p->x) || !aligned16(p->out) || !aligned16(ws)) return MOE_ERR_ALIGNMENT;
+
+    const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant);
+    char* w = static_cast<char*>(ws);
+    DevError* err = reinterpret_cast<DevError*>(w);
+    int32_t* ids = p->topk_ids_out ? p->topk_ids_out : reinterpret_cast<int32_t*>(w + L.ids);
+    float* tw = p->topk_w_out ? p->topk_w_out : reinterpret_cast<float*>(w + L.w);
+    int32_t* cu = reinterpret_cast<int32_t*>(w + L.cu);
+    int32_t* perm_token = reinterpret_cast<int32_t*>(w + L.perm_token);
+    float* perm_w = reinterpret_cast<float*>(w + L.perm_w);
+    int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+    void* xperm = w + L.xperm;
+    float* tscale = reinterpret_cast<float*>(w + L.tscale);
+    void* act = w + L.act;
+    __half* act2 = reinterpret_cast<__half*>(w + L.act2);
+    float* act2_scale = reinterpret_cast<float*>(w + L.act2_scale);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(w + L.y);
+    const int NvS = T * k;
+    cudaStream_t st = S(stream);
+    cudaError_t e;
+
+    // S1 route
+    e = launch_route_topk(p->router_logits, T, E, k, ids, tw, st, false);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // S2 permute
+    e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
+                       true);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // S2 gather (+ S2q)
+    if (fmt == MOE_W_BF16) {
+        e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, true);
+    } else if (p->act_quant) {
+        e = launch_quant_nvfp4(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes),
+                               reinterpret_cast<uint8_t*>(w + L.xq_sb), reinterpret_cast<float*>(w + L.xq_s),
+                               reinterpret_cast<__half*>(w + L.xq_deq), st, true);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_gather(1, w + L.xq_deq, H, perm_token, NvS, xperm, reinterpret_cast<float*>(w + L.xq_s), tscale,
+                          st, true);
+    } else {
+        e = launch_gather(2, p->x, H, perm_token, NvS, xperm, nullptr, tscale, st, true);
+    }
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    // S3 + S4: gate/up grouped GEMM with the activation epilogue
+    const bool situ = p->act.act == MOE_ACT_SITU;
+    GemmProblem g1{};
+    g1.x = xperm;
+    g1.M_alloc = NvS;
+    g1.cu_seqlens = cu;
+    g1.G = G;
+    g1.N = I;
+    g1.K = H;
+    g1.wfmt = fmt;
+    g1.dual = true;
+    g1.w0 = p->w_gate.data;
+    g1.w1 = p->w_up.data;
+    g1.kdata0 = p->w_gate.kdata;
+    g1.kscale0 = p->w_gate.kscale;
+    g1.kdata1 = p->w_up.kdata;
+    g1.kscale1 = p->w_up.kscale;
+    g1.alpha0 = weight_alpha(p->w_gate);
+    g1.alpha1 = weight_alpha(p->w_up);
+    g1.perm_w = p->apply_topk_in_fc1 ? perm_w : nullptr;
+    g1.tscale = fmt == MOE_W_BF16 ? nullptr : tscale;
+    g1.out_scale = 1.0f;
+    g1.act = p->act.act;
+    g1.situ_a = p->act.situ_alpha;
+    g1.situ_b = p->act.situ_beta;
+    g1.out = act;
+    g1.err = err;
+    // The down projection's operand: bf16 for BF16 weights; for FP4 weights f16 with a
+    // per-row power-of-two scale (or a fixed one when SITU bounds |h| by alpha*beta),
+    // or NVFP4-quantised rows when act_quant.
+    float fc2_out_scale = 1.0f;
+    const void* fc2_x = act;
+    const float* fc2_tscale = nullptr;
+    bool row_pass = false;
+    if (fmt == MOE_W_BF16) {
+        g1.out_kind = OUT_BF16;
+    } else if (situ && !p->act_quant) {
+        // |h| <= alpha*beta*|route weight| <= alpha*beta: one fixed power of two keeps it below 2^15
+        const double bound = (double)p->act.situ_alpha * p->act.situ_beta;
+        int ex = 0;
+        std::frexp(bound, &ex);
+        const int sh = std::max(0, ex - 15);
+        g1.out_scale = std::ldexp(1.0f, -sh);
+        fc2_out_scale = std::ldexp(1.0f, sh);
+        g1.out_kind = OUT_F16;
+    } else {
+        g1.out_kind = OUT_F32;
+        row_pass = true;
+    }
+    e = launch_grouped_gemm(g1, st, true);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (row_pass) {
+        if (p->act_quant) {
+            e = launch_quant_nvfp4(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.act_codes),
+                                   reinterpret_cast<uint8_t*>(w + L.act_sb), act2_scale, act2, st, true);
+        } else {
+            e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, true);
+        }
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        fc2_x = act2;
+        fc2_tscale = act2_scale;
+    }
+    // S5: down grouped GEMM
+    GemmProblem g2{};
+    g2.x = fc2_x;
+    g2.M_alloc = NvS;
+    g2.cu_seqlens = cu;
+    g2.G = G;
+    g2.N = H;
+    g2.K = I;
+    g2.wfmt = fmt;
+    g2.dual = false;
+    g2.w0 = p->w_down.data;
+    g2.kdata0 = p->w_down.kdata;
+    g2.kscale0 = p->w_down.kscale;
+    g2.alpha0 = weight_alpha(p->w_down);
+    g2.tscale = fc2_tscale;
+    g2.out_scale = fc2_out_scale;
+    g2.out = y;
+    g2.out_kind = OUT_BF16;
+    g2.err = err;
+    e = launch_grouped_gemm(g2, st, true);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // S6: combine
+    e = launch_combine(y, inv, p->apply_topk_in_fc1 ? nullptr : tw, T, k, H, static_cast<__nv_bfloat16*>(p->out), st,
+                       true);
+    return cuda_status(e);
+}
+
+moe_status_t moe_get_device_error(void* ws, moe_stream_t stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    DevError h{0, 0};
+    if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (h.code != 0) {
+        if (cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return MOE_ERR_CUDA;
+        return static_cast<moe_status_t>(h.code);
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+// Internal launch interfaces shared by the .cu files of the library.
+#pragma once
+
+#include <algorithm>
+#include <cstddef>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Launches a kernel with cudaLaunchKernelEx; with `pdl` the launch may begin
+// while the previous kernel on the stream is still running (programmatic
+// dependent launch); every kernel calls griddepcontrol.wait before it reads
+// what its predecessor wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ---------------------------------------------------------------- S1/S2
+cudaError_t launch_route_topk(const float* logits, int T, int E, int topk, int32_t* ids, float* w,
+                              cudaStream_t st, bool pdl);
+
+struct PermuteWs {
+    int nblk;
+    size_t blkcnt, blkoff, total, nrep, rep_ptr, rep_rows, rowstart, bytes;
+};
+PermuteWs permute_ws_layout(int T, int topk, int E, int B);
+cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int topk, int E, int B,
+                           const int32_t* replica_src, int32_t* cu_seqlens, int32_t* perm_token,
+                           float* perm_w, int32_t* inv_perm, DevError* err, char* scratch,
+                           cudaStream_t st, bool pdl);
+cudaError_t launch_gather(int mode, const void* src, int H, const int32_t* perm_token, int NvS,
+                          void* dst, const float* src_scale, float* dst_scale, cudaStream_t st,
+                          bool pdl);
+cudaError_t launch_rows_to_f16(const void* src, bool in_f32, int R, int K, __half* dst, float* scale,
+                               cudaStream_t st, bool pdl);
+
+// ---------------------------------------------------------------- S4/S6/S2q
+cudaError_t launch_act_and_mul(const __nv_bfloat16* gate, const __nv_bfloat16* up,
+                               const float* perm_w, int M, int I, int act, float sa, float sb,
+                               __nv_bfloat16* out, cudaStream_t st, bool pdl);
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, const float* topk_w,
+                           int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
+cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes,
+                               uint8_t* sb, float* s, __half* deq, cudaStream_t st, bool pdl);
+
+// ---------------------------------------------------------------- grouped GEMM
+// Output kinds of the GEMM epilogue.
+enum OutKind { OUT_BF16 = 0, OUT_F16 = 1, OUT_F32 = 2 };
+
+struct GemmProblem {
+    // tokens: [M_alloc, K] bf16 (BF16 weights) or f16 (FP4 weights), row-major
+    const void* x;
+    int M_alloc;
+    const int32_t* cu_seqlens;  // [G] inclusive ends, device
+    int G, N, K;
+    int wfmt;                   // moe_wfmt_t
+    bool dual;                  // gate+up with the activation epilogue
+    // weights: BF16 [G,N,K] (w0 = gate or plain, w1 = up)
+    const void* w0;
+    const void* w1;
+    // FP4 kernel format (prepared)
+    const void* kdata0;
+    const void* kscale0;
+    const void* kdata1;
+    const void* kscale1;
+    const float* alpha0;        // per-row global scale or NULL
+    const float* alpha1;
+    const float* perm_w;        // route weight per token row (dual only) or NULL
+    const float* tscale;        // per token-row scale or NULL
+    float out_scale;
+    int act;
+    float situ_a, situ_b;
+    void* out;                  // [M_alloc, N]
+    int out_kind;               // OutKind
+    bool zero_pad;              // write zeros to rows [cu[G-1], M_alloc)
+    int bt;                     // token tile (0 = choose)
+    DevError* err;
+};
+cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
+int choose_token_tile(long long NvS, int G);
+
+// FP4 kernel layout: tiles of 128 weight rows x 64 K values.
+constexpr int kTileN = 128;
+constexpr int kTileK = 64;
+inline int fp4_scale_bytes_per_row(int wfmt) { return wfmt == MOE_W_MXFP4 ? 2 : 4; }
+
+// ---------------------------------------------------------------- device info
+int num_sms();
+
+}  // namespace moe

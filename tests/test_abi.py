@@ -1,0 +1,150 @@
+"""The C ABI on the CPU: the library loads, exports every symbol include/moe.h declares,
+and rejects bad arguments on the host (status codes, nothing launched, no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_layer_21_b200 as m
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+L = m.lib()
+INVALID, UNSUP, ALIGN, WS_SMALL, NOT_PREP = 1, 2, 3, 4, 8
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 15
+    out = subprocess.run(["nm", "-D", "--defined-only", m.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert sorted(m.EXPORTS) == names
+
+
+def test_status_strings_and_version():
+    assert m.status_string(0) == "MOE_OK"
+    assert m.status_string(8) == "MOE_ERR_NOT_PREPARED"
+    assert m.status_string(99) == "MOE_ERR_UNKNOWN"
+    assert "sm_100a" in m.version()
+
+
+def test_workspace_sizes():
+    assert L.moe_permute_workspace_size(64, 8, 256, 16) > 0
+    assert L.moe_permute_workspace_size(8192, 8, 256, 16) > L.moe_permute_workspace_size(64, 8, 256, 16)
+    a = L.moe_forward_workspace_size(64, 7168, 2048, 256, 16, 8, 0, 0)
+    b = L.moe_forward_workspace_size(8192, 7168, 2048, 256, 16, 8, 0, 0)
+    assert 0 < a < b
+    assert L.moe_forward_workspace_size(1024, 7168, 2048, 256, 0, 8, 2, 1) > \
+        L.moe_forward_workspace_size(1024, 7168, 2048, 256, 0, 8, 0, 0)
+    assert L.moe_forward_workspace_size(-1, 1, 1, 1, 0, 1, 0, 0) == 0
+
+
+def test_prepared_bytes():
+    w = m.moe_weight_t(1, 4, 300, 96)         # MXFP4, G=4, N=300 (3 row tiles), K=96 (2 K tiles)
+    assert L.moe_prepared_weight_bytes(ctypes.byref(w)) >= 4 * 3 * 2 * (128 * 32 + 128 * 2)
+    w.fmt = 0
+    assert L.moe_prepared_weight_bytes(ctypes.byref(w)) == 0
+
+
+def test_route_validation():
+    f = L.moe_route_topk
+    assert f(None, -1, 8, 2, None, None, None) == INVALID
+    assert f(None, 4, 8, 9, None, None, None) == INVALID       # topk > E
+    assert f(None, 4, 8, 0, None, None, None) == INVALID
+    assert f(None, 4, 2048, 2, None, None, None) == UNSUP      # E > 1024
+    assert f(None, 4, 64, 33, None, None, None) == UNSUP      # topk > 32
+    assert f(None, 0, 8, 2, None, None, None) == 0             # no tokens: no-op
+    assert f(None, 4, 8, 2, None, None, None) == INVALID       # null pointers
+
+
+def test_permute_validation():
+    f = L.moe_permute
+    args = lambda **kw: dict(dict(ids=None, w=None, T=4, k=2, E=8, B=0, src=None, x=None, H=0, cu=1,
+                                  pt=None, pw=None, inv=None, xp=None, M=0, ws=1, nws=1 << 20), **kw)
+    call = lambda d: f(d["ids"], d["w"], d["T"], d["k"], d["E"], d["B"], d["src"], d["x"], d["H"],
+                       d["cu"], d["pt"], d["pw"], d["inv"], d["xp"], d["M"], d["ws"], d["nws"], None)
+    assert call(args(k=9)) == INVALID
+    assert call(args(B=2)) == INVALID                         # B > 0 needs replica_src
+    assert call(args(nws=16)) == WS_SMALL
+    assert call(args(xp=16, x=16, H=12, M=8)) == ALIGN        # H % 8
+    assert call(args(xp=16, x=16, H=16, M=4)) == INVALID      # M_alloc < T*k
+    assert call(args()) == INVALID                            # T > 0 with null outputs
+
+
+def _w(fmt, G, N, K, data=16, scale=16, kdata=None):
+    w = m.moe_weight_t(fmt, G, N, K, data, scale if fmt else None, None)
+    if kdata:
+        w.kdata, w.kscale, w.kalpha = kdata, kdata, kdata
+    return w
+
+
+def _fwd(**kw):
+    p = m.moe_forward_args_t()
+    d = dict(T=8, H=64, I=128, E=4, B=0, topk=2, fmt=0, act=0, sa=1.0, sb=1.0, aq=0, T_max=8)
+    d.update(kw)
+    p.x, p.router_logits, p.out = 16, 16, 16
+    p.T, p.H, p.I, p.E, p.B, p.topk, p.T_max = d["T"], d["H"], d["I"], d["E"], d["B"], d["topk"], d["T_max"]
+    G = d["E"] + d["B"]
+    kd = kw.get("kdata")
+    p.w_gate = _w(d["fmt"], G, d["I"], d["H"], kdata=kd)
+    p.w_up = _w(d["fmt"], G, d["I"], d["H"], kdata=kd)
+    p.w_down = _w(d["fmt"], G, d["H"], d["I"], kdata=kd)
+    p.act = m.moe_act_params_t(d["act"], d["sa"], d["sb"])
+    p.act_quant = d["aq"]
+    p.apply_topk_in_fc1 = 1
+    nws = L.moe_forward_workspace_size(d["T_max"], d["H"], d["I"], d["E"], d["B"], d["topk"], d["fmt"], d["aq"])
+    return p, nws
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(act=1, sa=0.0), INVALID),                 # SITU needs alpha > 0
+    (dict(act=1, sb=-1.0), INVALID),
+    (dict(act=7), INVALID),
+    (dict(T=9), INVALID),                           # T > T_max: buffer sized for fewer tokens
+    (dict(topk=5), INVALID),                        # topk > E
+    (dict(fmt=1), NOT_PREP),                        # FP4 weights not prepared
+    (dict(fmt=1, H=48, kdata=16), ALIGN),           # MXFP4 needs K % 32
+    (dict(aq=1), UNSUP),                            # dynamic NVFP4 activations need NVFP4 weights
+    (dict(H=72, I=128), ALIGN),                     # H % 16
+    (dict(B=2), INVALID),                           # replicas without replica_src
+    (dict(E=1100, topk=2), UNSUP),
+])
+def test_forward_validation(kw, expect):
+    p, nws = _fwd(**kw)
+    assert L.moe_forward(ctypes.byref(p), 16, max(nws, 1 << 30), None) == expect
+
+
+def test_forward_small_workspace_and_empty():
+    p, nws = _fwd()
+    assert L.moe_forward(ctypes.byref(p), 16, nws - 1, None) == WS_SMALL
+    p, nws = _fwd(T=0)
+    assert L.moe_forward(ctypes.byref(p), 16, nws, None) == 0   # no tokens: nothing launched
+    p.w_down.N = 63
+    assert L.moe_forward(ctypes.byref(p), 16, nws, None) == INVALID
+
+
+def test_grouped_gemm_and_misc_validation():
+    w = _w(2, 4, 128, 64)
+    assert L.moe_grouped_gemm(16, 8, ctypes.byref(w), 16, 16, 16, 1 << 20, None) == NOT_PREP
+    w = _w(0, 4, 128, 60)
+    assert L.moe_grouped_gemm(16, 8, ctypes.byref(w), 16, 16, 16, 1 << 20, None) == ALIGN
+    w = _w(0, 4, 128, 64)
+    assert L.moe_grouped_gemm(16, 0, ctypes.byref(w), 16, 16, 16, 1 << 20, None) == 0   # no rows
+    assert L.moe_grouped_gemm(16, 8, ctypes.byref(w), 16, 16, 16, 100, None) == WS_SMALL
+    assert L.moe_quantize_nvfp4(16, 0, 4, 24, 16, 16, 16, None, None) == ALIGN
+    assert L.moe_quantize_nvfp4(16, 0, 0, 32, 16, 16, 16, None, None) == 0
+    assert L.moe_combine(16, 16, None, 4, 2, 12, 16, None) == ALIGN
+    assert L.moe_act_and_mul(16, 16, None, 4, 16, m.moe_act_params_t(1, 0.0, 1.0), 16, None) == INVALID
+    wb = _w(0, 4, 128, 64)
+    assert L.moe_prepare_weights(ctypes.byref(wb), None, 0, None) == 0                   # BF16: no-op
+    wm = _w(1, 4, 128, 48)
+    assert L.moe_prepare_weights(ctypes.byref(wm), 16, 1 << 20, None) == ALIGN
