@@ -1,0 +1,434 @@
+"""Benchmark of the fused MoE expert layer on B200s: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one full forward of the layer (route -> permute -> gate/up GEMM with the
+activation -> down GEMM -> combine) over one batch of seeded synthetic inputs. The
+default workload is the Mixtral-shaped BF16 prefill (T=4096, H=4096, I=14336, E=8,
+top-2). With N GPUs (torchrun, one process per GPU) every rank runs its own replica of
+the layer on its own batch: there is no data-path collective ("weak" scaling); the time
+is the max over ranks of the device time.
+
+value   tokens/s over all ranks, inputs resident in HBM, CUDA events on the stream.
+e2e     the same through the public call with pinned host buffers: the H2D copy of x
+        and the router logits and the D2H copy of the output are inside the timed region.
+roofline  the dominant kernel (the gate/up grouped GEMM), algorithmic FLOPs or bytes per
+        launch over its event-timed duration, against MEASURED_PEAKS.json.
+cpu_baseline  the CPU oracle on a bounded token sample, rank 0, N = 1 only.
+
+--impl reference times the CPU oracle alone (the only reference there is: the pages
+describe closed or library kernels), rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer tokens/s on 1 B200; grouped-GEMM TFLOP/s & HBM GB/s as % roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+# ---------------------------------------------------------------------------- accounting
+
+def weight_bytes_per_row(ws: W.WeightSet) -> int:
+    """Bytes of one weight row [N,K] including its scales and alpha."""
+    b = ws.data[0].numel() * ws.data.element_size()
+    if ws.scale is not None:
+        b += ws.scale[0].numel()
+    if ws.alpha is not None:
+        b += 4
+    return b
+
+
+def segment_stats(cfg: W.MoEConfig, topk_ids: torch.Tensor, replica_src: torch.Tensor):
+    """Non-empty weight rows and the largest segment of one step, from the top-k ids the
+    library produced (bookkeeping for the roofline, outside the timed region): expert e
+    with n_e assignments and R_e rows (itself plus its used replicas) fills min(n_e, R_e)
+    rows, the largest holding ceil(n_e / R_e)."""
+    n = torch.bincount(topk_ids.reshape(-1).long().cpu(), minlength=cfg.E).numpy()
+    R = np.ones(cfg.E, dtype=np.int64)
+    for s in replica_src.tolist():
+        if s >= 0:
+            R[s] += 1
+    nonempty = int(np.minimum(n, R).sum())
+    max_seg = int(np.max(-(-n // R))) if cfg.E else 0
+    return nonempty, max_seg
+
+
+def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) -> dict:
+    NvS = cfg.NvS
+    wg, wu, wd = (weight_bytes_per_row(inp.w_gate), weight_bytes_per_row(inp.w_up),
+                  weight_bytes_per_row(inp.w_down))
+    act_out = 2 if cfg.wfmt == "bf16" or (cfg.act == "situ" and not cfg.act_quant) else 4
+    fc1_flops = 4.0 * NvS * cfg.H * cfg.I
+    fc2_flops = 2.0 * NvS * cfg.H * cfg.I
+    fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * 2 + NvS * cfg.I * act_out
+    fc2_bytes = nonempty * wd + NvS * cfg.I * 2 + NvS * cfg.H * 2
+    layer_bytes = nonempty * (wg + wu + wd) + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
+    return dict(nonempty=nonempty, max_seg=max_seg,
+                fc1_flops=fc1_flops, fc2_flops=fc2_flops, fc1_bytes=fc1_bytes, fc2_bytes=fc2_bytes,
+                layer_flops=fc1_flops + fc2_flops, layer_bytes=layer_bytes,
+                weight_bytes_total=nonempty * (wg + wu + wd))
+
+
+def load_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "common.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_21_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str) -> float | None:
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary, if the
+    summary was taken on the kernel source as it is now; else None."""
+    p = os.path.join(ROOT, "profiles", f"grouped_gemm_fc1_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            p = torch.cuda.get_device_properties(index)
+            ids = [getattr(p, n, None) for n in ("pci_domain_id", "pci_bus_id", "pci_device_id")]
+            if all(isinstance(v, int) for v in ids):
+                bus = "%08X:%02X:%02X.0" % tuple(ids)   # NVML wants the string form
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: report it
+            self.err = str(e)
+        self.period = period_s
+        self.samples = []
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = self._reasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self) -> dict:
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        mhz = [s[0] for s in busy]
+        reasons = set()
+        for _, r, _ in busy:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(busy), "source": "nvml"}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(cfg, inp, tokens):
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
+                  inp.w_down, tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def default_sample(cfg) -> int:
+    """Token sample for one oracle call: about a few seconds of fp64 work on 8+ cores."""
+    flops_per_token = 6.0 * cfg.topk * cfg.H * cfg.I
+    return int(max(1, min(cfg.T, 1.5e11 // flops_per_token)))
+
+
+# ---------------------------------------------------------------------------- arms
+
+def kernel_launches(cfg) -> int:
+    n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
+    if cfg.act_quant:
+        n += 2                            # x quantisation, activation quantisation
+    elif cfg.wfmt != "bf16" and cfg.act != "situ":
+        n += 1                            # activation row pass to f16
+    return n
+
+
+def run_ours(args, cfg, rank, world):
+    import mixture_experts_layer_21_b200 as m
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = W.gen_inputs(cfg)
+    ws = [m.Weight.from_host(w, dev) for w in (inp.w_gate, inp.w_up, inp.w_down)]
+    layer = m.MoEForward(*ws, cfg.E, cfg.topk, cfg.B,
+                         inp.replica_src.to(dev) if cfg.B else None, cfg.act, cfg.situ_alpha,
+                         cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T)
+    x_d, l_d = inp.x.to(dev), inp.logits.to(dev)
+    out_d = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    K, Wm = args.steps, args.warmup
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+            torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    ids_d = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device=dev)
+    for _ in range(Wm):
+        layer(x_d, l_d, out=out_d, topk_ids=ids_d)
+    assert layer.device_error() == 0, "device error in warm-up"
+    acc = accounting(cfg, inp, *segment_stats(cfg, ids_d, inp.replica_src))
+
+    # ---- device-resident timed region, stage events on the launching stream
+    nst = m.MOE_FWD_STAGE_EVENTS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(stream)
+        for i in range(K):
+            layer(x_d, l_d, out=out_d, stage_events=evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nst - 1)]
+                         for i in range(K)]).mean(axis=0)
+    assert layer.device_error() == 0, "device error in timed region"
+
+    # ---- end to end through the public call, host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_h = inp.x.pin_memory()
+        l_h = inp.logits.pin_memory()
+        o_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            l_d.copy_(l_h, non_blocking=True)
+            layer(x_d, l_d, out=out_d)
+            o_h.copy_(out_d, non_blocking=True)
+
+        for _ in range(Wm):
+            e2e_step()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1))
+        e2e = {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 4),
+               "d2h_bytes_per_step": int(o_h.numel() * 2)}
+
+    peaks, peak_src = load_peaks()
+    ms_step = ms_total / K
+    fc1_ms = float(stage_ms[2])
+    t_fc1_tensor = acc["fc1_flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_fc1_hbm = acc["fc1_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    traffic = profiled_traffic(args.config)
+    if t_fc1_tensor >= t_fc1_hbm:
+        ach = acc["fc1_flops"] / (fc1_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"]}
+    else:
+        ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    roof.update({"traffic": traffic, "kernel": "grouped_gemm_kernel gate+up (fused activation)",
+                 "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
+                 "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst)"})
+    t_layer_roof = max(acc["layer_flops"] / (peaks["bf16_tflops"] * 1e12),
+                       acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    tok_s = world * cfg.T * K / (ms_total / 1e3)
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        S = default_sample(cfg)
+        toks = list(range(S))
+        dt = oracle_sample(cfg, inp, toks)
+        cpu = {"value": S / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{S} of {cfg.T} tokens (routing and permutation of all {cfg.T}), "
+                         f"fp64 NumPy, {dt:.1f} s"}
+
+    res = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.wfmt == "bf16" else "f16",
+        "data": "synthetic (seeded; random weights of the workload's shapes)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
+                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: weights touched per step {acc['weight_bytes_total'] / 1e9:.2f} GB "
+                         f"> L2 {L2_BYTES / 2 ** 20:.0f} MiB",
+                   "nonempty_segments": acc["nonempty"], "max_segment": acc["max_seg"]},
+        "roofline": roof,
+        "layer_roofline": {"t_roof_ms": t_layer_roof * 1e3, "frac": t_layer_roof * 1e3 / ms_step,
+                           "flops": acc["layer_flops"], "bytes": acc["layer_bytes"],
+                           "tflops": acc["layer_flops"] / (ms_step * 1e-3) / 1e12,
+                           "gbs": acc["layer_bytes"] / (ms_step * 1e-3) / 1e9},
+        "stage_ms": {n: float(v) for n, v in zip(
+            ["route", "permute_gather", "gate_up_gemm", "act_row_pass", "down_gemm", "combine"], stage_ms)},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernel_launches(cfg) * K,
+        "clocks": clk.summary(),
+    }
+    return res
+
+
+def run_reference(args, cfg):
+    """The CPU oracle on the host cores, each step a bounded token sample."""
+    inp = W.gen_inputs(cfg)
+    S = max(1, default_sample(cfg) // 4)
+    K, Wm = args.steps, args.warmup
+    # keep the whole run within a few minutes: shrink the sample if a calibration step is slow
+    dt0 = oracle_sample(cfg, inp, list(range(min(S, cfg.T))))
+    while S > 1 and dt0 * (K + Wm) > 240:
+        S = max(1, S // 2)
+        dt0 = oracle_sample(cfg, inp, list(range(min(S, cfg.T))))
+    for i in range(Wm):
+        oracle_sample(cfg, inp, [(i * S + j) % cfg.T for j in range(S)])
+    t = 0.0
+    for i in range(K):
+        t += oracle_sample(cfg, inp, [((Wm + i) * S + j) % cfg.T for j in range(S)])
+    val = S * K / t
+    cores = cpu_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1,
+        "steps": K, "warmup": Wm, "ms_per_step": t / K * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
+                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{S} tokens per step of {cfg.T} (routing of all), fp64 NumPy"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="mixtral_prefill", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = W.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, cfg, rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

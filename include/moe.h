@@ -210,7 +210,14 @@ moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,
  *   0 applies it in the combine (FlashInfer MoE-EP page, apply_topk_in_fc1).
  *   topk_ids_out/topk_w_out: optional [T,topk] copies of the routing.
  *   T <= T_max given to moe_forward_workspace_size, else INVALID_ARG.
+ *   stage_events: optional array of MOE_FWD_STAGE_EVENTS caller-created cudaEvent_t,
+ *   recorded on `stream` at the stage boundaries: [0] start, [1] after S1 routing,
+ *   [2] after S2 permutation/gather (and x quantisation), [3] after S3+S4 gate/up
+ *   GEMM, [4] after the activation row pass (== [3] when there is none),
+ *   [5] after S5 down GEMM, [6] after S6 combine. Recording an event between two
+ *   kernels stops them overlapping through programmatic dependent launch.
  */
+#define MOE_FWD_STAGE_EVENTS 7
 typedef struct {
     const void* x;
     const float* router_logits;
@@ -224,6 +231,7 @@ typedef struct {
     int32_t* topk_ids_out;          /* optional */
     float* topk_w_out;              /* optional */
     int32_t T_max;                  /* capacity the workspace was sized for */
+    void* const* stage_events;      /* optional: MOE_FWD_STAGE_EVENTS cudaEvent_t */
 } moe_forward_args_t;
 
 size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,

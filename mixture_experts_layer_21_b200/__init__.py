@@ -65,7 +65,9 @@ class moe_forward_args_t(ctypes.Structure):
                 ("act", moe_act_params_t), ("apply_topk_in_fc1", ctypes.c_int32),
                 ("act_quant", ctypes.c_int32), ("out", ctypes.c_void_p),
                 ("topk_ids_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
-                ("T_max", ctypes.c_int32)]
+                ("T_max", ctypes.c_int32), ("stage_events", ctypes.c_void_p)]
+
+MOE_FWD_STAGE_EVENTS = 7
 
 
 _P, _I, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -283,8 +285,18 @@ class MoEForward:
                                     w_gate.data.device)
         self.args = moe_forward_args_t()
 
-    def __call__(self, x, router_logits, out=None, topk_ids=None, topk_w=None, stream=None):
+    def __call__(self, x, router_logits, out=None, topk_ids=None, topk_w=None, stream=None,
+                 stage_events=None):
+        """``stage_events``: None, or MOE_FWD_STAGE_EVENTS recorded torch.cuda.Event objects
+        (created with enable_timing and recorded once, so that their handles exist)."""
         T = x.shape[0]
+        if stage_events is not None:
+            if len(stage_events) != MOE_FWD_STAGE_EVENTS:
+                raise ValueError(f"need {MOE_FWD_STAGE_EVENTS} events")
+            self._ev = (ctypes.c_void_p * MOE_FWD_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
+            self.args.stage_events = ctypes.cast(self._ev, ctypes.c_void_p)
+        else:
+            self.args.stage_events = None
         out = out if out is not None else torch.empty(T, self.H, dtype=torch.bfloat16, device=x.device)
         a = self.args
         a.x, a.router_logits = _ptr(x), _ptr(router_logits)
