@@ -6,7 +6,7 @@ entry points' names (see ``include/moe.h``); each takes and returns torch
 tensors on the current CUDA device and launches on the current stream.
 
 There is no fallback: if the shared library is missing the import fails.
-Build it with ``python -m mixture_experts_layer_21_b200.build``.
+Build it with ``python mixture_experts_layer_21_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: run `python -m mixture_experts_layer_21_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: run `python mixture_experts_layer_21_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

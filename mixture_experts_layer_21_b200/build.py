@@ -5,7 +5,9 @@ the FP4 conversions need it) into an object, in parallel, then linked into one
 shared library with the CUDA runtime linked statically. Objects are rebuilt only
 when a source or header is newer.
 
-    python -m mixture_experts_layer_21_b200.build [--force] [-j N] [--verbose]
+    python mixture_experts_layer_21_b200/build.py [--force] [-j N] [--verbose] [--ptxas-v]
+
+(run it by path: importing the package loads the library, which may not exist yet)
 """
 from __future__ import annotations
 
