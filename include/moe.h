@@ -136,6 +136,31 @@ moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, in
                          void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_permute without a workspace argument. The pages have no counterpart: it
+ * exists for callers that cannot allocate, such as an operator that is handed only
+ * its input and output pointers by another runtime, or a serving loop with a fixed
+ * memory plan where cudaMalloc (which also synchronises the device) is not allowed.
+ * Arguments and results are those of moe_permute, minus ws/ws_bytes; it calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   Scratch: a 1 MiB array of device memory inside the library, present on every
+ *   GPU that loads it until the process exits. Sizes whose scratch would not fit
+ *   (about 2*ceil(T/256)*E*4 bytes plus small tables) return
+ *   MOE_ERR_WORKSPACE_TOO_SMALL with nothing launched.
+ *   The first call on a device looks up that array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (two streams,
+ *   two host threads) race and must be serialised by the caller. An expert id
+ *   outside [0,E) is skipped (its inv_perm entry is -1); unlike moe_permute the
+ *   error word is internal and cleared at every call.
+ */
+moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w, int T, int topk,
+                                 int E, int B, const int32_t* replica_src,
+                                 const void* x, int H,
+                                 int32_t* cu_seqlens, int32_t* perm_token, float* perm_w,
+                                 int32_t* inv_perm, void* x_perm, int M_alloc,
+                                 moe_stream_t stream);
+
+/*
  * S3/S5 — grouped GEMM: out[seg_g] = alpha_g * a[seg_g] @ W[g]^T for every
  * cu_seqlens segment; rows [cu_seqlens[G-1], M_alloc) of out are written as zero
  * (MoonEP page, moonep_grouped_gemm). Empty segments are skipped.

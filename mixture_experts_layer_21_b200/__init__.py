@@ -35,7 +35,7 @@ WFMT = {"bf16": 0, "mxfp4": 1, "nvfp4": 2}
 EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_workspace_size",
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
-           "moe_forward_workspace_size", "moe_forward", "moe_get_device_error"]
+           "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc"]
 
 
 class MoEError(RuntimeError):
@@ -87,6 +87,7 @@ _sig = {
     "moe_forward_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "moe_forward": (_I, [ctypes.POINTER(moe_forward_args_t), _P, _S, _P]),
     "moe_get_device_error": (_I, [_P, _P]),
+    "moe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
