@@ -94,7 +94,7 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.act2_scale = take(fp4 ? 4 * NvS : 0);
     L.act_codes = take(act_quant ? NvS * I / 2 : 0);
     L.act_sb = take(act_quant ? NvS * I / 16 : 0);
-    L.y = take(2 * NvS * H);
+    L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
     L.bytes = off;
     return L;
 }
@@ -308,7 +308,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     void* act = w + L.act;
     __half* act2 = reinterpret_cast<__half*>(w + L.act2);
     float* act2_scale = reinterpret_cast<float*>(w + L.act2_scale);
-    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(w + L.y);
+    float* y = reinterpret_cast<float*>(w + L.y);
     const int NvS = T * k;
     cudaStream_t st = S(stream);
     cudaError_t e;
@@ -422,13 +422,13 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.tscale = fc2_tscale;
     g2.out_scale = fc2_out_scale;
     g2.out = y;
-    g2.out_kind = OUT_BF16;
+    g2.out_kind = OUT_F32;
     g2.err = err;
     e = launch_grouped_gemm(g2, st, pdl);
     if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
     // S6: combine
-    e = launch_combine(y, inv, p->apply_topk_in_fc1 ? nullptr : tw, T, k, H, static_cast<__nv_bfloat16*>(p->out), st,
-                       pdl);
+    e = launch_combine_f32(y, inv, p->apply_topk_in_fc1 ? nullptr : tw, T, k, H, static_cast<__nv_bfloat16*>(p->out),
+                           st, pdl);
     if (e != cudaSuccess || !mark(6)) return MOE_ERR_CUDA;
     return MOE_OK;
 }

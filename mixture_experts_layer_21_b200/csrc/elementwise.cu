@@ -48,8 +48,28 @@ cudaError_t launch_act_and_mul(const __nv_bfloat16* gate, const __nv_bfloat16* u
 
 // ----------------------------------------------------------------- S6
 // out[t] = sum_k w[t,k] * y[inv_perm[t,k]], fp32 in k order, one bf16 rounding.
-// Grid (T, ceil(H / 1024)); each thread owns 8 contiguous columns.
-__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __restrict__ y,
+// Grid (T, ceil(H / 1024)); each thread owns 8 contiguous columns. y is bf16 (the
+// standalone entry point) or fp32 (the fused layer keeps the down projection's rows
+// in fp32 so that the output is rounded to bf16 once).
+__device__ __forceinline__ void load8(const __nv_bfloat16* y, size_t row, int H, int c8, float (&f)[8]) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + row * H) + c8);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 g = __bfloat1622float2(p[q]);
+        f[2 * q] = g.x;
+        f[2 * q + 1] = g.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* y, size_t row, int H, int c8, float (&f)[8]) {
+    const float4* p = reinterpret_cast<const float4*>(y + row * H) + 2 * c8;
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <typename YT>
+__global__ void __launch_bounds__(128) combine_kernel(const YT* __restrict__ y,
                                                       const int32_t* __restrict__ inv_perm,
                                                       const float* __restrict__ topk_w, int T,
                                                       int topk, int H,
@@ -64,19 +84,10 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16* __res
         for (int j = 0; j < topk; ++j) {
             const int r = inv_perm[(size_t)t * topk + j];
             const float wj = topk_w ? topk_w[(size_t)t * topk + j] : 1.0f;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + (size_t)r * H) + c8);
-            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+            float f[8];
+            load8(y, (size_t)r, H, c8, f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __bfloat1622float2(p[q]);
-                if (topk_w) {
-                    acc[2 * q] = fmaf(wj, f.x, acc[2 * q]);
-                    acc[2 * q + 1] = fmaf(wj, f.y, acc[2 * q + 1]);
-                } else {
-                    acc[2 * q] += f.x;
-                    acc[2 * q + 1] += f.y;
-                }
-            }
+            for (int q = 0; q < 8; ++q) acc[q] = topk_w ? fmaf(wj, f[q], acc[q]) : acc[q] + f[q];
         }
         uint4 o;
         __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -92,7 +103,15 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, cons
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl) {
     if (T == 0) return cudaSuccess;
     dim3 grid(T, (H / 8 + 127) / 128);
-    return launch_k(combine_kernel, grid, dim3(128), 0, st, pdl, y, inv_perm, topk_w, T, topk, H, out);
+    return launch_k(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, pdl, y, inv_perm, topk_w, T, topk,
+                    H, out);
+}
+
+cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T, int topk,
+                               int H, __nv_bfloat16* out, cudaStream_t st, bool pdl) {
+    if (T == 0) return cudaSuccess;
+    dim3 grid(T, (H / 8 + 127) / 128);
+    return launch_k(combine_kernel<float>, grid, dim3(128), 0, st, pdl, y, inv_perm, topk_w, T, topk, H, out);
 }
 
 // ----------------------------------------------------------------- S2q

@@ -14,11 +14,17 @@
 // CTAs working on one weight block at the same time share it through L2.
 //
 // Warp roles (one CTA per SM):
-//   warp 0      TMA producer (one thread): weight tile(s) + token tile per K step
-//   warp 1      MMA issuer (one thread) + TMEM owner; accumulators double-buffered
-//   warps 2..5  epilogue: TMEM -> registers -> alpha / activation / scales -> global
-//   warps 6..9  (FP4 weights only) e2m1 -> f16 converters writing the swizzled
-//               operand the MMA reads (FP4 dequant fused into the mainloop)
+//   warp 0       producer (one thread): TMA / bulk copies per K step
+//   warp 1       MMA issuer (one thread) + TMEM owner; accumulators double-buffered
+//   warps 2..5   epilogue: TMEM -> registers -> alpha / activation / scales -> global
+//   warps 6..13  (FP4 weights only) e2m1 -> f16 converters writing the swizzled
+//                operand the MMA reads (FP4 dequant fused into the mainloop)
+// Pipelines:
+//   BF16 weights: one ring of stages {gate tile, [up tile], token tile}.
+//   FP4 weights: a deep ring of small raw stages {token tile, packed e2m1 codes,
+//   block scales} that keeps enough bytes in flight to stream HBM, feeding a
+//   shallow ring of converted f16 weight tiles. The MMA reads weights from the
+//   converted ring and tokens straight from the raw stage.
 // Every wait is bounded; a timeout records MOE_ERR_TIMEOUT in the error word,
 // stops all roles, lets copies in flight land, frees TMEM and returns.
 #include <mutex>
@@ -27,27 +33,36 @@
 
 namespace moe {
 
-constexpr int kMaxG = 1024;  // segment table capacity (weight rows)
+constexpr int kMaxG = 1024;      // segment table capacity (weight rows)
+constexpr int kMaxStages = 16;
+
+__host__ __device__ constexpr int round1024(int b) { return (b + 1023) & ~1023; }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 template <int BT, bool DUAL, int WFMT>
 struct GemmCfg {
+    static constexpr bool FP4 = WFMT != MOE_W_BF16;
     static constexpr int NB = DUAL ? 2 : 1;
     static constexpr int A_BYTES = kTileN * kTileK * 2;      // 16 KB: 128 rows x 64 x 16-bit
     static constexpr int B_BYTES = BT * kTileK * 2;          // BT rows x 64 x 16-bit
     static constexpr int RAW_D = kTileN * kTileK / 2;        // 4 KB of packed e2m1
     static constexpr int RAW_S = WFMT == MOE_W_MXFP4 ? kTileN * 2 : (WFMT == MOE_W_NVFP4 ? kTileN * 4 : 0);
-    static constexpr int RAW_BYTES = WFMT == MOE_W_BF16 ? 0 : NB * (RAW_D + RAW_S);
-    static constexpr int STAGE_BYTES = NB * A_BYTES + B_BYTES + RAW_BYTES;
+    // operand stage: weights (+ tokens for BF16); raw stage (FP4): tokens, codes, scales
+    static constexpr int OP_STAGE = NB * A_BYTES + (FP4 ? 0 : B_BYTES);
+    static constexpr int RAW_STAGE = FP4 ? round1024(B_BYTES + NB * (RAW_D + RAW_S)) : 0;
     static constexpr int CTRL_BYTES = 12288;
     static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int BUDGET = SMEM_LIMIT - 1024 - CTRL_BYTES;
+    static constexpr int STAGES = FP4 ? (BT >= 64 ? 4 : 3) : cmin(kMaxStages, BUDGET / OP_STAGE);
+    static constexpr int RSTAGES = FP4 ? cmin(kMaxStages, (BUDGET - STAGES * OP_STAGE) / RAW_STAGE) : 0;
     static constexpr int TMEM_USED = 2 * NB * BT;
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
-    static constexpr int CONV_WARPS = WFMT == MOE_W_BF16 ? 0 : 4;
+    static constexpr int CONV_WARPS = FP4 ? 8 : 0;
+    static constexpr int CONV_THREADS = CONV_WARPS * 32;
     static constexpr int THREADS = (6 + CONV_WARPS) * 32;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
-    static_assert(STAGES >= 2, "pipeline needs two stages");
+    static constexpr int SMEM_BYTES = 1024 + STAGES * OP_STAGE + RSTAGES * RAW_STAGE + CTRL_BYTES;
+    static_assert(STAGES >= 2 && (!FP4 || RSTAGES >= 2), "pipeline needs two stages");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
     static_assert(TMEM_USED <= 512, "accumulators exceed TMEM");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
 };
@@ -72,7 +87,9 @@ struct GemmArgs {
 };
 
 struct CtrlBlock {
-    uint64_t full[8], empty[8], raw_full[8], tfull[2], tempty[2], drain;
+    uint64_t full[kMaxStages], empty[kMaxStages];          // operand ring
+    uint64_t raw_full[kMaxStages], raw_empty[kMaxStages];  // raw ring (FP4)
+    uint64_t tfull[2], tempty[2], drain;
     uint32_t tmem_slot;
     int abort;
     uint16_t lut[256];
@@ -100,29 +117,28 @@ __device__ __forceinline__ void decode_tile(int L, const CtrlBlock* c, int G, in
     rows = min(BT, c->cu[g] - row0);
 }
 
-__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
-    uint32_t r;
-    asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(r) : "r"(byte));
-    return r;
-}
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
     return *reinterpret_cast<uint32_t*>(&r);
 }
-// 32 packed e2m1 values (16 bytes) times one f16 scale -> 4 x 16-byte swizzled chunks.
+// 8 packed e2m1 values (one 32-bit word, even k in the low nibble) -> 4 x f16x2, times a scale.
+__device__ __forceinline__ uint4 e2m1x8_to_f16(uint32_t w, uint32_t sc2) {
+    uint32_t o0, o1, o2, o3;
+    asm("{ .reg .b8 b0,b1,b2,b3; mov.b32 {b0,b1,b2,b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(w));
+    return make_uint4(hmul2_u32(o0, sc2), hmul2_u32(o1, sc2), hmul2_u32(o2, sc2), hmul2_u32(o3, sc2));
+}
+// 32 values (half a 64-value row) -> 4 x 16-byte chunks of the 128-byte-swizzled operand row.
 __device__ __forceinline__ void convert_half_row(const uint4 raw, uint32_t sc2_lo, uint32_t sc2_hi,
                                                  uint8_t* row_base, int r, int c_first) {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t sc = i < 2 ? sc2_lo : sc2_hi;
-        uint4 o;
-        o.x = hmul2_u32(e2m1x2_f16x2(w[i] & 0xFF), sc);
-        o.y = hmul2_u32(e2m1x2_f16x2((w[i] >> 8) & 0xFF), sc);
-        o.z = hmul2_u32(e2m1x2_f16x2((w[i] >> 16) & 0xFF), sc);
-        o.w = hmul2_u32(e2m1x2_f16x2(w[i] >> 24), sc);
-        const int c = c_first + i;
-        *reinterpret_cast<uint4*>(row_base + ((c ^ (r & 7)) << 4)) = o;
+        const uint4 o = e2m1x8_to_f16(w[i], i < 2 ? sc2_lo : sc2_hi);
+        *reinterpret_cast<uint4*>(row_base + (((c_first + i) ^ (r & 7)) << 4)) = o;
     }
 }
 
@@ -134,12 +150,18 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     using C = GemmCfg<BT, DUAL, WFMT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA0 = smem;
-    uint8_t* sA1 = sA0 + C::STAGES * C::A_BYTES;
-    uint8_t* sB = sA1 + (DUAL ? C::STAGES * C::A_BYTES : 0);
-    uint8_t* sRaw = sB + C::STAGES * C::B_BYTES;
-    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(sRaw + C::STAGES * C::RAW_BYTES);
+    // operand ring: stage s = [A0][A1 if dual][B if BF16]; raw ring (FP4): [B][D0][D1][S0][S1]
+    uint8_t* sOp = smem;
+    uint8_t* sRaw = sOp + C::STAGES * C::OP_STAGE;
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(sRaw + C::RSTAGES * C::RAW_STAGE);
     volatile int* abort_flag = &ctl->abort;
+    auto opA = [&](int s, int m) { return sOp + s * C::OP_STAGE + m * C::A_BYTES; };
+    auto opB = [&](int s) { return sOp + s * C::OP_STAGE + C::NB * C::A_BYTES; };
+    auto rawB = [&](int r) { return sRaw + r * C::RAW_STAGE; };
+    auto rawD = [&](int r, int m) { return sRaw + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_D; };
+    auto rawS = [&](int r, int m) {
+        return sRaw + r * C::RAW_STAGE + C::B_BYTES + C::NB * C::RAW_D + m * C::RAW_S;
+    };
 
     const int warp = warp_id(), lane = lane_id();
     const int G = a.G, NT = a.NT, KB = a.KB;
@@ -147,9 +169,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     // ---------------- prologue: independent of the previous kernel's output
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1 + C::CONV_WARPS);
+            mbar_init(&ctl->full[s], C::FP4 ? C::CONV_WARPS : 1);
             mbar_init(&ctl->empty[s], 1);
-            mbar_init(&ctl->raw_full[s], 1);
+        }
+        for (int r = 0; r < C::RSTAGES; ++r) {
+            mbar_init(&ctl->raw_full[r], 1);
+            mbar_init(&ctl->raw_empty[r], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
@@ -161,7 +186,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     }
     if (threadIdx.x == 32) {
         tma_prefetch_desc(&tm_x);
-        if (WFMT == MOE_W_BF16) {
+        if (!C::FP4) {
             tma_prefetch_desc(&tm_w0);
             if (DUAL) tma_prefetch_desc(&tm_w1);
         }
@@ -183,7 +208,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     }
     pdl_wait();
     if (warp == 0) {
-        // segment table: cu (inclusive ends) and the running tile count
+        // segment table: cu (inclusive ends) and the running tile count.
         // Ends are clamped to [0, M_alloc] and a segment whose end lies before the
         // previous end counts as empty, so no tile can touch rows outside the buffers.
         int carry = 0, prev_chunk_end = 0;
@@ -207,7 +232,6 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                 ctl->tpre[g + 1] = carry + incl;
             }
             carry += __shfl_sync(0xffffffffu, incl, 31);
-            // running end for the next chunk: the last lane's effective end
             const int eff = g < G ? (len > 0 ? end : prev) : prev;
             prev_chunk_end = __shfl_sync(0xffffffffu, eff, 31);
         }
@@ -221,42 +245,41 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     const int total = ctl->tpre[G];
 
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- producer
         if (lane == 0) {
+            constexpr int NS = C::FP4 ? C::RSTAGES : C::STAGES;
+            uint64_t* fullb = C::FP4 ? ctl->raw_full : ctl->full;
+            uint64_t* emptyb = C::FP4 ? ctl->raw_empty : ctl->empty;
             int s = 0;
-            uint32_t ph = 0;
-            uint32_t issued_mask = 0, issued_par = 0;
+            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&emptyb[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (WFMT == MOE_W_BF16) {
-                        mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
-                        tma_load_3d(sA0 + s * C::A_BYTES, &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g);
-                        if (DUAL)
-                            tma_load_3d(sA1 + s * C::A_BYTES, &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g);
+                    if (!C::FP4) {
+                        mbar_arrive_expect_tx(&fullb[s], C::NB * C::A_BYTES + C::B_BYTES);
+                        tma_load_3d(opA(s, 0), &tm_w0, &fullb[s], kb * kTileK, nt * kTileN, g);
+                        if (DUAL) tma_load_3d(opA(s, 1), &tm_w1, &fullb[s], kb * kTileK, nt * kTileN, g);
+                        tma_load_2d(opB(s), &tm_x, &fullb[s], kb * kTileK, row0);
                     } else {
-                        uint8_t* raw = sRaw + s * C::RAW_BYTES;
                         const size_t tile = ((size_t)g * NT + nt) * KB + kb;
-                        mbar_arrive_expect_tx(&ctl->raw_full[s], C::RAW_BYTES);
-                        bulk_load(raw, a.kd0 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[s]);
-                        bulk_load(raw + C::NB * C::RAW_D, a.ks0 + tile * C::RAW_S, C::RAW_S, &ctl->raw_full[s]);
+                        mbar_arrive_expect_tx(&fullb[s], C::B_BYTES + C::NB * (C::RAW_D + C::RAW_S));
+                        bulk_load(rawD(s, 0), a.kd0 + tile * C::RAW_D, C::RAW_D, &fullb[s]);
+                        bulk_load(rawS(s, 0), a.ks0 + tile * C::RAW_S, C::RAW_S, &fullb[s]);
                         if (DUAL) {
-                            bulk_load(raw + C::RAW_D, a.kd1 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[s]);
-                            bulk_load(raw + C::NB * C::RAW_D + C::RAW_S, a.ks1 + tile * C::RAW_S, C::RAW_S,
-                                      &ctl->raw_full[s]);
+                            bulk_load(rawD(s, 1), a.kd1 + tile * C::RAW_D, C::RAW_D, &fullb[s]);
+                            bulk_load(rawS(s, 1), a.ks1 + tile * C::RAW_S, C::RAW_S, &fullb[s]);
                         }
-                        mbar_arrive_expect_tx(&ctl->full[s], C::B_BYTES);
+                        tma_load_2d(rawB(s), &tm_x, &fullb[s], kb * kTileK, row0);
                     }
-                    tma_load_2d(sB + s * C::B_BYTES, &tm_x, &ctl->full[s], kb * kTileK, row0);
                     issued_mask |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
-                    if (++s == C::STAGES) {
+                    if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -267,21 +290,16 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                 ctl->abort = 1;
                 // let every copy this thread issued land before the CTA exits
                 int never = 0;
-                for (int q = 0; q < C::STAGES; ++q) {
-                    if (issued_mask >> q & 1u) {
-                        const uint32_t p = issued_par >> q & 1u;
-                        mbar_wait(&ctl->full[q], p, &never);
-                        if (WFMT != MOE_W_BF16) mbar_wait(&ctl->raw_full[q], p, &never);
-                    }
-                }
+                for (int q = 0; q < NS; ++q)
+                    if (issued_mask >> q & 1u) mbar_wait(&fullb[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(WFMT == MOE_W_BF16 ? 1 : 0, kTileN, BT);
-            int s = 0, b = 0;
-            uint32_t ph = 0, bph = 0;
+            constexpr uint32_t idesc = idesc_f16(C::FP4 ? 0 : 1, kTileN, BT);
+            int s = 0, r = 0, b = 0;
+            uint32_t ph = 0, rph = 0, bph = 0;
             bool ok = true, issued = false;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
@@ -291,14 +309,15 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::NB * BT);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag)) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) ||
+                        (C::FP4 && !mbar_wait(&ctl->raw_full[r], rph, abort_flag))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA0 + s * C::A_BYTES);
-                    const uint32_t a1 = smem_u32(sA1 + s * C::A_BYTES);
-                    const uint32_t bb = smem_u32(sB + s * C::B_BYTES);
+                    const uint32_t a0 = smem_u32(opA(s, 0));
+                    const uint32_t a1 = smem_u32(opA(s, DUAL ? 1 : 0));
+                    const uint32_t bb = smem_u32(C::FP4 ? rawB(r) : opB(s));
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint64_t bdesc = sw128_kmajor_desc(bb + kk * 32);
@@ -311,6 +330,13 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                     if (++s == C::STAGES) {
                         s = 0;
                         ph ^= 1u;
+                    }
+                    if (C::FP4) {
+                        mma_commit(&ctl->raw_empty[r]);
+                        if (++r == C::RSTAGES) {
+                            r = 0;
+                            rph ^= 1u;
+                        }
                     }
                 }
                 if (!ok) break;
@@ -395,42 +421,41 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
         }
     } else if (C::CONV_WARPS > 0) {
         // ---------------- FP4 -> f16 converters (FP4 dequant fused into the mainloop)
-        const int ct = threadIdx.x - 6 * 32;  // 0..127
-        int s = 0;
-        uint32_t ph = 0;
-        for (int L = blockIdx.x; L < total; L += gridDim.x) {
-            bool ok = true;
+        const int ct = threadIdx.x - 6 * 32;  // 0 .. CONV_THREADS-1
+        int s = 0, r = 0;
+        uint32_t ph = 0, rph = 0;
+        bool ok = true;
+        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&ctl->raw_full[s], ph, abort_flag)) {
+                if (!mbar_wait(&ctl->raw_full[r], rph, abort_flag) ||
+                    !mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                     if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 4);
                     ctl->abort = 1;
                     ok = false;
                     break;
                 }
-                const uint8_t* raw = sRaw + s * C::RAW_BYTES;
+                // items: (matrix m, row, half) -> 16 raw bytes = 32 values each; contiguous reads
+                constexpr int ITEMS = C::NB * kTileN * 2;
 #pragma unroll
-                for (int m = 0; m < C::NB; ++m) {
-                    const uint8_t* rd = raw + m * C::RAW_D;
-                    const uint8_t* rs = raw + C::NB * C::RAW_D + m * C::RAW_S;
-                    uint8_t* dst = (m == 0 ? sA0 : sA1) + s * C::A_BYTES;
-#pragma unroll
-                    for (int it = 0; it < 2; ++it) {
-                        const int item = ct + 128 * it;  // (row, half) pairs; contiguous reads
-                        const int r = item >> 1, h = item & 1;
-                        const uint4 v = *reinterpret_cast<const uint4*>(rd + item * 16);
-                        uint32_t lo, hi;
-                        if (WFMT == MOE_W_MXFP4) {
-                            const uint32_t bits = ctl->lut[rs[r * 2 + h]];
-                            lo = hi = bits | (bits << 16);
-                        } else {
-                            const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + r * 4 + h * 2);
-                            uint32_t s2;
-                            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(pair));
-                            lo = (s2 & 0xFFFFu) | (s2 << 16);
-                            hi = (s2 >> 16) | (s2 & 0xFFFF0000u);
-                        }
-                        convert_half_row(v, lo, hi, dst + r * 128, r, h * 4);
+                for (int it = 0; it < ITEMS / C::CONV_THREADS; ++it) {
+                    const int item = ct + C::CONV_THREADS * it;
+                    const int m = item / (kTileN * 2);
+                    const int ri = item - m * (kTileN * 2);
+                    const int row = ri >> 1, h = ri & 1;
+                    const uint4 v = *reinterpret_cast<const uint4*>(rawD(r, m) + ri * 16);
+                    const uint8_t* rs = rawS(r, m);
+                    uint32_t lo, hi;
+                    if (WFMT == MOE_W_MXFP4) {
+                        const uint32_t bits = ctl->lut[rs[row * 2 + h]];
+                        lo = hi = bits | (bits << 16);
+                    } else {
+                        const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + row * 4 + h * 2);
+                        uint32_t s2;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(pair));
+                        lo = (s2 & 0xFFFFu) | (s2 << 16);
+                        hi = (s2 >> 16) | (s2 & 0xFFFF0000u);
                     }
+                    convert_half_row(v, lo, hi, opA(s, m) + row * 128, row, h * 4);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -439,8 +464,11 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                     s = 0;
                     ph ^= 1u;
                 }
+                if (++r == C::RSTAGES) {
+                    r = 0;
+                    rph ^= 1u;
+                }
             }
-            if (!ok) break;
         }
     }
 
@@ -508,11 +536,14 @@ cudaError_t run(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& t
                 const CUtensorMap& t1, cudaStream_t st, bool pdl) {
     using C = GemmCfg<BT, DUAL, WFMT>;
     auto kern = grouped_gemm_kernel<BT, DUAL, WFMT, OUT>;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static int attr_set[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[dev] = 1;
     }
     const long long tiles_ub = ((long long)(p.M_alloc + BT - 1) / BT + p.G) * args.NT;
     const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles_ub));
@@ -528,7 +559,13 @@ cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtens
             if (p.out_kind == OUT_F16) return run<BT, true, MOE_W_MXFP4, OUT_F16>(p, args, tx, t0, t1, st, pdl);
             return run<BT, true, MOE_W_MXFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
         }
+        if (p.out_kind == OUT_F16) return run<BT, true, MOE_W_NVFP4, OUT_F16>(p, args, tx, t0, t1, st, pdl);
         return run<BT, true, MOE_W_NVFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
+    }
+    if (p.out_kind == OUT_F32) {
+        if (p.wfmt == MOE_W_BF16) return run<BT, false, MOE_W_BF16, OUT_F32>(p, args, tx, t0, t1, st, pdl);
+        if (p.wfmt == MOE_W_MXFP4) return run<BT, false, MOE_W_MXFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
+        return run<BT, false, MOE_W_NVFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
     }
     if (p.wfmt == MOE_W_BF16) return run<BT, false, MOE_W_BF16, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
     if (p.wfmt == MOE_W_MXFP4) return run<BT, false, MOE_W_MXFP4, OUT_BF16>(p, args, tx, t0, t1, st, pdl);

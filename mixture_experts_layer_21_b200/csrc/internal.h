@@ -53,6 +53,8 @@ cudaError_t launch_act_and_mul(const __nv_bfloat16* gate, const __nv_bfloat16* u
                                __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, const float* topk_w,
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
+cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T,
+                               int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes,
                                uint8_t* sb, float* s, __half* deq, cudaStream_t st, bool pdl);
 
