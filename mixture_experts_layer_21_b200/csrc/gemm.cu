@@ -1,4 +1,4 @@
-// S3/S4/S5 — persistent grouped GEMM on the 5th-generation tensor cores.
+// S3/S4/S5 — persistent grouped GEMMs on the 5th-generation tensor cores.
 //
 // Computes out[seg_g] = alpha_g * x[seg_g] @ W[g]^T over the expert-contiguous
 // segments of cu_seqlens (MoonEP experts page, moonep_grouped_gemm), optionally
@@ -13,18 +13,25 @@
 // (segment, weight block, token block) with the token block fastest, so the
 // CTAs working on one weight block at the same time share it through L2.
 //
+// Two kernels share the tile schedule and the epilogue:
+//
+// grouped_gemm_kernel (BF16 weights): a ring of shared-memory stages
+//   {gate tile, [up tile], token tile} filled by TMA; MMA operands from smem.
+//
+// grouped_gemm_fp4_kernel (MXFP4 / NVFP4 weights): a deep shared-memory ring of
+//   small raw stages {token tile, packed e2m1 codes, block scales} filled by bulk
+//   copies and TMA; converter warps expand the codes to f16 (times the block
+//   scale, exact) straight into a ring of weight tiles in tensor memory, and the
+//   MMA reads A from TMEM and the token tile from smem. Keeping the expanded
+//   weights out of shared memory matters: with f16 weights in smem every weight
+//   costs 4 bytes of smem traffic (converter write + MMA read), which caps an FP4
+//   weight stream well below HBM bandwidth.
+//
 // Warp roles (one CTA per SM):
-//   warp 0       producer (one thread): TMA / bulk copies per K step
-//   warp 1       MMA issuer (one thread) + TMEM owner; accumulators double-buffered
-//   warps 2..5   epilogue: TMEM -> registers -> alpha / activation / scales -> global
-//   warps 6..13  (FP4 weights only) e2m1 -> f16 converters writing the swizzled
-//                operand the MMA reads (FP4 dequant fused into the mainloop)
-// Pipelines:
-//   BF16 weights: one ring of stages {gate tile, [up tile], token tile}.
-//   FP4 weights: a deep ring of small raw stages {token tile, packed e2m1 codes,
-//   block scales} that keeps enough bytes in flight to stream HBM, feeding a
-//   shallow ring of converted f16 weight tiles. The MMA reads weights from the
-//   converted ring and tokens straight from the raw stage.
+//   warp 0        producer (one thread)
+//   warp 1        MMA issuer (one thread) + TMEM owner
+//   warps 2..5    epilogue: TMEM -> registers -> alpha / activation / scales -> global
+//   warps 6..13   (FP4 kernel) converters, two warps per TMEM lane quarter
 // Every wait is bounded; a timeout records MOE_ERR_TIMEOUT in the error word,
 // stops all roles, lets copies in flight land, frees TMEM and returns.
 #include <mutex>
@@ -35,37 +42,15 @@ namespace moe {
 
 constexpr int kMaxG = 1024;      // segment table capacity (weight rows)
 constexpr int kMaxStages = 16;
+constexpr int kCtrlBytes = 12288;
+constexpr int kSmemLimit = 232448;
+constexpr int kSmemBudget = kSmemLimit - 1024 - kCtrlBytes;
 
 __host__ __device__ constexpr int round1024(int b) { return (b + 1023) & ~1023; }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
-
-template <int BT, bool DUAL, int WFMT>
-struct GemmCfg {
-    static constexpr bool FP4 = WFMT != MOE_W_BF16;
-    static constexpr int NB = DUAL ? 2 : 1;
-    static constexpr int A_BYTES = kTileN * kTileK * 2;      // 16 KB: 128 rows x 64 x 16-bit
-    static constexpr int B_BYTES = BT * kTileK * 2;          // BT rows x 64 x 16-bit
-    static constexpr int RAW_D = kTileN * kTileK / 2;        // 4 KB of packed e2m1
-    static constexpr int RAW_S = WFMT == MOE_W_MXFP4 ? kTileN * 2 : (WFMT == MOE_W_NVFP4 ? kTileN * 4 : 0);
-    // operand stage: weights (+ tokens for BF16); raw stage (FP4): tokens, codes, scales
-    static constexpr int OP_STAGE = NB * A_BYTES + (FP4 ? 0 : B_BYTES);
-    static constexpr int RAW_STAGE = FP4 ? round1024(B_BYTES + NB * (RAW_D + RAW_S)) : 0;
-    static constexpr int CTRL_BYTES = 12288;
-    static constexpr int SMEM_LIMIT = 232448;
-    static constexpr int BUDGET = SMEM_LIMIT - 1024 - CTRL_BYTES;
-    static constexpr int STAGES = FP4 ? (BT >= 64 ? 4 : 3) : cmin(kMaxStages, BUDGET / OP_STAGE);
-    static constexpr int RSTAGES = FP4 ? cmin(kMaxStages, (BUDGET - STAGES * OP_STAGE) / RAW_STAGE) : 0;
-    static constexpr int TMEM_USED = 2 * NB * BT;
-    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
-    static constexpr int CONV_WARPS = FP4 ? 8 : 0;
-    static constexpr int CONV_THREADS = CONV_WARPS * 32;
-    static constexpr int THREADS = (6 + CONV_WARPS) * 32;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * OP_STAGE + RSTAGES * RAW_STAGE + CTRL_BYTES;
-    static_assert(STAGES >= 2 && (!FP4 || RSTAGES >= 2), "pipeline needs two stages");
-    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
-    static_assert(TMEM_USED <= 512, "accumulators exceed TMEM");
-    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
-};
+__host__ __device__ constexpr int tmem_cols_pow2(int c) {
+    return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
+}
 
 struct GemmArgs {
     const int32_t* cu;
@@ -87,16 +72,18 @@ struct GemmArgs {
 };
 
 struct CtrlBlock {
-    uint64_t full[kMaxStages], empty[kMaxStages];          // operand ring
+    uint64_t full[kMaxStages], empty[kMaxStages];          // operand ring (smem or TMEM)
     uint64_t raw_full[kMaxStages], raw_empty[kMaxStages];  // raw ring (FP4)
-    uint64_t tfull[2], tempty[2], drain;
+    uint64_t tfull[2], tempty[2], drain[4];
     uint32_t tmem_slot;
     int abort;
     uint16_t lut[256];
     int cu[kMaxG];
     int tpre[kMaxG + 1];
 };
-static_assert(sizeof(CtrlBlock) <= 12288, "control block");
+static_assert(sizeof(CtrlBlock) <= kCtrlBytes, "control block");
+
+// ------------------------------------------------------------------ shared pieces
 
 template <int BT>
 __device__ __forceinline__ void decode_tile(int L, const CtrlBlock* c, int G, int NT, int& g, int& nt,
@@ -117,126 +104,162 @@ __device__ __forceinline__ void decode_tile(int L, const CtrlBlock* c, int G, in
     rows = min(BT, c->cu[g] - row0);
 }
 
-__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
-    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-// 8 packed e2m1 values (one 32-bit word, even k in the low nibble) -> 4 x f16x2, times a scale.
-__device__ __forceinline__ uint4 e2m1x8_to_f16(uint32_t w, uint32_t sc2) {
-    uint32_t o0, o1, o2, o3;
-    asm("{ .reg .b8 b0,b1,b2,b3; mov.b32 {b0,b1,b2,b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
-        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
-        : "r"(w));
-    return make_uint4(hmul2_u32(o0, sc2), hmul2_u32(o1, sc2), hmul2_u32(o2, sc2), hmul2_u32(o3, sc2));
-}
-// 32 values (half a 64-value row) -> 4 x 16-byte chunks of the 128-byte-swizzled operand row.
-__device__ __forceinline__ void convert_half_row(const uint4 raw, uint32_t sc2_lo, uint32_t sc2_hi,
-                                                 uint8_t* row_base, int r, int c_first) {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+// One warp: the segment table (cu, clamped, and the running tile count tpre).
+// Ends are clamped to [0, M_alloc] and a segment whose end lies before the previous
+// end counts as empty, so no tile can touch rows outside the buffers.
+template <int BT>
+__device__ __forceinline__ void build_segment_table(const GemmArgs& a, CtrlBlock* ctl, int lane) {
+    const int G = a.G, NT = a.NT;
+    int carry = 0, prev_chunk_end = 0;
+    for (int base = 0; base < G; base += 32) {
+        const int g = base + lane;
+        const int raw = g < G ? a.cu[g] : 0;
+        const int end = min(max(raw, 0), a.M_alloc);
+        int prev = __shfl_up_sync(0xffffffffu, end, 1);
+        if (lane == 0) prev = prev_chunk_end;
+        if (g < G && (raw != end || end < prev)) report_error(a.err, MOE_ERR_DEVICE, 1000000 + g);
+        const int len = g < G ? max(0, end - prev) : 0;
+        const int tiles = ((len + BT - 1) / BT) * NT;
+        int incl = tiles;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 o = e2m1x8_to_f16(w[i], i < 2 ? sc2_lo : sc2_hi);
-        *reinterpret_cast<uint4*>(row_base + (((c_first + i) ^ (r & 7)) << 4)) = o;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += n;
+        }
+        if (g < G) {
+            ctl->cu[g] = len > 0 ? end : prev;
+            ctl->tpre[g + 1] = carry + incl;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        const int eff = g < G ? (len > 0 ? end : prev) : prev;
+        prev_chunk_end = __shfl_sync(0xffffffffu, eff, 31);
+    }
+    if (lane == 0) ctl->tpre[0] = 0;
+}
+
+// Epilogue of one tile for the warp owning TMEM lanes [32q, 32q+32). The accumulator
+// buffer at column tb holds NPART partial sums per matrix (one per MMA-issuing thread):
+// with two matrices, partial j of gate at tb + 2j*BT and of up at tb + (2j+1)*BT; with
+// one, partial j at tb + j*BT.
+template <int BT, bool DUAL, int OUT, int NPART = 1>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, int g, int nt, int row0, int rows,
+                                              int q, int lane) {
+    const int n = nt * kTileN + q * 32 + lane;
+    const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
+    const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
+    constexpr int STRIDE = DUAL ? 2 * BT : BT;   // column distance between partials of one matrix
+#pragma unroll 1
+    for (int c0 = 0; c0 < BT; c0 += 16) {
+        if (c0 >= rows) break;
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tb + c0, r0);
+        if (DUAL) tmem_ld16(tb + BT + c0, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int pj = 1; pj < NPART; ++pj) {
+            uint32_t p0[16], p1[16];
+            tmem_ld16(tb + pj * STRIDE + c0, p0);
+            if (DUAL) tmem_ld16(tb + pj * STRIDE + BT + c0, p1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                r0[j] = __float_as_uint(__uint_as_float(r0[j]) + __uint_as_float(p0[j]));
+                if (DUAL) r1[j] = __float_as_uint(__uint_as_float(r1[j]) + __uint_as_float(p1[j]));
+            }
+        }
+        if (n < a.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (c0 + j < rows) {
+                    const int row = row0 + c0 + j;
+                    const float ts = a.tscale ? a.tscale[row] : 1.0f;
+                    float v;
+                    if (DUAL) {
+                        const float gv = __uint_as_float(r0[j]) * al0 * ts;
+                        const float uv = __uint_as_float(r1[j]) * al1 * ts;
+                        v = act_apply(a.act, gv, uv, a.sa, a.sb);
+                        if (a.perm_w) v *= a.perm_w[row];
+                    } else {
+                        v = __uint_as_float(r0[j]) * al0 * ts;
+                    }
+                    v *= a.out_scale;
+                    const size_t idx = (size_t)row * a.N + n;
+                    if (OUT == OUT_BF16) reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
+                    else if (OUT == OUT_F16) reinterpret_cast<__half*>(a.out)[idx] = __float2half_rn(v);
+                    else reinterpret_cast<float*>(a.out)[idx] = v;
+                }
+            }
+        }
     }
 }
 
-template <int BT, bool DUAL, int WFMT, int OUT>
-__global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
+// Rows [cu[G-1], M_alloc) of a bf16 output are zero (standalone grouped GEMM).
+__device__ __forceinline__ void zero_padding_rows(const GemmArgs& a, const CtrlBlock* ctl, int tid128) {
+    const int start = a.G > 0 ? ctl->cu[a.G - 1] : 0;
+    const long long count = (long long)(a.M_alloc - start) * a.N;
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)start * a.N;
+    const long long stride = (long long)gridDim.x * 128;
+    for (long long i = (long long)blockIdx.x * 128 + tid128; i < count; i += stride) o[i] = __float2bfloat16_rn(0.0f);
+}
+
+// ------------------------------------------------------------------ BF16 kernel
+
+template <int BT, bool DUAL>
+struct Bf16Cfg {
+    static constexpr int NB = DUAL ? 2 : 1;
+    static constexpr int A_BYTES = kTileN * kTileK * 2;      // 16 KB: 128 rows x 64 bf16
+    static constexpr int B_BYTES = BT * kTileK * 2;
+    static constexpr int STAGE = NB * A_BYTES + B_BYTES;
+    static constexpr int STAGES = cmin(kMaxStages, kSmemBudget / STAGE);
+    static constexpr int ACC_COLS = NB * BT;
+    static constexpr int TMEM_COLS = tmem_cols_pow2(2 * ACC_COLS);
+    static constexpr int THREADS = 6 * 32;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
+    static_assert(STAGES >= 2 && SMEM_BYTES <= kSmemLimit && 2 * ACC_COLS <= 512, "BF16 GEMM config");
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
+};
+
+template <int BT, bool DUAL, int OUT>
+__global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_w0,
                         const __grid_constant__ CUtensorMap tm_w1, const GemmArgs a) {
-    using C = GemmCfg<BT, DUAL, WFMT>;
+    using C = Bf16Cfg<BT, DUAL>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // operand ring: stage s = [A0][A1 if dual][B if BF16]; raw ring (FP4): [B][D0][D1][S0][S1]
-    uint8_t* sOp = smem;
-    uint8_t* sRaw = sOp + C::STAGES * C::OP_STAGE;
-    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(sRaw + C::RSTAGES * C::RAW_STAGE);
+    // 1024-byte alignment by offsetting the shared array itself (no integer round trip),
+    // so that every access below stays a shared-memory access
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
     volatile int* abort_flag = &ctl->abort;
-    auto opA = [&](int s, int m) { return sOp + s * C::OP_STAGE + m * C::A_BYTES; };
-    auto opB = [&](int s) { return sOp + s * C::OP_STAGE + C::NB * C::A_BYTES; };
-    auto rawB = [&](int r) { return sRaw + r * C::RAW_STAGE; };
-    auto rawD = [&](int r, int m) { return sRaw + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_D; };
-    auto rawS = [&](int r, int m) {
-        return sRaw + r * C::RAW_STAGE + C::B_BYTES + C::NB * C::RAW_D + m * C::RAW_S;
-    };
-
+    auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
+    auto opB = [&](int s) { return smem + s * C::STAGE + C::NB * C::A_BYTES; };
     const int warp = warp_id(), lane = lane_id();
     const int G = a.G, NT = a.NT, KB = a.KB;
 
-    // ---------------- prologue: independent of the previous kernel's output
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], C::FP4 ? C::CONV_WARPS : 1);
+            mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
-        }
-        for (int r = 0; r < C::RSTAGES; ++r) {
-            mbar_init(&ctl->raw_full[r], 1);
-            mbar_init(&ctl->raw_empty[r], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
             mbar_init(&ctl->tempty[b], 4);
         }
-        mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->drain[0], 1);
         ctl->abort = 0;
         fence_barrier_init();
     }
     if (threadIdx.x == 32) {
         tma_prefetch_desc(&tm_x);
-        if (!C::FP4) {
-            tma_prefetch_desc(&tm_w0);
-            if (DUAL) tma_prefetch_desc(&tm_w1);
-        }
+        tma_prefetch_desc(&tm_w0);
+        if (DUAL) tma_prefetch_desc(&tm_w1);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (WFMT == MOE_W_MXFP4) {
-        // e8m0 (already re-biased by the weight preparation) -> f16 bits of 2^(e-127)
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-            const int e = i - 127;
-            uint16_t bits;
-            if (e >= -14 && e <= 15) bits = (uint16_t)((e + 15) << 10);
-            else if (e >= -24 && e < -14) bits = (uint16_t)(1u << (e + 24));
-            else bits = e > 15 ? (uint16_t)0x7C00 : (uint16_t)0;
-            ctl->lut[i] = bits;
-        }
-    }
     pdl_wait();
-    if (warp == 0) {
-        // segment table: cu (inclusive ends) and the running tile count.
-        // Ends are clamped to [0, M_alloc] and a segment whose end lies before the
-        // previous end counts as empty, so no tile can touch rows outside the buffers.
-        int carry = 0, prev_chunk_end = 0;
-        for (int base = 0; base < G; base += 32) {
-            const int g = base + lane;
-            const int raw = g < G ? a.cu[g] : 0;
-            const int end = min(max(raw, 0), a.M_alloc);
-            int prev = __shfl_up_sync(0xffffffffu, end, 1);
-            if (lane == 0) prev = prev_chunk_end;
-            if (g < G && (raw != end || end < prev)) report_error(a.err, MOE_ERR_DEVICE, 1000000 + g);
-            const int len = g < G ? max(0, end - prev) : 0;
-            const int tiles = ((len + BT - 1) / BT) * NT;
-            int incl = tiles;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += n;
-            }
-            if (g < G) {
-                ctl->cu[g] = len > 0 ? end : prev;
-                ctl->tpre[g + 1] = carry + incl;
-            }
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-            const int eff = g < G ? (len > 0 ? end : prev) : prev;
-            prev_chunk_end = __shfl_sync(0xffffffffu, eff, 31);
-        }
-        if (lane == 0) ctl->tpre[0] = 0;
-    }
+    if (warp == 0) build_segment_table<BT>(a, ctl, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -245,11 +268,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
     const int total = ctl->tpre[G];
 
     if (warp == 0) {
-        // ---------------- producer
-        if (lane == 0) {
-            constexpr int NS = C::FP4 ? C::RSTAGES : C::STAGES;
-            uint64_t* fullb = C::FP4 ? ctl->raw_full : ctl->full;
-            uint64_t* emptyb = C::FP4 ? ctl->raw_empty : ctl->empty;
+        if (lane == 0) {  // ---------------- TMA producer
             int s = 0;
             uint32_t ph = 0, issued_mask = 0, issued_par = 0;
             bool ok = true;
@@ -257,29 +276,17 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&emptyb[s], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (!C::FP4) {
-                        mbar_arrive_expect_tx(&fullb[s], C::NB * C::A_BYTES + C::B_BYTES);
-                        tma_load_3d(opA(s, 0), &tm_w0, &fullb[s], kb * kTileK, nt * kTileN, g);
-                        if (DUAL) tma_load_3d(opA(s, 1), &tm_w1, &fullb[s], kb * kTileK, nt * kTileN, g);
-                        tma_load_2d(opB(s), &tm_x, &fullb[s], kb * kTileK, row0);
-                    } else {
-                        const size_t tile = ((size_t)g * NT + nt) * KB + kb;
-                        mbar_arrive_expect_tx(&fullb[s], C::B_BYTES + C::NB * (C::RAW_D + C::RAW_S));
-                        bulk_load(rawD(s, 0), a.kd0 + tile * C::RAW_D, C::RAW_D, &fullb[s]);
-                        bulk_load(rawS(s, 0), a.ks0 + tile * C::RAW_S, C::RAW_S, &fullb[s]);
-                        if (DUAL) {
-                            bulk_load(rawD(s, 1), a.kd1 + tile * C::RAW_D, C::RAW_D, &fullb[s]);
-                            bulk_load(rawS(s, 1), a.ks1 + tile * C::RAW_S, C::RAW_S, &fullb[s]);
-                        }
-                        tma_load_2d(rawB(s), &tm_x, &fullb[s], kb * kTileK, row0);
-                    }
+                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
+                    tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g);
+                    if (DUAL) tma_load_3d(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g);
+                    tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * kTileK, row0);
                     issued_mask |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
-                    if (++s == NS) {
+                    if (++s == C::STAGES) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -288,18 +295,16 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 1);
                 ctl->abort = 1;
-                // let every copy this thread issued land before the CTA exits
-                int never = 0;
-                for (int q = 0; q < NS; ++q)
-                    if (issued_mask >> q & 1u) mbar_wait(&fullb[q], issued_par >> q & 1u, &never);
+                int never = 0;  // let every copy this thread issued land before the CTA exits
+                for (int q = 0; q < C::STAGES; ++q)
+                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(C::FP4 ? 0 : 1, kTileN, BT);
-            int s = 0, r = 0, b = 0;
-            uint32_t ph = 0, rph = 0, bph = 0;
+        if (lane == 0) {  // ---------------- MMA issuer
+            constexpr uint32_t idesc = idesc_f16(1, kTileN, BT);
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0;
             bool ok = true, issued = false;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
@@ -307,17 +312,16 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + (uint32_t)(b * C::NB * BT);
+                const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) ||
-                        (C::FP4 && !mbar_wait(&ctl->raw_full[r], rph, abort_flag))) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(opA(s, 0));
                     const uint32_t a1 = smem_u32(opA(s, DUAL ? 1 : 0));
-                    const uint32_t bb = smem_u32(C::FP4 ? rawB(r) : opB(s));
+                    const uint32_t bb = smem_u32(opB(s));
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint64_t bdesc = sw128_kmajor_desc(bb + kk * 32);
@@ -331,13 +335,6 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                         s = 0;
                         ph ^= 1u;
                     }
-                    if (C::FP4) {
-                        mma_commit(&ctl->raw_empty[r]);
-                        if (++r == C::RSTAGES) {
-                            r = 0;
-                            rph ^= 1u;
-                        }
-                    }
                 }
                 if (!ok) break;
                 mma_commit(&ctl->tfull[b]);
@@ -347,16 +344,15 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {
-                    // wait (bounded) for the MMAs in flight before TMEM is released
+                if (issued) {  // wait (bounded) for the MMAs in flight before TMEM is released
                     int never = 0;
-                    mma_commit(&ctl->drain);
-                    mbar_wait(&ctl->drain, 0, &never);
+                    mma_commit(&ctl->drain[0]);
+                    mbar_wait(&ctl->drain[0], 0, &never);
                 }
             }
         }
-    } else if (warp < 6) {
-        // ---------------- epilogue
+    } else {
+        // ---------------- epilogue (warps 2..5)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         int b = 0;
         uint32_t bph = 0;
@@ -369,98 +365,344 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const int n = nt * kTileN + q * 32 + lane;
-            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::NB * BT);
-            const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
-            const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += 16) {
-                if (c0 >= rows) break;
-                uint32_t r0[16], r1[16];
-                tmem_ld16(tb + c0, r0);
-                if (DUAL) tmem_ld16(tb + BT + c0, r1);
-                tmem_ld_wait();
-                if (n < a.N) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (c0 + j < rows) {
-                            const int row = row0 + c0 + j;
-                            const float ts = a.tscale ? a.tscale[row] : 1.0f;
-                            float v;
-                            if (DUAL) {
-                                const float gv = __uint_as_float(r0[j]) * al0 * ts;
-                                const float uv = __uint_as_float(r1[j]) * al1 * ts;
-                                v = act_apply(a.act, gv, uv, a.sa, a.sb);
-                                if (a.perm_w) v *= a.perm_w[row];
-                            } else {
-                                v = __uint_as_float(r0[j]) * al0 * ts;
-                            }
-                            v *= a.out_scale;
-                            const size_t idx = (size_t)row * a.N + n;
-                            if (OUT == OUT_BF16) reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
-                            else if (OUT == OUT_F16) reinterpret_cast<__half*>(a.out)[idx] = __float2half_rn(v);
-                            else reinterpret_cast<float*>(a.out)[idx] = v;
-                        }
-                    }
-                }
-            }
+            epilogue_tile<BT, DUAL, OUT>(a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g,
+                                         nt, row0, rows, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[b]);
             b ^= 1;
             if (b == 0) bph ^= 1u;
         }
-        if (a.zero_pad && OUT == OUT_BF16) {
-            // rows [cu[G-1], M_alloc) of the output are zero
-            const int start = G > 0 ? ctl->cu[G - 1] : 0;
-            const long long count = (long long)(a.M_alloc - start) * a.N;
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + (size_t)start * a.N;
-            const long long tid = (long long)blockIdx.x * 128 + (threadIdx.x - 64);
-            const long long stride = (long long)gridDim.x * 128;
-            for (long long i = tid; i < count; i += stride) o[i] = __float2bfloat16_rn(0.0f);
+        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 64);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ FP4 kernel
+
+template <int BT, bool DUAL, int WFMT>
+struct Fp4Cfg {
+    static constexpr int NB = DUAL ? 2 : 1;
+    static constexpr int B_BYTES = BT * kTileK * 2;          // token tile, f16
+    static constexpr int RAW_D = kTileN * kTileK / 2;        // 4 KB of packed e2m1
+    static constexpr int RAW_S = WFMT == MOE_W_MXFP4 ? kTileN * 2 : kTileN * 4;
+    static constexpr int RAW_STAGE = round1024(B_BYTES + NB * (RAW_D + RAW_S));
+    static constexpr int RSTAGES = cmin(kMaxStages, kSmemBudget / RAW_STAGE);
+    // MMA-issuing threads. A 128 x N x 16 MMA costs an issuing thread ~45 cycles for any
+    // N <= 64, so narrow token tiles are issue-bound with one issuer; four issuers (each
+    // with its own partial accumulator: matrix x K-half, or K-quarter for one matrix)
+    // reach the tensor pipe's rate. Wide tiles (N = 128) run at full rate with one.
+    static constexpr int NI = BT <= 64 ? 4 : 1;
+    static constexpr int NPART = NI == 1 ? 1 : (DUAL ? 2 : 4);  // partial sums per matrix
+    // TMEM: accumulators [ACC_BUFS x ACC_COLS] then the weight ring [A_STAGES x NB x 32 cols]
+    static constexpr int ACC_COLS = NB * NPART * BT;
+    static constexpr int ACC_BUFS = 2 * ACC_COLS <= 256 ? 2 : 1;
+    static constexpr int A_COLS = 32;                        // 128 rows x 64 f16 = 32 columns
+    static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
+    static constexpr int A_STAGES = cmin(8, (512 - A_BASE) / (NB * A_COLS));
+    static constexpr int CONV_WARPS = 8;
+    // warps: 0 producer, [1, 1+NI) issuers, then 4 epilogue, then the converters
+    static constexpr int EPI_WARP0 = 1 + NI;
+    static constexpr int CONV_WARP0 = EPI_WARP0 + 4;
+    static constexpr int THREADS = (CONV_WARP0 + CONV_WARPS) * 32;
+    static constexpr int SMEM_BYTES = 1024 + RSTAGES * RAW_STAGE + kCtrlBytes;
+    static_assert(RSTAGES >= 2 && A_STAGES >= 2 && SMEM_BYTES <= kSmemLimit, "FP4 GEMM config");
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
+};
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+// 8 packed e2m1 values (one 32-bit word, even k in the low nibble) -> 4 x f16x2, times a scale.
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t sc2, uint32_t* o) {
+    uint32_t o0, o1, o2, o3;
+    asm("{ .reg .b8 b0,b1,b2,b3; mov.b32 {b0,b1,b2,b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(w));
+    o[0] = hmul2_u32(o0, sc2);
+    o[1] = hmul2_u32(o1, sc2);
+    o[2] = hmul2_u32(o2, sc2);
+    o[3] = hmul2_u32(o3, sc2);
+}
+// f16x2 holding `bits` in both halves
+__device__ __forceinline__ uint32_t dup16(uint32_t bits) { return (bits & 0xFFFFu) | (bits << 16); }
+
+template <int BT, bool DUAL, int WFMT, int OUT>
+__global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
+    grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
+    using C = Fp4Cfg<BT, DUAL, WFMT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::RSTAGES * C::RAW_STAGE);
+    volatile int* abort_flag = &ctl->abort;
+    auto rawB = [&](int r) { return smem + r * C::RAW_STAGE; };
+    auto rawD = [&](int r, int m) { return smem + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_D; };
+    auto rawS = [&](int r, int m) {
+        return smem + r * C::RAW_STAGE + C::B_BYTES + C::NB * C::RAW_D + m * C::RAW_S;
+    };
+    const int warp = warp_id(), lane = lane_id();
+    const int G = a.G, NT = a.NT, KB = a.KB;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::A_STAGES; ++s) {
+            mbar_init(&ctl->full[s], C::CONV_WARPS);
+            mbar_init(&ctl->empty[s], C::NI);       // every issuer commits once per stage
         }
-    } else if (C::CONV_WARPS > 0) {
-        // ---------------- FP4 -> f16 converters (FP4 dequant fused into the mainloop)
-        const int ct = threadIdx.x - 6 * 32;  // 0 .. CONV_THREADS-1
+        for (int r = 0; r < C::RSTAGES; ++r) {
+            mbar_init(&ctl->raw_full[r], 1);
+            mbar_init(&ctl->raw_empty[r], C::NI);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], C::NI);
+            mbar_init(&ctl->tempty[b], 4);
+        }
+        for (int i = 0; i < 4; ++i) mbar_init(&ctl->drain[i], 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 0) tma_prefetch_desc(&tm_x);
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (WFMT == MOE_W_MXFP4) {
+        // e8m0 (re-biased by the weight preparation) -> f16 bits of 2^(e-127)
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+            const int e = i - 127;
+            uint16_t bits;
+            if (e >= -14 && e <= 15) bits = (uint16_t)((e + 15) << 10);
+            else if (e >= -24 && e < -14) bits = (uint16_t)(1u << (e + 24));
+            else bits = e > 15 ? (uint16_t)0x7C00 : (uint16_t)0;
+            ctl->lut[i] = bits;
+        }
+    }
+    pdl_wait();
+    if (warp == 0) build_segment_table<BT>(a, ctl, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch();
+    const uint32_t tmem_base = ctl->tmem_slot;
+    const int total = ctl->tpre[G];
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------- producer: token tile (TMA) + codes and scales (bulk)
+            int r = 0;
+            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            bool ok = true;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->raw_empty[r], ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const size_t tile = ((size_t)g * NT + nt) * KB + kb;
+                    mbar_arrive_expect_tx(&ctl->raw_full[r], C::B_BYTES + C::NB * (C::RAW_D + C::RAW_S));
+                    bulk_load(rawD(r, 0), a.kd0 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[r]);
+                    bulk_load(rawS(r, 0), a.ks0 + tile * C::RAW_S, C::RAW_S, &ctl->raw_full[r]);
+                    if (DUAL) {
+                        bulk_load(rawD(r, 1), a.kd1 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[r]);
+                        bulk_load(rawS(r, 1), a.ks1 + tile * C::RAW_S, C::RAW_S, &ctl->raw_full[r]);
+                    }
+                    tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * kTileK, row0);
+                    issued_mask |= 1u << r;
+                    issued_par = (issued_par & ~(1u << r)) | (ph << r);
+                    if (++r == C::RSTAGES) {
+                        r = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+                int never = 0;
+                for (int q = 0; q < C::RSTAGES; ++q)
+                    if (issued_mask >> q & 1u) mbar_wait(&ctl->raw_full[q], issued_par >> q & 1u, &never);
+            }
+        }
+    } else if (warp < C::EPI_WARP0) {
+        if (lane == 0) {  // ---------------- MMA issuers: A from TMEM, B (tokens) from smem
+            // issuer i: with NI == 1 all four K steps of both matrices; with NI == 4 and two
+            // matrices, matrix i&1 over K steps {2(i>>1), 2(i>>1)+1} into partial i>>1; with
+            // one matrix, K step i into partial i. Partial p of matrix m sits at column
+            // (p*NB + m)*BT of the accumulator buffer.
+            const int i = warp - 1;
+            constexpr uint32_t idesc = idesc_f16(0, kTileN, BT);
+            constexpr int KPI = (kTileK / 16) / (C::NI == 1 ? 1 : (DUAL ? 2 : 4));  // K steps per issuer
+            const int m_i = (C::NI == 1 || !DUAL) ? 0 : (i & 1);
+            const int p_i = C::NI == 1 ? 0 : (DUAL ? (i >> 1) : i);
+            const int kk0 = p_i * KPI;
+            int s = 0, r = 0, b = 0;
+            uint32_t ph = 0, rph = 0, bph = 0;
+            bool ok = true, issued = false;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&ctl->raw_full[r], rph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t bb = smem_u32(rawB(r));
+                    const uint32_t a0 = tmem_base + (uint32_t)(C::A_BASE + (s * C::NB) * C::A_COLS);
+                    if (C::NI == 1) {
+#pragma unroll
+                        for (int kk = 0; kk < kTileK / 16; ++kk) {
+                            const uint64_t bdesc = sw128_kmajor_desc(bb + kk * 32);
+                            const uint32_t acc = (kb | kk) != 0;
+                            mma_f16_ts(d0, a0 + kk * 8, bdesc, idesc, acc);
+                            if (DUAL) mma_f16_ts(d0 + BT, a0 + C::A_COLS + kk * 8, bdesc, idesc, acc);
+                        }
+                    } else {
+                        const uint32_t dm = d0 + (uint32_t)((p_i * C::NB + m_i) * BT);
+#pragma unroll
+                        for (int j = 0; j < KPI; ++j) {
+                            const int kk = kk0 + j;
+                            mma_f16_ts(dm, a0 + m_i * C::A_COLS + kk * 8, sw128_kmajor_desc(bb + kk * 32), idesc,
+                                       (kb > 0 || j > 0) ? 1u : 0u);
+                        }
+                    }
+                    issued = true;
+                    mma_commit(&ctl->empty[s]);
+                    mma_commit(&ctl->raw_empty[r]);
+                    if (++s == C::A_STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                    if (++r == C::RSTAGES) {
+                        r = 0;
+                        rph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[b]);
+                if (++b == C::ACC_BUFS) {
+                    b = 0;
+                    bph ^= 1u;
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 2);
+                ctl->abort = 1;
+                if (issued) {
+                    int never = 0;
+                    mma_commit(&ctl->drain[i]);
+                    mbar_wait(&ctl->drain[i], 0, &never);
+                }
+            }
+        }
+    } else if (warp < C::CONV_WARP0) {
+        // ---------------- epilogue (warps 2..5)
+        const int q = warp & 3;
+        int b = 0;
+        uint32_t bph = 0;
+        for (int L = blockIdx.x; L < total; L += gridDim.x) {
+            int g, nt, row0, rows;
+            decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+                if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after();
+            epilogue_tile<BT, DUAL, OUT, C::NPART>(a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g,
+                                         nt, row0, rows, q, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            if (++b == C::ACC_BUFS) {
+                b = 0;
+                bph ^= 1u;
+            }
+        }
+        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
+    } else {
+        // ---------------- converters (warps 6..13): e2m1 x block scale -> f16 rows in TMEM.
+        // Warp w owns TMEM lanes [32q, 32q+32), q = w % 4, so thread `lane` converts weight
+        // row 32q + lane. With two matrices the second warp of the quarter takes the up
+        // projection; with one, the two warps split the 64 K values of the stage.
+        const int q = warp & 3, grp = (warp - C::CONV_WARP0) >> 2;
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         int s = 0, r = 0;
         uint32_t ph = 0, rph = 0;
         bool ok = true;
         for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&ctl->raw_full[r], rph, abort_flag) ||
-                    !mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                if (!mbar_wait(&ctl->raw_full[r], rph, abort_flag) || !mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
                     if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 4);
                     ctl->abort = 1;
                     ok = false;
                     break;
                 }
-                // items: (matrix m, row, half) -> 16 raw bytes = 32 values each; contiguous reads
-                constexpr int ITEMS = C::NB * kTileN * 2;
-#pragma unroll
-                for (int it = 0; it < ITEMS / C::CONV_THREADS; ++it) {
-                    const int item = ct + C::CONV_THREADS * it;
-                    const int m = item / (kTileN * 2);
-                    const int ri = item - m * (kTileN * 2);
-                    const int row = ri >> 1, h = ri & 1;
-                    const uint4 v = *reinterpret_cast<const uint4*>(rawD(r, m) + ri * 16);
+                tc_fence_after();
+                if (DUAL) {
+                    const int m = grp;
+                    const uint8_t* rd = rawD(r, m) + row * 32;
                     const uint8_t* rs = rawS(r, m);
-                    uint32_t lo, hi;
+                    const uint4 v0 = *reinterpret_cast<const uint4*>(rd);
+                    const uint4 v1 = *reinterpret_cast<const uint4*>(rd + 16);
+                    uint32_t sc[4];
                     if (WFMT == MOE_W_MXFP4) {
-                        const uint32_t bits = ctl->lut[rs[row * 2 + h]];
-                        lo = hi = bits | (bits << 16);
+                        sc[0] = sc[1] = dup16(ctl->lut[rs[row * 2]]);
+                        sc[2] = sc[3] = dup16(ctl->lut[rs[row * 2 + 1]]);
+                    } else {
+                        const uint32_t four = *reinterpret_cast<const uint32_t*>(rs + row * 4);
+                        uint32_t s01, s23;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"((uint16_t)(four & 0xFFFF)));
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s23) : "h"((uint16_t)(four >> 16)));
+                        sc[0] = dup16(s01);
+                        sc[1] = dup16(s01 >> 16);
+                        sc[2] = dup16(s23);
+                        sc[3] = dup16(s23 >> 16);
+                    }
+                    uint32_t o[32];
+                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
+                    tmem_st32(lane_base + (uint32_t)(C::A_BASE + (s * C::NB + m) * C::A_COLS), o);
+                } else {
+                    const int h = grp;  // K half
+                    const uint4 v = *reinterpret_cast<const uint4*>(rawD(r, 0) + row * 32 + h * 16);
+                    const uint8_t* rs = rawS(r, 0);
+                    uint32_t sc[2];
+                    if (WFMT == MOE_W_MXFP4) {
+                        sc[0] = sc[1] = dup16(ctl->lut[rs[row * 2 + h]]);
                     } else {
                         const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + row * 4 + h * 2);
-                        uint32_t s2;
-                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(pair));
-                        lo = (s2 & 0xFFFFu) | (s2 << 16);
-                        hi = (s2 >> 16) | (s2 & 0xFFFF0000u);
+                        uint32_t s01;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"(pair));
+                        sc[0] = dup16(s01);
+                        sc[1] = dup16(s01 >> 16);
                     }
-                    convert_half_row(v, lo, hi, opA(s, m) + row * 128, row, h * 4);
+                    uint32_t o[16];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
+                    tmem_st16(lane_base + (uint32_t)(C::A_BASE + s * C::A_COLS + h * 16), o);
                 }
-                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->full[s]);
-                if (++s == C::STAGES) {
+                if (++s == C::A_STAGES) {
                     s = 0;
                     ph ^= 1u;
                 }
@@ -472,12 +714,11 @@ __global__ void __launch_bounds__(GemmCfg<BT, DUAL, WFMT>::THREADS, 1)
         }
     }
 
-    // ---------------- teardown
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        tmem_dealloc(tmem_base, 512);
     }
 }
 
@@ -531,45 +772,68 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BT, bool DUAL, int WFMT, int OUT>
-cudaError_t run(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& t0,
-                const CUtensorMap& t1, cudaStream_t st, bool pdl) {
-    using C = GemmCfg<BT, DUAL, WFMT>;
-    auto kern = grouped_gemm_kernel<BT, DUAL, WFMT, OUT>;
-    static int attr_set[64] = {0};
+// `done` belongs to the caller's instantiation: kernels of one signature share a
+// function-pointer type, so the flag cannot live in a template on that type.
+template <typename Kern>
+cudaError_t set_smem_once(Kern kern, int bytes, int (&done)[64]) {
     int dev = 0;
-    cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = 1;
+        done[dev] = 1;
     }
-    const long long tiles_ub = ((long long)(p.M_alloc + BT - 1) / BT + p.G) * args.NT;
-    const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles_ub));
-    return launch_k(kern, dim3(grid), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, t0, t1, args);
+    return cudaSuccess;
+}
+
+int grid_for(const GemmProblem& p, const GemmArgs& args, int bt) {
+    const long long tiles_ub = ((long long)(p.M_alloc + bt - 1) / bt + p.G) * args.NT;
+    return (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles_ub));
+}
+
+template <int BT, bool DUAL, int OUT>
+cudaError_t run_bf16(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& t0,
+                     const CUtensorMap& t1, cudaStream_t st, bool pdl) {
+    using C = Bf16Cfg<BT, DUAL>;
+    auto kern = grouped_gemm_kernel<BT, DUAL, OUT>;
+    static int done[64] = {0};
+    cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, t0, t1,
+                    args);
+}
+
+template <int BT, bool DUAL, int WFMT, int OUT>
+cudaError_t run_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st, bool pdl) {
+    using C = Fp4Cfg<BT, DUAL, WFMT>;
+    auto kern = grouped_gemm_fp4_kernel<BT, DUAL, WFMT, OUT>;
+    static int done[64] = {0};
+    cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, args);
+}
+
+template <int BT, int WFMT>
+cudaError_t dispatch_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st,
+                         bool pdl) {
+    if (p.dual) {
+        if (p.out_kind == OUT_F16) return run_fp4<BT, true, WFMT, OUT_F16>(p, args, tx, st, pdl);
+        return run_fp4<BT, true, WFMT, OUT_F32>(p, args, tx, st, pdl);
+    }
+    if (p.out_kind == OUT_F32) return run_fp4<BT, false, WFMT, OUT_F32>(p, args, tx, st, pdl);
+    return run_fp4<BT, false, WFMT, OUT_BF16>(p, args, tx, st, pdl);
 }
 
 template <int BT>
 cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx,
                         const CUtensorMap& t0, const CUtensorMap& t1, cudaStream_t st, bool pdl) {
-    if (p.dual) {
-        if (p.wfmt == MOE_W_BF16) return run<BT, true, MOE_W_BF16, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
-        if (p.wfmt == MOE_W_MXFP4) {
-            if (p.out_kind == OUT_F16) return run<BT, true, MOE_W_MXFP4, OUT_F16>(p, args, tx, t0, t1, st, pdl);
-            return run<BT, true, MOE_W_MXFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
-        }
-        if (p.out_kind == OUT_F16) return run<BT, true, MOE_W_NVFP4, OUT_F16>(p, args, tx, t0, t1, st, pdl);
-        return run<BT, true, MOE_W_NVFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
-    }
-    if (p.out_kind == OUT_F32) {
-        if (p.wfmt == MOE_W_BF16) return run<BT, false, MOE_W_BF16, OUT_F32>(p, args, tx, t0, t1, st, pdl);
-        if (p.wfmt == MOE_W_MXFP4) return run<BT, false, MOE_W_MXFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
-        return run<BT, false, MOE_W_NVFP4, OUT_F32>(p, args, tx, t0, t1, st, pdl);
-    }
-    if (p.wfmt == MOE_W_BF16) return run<BT, false, MOE_W_BF16, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
-    if (p.wfmt == MOE_W_MXFP4) return run<BT, false, MOE_W_MXFP4, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
-    return run<BT, false, MOE_W_NVFP4, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
+    if (p.wfmt == MOE_W_MXFP4) return dispatch_fp4<BT, MOE_W_MXFP4>(p, args, tx, st, pdl);
+    if (p.wfmt == MOE_W_NVFP4) return dispatch_fp4<BT, MOE_W_NVFP4>(p, args, tx, st, pdl);
+    if (p.dual) return run_bf16<BT, true, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
+    if (p.out_kind == OUT_F32) return run_bf16<BT, false, OUT_F32>(p, args, tx, t0, t1, st, pdl);
+    return run_bf16<BT, false, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
 }
 
 }  // namespace
