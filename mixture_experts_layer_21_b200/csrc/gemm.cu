@@ -389,10 +389,13 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 template <int BT, bool DUAL, int WFMT>
 struct Fp4Cfg {
     static constexpr int NB = DUAL ? 2 : 1;
-    static constexpr int B_BYTES = BT * kTileK * 2;          // token tile, f16
-    static constexpr int RAW_D = kTileN * kTileK / 2;        // 4 KB of packed e2m1
-    static constexpr int RAW_S = WFMT == MOE_W_MXFP4 ? kTileN * 2 : kTileN * 4;
-    static constexpr int RAW_STAGE = round1024(B_BYTES + NB * (RAW_D + RAW_S));
+    static constexpr int KS = kFp4StageK;                    // 128 K values per stage
+    static constexpr int BOX_BYTES = BT * kTileK * 2;        // one 64-K token box, f16
+    static constexpr int B_BYTES = 2 * BOX_BYTES;            // token tile of a stage
+    static constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;    // scale bytes per row per 64 K
+    static constexpr int CHUNK = kTileN * 32 + kTileN * S;   // prepared 128 x 64 chunk
+    static constexpr int RAW_M = 2 * CHUNK;                  // one matrix's raw bytes per stage
+    static constexpr int RAW_STAGE = round1024(B_BYTES + NB * RAW_M);
     static constexpr int RSTAGES = cmin(kMaxStages, kSmemBudget / RAW_STAGE);
     // MMA-issuing threads. A 128 x N x 16 MMA costs an issuing thread ~45 cycles for any
     // N <= 64, so narrow token tiles are issue-bound with one issuer; four issuers (each
@@ -400,10 +403,10 @@ struct Fp4Cfg {
     // reach the tensor pipe's rate. Wide tiles (N = 128) run at full rate with one.
     static constexpr int NI = BT <= 64 ? 4 : 1;
     static constexpr int NPART = NI == 1 ? 1 : (DUAL ? 2 : 4);  // partial sums per matrix
-    // TMEM: accumulators [ACC_BUFS x ACC_COLS] then the weight ring [A_STAGES x NB x 32 cols]
+    // TMEM: accumulators [ACC_BUFS x ACC_COLS] then the weight ring [A_STAGES x NB x 64 cols]
     static constexpr int ACC_COLS = NB * NPART * BT;
     static constexpr int ACC_BUFS = 2 * ACC_COLS <= 256 ? 2 : 1;
-    static constexpr int A_COLS = 32;                        // 128 rows x 64 f16 = 32 columns
+    static constexpr int A_COLS = KS / 2;                    // 128 rows x 128 f16 = 64 columns
     static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
     static constexpr int A_STAGES = cmin(8, (512 - A_BASE) / (NB * A_COLS));
     static constexpr int CONV_WARPS = 8;
@@ -414,6 +417,7 @@ struct Fp4Cfg {
     static constexpr int SMEM_BYTES = 1024 + RSTAGES * RAW_STAGE + kCtrlBytes;
     static_assert(RSTAGES >= 2 && A_STAGES >= 2 && SMEM_BYTES <= kSmemLimit, "FP4 GEMM config");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
+    static_assert(BOX_BYTES % 1024 == 0, "token boxes must stay 1024-byte aligned");
 };
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
@@ -436,6 +440,33 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t sc2, uint32_t
 // f16x2 holding `bits` in both halves
 __device__ __forceinline__ uint32_t dup16(uint32_t bits) { return (bits & 0xFFFFu) | (bits << 16); }
 
+// One weight row's 64 K values of one prepared chunk -> 32 f16x2 words (scale applied).
+template <int WFMT>
+__device__ __forceinline__ void convert_chunk_row(const uint8_t* chunk, int row, const uint16_t* lut,
+                                                  uint32_t (&o)[32]) {
+    constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;
+    const uint4 v0 = *reinterpret_cast<const uint4*>(chunk + row * 32);
+    const uint4 v1 = *reinterpret_cast<const uint4*>(chunk + row * 32 + 16);
+    const uint8_t* rs = chunk + kTileN * 32 + row * S;
+    uint32_t sc[4];
+    if (WFMT == MOE_W_MXFP4) {
+        sc[0] = sc[1] = dup16(lut[rs[0]]);
+        sc[2] = sc[3] = dup16(lut[rs[1]]);
+    } else {
+        const uint32_t four = *reinterpret_cast<const uint32_t*>(rs);
+        uint32_t s01, s23;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"((uint16_t)(four & 0xFFFF)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s23) : "h"((uint16_t)(four >> 16)));
+        sc[0] = dup16(s01);
+        sc[1] = dup16(s01 >> 16);
+        sc[2] = dup16(s23);
+        sc[3] = dup16(s23 >> 16);
+    }
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
+}
+
 template <int BT, bool DUAL, int WFMT, int OUT>
 __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
@@ -444,13 +475,11 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::RSTAGES * C::RAW_STAGE);
     volatile int* abort_flag = &ctl->abort;
+    // raw stage r: [token box 0][token box 1][matrix 0: chunk kb, chunk kb+1][matrix 1: ...]
     auto rawB = [&](int r) { return smem + r * C::RAW_STAGE; };
-    auto rawD = [&](int r, int m) { return smem + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_D; };
-    auto rawS = [&](int r, int m) {
-        return smem + r * C::RAW_STAGE + C::B_BYTES + C::NB * C::RAW_D + m * C::RAW_S;
-    };
+    auto rawM = [&](int r, int m) { return smem + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_M; };
     const int warp = warp_id(), lane = lane_id();
-    const int G = a.G, NT = a.NT, KB = a.KB;
+    const int G = a.G, NT = a.NT, KB = a.KB;   // KB: stages of 128 K per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::A_STAGES; ++s) {
@@ -495,27 +524,25 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
     const int total = ctl->tpre[G];
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- producer: token tile (TMA) + codes and scales (bulk)
+        if (lane == 0) {  // ---------------- producer: two token boxes (TMA) + one copy per matrix
             int r = 0;
             uint32_t ph = 0, issued_mask = 0, issued_par = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const size_t chunk0 = ((size_t)g * NT + nt) * (2 * KB);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&ctl->raw_empty[r], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const size_t tile = ((size_t)g * NT + nt) * KB + kb;
-                    mbar_arrive_expect_tx(&ctl->raw_full[r], C::B_BYTES + C::NB * (C::RAW_D + C::RAW_S));
-                    bulk_load(rawD(r, 0), a.kd0 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[r]);
-                    bulk_load(rawS(r, 0), a.ks0 + tile * C::RAW_S, C::RAW_S, &ctl->raw_full[r]);
-                    if (DUAL) {
-                        bulk_load(rawD(r, 1), a.kd1 + tile * C::RAW_D, C::RAW_D, &ctl->raw_full[r]);
-                        bulk_load(rawS(r, 1), a.ks1 + tile * C::RAW_S, C::RAW_S, &ctl->raw_full[r]);
-                    }
-                    tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * kTileK, row0);
+                    mbar_arrive_expect_tx(&ctl->raw_full[r], C::B_BYTES + C::NB * C::RAW_M);
+                    const size_t off = (chunk0 + 2 * kb) * C::CHUNK;
+                    bulk_load(rawM(r, 0), a.kd0 + off, C::RAW_M, &ctl->raw_full[r]);
+                    if (DUAL) bulk_load(rawM(r, 1), a.kd1 + off, C::RAW_M, &ctl->raw_full[r]);
+                    tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0);
+                    tma_load_2d(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0);
                     issued_mask |= 1u << r;
                     issued_par = (issued_par & ~(1u << r)) | (ph << r);
                     if (++r == C::RSTAGES) {
@@ -534,13 +561,15 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
         }
     } else if (warp < C::EPI_WARP0) {
         if (lane == 0) {  // ---------------- MMA issuers: A from TMEM, B (tokens) from smem
-            // issuer i: with NI == 1 all four K steps of both matrices; with NI == 4 and two
-            // matrices, matrix i&1 over K steps {2(i>>1), 2(i>>1)+1} into partial i>>1; with
-            // one matrix, K step i into partial i. Partial p of matrix m sits at column
-            // (p*NB + m)*BT of the accumulator buffer.
+            // A stage: matrix m at columns (s*NB + m)*64, K step kk (0..7) at +8*kk.
+            // B: K step kk in token box kk/4 at byte offset (kk%4)*32.
+            // Issuer i with NI == 4: two matrices -> matrix i&1, K steps 4(i>>1)..+3,
+            // partial i>>1; one matrix -> K steps 2i, 2i+1, partial i. Partial p of matrix m
+            // at column (p*NB + m)*BT of the accumulator buffer.
             const int i = warp - 1;
             constexpr uint32_t idesc = idesc_f16(0, kTileN, BT);
-            constexpr int KPI = (kTileK / 16) / (C::NI == 1 ? 1 : (DUAL ? 2 : 4));  // K steps per issuer
+            constexpr int KSTEPS = C::KS / 16;
+            constexpr int KPI = C::NI == 1 ? KSTEPS : (DUAL ? KSTEPS / 2 : KSTEPS / 4);
             const int m_i = (C::NI == 1 || !DUAL) ? 0 : (i & 1);
             const int p_i = C::NI == 1 ? 0 : (DUAL ? (i >> 1) : i);
             const int kk0 = p_i * KPI;
@@ -562,20 +591,22 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                     tc_fence_after();
                     const uint32_t bb = smem_u32(rawB(r));
                     const uint32_t a0 = tmem_base + (uint32_t)(C::A_BASE + (s * C::NB) * C::A_COLS);
+                    auto bdesc = [&](int kk) {
+                        return sw128_kmajor_desc(bb + (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32);
+                    };
                     if (C::NI == 1) {
 #pragma unroll
-                        for (int kk = 0; kk < kTileK / 16; ++kk) {
-                            const uint64_t bdesc = sw128_kmajor_desc(bb + kk * 32);
+                        for (int kk = 0; kk < KSTEPS; ++kk) {
                             const uint32_t acc = (kb | kk) != 0;
-                            mma_f16_ts(d0, a0 + kk * 8, bdesc, idesc, acc);
-                            if (DUAL) mma_f16_ts(d0 + BT, a0 + C::A_COLS + kk * 8, bdesc, idesc, acc);
+                            mma_f16_ts(d0, a0 + kk * 8, bdesc(kk), idesc, acc);
+                            if (DUAL) mma_f16_ts(d0 + BT, a0 + C::A_COLS + kk * 8, bdesc(kk), idesc, acc);
                         }
                     } else {
                         const uint32_t dm = d0 + (uint32_t)((p_i * C::NB + m_i) * BT);
 #pragma unroll
                         for (int j = 0; j < KPI; ++j) {
                             const int kk = kk0 + j;
-                            mma_f16_ts(dm, a0 + m_i * C::A_COLS + kk * 8, sw128_kmajor_desc(bb + kk * 32), idesc,
+                            mma_f16_ts(dm, a0 + m_i * C::A_COLS + kk * 8, bdesc(kk), idesc,
                                        (kb > 0 || j > 0) ? 1u : 0u);
                         }
                     }
@@ -601,7 +632,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {
+                if (issued) {  // wait (bounded) for this issuer's MMAs before TMEM is released
                     int never = 0;
                     mma_commit(&ctl->drain[i]);
                     mbar_wait(&ctl->drain[i], 0, &never);
@@ -609,7 +640,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
             }
         }
     } else if (warp < C::CONV_WARP0) {
-        // ---------------- epilogue (warps 2..5)
+        // ---------------- epilogue (4 warps)
         const int q = warp & 3;
         int b = 0;
         uint32_t bph = 0;
@@ -622,8 +653,8 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT, C::NPART>(a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g,
-                                         nt, row0, rows, q, lane);
+            epilogue_tile<BT, DUAL, OUT, C::NPART>(
+                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[b]);
@@ -634,10 +665,10 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
         }
         if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
     } else {
-        // ---------------- converters (warps 6..13): e2m1 x block scale -> f16 rows in TMEM.
+        // ---------------- converters (8 warps): e2m1 x block scale -> f16 rows in TMEM.
         // Warp w owns TMEM lanes [32q, 32q+32), q = w % 4, so thread `lane` converts weight
-        // row 32q + lane. With two matrices the second warp of the quarter takes the up
-        // projection; with one, the two warps split the 64 K values of the stage.
+        // row 32q + lane. With two matrices the second warp of a quarter takes the up
+        // projection (both 64-K chunks); with one, the two warps take one chunk each.
         const int q = warp & 3, grp = (warp - C::CONV_WARP0) >> 2;
         const int row = q * 32 + lane;
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -653,50 +684,18 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                const uint32_t acol = (uint32_t)(C::A_BASE + s * C::NB * C::A_COLS);
+                uint32_t o[32];
                 if (DUAL) {
-                    const int m = grp;
-                    const uint8_t* rd = rawD(r, m) + row * 32;
-                    const uint8_t* rs = rawS(r, m);
-                    const uint4 v0 = *reinterpret_cast<const uint4*>(rd);
-                    const uint4 v1 = *reinterpret_cast<const uint4*>(rd + 16);
-                    uint32_t sc[4];
-                    if (WFMT == MOE_W_MXFP4) {
-                        sc[0] = sc[1] = dup16(ctl->lut[rs[row * 2]]);
-                        sc[2] = sc[3] = dup16(ctl->lut[rs[row * 2 + 1]]);
-                    } else {
-                        const uint32_t four = *reinterpret_cast<const uint32_t*>(rs + row * 4);
-                        uint32_t s01, s23;
-                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"((uint16_t)(four & 0xFFFF)));
-                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s23) : "h"((uint16_t)(four >> 16)));
-                        sc[0] = dup16(s01);
-                        sc[1] = dup16(s01 >> 16);
-                        sc[2] = dup16(s23);
-                        sc[3] = dup16(s23 >> 16);
+                    const uint8_t* raw = rawM(r, grp);
+#pragma unroll 1
+                    for (int c = 0; c < 2; ++c) {
+                        convert_chunk_row<WFMT>(raw + c * C::CHUNK, row, ctl->lut, o);
+                        tmem_st32(lane_base + acol + grp * C::A_COLS + c * 32, o);
                     }
-                    uint32_t o[32];
-                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
-                    tmem_st32(lane_base + (uint32_t)(C::A_BASE + (s * C::NB + m) * C::A_COLS), o);
                 } else {
-                    const int h = grp;  // K half
-                    const uint4 v = *reinterpret_cast<const uint4*>(rawD(r, 0) + row * 32 + h * 16);
-                    const uint8_t* rs = rawS(r, 0);
-                    uint32_t sc[2];
-                    if (WFMT == MOE_W_MXFP4) {
-                        sc[0] = sc[1] = dup16(ctl->lut[rs[row * 2 + h]]);
-                    } else {
-                        const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + row * 4 + h * 2);
-                        uint32_t s01;
-                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"(pair));
-                        sc[0] = dup16(s01);
-                        sc[1] = dup16(s01 >> 16);
-                    }
-                    uint32_t o[16];
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
-                    tmem_st16(lane_base + (uint32_t)(C::A_BASE + s * C::A_COLS + h * 16), o);
+                    convert_chunk_row<WFMT>(rawM(r, 0) + grp * C::CHUNK, row, ctl->lut, o);
+                    tmem_st32(lane_base + acol + grp * 32, o);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -854,7 +853,8 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.G = p.G;
     a.N = p.N;
     a.K = p.K;
-    a.KB = (p.K + kTileK - 1) / kTileK;
+    // pipeline stages per tile: 64 K values (BF16) or 128 (FP4, two prepared chunks)
+    a.KB = p.wfmt == MOE_W_BF16 ? (p.K + kTileK - 1) / kTileK : (p.K + kFp4StageK - 1) / kFp4StageK;
     a.NT = (p.N + kTileN - 1) / kTileN;
     a.M_alloc = p.M_alloc;
     a.out = p.out;

@@ -98,6 +98,9 @@ int choose_token_tile(long long NvS, int G);
 constexpr int kTileN = 128;
 constexpr int kTileK = 64;
 inline int fp4_scale_bytes_per_row(int wfmt) { return wfmt == MOE_W_MXFP4 ? 2 : 4; }
+// Prepared FP4 chunk (128 rows x 64 K): codes then scales, contiguous.
+inline int fp4_chunk_bytes(int wfmt) { return kTileN * 32 + kTileN * fp4_scale_bytes_per_row(wfmt); }
+constexpr int kFp4StageK = 128;  // K values per FP4 pipeline stage (two chunks)
 
 // ---------------------------------------------------------------- device info
 int num_sms();

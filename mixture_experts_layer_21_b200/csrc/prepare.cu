@@ -2,10 +2,12 @@
 // (the "kernel format" of the FlashInfer MoE-EP page's
 // process_weights_after_loading and the DeepSeek-V4 FI page's finalize_weights).
 //
-// Layout, per weight row g, per 128-row block nt, per 64-value K block kb:
-//   kdata : 128 rows x 32 bytes of packed e2m1 (even k in the low nibble),
-//           zero past N and past K: one 4 KB contiguous tile per pipeline stage.
-//   kscale: 128 rows x S bytes, S = 2 (MXFP4, two e8m0 per 64) or 4 (NVFP4, four e4m3).
+// Layout: chunks [g][nt][kb] for weight row g, 128-row block nt and 64-value K block
+// kb, the number of K blocks padded to even (a pipeline stage covers 128 K values);
+// each chunk of kFp4ChunkBytes(fmt) = 4096 + 128*S bytes holds
+//   128 rows x 32 bytes of packed e2m1 (even k in the low nibble), zero past N and K,
+//   then 128 rows x S scale bytes, S = 2 (MXFP4, two e8m0 per 64) or 4 (NVFP4, four e4m3),
+// so one stage is one contiguous copy per matrix. kdata and kscale both point at it.
 //   kalpha: fp32 [G]. NVFP4: weight_scale_2 (1 if absent). MXFP4: 2^bias_g, where
 //           bias_g re-bases expert g's e8m0 exponents so its largest block scale is
 //           2^13; the GEMM stages e2m1 * 2^(e-127-bias) in f16, exact while the
@@ -29,17 +31,17 @@ struct PrepLayout {
 PrepLayout prep_layout(const moe_weight_t* w) {
     PrepLayout L{};
     L.NT = (w->N + kTileN - 1) / kTileN;
-    L.KB = (w->K + kTileK - 1) / kTileK;
+    L.KB = 2 * ((w->K + 2 * kTileK - 1) / (2 * kTileK));  // padded to even
     L.S = fp4_scale_bytes_per_row(w->fmt);
-    const size_t tiles = (size_t)w->G * L.NT * L.KB;
+    const size_t chunks = (size_t)w->G * L.NT * L.KB;
     size_t off = 0;
     auto take = [&](size_t b) {
         const size_t o = off;
         off += (b + 255) & ~size_t(255);
         return o;
     };
-    L.data_off = take(tiles * kTileN * 32);
-    L.scale_off = take(tiles * kTileN * L.S);
+    L.data_off = take(chunks * fp4_chunk_bytes(w->fmt));
+    L.scale_off = L.data_off;
     L.alpha_off = take(sizeof(float) * w->G);
     L.scratch_off = take(sizeof(int) * 2 * w->G + 16);
     L.bytes = off;
@@ -79,13 +81,12 @@ __global__ void mx_scale_range_kernel(const uint8_t* __restrict__ scale, int N, 
     }
 }
 
-// One block per (g, nt, kb) tile; thread r copies weight row nt*128 + r.
+// One block per (g, nt, kb) chunk; thread r copies weight row nt*128 + r.
 __global__ void __launch_bounds__(128) relayout_kernel(const uint8_t* __restrict__ data,
                                                        const uint8_t* __restrict__ scale, int fmt,
                                                        int G, int N, int K, int NT, int KB,
                                                        const int* __restrict__ bias,
-                                                       uint8_t* __restrict__ kdata,
-                                                       uint8_t* __restrict__ kscale) {
+                                                       uint8_t* __restrict__ chunks) {
     const size_t tile = blockIdx.x;
     const int kb = (int)(tile % KB);
     const int nt = (int)((tile / KB) % NT);
@@ -96,14 +97,16 @@ __global__ void __launch_bounds__(128) relayout_kernel(const uint8_t* __restrict
     const int S = fmt == MOE_W_MXFP4 ? 2 : 4;
     const int per = fmt == MOE_W_MXFP4 ? 32 : 16;  // values per scale
     const int KS = K / per;
+    uint8_t* chunk = chunks + tile * (size_t)(kTileN * 32 + kTileN * S);
     uint8_t out[32];
     for (int i = 0; i < 32; ++i) {
         const int byte = kb * 32 + i;
         out[i] = (n < N && byte < row_bytes) ? data[((size_t)g * N + n) * row_bytes + byte] : (uint8_t)0;
     }
-    uint4* d = reinterpret_cast<uint4*>(kdata + tile * (kTileN * 32) + r * 32);
+    uint4* d = reinterpret_cast<uint4*>(chunk + r * 32);
     d[0] = *reinterpret_cast<uint4*>(out);
     d[1] = *reinterpret_cast<uint4*>(out + 16);
+    uint8_t* kscale = chunk + kTileN * 32;
     for (int i = 0; i < S; ++i) {
         const int si = kb * S + i;
         uint8_t v = 0;
@@ -113,7 +116,7 @@ __global__ void __launch_bounds__(128) relayout_kernel(const uint8_t* __restrict
         } else if (fmt == MOE_W_MXFP4) {
             v = 127;  // any finite scale: these codes are zero
         }
-        kscale[tile * (kTileN * S) + r * S + i] = v;
+        kscale[r * S + i] = v;
     }
     (void)G;
 }
@@ -164,7 +167,7 @@ moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaS
     if (tiles > 0) {
         relayout_kernel<<<(unsigned)tiles, 128, 0, st>>>(static_cast<const uint8_t*>(w->data),
                                                           static_cast<const uint8_t*>(w->scale), w->fmt, w->G, w->N,
-                                                          w->K, L.NT, L.KB, d_bias, kdata, kscale);
+                                                          w->K, L.NT, L.KB, d_bias, kdata);
     }
     alpha_kernel<<<(w->G + 255) / 256, 256, 0, st>>>(w->alpha, d_bias, w->fmt, w->G, kalpha);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
