@@ -226,4 +226,14 @@ MOE_DEV float act_apply(int act, float g, float u, float a, float b) {
     return silu_f(g) * u;
 }
 
+// The same activations for the GEMM epilogue, from the exponential intrinsic and
+// approximate division (relative error ~1e-6, far below the 16-bit output rounding):
+// sigmoid(x) = 1/(1+e^-x), tanh(y) = 1 - 2/(1+e^(2y)) (exact limits +-1 as e^(2y) -> inf / 0).
+MOE_DEV float fast_sigmoid(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+MOE_DEV float fast_tanh(float y) { return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * y)); }
+MOE_DEV float act_apply_fast(int act, float g, float u, float a, float b, float inv_a, float inv_b) {
+    if (act == MOE_ACT_SITU) return a * fast_tanh(g * inv_a) * fast_sigmoid(g) * (b * fast_tanh(u * inv_b));
+    return g * fast_sigmoid(g) * u;
+}
+
 }  // namespace moe

@@ -147,6 +147,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
     const int n = nt * kTileN + q * 32 + lane;
     const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
     const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
+    const float inv_sa = 1.0f / a.sa, inv_sb = 1.0f / a.sb;
     constexpr int STRIDE = DUAL ? 2 * BT : BT;   // column distance between partials of one matrix
 #pragma unroll 1
     for (int c0 = 0; c0 < BT; c0 += 16) {
@@ -167,18 +168,24 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
                 if (DUAL) r1[j] = __float_as_uint(__uint_as_float(r1[j]) + __uint_as_float(p1[j]));
             }
         }
-        if (n < a.N) {
+        // per-token factors of this 16-token chunk: one coalesced load, then broadcasts
+        const int my_row = row0 + c0 + (lane & 15);
+        const bool row_ok = c0 + (lane & 15) < rows;
+        const float my_ts = (a.tscale && row_ok) ? a.tscale[my_row] : 1.0f;
+        const float my_pw = (DUAL && a.perm_w && row_ok) ? a.perm_w[my_row] : 1.0f;
+        {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                if (c0 + j < rows) {
+                // every lane takes part in the shuffles; only in-range outputs are stored
+                const float ts = __shfl_sync(0xffffffffu, my_ts, j);
+                const float pw = __shfl_sync(0xffffffffu, my_pw, j);
+                if (n < a.N && c0 + j < rows) {
                     const int row = row0 + c0 + j;
-                    const float ts = a.tscale ? a.tscale[row] : 1.0f;
                     float v;
                     if (DUAL) {
                         const float gv = __uint_as_float(r0[j]) * al0 * ts;
                         const float uv = __uint_as_float(r1[j]) * al1 * ts;
-                        v = act_apply(a.act, gv, uv, a.sa, a.sb);
-                        if (a.perm_w) v *= a.perm_w[row];
+                        v = act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb) * pw;
                     } else {
                         v = __uint_as_float(r0[j]) * al0 * ts;
                     }
@@ -409,7 +416,7 @@ struct Fp4Cfg {
     static constexpr int A_COLS = KS / 2;                    // 128 rows x 128 f16 = 64 columns
     static constexpr int A_BASE = ACC_BUFS * ACC_COLS;
     static constexpr int A_STAGES = cmin(8, (512 - A_BASE) / (NB * A_COLS));
-    static constexpr int CONV_WARPS = 8;
+    static constexpr int CONV_WARPS = 16;
     // warps: 0 producer, [1, 1+NI) issuers, then 4 epilogue, then the converters
     static constexpr int EPI_WARP0 = 1 + NI;
     static constexpr int CONV_WARP0 = EPI_WARP0 + 4;
@@ -465,6 +472,28 @@ __device__ __forceinline__ void convert_chunk_row(const uint8_t* chunk, int row,
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
+}
+
+// Half of it: the 32 values [32h, 32h+32) of the chunk row -> 16 f16x2 words.
+template <int WFMT>
+__device__ __forceinline__ void convert_half_chunk_row(const uint8_t* chunk, int row, int h, const uint16_t* lut,
+                                                       uint32_t (&o)[16]) {
+    constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;
+    const uint4 v = *reinterpret_cast<const uint4*>(chunk + row * 32 + h * 16);
+    const uint8_t* rs = chunk + kTileN * 32 + row * S;
+    uint32_t sc[2];
+    if (WFMT == MOE_W_MXFP4) {
+        sc[0] = sc[1] = dup16(lut[rs[h]]);
+    } else {
+        const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + 2 * h);
+        uint32_t s01;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"(pair));
+        sc[0] = dup16(s01);
+        sc[1] = dup16(s01 >> 16);
+    }
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
 }
 
 template <int BT, bool DUAL, int WFMT, int OUT>
@@ -665,10 +694,10 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
         }
         if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
     } else {
-        // ---------------- converters (8 warps): e2m1 x block scale -> f16 rows in TMEM.
+        // ---------------- converters (16 warps): e2m1 x block scale -> f16 rows in TMEM.
         // Warp w owns TMEM lanes [32q, 32q+32), q = w % 4, so thread `lane` converts weight
-        // row 32q + lane. With two matrices the second warp of a quarter takes the up
-        // projection (both 64-K chunks); with one, the two warps take one chunk each.
+        // row 32q + lane; the four warps of a quarter split a stage's row into four units
+        // (two matrices x two 64-K chunks, or two chunks x two halves).
         const int q = warp & 3, grp = (warp - C::CONV_WARP0) >> 2;
         const int row = q * 32 + lane;
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -685,17 +714,16 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t acol = (uint32_t)(C::A_BASE + s * C::NB * C::A_COLS);
-                uint32_t o[32];
-                if (DUAL) {
-                    const uint8_t* raw = rawM(r, grp);
-#pragma unroll 1
-                    for (int c = 0; c < 2; ++c) {
-                        convert_chunk_row<WFMT>(raw + c * C::CHUNK, row, ctl->lut, o);
-                        tmem_st32(lane_base + acol + grp * C::A_COLS + c * 32, o);
-                    }
-                } else {
-                    convert_chunk_row<WFMT>(rawM(r, 0) + grp * C::CHUNK, row, ctl->lut, o);
-                    tmem_st32(lane_base + acol + grp * 32, o);
+                if (DUAL) {  // unit grp: matrix grp>>1, chunk grp&1 (64 values)
+                    const int m = grp >> 1, c = grp & 1;
+                    uint32_t o[32];
+                    convert_chunk_row<WFMT>(rawM(r, m) + c * C::CHUNK, row, ctl->lut, o);
+                    tmem_st32(lane_base + acol + m * C::A_COLS + c * 32, o);
+                } else {     // unit grp: chunk grp>>1, half grp&1 (32 values)
+                    const int c = grp >> 1, h = grp & 1;
+                    uint32_t o[16];
+                    convert_half_chunk_row<WFMT>(rawM(r, 0) + c * C::CHUNK, row, h, ctl->lut, o);
+                    tmem_st16(lane_base + acol + c * 32 + h * 16, o);
                 }
                 tmem_st_wait();
                 tc_fence_before();
