@@ -122,6 +122,22 @@ def profiled_traffic(workload: str) -> float | None:
         return None
 
 
+# ---------------------------------------------------------------------------- ranks
+
+def reduce_max(v: float, world: int, device) -> float:
+    """Max of a per-rank value over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank runs its own replica on its own batch."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 # ---------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -249,11 +265,7 @@ def run_ours(args, cfg, rank, world):
             torch.cuda.synchronize()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     ids_d = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device=dev)
     for _ in range(Wm):
@@ -305,7 +317,7 @@ def run_ours(args, cfg, rank, world):
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(a0.elapsed_time(a1))
-        e2e = {"value": world * cfg.T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_tokens_per_s(world, cfg.T, K, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 4),
                "d2h_bytes_per_step": int(o_h.numel() * 2)}
 
@@ -328,7 +340,7 @@ def run_ours(args, cfg, rank, world):
                  "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst)"})
     t_layer_roof = max(acc["layer_flops"] / (peaks["bf16_tflops"] * 1e12),
                        acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
-    tok_s = world * cfg.T * K / (ms_total / 1e3)
+    tok_s = job_tokens_per_s(world, cfg.T, K, ms_total)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
