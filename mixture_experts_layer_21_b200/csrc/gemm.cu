@@ -865,13 +865,18 @@ cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtens
 
 }  // namespace
 
-int choose_token_tile(long long NvS, int G) {
+// Token tile from the mean segment length. 256-token tiles exist for the single-matrix
+// BF16 GEMM only: at 128 x 128 it needs about twice the shared-memory bandwidth per FLOP
+// that an SM has, and a 256-wide tile halves the weight-tile traffic per FLOP while its
+// double-buffered accumulators (2 x 256 columns) still fit in TMEM.
+int choose_token_tile(long long NvS, int G, bool wide_ok) {
     const long long segs = std::max<long long>(1, std::min<long long>(G, NvS));
     const long long avg = (NvS + segs - 1) / segs;
     if (avg <= 16) return 16;
     if (avg <= 32) return 32;
     if (avg <= 64) return 64;
-    return 128;
+    if (avg <= 128 || !wide_ok) return 128;
+    return 256;
 }
 
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl) {
@@ -900,13 +905,16 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.ks1 = static_cast<const uint8_t*>(p.kscale1);
     a.zero_pad = p.zero_pad ? 1 : 0;
     a.err = p.err;
+    const bool wide_ok = p.wfmt == MOE_W_BF16 && !p.dual;
     int bt = p.bt;
     if (!bt) {
-        // MOE_TOKEN_TILE=16|32|64|128 overrides the token-tile choice (tests, tuning)
+        // MOE_TOKEN_TILE=16|32|64|128|256 overrides the token-tile choice (tests, tuning)
         const char* env = getenv("MOE_TOKEN_TILE");
         const int v = env ? atoi(env) : 0;
-        bt = (v == 16 || v == 32 || v == 64 || v == 128) ? v : choose_token_tile(p.M_alloc, p.G);
+        bt = (v == 16 || v == 32 || v == 64 || v == 128 || (v == 256 && wide_ok)) ? v
+                                                                                   : choose_token_tile(p.M_alloc, p.G, wide_ok);
     }
+    if (bt == 256 && !wide_ok) bt = 128;
     const CUtensorMapDataType xdt =
         p.wfmt == MOE_W_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tx, t0, t1;
@@ -922,6 +930,9 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
         case 16: return dispatch_bt<16>(p, a, tx, t0, t1, st, pdl);
         case 32: return dispatch_bt<32>(p, a, tx, t0, t1, st, pdl);
         case 64: return dispatch_bt<64>(p, a, tx, t0, t1, st, pdl);
+        case 256:
+            if (p.out_kind == OUT_F32) return run_bf16<256, false, OUT_F32>(p, a, tx, t0, t1, st, pdl);
+            return run_bf16<256, false, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
         default: return dispatch_bt<128>(p, a, tx, t0, t1, st, pdl);
     }
 }

@@ -92,7 +92,7 @@ struct GemmProblem {
     DevError* err;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
-int choose_token_tile(long long NvS, int G);
+int choose_token_tile(long long NvS, int G, bool wide_ok);
 
 // FP4 kernel layout: tiles of 128 weight rows x 64 K values.
 constexpr int kTileN = 128;

@@ -123,6 +123,20 @@ def test_grouped_gemm_every_token_tile(lib, bt, fmt, monkeypatch):
     check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what=f"bt{bt}")
 
 
+def test_grouped_gemm_bf16_256_token_tile(lib, monkeypatch):
+    # the wide tile of the single-matrix BF16 GEMM: segments spanning 1, 2 and 3 tiles, ragged N
+    monkeypatch.setenv("MOE_TOKEN_TILE", "256")
+    seg = [300, 0, 17, 600, 1]
+    M, N, K = sum(seg) + 9, 200, 192
+    a, wt, _ = W.gen_grouped_gemm_case(M, seg, N, K, seed=256)
+    cu = np.cumsum(seg).astype(np.int32)
+    w = lib.Weight("bf16", to_dev(wt))
+    out = lib.moe_grouped_gemm(to_dev(a), w, to_dev(torch.from_numpy(cu)))
+    torch.cuda.synchronize()
+    ref = O.grouped_gemm(O.to_f64(a), W.WeightSet("bf16", wt), cu, M_alloc=M)
+    check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what="bt256")
+
+
 def test_grouped_gemm_bf16_matches_torch_grouped_mm(lib):
     if not hasattr(torch, "_grouped_mm"):
         pytest.skip("torch._grouped_mm unavailable")
