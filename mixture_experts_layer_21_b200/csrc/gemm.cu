@@ -68,6 +68,7 @@ struct GemmArgs {
     const uint8_t* kd1;
     const uint8_t* ks1;
     int zero_pad;
+    int x3d;          // FP4: the token map is 3-D {64, rows, K/64}: one copy per 128-K stage
     DevError* err;
 };
 
@@ -423,6 +424,7 @@ struct Fp4Cfg {
     static constexpr int THREADS = (CONV_WARP0 + CONV_WARPS) * 32;
     static constexpr int SMEM_BYTES = 1024 + RSTAGES * RAW_STAGE + kCtrlBytes;
     static_assert(RSTAGES >= 2 && A_STAGES >= 2 && SMEM_BYTES <= kSmemLimit, "FP4 GEMM config");
+    static_assert(RSTAGES > A_STAGES, "TMEM slot reuse is read from the raw ring's barriers");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
     static_assert(BOX_BYTES % 1024 == 0, "token boxes must stay 1024-byte aligned");
 };
@@ -570,8 +572,12 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                     const size_t off = (chunk0 + 2 * kb) * C::CHUNK;
                     bulk_load(rawM(r, 0), a.kd0 + off, C::RAW_M, &ctl->raw_full[r]);
                     if (DUAL) bulk_load(rawM(r, 1), a.kd1 + off, C::RAW_M, &ctl->raw_full[r]);
-                    tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0);
-                    tma_load_2d(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0);
+                    if (a.x3d) {  // both 64-K boxes of the token tile in one copy: {64, rows, chunks}
+                        tma_load_3d(rawB(r), &tm_x, &ctl->raw_full[r], 0, row0, 2 * kb);
+                    } else {
+                        tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0);
+                        tma_load_2d(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0);
+                    }
                     issued_mask |= 1u << r;
                     issued_par = (issued_par & ~(1u << r)) | (ph << r);
                     if (++r == C::RSTAGES) {
@@ -613,7 +619,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&ctl->raw_full[r], rph, abort_flag)) {
+                    // the converters arrive on full[s] only after they saw raw stage r land, so
+                    // this one wait also orders the token tile before the MMA
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -640,7 +648,8 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                         }
                     }
                     issued = true;
-                    mma_commit(&ctl->empty[s]);
+                    // one commit per stage: it frees raw stage r and, for the converters, the
+                    // TMEM weight slot of this stage
                     mma_commit(&ctl->raw_empty[r]);
                     if (++s == C::A_STAGES) {
                         s = 0;
@@ -703,10 +712,19 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         int s = 0, r = 0;
         uint32_t ph = 0, rph = 0;
+        long long it = 0;  // stages converted so far
         bool ok = true;
         for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-            for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&ctl->raw_full[r], rph, abort_flag) || !mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                // The TMEM weight slot s is free once the MMAs of stage it - A_STAGES are done,
+                // which the issuers' commit on that stage's raw barrier records. That barrier
+                // cannot run a phase ahead: it would need stage it - A_STAGES + RSTAGES > it.
+                bool got = mbar_wait(&ctl->raw_full[r], rph, abort_flag);
+                if (got && it >= C::A_STAGES) {
+                    const long long j = it - C::A_STAGES;
+                    got = mbar_wait(&ctl->raw_empty[j % C::RSTAGES], (uint32_t)((j / C::RSTAGES) & 1), abort_flag);
+                }
+                if (!got) {
                     if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 4);
                     ctl->abort = 1;
                     ok = false;
@@ -781,6 +799,22 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64
     const cuuint32_t box[2] = {(cuuint32_t)kTileK, box_rows};
     const cuuint32_t es[2] = {1, 1};
     return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A row-major [rows, K] matrix of 16-bit elements seen as {64 columns, rows, K/64 chunks}
+// (chunk stride 128 bytes); box = 64 x box_rows x 2 lands as two consecutive 64-column
+// boxes, i.e. a 128-K token tile in one copy. Needs K % 64 == 0 (no column past K is read).
+bool make_map_3d_chunks(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t K, uint64_t rows,
+                        uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc || K % kTileK) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kTileK, rows, K / kTileK};
+    const cuuint64_t strides[2] = {K * 2, (cuuint64_t)kTileK * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kTileK, box_rows, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -920,7 +954,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     CUtensorMap tx, t0, t1;
     memset(&t0, 0, sizeof(t0));
     memset(&t1, 0, sizeof(t1));
-    if (!make_map_2d(&tx, p.x, xdt, p.K, p.M_alloc, bt)) return cudaErrorInvalidValue;
+    a.x3d = p.wfmt != MOE_W_BF16 && p.K % kTileK == 0;
+    if (a.x3d) {
+        if (!make_map_3d_chunks(&tx, p.x, xdt, p.K, p.M_alloc, bt)) return cudaErrorInvalidValue;
+    } else if (!make_map_2d(&tx, p.x, xdt, p.K, p.M_alloc, bt)) {
+        return cudaErrorInvalidValue;
+    }
     if (p.wfmt == MOE_W_BF16) {
         if (!make_map_3d(&t0, p.w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G)) return cudaErrorInvalidValue;
         if (p.dual && !make_map_3d(&t1, p.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G))
