@@ -273,25 +273,38 @@ def run_ours(args, cfg, rank, world):
     assert layer.device_error() == 0, "device error in warm-up"
     acc = accounting(cfg, inp, *segment_stats(cfg, ids_d, inp.replica_src))
 
-    # ---- device-resident timed region, stage events on the launching stream
+    # ---- device-resident timed region. Only the two events around the gate/up GEMM are
+    # recorded (on the launching stream): every other kernel boundary keeps its
+    # programmatic-dependent-launch overlap.
     nst = m.MOE_FWD_STAGE_EVENTS
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(K)]
-    for row in evs:
+
+    def new_events():
+        row = [torch.cuda.Event(enable_timing=True) for _ in range(nst)]
         for e in row:
-            e.record(stream)
+            e.record(stream)  # creates the handle
+        return row
+
+    fc1_evs = [new_events() for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0.record(stream)
         for i in range(K):
-            layer(x_d, l_d, out=out_d, stage_events=evs[i])
+            ev = fc1_evs[i]
+            layer(x_d, l_d, out=out_d, stage_events=[None, None, ev[2], ev[3], None, None, None])
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
     ms_total = max_over_ranks(t0.elapsed_time(t1))
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nst - 1)]
-                         for i in range(K)]).mean(axis=0)
+    fc1_ms = float(np.mean([fc1_evs[i][2].elapsed_time(fc1_evs[i][3]) for i in range(K)]))
     assert layer.device_error() == 0, "device error in timed region"
+
+    # ---- stage breakdown (separate pass, all seven events; not part of the value)
+    br_evs = [new_events() for _ in range(min(K, 10))]
+    for row in br_evs:
+        layer(x_d, l_d, out=out_d, stage_events=row)
+    torch.cuda.synchronize()
+    stage_ms = np.array([[row[j].elapsed_time(row[j + 1]) for j in range(nst - 1)] for row in br_evs]).mean(axis=0)
 
     # ---- end to end through the public call, host buffers
     e2e = None
@@ -323,7 +336,6 @@ def run_ours(args, cfg, rank, world):
 
     peaks, peak_src = load_peaks()
     ms_step = ms_total / K
-    fc1_ms = float(stage_ms[2])
     t_fc1_tensor = acc["fc1_flops"] / (peaks["bf16_tflops"] * 1e12)
     t_fc1_hbm = acc["fc1_bytes"] / (peaks["hbm_gbs"] * 1e9)
     traffic = profiled_traffic(args.config)

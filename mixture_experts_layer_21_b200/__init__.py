@@ -288,13 +288,15 @@ class MoEForward:
 
     def __call__(self, x, router_logits, out=None, topk_ids=None, topk_w=None, stream=None,
                  stage_events=None):
-        """``stage_events``: None, or MOE_FWD_STAGE_EVENTS recorded torch.cuda.Event objects
-        (created with enable_timing and recorded once, so that their handles exist)."""
+        """``stage_events``: None, or a list of MOE_FWD_STAGE_EVENTS entries, each None (not
+        recorded) or a torch.cuda.Event created with enable_timing and recorded once (so that
+        its handle exists)."""
         T = x.shape[0]
         if stage_events is not None:
             if len(stage_events) != MOE_FWD_STAGE_EVENTS:
                 raise ValueError(f"need {MOE_FWD_STAGE_EVENTS} events")
-            self._ev = (ctypes.c_void_p * MOE_FWD_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
+            self._ev = (ctypes.c_void_p * MOE_FWD_STAGE_EVENTS)(
+                *[None if e is None else e.cuda_event for e in stage_events])
             self.args.stage_events = ctypes.cast(self._ev, ctypes.c_void_p)
         else:
             self.args.stage_events = None

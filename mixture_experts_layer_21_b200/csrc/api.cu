@@ -312,12 +312,19 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     const int NvS = T * k;
     cudaStream_t st = S(stream);
     cudaError_t e;
-    // optional stage events (tracing); a recorded event ends the PDL overlap at that boundary
+    // Optional stage events (tracing). An event recorded between two kernels ends their
+    // programmatic-dependent-launch overlap, so only that boundary launches without it.
+    bool ev = false;
     auto mark = [&](int i) -> bool {
         if (!p->stage_events || !p->stage_events[i]) return true;
+        ev = true;
         return cudaEventRecord(static_cast<cudaEvent_t>(p->stage_events[i]), st) == cudaSuccess;
     };
-    const bool pdl = p->stage_events == nullptr;
+    auto pdl = [&]() {
+        const bool r = !ev;
+        ev = false;
+        return r;
+    };
 
     if (!mark(0)) return MOE_ERR_CUDA;
     // S1 route
@@ -325,20 +332,20 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (e != cudaSuccess || !mark(1)) return MOE_ERR_CUDA;
     // S2 permute
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
-                       pdl);
+                       pdl());
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     // S2 gather (+ S2q)
     if (fmt == MOE_W_BF16) {
-        e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl);
+        e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (p->act_quant) {
         e = launch_quant_nvfp4(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes),
                                reinterpret_cast<uint8_t*>(w + L.xq_sb), reinterpret_cast<float*>(w + L.xq_s),
-                               reinterpret_cast<__half*>(w + L.xq_deq), st, pdl);
+                               reinterpret_cast<__half*>(w + L.xq_deq), st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(1, w + L.xq_deq, H, perm_token, NvS, xperm, reinterpret_cast<float*>(w + L.xq_s), tscale,
-                          st, pdl);
+                          st, pdl());
     } else {
-        e = launch_gather(2, p->x, H, perm_token, NvS, xperm, nullptr, tscale, st, pdl);
+        e = launch_gather(2, p->x, H, perm_token, NvS, xperm, nullptr, tscale, st, pdl());
     }
     if (e != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
 
@@ -391,14 +398,14 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         g1.out_kind = OUT_F32;
         row_pass = true;
     }
-    e = launch_grouped_gemm(g1, st, pdl);
+    e = launch_grouped_gemm(g1, st, pdl());
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
     if (row_pass) {
         if (p->act_quant) {
             e = launch_quant_nvfp4(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.act_codes),
-                                   reinterpret_cast<uint8_t*>(w + L.act_sb), act2_scale, act2, st, pdl);
+                                   reinterpret_cast<uint8_t*>(w + L.act_sb), act2_scale, act2, st, pdl());
         } else {
-            e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, pdl);
+            e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, pdl());
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         fc2_x = act2;
@@ -424,11 +431,11 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.out = y;
     g2.out_kind = OUT_F32;
     g2.err = err;
-    e = launch_grouped_gemm(g2, st, pdl);
+    e = launch_grouped_gemm(g2, st, pdl());
     if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
     // S6: combine
     e = launch_combine_f32(y, inv, p->apply_topk_in_fc1 ? nullptr : tw, T, k, H, static_cast<__nv_bfloat16*>(p->out),
-                           st, pdl);
+                           st, pdl());
     if (e != cudaSuccess || !mark(6)) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -296,12 +296,13 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
         if (e != cudaSuccess) return e;
     }
     const size_t scan_smem = sizeof(int) * (E + B + 1024);
-    e = launch_k(permute_scan_kernel, dim3(1), dim3(1024), scan_smem, st, pdl && L.nblk > 0,
+    // the scan and scatter follow this function's own kernels: they always overlap with them
+    e = launch_k(permute_scan_kernel, dim3(1), dim3(1024), scan_smem, st, L.nblk > 0 ? true : pdl,
                  (const int*)blkcnt, L.nblk, E, B, replica_src, blkoff, total, nrep, rep_ptr, rep_rows,
                  rowstart, cu_seqlens, err);
     if (e != cudaSuccess) return e;
     if (L.nblk > 0) {
-        e = launch_k(permute_scatter_kernel, dim3(L.nblk), dim3(kPermBlock), mask_smem, st, pdl, ids,
+        e = launch_k(permute_scatter_kernel, dim3(L.nblk), dim3(kPermBlock), mask_smem, st, true, ids,
                      topk_w, T, topk, E, (const int*)blkoff, (const int*)total, (const int*)nrep,
                      (const int*)rep_ptr, (const int*)rep_rows, (const int*)rowstart, perm_token,
                      perm_w, inv_perm, err);
