@@ -69,6 +69,10 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt_t;
  *           epilogue_from_quant_config: finite, > 0, one per expert).
  *   kdata, kscale, kalpha : the kernel-format copy that moe_prepare_weights
  *           writes into caller memory; NULL until then. BF16 needs none.
+ *           kdata: tiles of 128 rows x 64 K (codes, then scales) for the GEMM that
+ *           stages FP4 weights as f16. kscale: for NVFP4 with K % 256 == 0, tiles of
+ *           128 rows x 256 K for the block-scaled GEMM (moe_grouped_gemm_nvfp4);
+ *           otherwise equal to kdata. kalpha: the epilogue alphas.
  */
 typedef struct {
     int32_t fmt;            /* moe_wfmt_t */
@@ -177,6 +181,25 @@ moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * S3/S5 with NVFP4 activations — the block-scaled grouped GEMM (FlashInfer MoE-EP page:
+ * NVFP4 experts quantise activations inside the kernel; DeepSeek-V4 FI page: fc1/fc2
+ * alphas in the epilogue). For every cu_seqlens segment g and row r in it:
+ *   out[r, n] = alpha_g * a_s[r] * sum_k e2m1(a[r,k]) * e4m3(a_sb[r,k/16])
+ *                                      * e2m1(W[g][n,k]) * e4m3(W_scale[g][n,k/16])
+ * with the products summed in fp32 by the tensor cores (kind::mxf4nvf4), rounded once
+ * to bf16; rows [cu_seqlens[G-1], M_alloc) of out are written as zero.
+ *   a_codes uint8 [M_alloc, K/2] packed e2m1 (even k in the low nibble);
+ *   a_sb    uint8 [M_alloc, K/16] e4m3;  a_s fp32 [M_alloc] — the three outputs of
+ *           moe_quantize_nvfp4 for the segment-ordered rows.
+ *   w       NVFP4 weights prepared by moe_prepare_weights; K % 256 == 0 (else
+ *           MOE_ERR_ALIGNMENT); other formats: MOE_ERR_UNSUPPORTED.
+ *   out bf16 [M_alloc, N]; cu_seqlens int32 [G] on device.
+ *   ws: at least 256 bytes (the error word).
+ */
+moe_status_t moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sb, const float* a_s,
+                                    int M_alloc, const moe_weight_t* w, const int32_t* cu_seqlens,
+                                    void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+/*
  * S4 — gated activation times route weight: out[r,i] = act(gate[r,i], up[r,i]) * perm_w[r]
  * (MoonEP page, MoonEPExperts.apply). gate/up/out bf16 [M, I]; perm_w fp32 [M]
  * or NULL (no scaling). Computed in fp32, rounded once to bf16.
@@ -230,7 +253,9 @@ moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,
  * finalized output out) are the two shapes this mirrors.
  *   x bf16 [T,H]; router_logits fp32 [T,E]; weights [E+B, I, H] gate/up and
  *   [E+B, H, I] down, all in one format; FP4 weights must be prepared.
- *   act_quant = 1: dynamic NVFP4 activations (NVFP4 weights only).
+ *   act_quant = 1: dynamic NVFP4 activations (NVFP4 weights only); each GEMM whose K
+ *   (H for gate/up, I for down) is a multiple of 256 then runs block-scaled as in
+ *   moe_grouped_gemm_nvfp4, the other one on f16-staged operands.
  *   apply_topk_in_fc1 = 1 applies the route weight in the activation (default);
  *   0 applies it in the combine (FlashInfer MoE-EP page, apply_topk_in_fc1).
  *   topk_ids_out/topk_w_out: optional [T,topk] copies of the routing.

@@ -35,7 +35,8 @@ WFMT = {"bf16": 0, "mxfp4": 1, "nvfp4": 2}
 EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_workspace_size",
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
-           "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc"]
+           "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc",
+           "moe_grouped_gemm_nvfp4"]
 
 
 class MoEError(RuntimeError):
@@ -88,6 +89,7 @@ _sig = {
     "moe_forward": (_I, [ctypes.POINTER(moe_forward_args_t), _P, _S, _P]),
     "moe_get_device_error": (_I, [_P, _P]),
     "moe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P]),
+    "moe_grouped_gemm_nvfp4": (_I, [_P, _P, _P, _I, ctypes.POINTER(moe_weight_t), _P, _P, _P, _S, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -221,6 +223,19 @@ def moe_grouped_gemm(a: torch.Tensor, w: Weight, cu_seqlens: torch.Tensor, out=N
         ws = torch.zeros(n, dtype=torch.uint8, device=a.device)
     _check(_lib.moe_grouped_gemm(_ptr(a), M, ctypes.byref(w.desc), _ptr(cu_seqlens), _ptr(out),
                                  _ptr(ws), ws.numel(), _stream(stream)), "moe_grouped_gemm")
+    return out
+
+
+def moe_grouped_gemm_nvfp4(a_codes: torch.Tensor, a_sb: torch.Tensor, a_s: torch.Tensor, w: Weight,
+                           cu_seqlens: torch.Tensor, out=None, ws=None, stream=None) -> torch.Tensor:
+    """Block-scaled grouped GEMM on NVFP4 activations (codes [M,K/2], e4m3 scales [M,K/16],
+    row scales [M]) and prepared NVFP4 weights; bf16 out [M,N]."""
+    M = a_codes.shape[0]
+    out = out if out is not None else torch.empty(M, w.N, dtype=torch.bfloat16, device=a_codes.device)
+    ws = ws if ws is not None else torch.zeros(256, dtype=torch.uint8, device=a_codes.device)
+    _check(_lib.moe_grouped_gemm_nvfp4(_ptr(a_codes), _ptr(a_sb), _ptr(a_s), M, ctypes.byref(w.desc),
+                                       _ptr(cu_seqlens), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_gemm_nvfp4")
     return out
 
 

@@ -62,8 +62,13 @@ const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? 
 // ----------------------------------------------------------------- forward workspace
 struct FwdWs {
     size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
-        xq_deq, act, act2, act2_scale, act_codes, act_sb, y, bytes;
+        xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, y, bytes;
 };
+
+// With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
+// tensor cores; its operand rows are records of K/2 code bytes followed by K/16 scales.
+inline bool nvf4_k(int act_quant, int K) { return act_quant && K % kNvf4StageK == 0; }
+inline int nvf4_rec_bytes(int K) { return K / 2 + K / 16; }
 
 FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
     FwdWs L{};
@@ -83,17 +88,22 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.perm_w = take(4 * NvS);
     L.inv = take(4 * NvS);
     L.perm_scratch = take(permute_ws_layout(T_max, topk, E, B).bytes);
-    L.xperm = take(2 * NvS * H);
+    const bool nat1 = nvf4_k(act_quant, H), nat2 = nvf4_k(act_quant, I);
+    const bool q1 = act_quant && !nat1, q2 = act_quant && !nat2;  // quantised, then staged as f16
+    L.xperm = take(nat1 ? 0 : 2 * NvS * H);
     L.tscale = take(fp4 ? 4 * NvS : 0);
-    L.xq_codes = take(act_quant ? (size_t)T_max * H / 2 : 0);
-    L.xq_sb = take(act_quant ? (size_t)T_max * H / 16 : 0);
+    L.xq_codes = take(q1 ? (size_t)T_max * H / 2 : 0);
+    L.xq_sb = take(q1 ? (size_t)T_max * H / 16 : 0);
     L.xq_s = take(act_quant ? 4 * (size_t)T_max : 0);
-    L.xq_deq = take(act_quant ? 2 * (size_t)T_max * H : 0);
+    L.xq_deq = take(q1 ? 2 * (size_t)T_max * H : 0);
+    L.xq_rec = take(nat1 ? (size_t)T_max * nvf4_rec_bytes(H) : 0);
+    L.xperm_rec = take(nat1 ? NvS * nvf4_rec_bytes(H) : 0);
     L.act = take((fp4 ? 4 : 2) * NvS * I);  // fp32 when a row pass follows
-    L.act2 = take(fp4 ? 2 * NvS * I : 0);
+    L.act2 = take(fp4 && !nat2 ? 2 * NvS * I : 0);
     L.act2_scale = take(fp4 ? 4 * NvS : 0);
-    L.act_codes = take(act_quant ? NvS * I / 2 : 0);
-    L.act_sb = take(act_quant ? NvS * I / 16 : 0);
+    L.act_codes = take(q2 ? NvS * I / 2 : 0);
+    L.act_sb = take(q2 ? NvS * I / 16 : 0);
+    L.act_rec = take(nat2 ? NvS * nvf4_rec_bytes(I) : 0);
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
     L.bytes = off;
     return L;
@@ -209,6 +219,44 @@ moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
     return cuda_status(launch_grouped_gemm(p, st, pdl));
 }
 
+moe_status_t moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sb, const float* a_s, int M_alloc,
+                                    const moe_weight_t* w, const int32_t* cu_seqlens, void* out, void* ws,
+                                    size_t ws_bytes, moe_stream_t stream) {
+    if (!w || M_alloc < 0 || w->G < 1 || w->N < 1 || w->K < 1) return MOE_ERR_INVALID_ARG;
+    if (w->G > 1024) return MOE_ERR_UNSUPPORTED;
+    if (w->fmt != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+    moe_status_t s = check_weight(*w, w->G, w->N, w->K);
+    if (s != MOE_OK) return s;
+    if (w->K % kNvf4StageK) return MOE_ERR_ALIGNMENT;
+    if (M_alloc == 0) return MOE_OK;
+    if (!a_codes || !a_sb || !a_s || !cu_seqlens || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sb) || !aligned16(out) || w->N % 8) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < kErrBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    GemmProblem p{};
+    p.x = a_codes;
+    p.x_stride = w->K / 2;
+    p.xsf = a_sb;
+    p.xsf_stride = w->K / 16;
+    p.nvf4 = true;
+    p.tscale = a_s;
+    p.M_alloc = M_alloc;
+    p.cu_seqlens = cu_seqlens;
+    p.G = w->G;
+    p.N = w->N;
+    p.K = w->K;
+    p.wfmt = w->fmt;
+    p.dual = false;
+    p.kdata0 = w->kdata;
+    p.kscale0 = w->kscale;
+    p.alpha0 = weight_alpha(*w);
+    p.out_scale = 1.0f;
+    p.out = out;
+    p.out_kind = OUT_BF16;
+    p.zero_pad = true;
+    p.err = reinterpret_cast<DevError*>(ws);
+    return cuda_status(launch_grouped_gemm(p, S(stream), false));
+}
+
 moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm_w, int M, int I,
                              moe_act_params_t act, void* out, moe_stream_t stream) {
     if (M < 0 || I < 0 || !act_ok(act)) return MOE_ERR_INVALID_ARG;
@@ -238,8 +286,8 @@ moe_status_t moe_quantize_nvfp4(const void* in, int in_is_f32, int R, int K, uin
     if ((size_t)R * K == 0) return MOE_OK;
     if (!in || !codes || !sb || !s) return MOE_ERR_INVALID_ARG;
     if (!aligned16(in) || !aligned16(codes) || (deq_f16 && !aligned16(deq_f16))) return MOE_ERR_ALIGNMENT;
-    return cuda_status(launch_quant_nvfp4(in, in_is_f32 != 0, R, K, codes, sb, s, static_cast<__half*>(deq_f16),
-                                          S(stream), false));
+    return cuda_status(launch_quant_nvfp4(in, in_is_f32 != 0, R, K, codes, K / 2, sb, K / 16, s,
+                                          static_cast<__half*>(deq_f16), S(stream), false));
 }
 
 size_t moe_prepared_weight_bytes(const moe_weight_t* w) {
@@ -310,6 +358,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     float* act2_scale = reinterpret_cast<float*>(w + L.act2_scale);
     float* y = reinterpret_cast<float*>(w + L.y);
     const int NvS = T * k;
+    const bool nat1 = nvf4_k(p->act_quant, H), nat2 = nvf4_k(p->act_quant, I);
     cudaStream_t st = S(stream);
     cudaError_t e;
     // Optional stage events (tracing). An event recorded between two kernels ends their
@@ -337,9 +386,18 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     // S2 gather (+ S2q)
     if (fmt == MOE_W_BF16) {
         e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
+    } else if (nat1) {
+        // quantise each token once into records, then gather the records into segment order
+        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.xq_rec);
+        const int rb = nvf4_rec_bytes(H);
+        e = launch_quant_nvfp4(p->x, false, T, H, rec, rb, rec + H / 2, rb, reinterpret_cast<float*>(w + L.xq_s),
+                               nullptr, st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_gather(1, rec, rb / 2, perm_token, NvS, w + L.xperm_rec, reinterpret_cast<float*>(w + L.xq_s),
+                          tscale, st, pdl());
     } else if (p->act_quant) {
-        e = launch_quant_nvfp4(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes),
-                               reinterpret_cast<uint8_t*>(w + L.xq_sb), reinterpret_cast<float*>(w + L.xq_s),
+        e = launch_quant_nvfp4(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes), H / 2,
+                               reinterpret_cast<uint8_t*>(w + L.xq_sb), H / 16, reinterpret_cast<float*>(w + L.xq_s),
                                reinterpret_cast<__half*>(w + L.xq_deq), st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(1, w + L.xq_deq, H, perm_token, NvS, xperm, reinterpret_cast<float*>(w + L.xq_s), tscale,
@@ -376,6 +434,14 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g1.situ_b = p->act.situ_beta;
     g1.out = act;
     g1.err = err;
+    if (nat1) {
+        const int rb = nvf4_rec_bytes(H);
+        g1.nvf4 = true;
+        g1.x = w + L.xperm_rec;
+        g1.x_stride = rb;
+        g1.xsf = w + L.xperm_rec + H / 2;
+        g1.xsf_stride = rb;
+    }
     // The down projection's operand: bf16 for BF16 weights; for FP4 weights f16 with a
     // per-row power-of-two scale (or a fixed one when SITU bounds |h| by alpha*beta),
     // or NVFP4-quantised rows when act_quant.
@@ -400,15 +466,19 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     }
     e = launch_grouped_gemm(g1, st, pdl());
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
+    const int rb2 = nvf4_rec_bytes(I);
     if (row_pass) {
-        if (p->act_quant) {
-            e = launch_quant_nvfp4(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.act_codes),
-                                   reinterpret_cast<uint8_t*>(w + L.act_sb), act2_scale, act2, st, pdl());
+        if (nat2) {
+            uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.act_rec);
+            e = launch_quant_nvfp4(act, true, NvS, I, rec, rb2, rec + I / 2, rb2, act2_scale, nullptr, st, pdl());
+        } else if (p->act_quant) {
+            e = launch_quant_nvfp4(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.act_codes), I / 2,
+                                   reinterpret_cast<uint8_t*>(w + L.act_sb), I / 16, act2_scale, act2, st, pdl());
         } else {
             e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, pdl());
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        fc2_x = act2;
+        fc2_x = nat2 ? static_cast<const void*>(w + L.act_rec) : act2;
         fc2_tscale = act2_scale;
     }
     if (!mark(4)) return MOE_ERR_CUDA;
@@ -431,6 +501,12 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.out = y;
     g2.out_kind = OUT_F32;
     g2.err = err;
+    if (nat2) {
+        g2.nvf4 = true;
+        g2.x_stride = rb2;
+        g2.xsf = w + L.act_rec + I / 2;
+        g2.xsf_stride = rb2;
+    }
     e = launch_grouped_gemm(g2, st, pdl());
     if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
     // S6: combine

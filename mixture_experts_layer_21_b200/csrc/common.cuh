@@ -178,6 +178,43 @@ __host__ __device__ constexpr uint32_t idesc_f16(int in_fmt, int M, int N) {
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- block-scaled FP4 MMA
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T with A, B packed e2m1 (two values per byte, the
+// even K index in the low nibble) in K-major 128-byte-swizzled smem, one fp8-e4m3
+// scale per 16 K values for every row of A and of B, read from tensor memory; fp32
+// accumulate; K = 64 per instruction (32 bytes of each row).
+MOE_DEV void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// Instruction descriptor of that MMA: A and B e2m1 (format 1 at bits [7,10) and
+// [10,13)), N >> 3 at [17,23), scale format 0 = ue4m3 at bit 23, M >> 4 at [24,29),
+// scale-factor ids 0, dense K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Copies 32 rows x 16 bytes of shared memory (rows 16 bytes apart) into tensor-memory
+// lanes 0..31, columns taddr..taddr+3 (bytes 4c..4c+3 of a row in column c), and the
+// same data into the other three lane quarters. Ordered with the MMAs this thread issues.
+MOE_DEV void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+// Shared-memory descriptor of a scale-factor block for that copy: no swizzle, 8-row
+// core matrices of 16-byte rows, consecutive 8-row groups 128 bytes apart.
+MOE_DEV uint64_t sf_block_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
 // 32 lanes x 32-bit, 16 consecutive columns per thread.
 MOE_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(

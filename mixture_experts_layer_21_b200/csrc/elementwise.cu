@@ -175,8 +175,8 @@ __device__ __forceinline__ void load16(const void* base, size_t off, float (&v)[
 
 template <bool IN_F32>
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict__ in, int R, int K,
-                                                          uint8_t* __restrict__ codes,
-                                                          uint8_t* __restrict__ sbo,
+                                                          uint8_t* __restrict__ codes, int cstride,
+                                                          uint8_t* __restrict__ sbo, int sstride,
                                                           float* __restrict__ so,
                                                           __half* __restrict__ deq) {
     pdl_wait();
@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
                     packed[i >> 2] |= (uint32_t)byte << (8 * (i & 3));
                 }
             }
-            *reinterpret_cast<uint2*>(codes + (size_t)r * (K / 2) + b * 8) = make_uint2(packed[0], packed[1]);
-            sbo[(size_t)r * nb + b] = sbc;
+            *reinterpret_cast<uint2*>(codes + (size_t)r * cstride + b * 8) = make_uint2(packed[0], packed[1]);
+            sbo[(size_t)r * sstride + b] = sbc;
             if (deq) {
                 const __half hsb = __float2half_rn(sbv);  // exact: e4m3 values are f16 values
                 const __half2 sb2 = __halves2half2(hsb, hsb);
@@ -235,12 +235,15 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
     pdl_launch();
 }
 
-cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes,
-                               uint8_t* sb, float* s, __half* deq, cudaStream_t st, bool pdl) {
+cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
+                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl) {
     if (R <= 0) return cudaSuccess;
     dim3 grid((R + 7) / 8), block(256);
-    if (in_f32) return launch_k(quant_nvfp4_kernel<true>, grid, block, 0, st, pdl, in, R, K, codes, sb, s, deq);
-    return launch_k(quant_nvfp4_kernel<false>, grid, block, 0, st, pdl, in, R, K, codes, sb, s, deq);
+    if (in_f32)
+        return launch_k(quant_nvfp4_kernel<true>, grid, block, 0, st, pdl, in, R, K, codes, codes_stride, sb,
+                        sb_stride, s, deq);
+    return launch_k(quant_nvfp4_kernel<false>, grid, block, 0, st, pdl, in, R, K, codes, codes_stride, sb, sb_stride,
+                    s, deq);
 }
 
 }  // namespace moe

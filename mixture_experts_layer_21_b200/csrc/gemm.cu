@@ -767,6 +767,241 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------ block-scaled NVFP4 kernel
+
+template <int BT, bool DUAL>
+struct Nvf4Cfg {
+    static constexpr int NB = DUAL ? 2 : 1;
+    static constexpr int A_BYTES = kNvf4TileBytes;              // codes image + 4 scale blocks
+    static constexpr int B_OFF = NB * A_BYTES;                  // token codes: BT rows x 128 bytes
+    static constexpr int B_BYTES = BT * kNvf4StageK / 2;
+    static constexpr int SFR_OFF = B_OFF + B_BYTES;             // token scales as loaded: BT x 16 bytes
+    static constexpr int SFR_BYTES = BT * 16;
+    static constexpr int SFB_OFF = SFR_OFF + (SFR_BYTES < 128 ? 128 : SFR_BYTES);  // 4 copy blocks
+    static constexpr int STAGE = round1024(SFB_OFF + 4 * 512);
+    static constexpr int STAGES = cmin(kMaxStages, kSmemBudget / STAGE);
+    // TMEM: two accumulator buffers, then the scale factors of one stage (four 4-column
+    // groups per matrix, then four for the tokens)
+    static constexpr int ACC_COLS = NB * BT;
+    static constexpr int SFA_COL = 2 * ACC_COLS;
+    static constexpr int SFB_COL = SFA_COL + NB * 16;
+    static constexpr int TMEM_COLS = tmem_cols_pow2(SFB_COL + 16);
+    static constexpr int THREADS = 6 * 32;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
+    static_assert(STAGES >= 2 && SMEM_BYTES <= kSmemLimit && SFB_COL + 16 <= 512, "NVFP4 GEMM config");
+    static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128, "token tile");
+    static_assert(B_OFF % 1024 == 0 && SFR_OFF % 128 == 0 && SFB_OFF % 128 == 0, "operand alignment");
+};
+
+// The token tile's scales arrive as BT rows of 16 bytes (one 32-bit word of four scales
+// per 64 K values j). The scale-factor copy wants, per j, a 512-byte block whose byte
+// 16*(r % 32) + 4*(r / 32) + i is scale i of row r. Lane l moves rows l, l+32, ...
+template <int BT>
+__device__ __forceinline__ void build_sfb_blocks(const uint8_t* raw, uint8_t* blk, int lane) {
+    constexpr int G32 = BT >= 32 ? BT / 32 : 1;
+    if (BT < 32 && lane >= BT) return;
+    uint32_t w[G32][4];
+#pragma unroll
+    for (int m1 = 0; m1 < G32; ++m1) {
+        const uint4 v = *reinterpret_cast<const uint4*>(raw + (32 * m1 + lane) * 16);
+        w[m1][0] = v.x;
+        w[m1][1] = v.y;
+        w[m1][2] = v.z;
+        w[m1][3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint8_t* d = blk + j * 512 + lane * 16;
+        if (G32 == 4) *reinterpret_cast<uint4*>(d) = make_uint4(w[0][j], w[1 % G32][j], w[2 % G32][j], w[3 % G32][j]);
+        else if (G32 == 2) *reinterpret_cast<uint2*>(d) = make_uint2(w[0][j], w[1 % G32][j]);
+        else *reinterpret_cast<uint32_t*>(d) = w[0][j];
+    }
+}
+
+// Weights in block-scaled tiles (bulk copies), tokens as packed e2m1 rows plus their
+// e4m3 scales (TMA); the tensor cores apply both scales. Warp roles as in the BF16 kernel;
+// the whole MMA warp rearranges the token scales before its lane 0 issues.
+template <int BT, bool DUAL, int OUT>
+__global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
+    grouped_gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sf,
+                             const GemmArgs a) {
+    using C = Nvf4Cfg<BT, DUAL>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
+    volatile int* abort_flag = &ctl->abort;
+    auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
+    auto opB = [&](int s) { return smem + s * C::STAGE + C::B_OFF; };
+    auto sfRaw = [&](int s) { return smem + s * C::STAGE + C::SFR_OFF; };
+    auto sfBlk = [&](int s) { return smem + s * C::STAGE + C::SFB_OFF; };
+    const int warp = warp_id(), lane = lane_id();
+    const int G = a.G, NT = a.NT, KB = a.KB;   // KB: 256-K stages per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 4);
+        }
+        mbar_init(&ctl->drain[0], 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_sf);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    if (warp == 0) build_segment_table<BT>(a, ctl, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch();
+    const uint32_t tmem_base = ctl->tmem_slot;
+    const int total = ctl->tpre[G];
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------- producer
+            int s = 0;
+            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            bool ok = true;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const size_t tile0 = ((size_t)g * NT + nt) * KB;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES + C::SFR_BYTES);
+                    const size_t off = (tile0 + kb) * (size_t)kNvf4TileBytes;
+                    bulk_load(opA(s, 0), a.ks0 + off, kNvf4TileBytes, &ctl->full[s]);
+                    if (DUAL) bulk_load(opA(s, 1), a.ks1 + off, kNvf4TileBytes, &ctl->full[s]);
+                    tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * (kNvf4StageK / 2), row0);
+                    tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], kb * (kNvf4StageK / 16), row0);
+                    issued_mask |= 1u << s;
+                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+                int never = 0;
+                for (int q = 0; q < C::STAGES; ++q)
+                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA warp: token scales rearranged by all lanes, issue by lane 0
+        constexpr uint32_t idesc = idesc_nvf4(kTileN, BT);
+        const uint32_t sfa = tmem_base + (uint32_t)C::SFA_COL;
+        const uint32_t sfb = tmem_base + (uint32_t)C::SFB_COL;
+        int s = 0, b = 0;
+        uint32_t ph = 0, bph = 0;
+        bool ok = true, issued = false;
+        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                build_sfb_blocks<BT>(sfRaw(s), sfBlk(s), lane);
+                fence_proxy_async_smem();  // the copies below read these bytes through the async proxy
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                        for (int m = 0; m < C::NB; ++m)
+                            tmem_cp_32x128b_x4(sfa + m * 16 + 4 * j,
+                                               sf_block_desc(smem_u32(opA(s, m)) + kNvf4CodeBytes + 512 * j));
+                        tmem_cp_32x128b_x4(sfb + 4 * j, sf_block_desc(smem_u32(sfBlk(s)) + 512 * j));
+                    }
+                    const uint32_t bb = smem_u32(opB(s));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t bdesc = sw128_kmajor_desc(bb + 32 * j);
+                        const uint32_t acc = (kb | j) != 0;
+#pragma unroll
+                        for (int m = 0; m < C::NB; ++m)
+                            mma_nvf4_ss(d0 + m * BT, sw128_kmajor_desc(smem_u32(opA(s, m)) + 32 * j), bdesc, idesc,
+                                        sfa + m * 16 + 4 * j, sfb + 4 * j, acc);
+                    }
+                    mma_commit(&ctl->empty[s]);
+                }
+                __syncwarp();
+                issued = true;
+                if (++s == C::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) mma_commit(&ctl->tfull[b]);
+            b ^= 1;
+            if (b == 0) bph ^= 1u;
+        }
+        if (!ok && lane == 0) {
+            report_error(a.err, MOE_ERR_TIMEOUT, 2);
+            ctl->abort = 1;
+            if (issued) {  // wait (bounded) for the copies and MMAs in flight before TMEM is released
+                int never = 0;
+                mma_commit(&ctl->drain[0]);
+                mbar_wait(&ctl->drain[0], 0, &never);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5)
+        const int q = warp & 3;
+        int b = 0;
+        uint32_t bph = 0;
+        for (int L = blockIdx.x; L < total; L += gridDim.x) {
+            int g, nt, row0, rows;
+            decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+                if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after();
+            epilogue_tile<BT, DUAL, OUT>(a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g,
+                                         nt, row0, rows, q, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            b ^= 1;
+            if (b == 0) bph ^= 1u;
+        }
+        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 64);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // ============================================================ host side
 
 namespace {
@@ -833,6 +1068,21 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over rows of bytes: [rows, cols] with rows `stride` bytes apart; box = box_cols
+// bytes x box_rows. Rows and columns past the ends read as zero.
+bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t stride,
+                 uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {stride};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // `done` belongs to the caller's instantiation: kernels of one signature share a
 // function-pointer type, so the flag cannot live in a template on that type.
 template <typename Kern>
@@ -874,6 +1124,57 @@ cudaError_t run_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMa
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
     return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, args);
+}
+
+template <int BT, bool DUAL, int OUT>
+cudaError_t run_nvf4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
+                     cudaStream_t st, bool pdl) {
+    using C = Nvf4Cfg<BT, DUAL>;
+    auto kern = grouped_gemm_nvf4_kernel<BT, DUAL, OUT>;
+    static int done[64] = {0};
+    cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, tsf,
+                    args);
+}
+
+template <int BT>
+cudaError_t dispatch_nvf4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
+                          cudaStream_t st, bool pdl) {
+    if constexpr (BT <= 64) {
+        if (p.dual) return run_nvf4<BT, true, OUT_F32>(p, args, tx, tsf, st, pdl);
+    }
+    if (p.dual) return cudaErrorInvalidValue;
+    if (p.out_kind == OUT_F32) return run_nvf4<BT, false, OUT_F32>(p, args, tx, tsf, st, pdl);
+    return run_nvf4<BT, false, OUT_BF16>(p, args, tx, tsf, st, pdl);
+}
+
+// The block-scaled NVFP4 GEMM. Token tile as for the other kernels, at most 64 for the
+// gate/up pair (two 2 x 64-column accumulator buffers plus the scale factors fill TMEM).
+cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool pdl) {
+    if (p.K % kNvf4StageK || !p.kscale0 || (p.dual && !p.kscale1) || !p.xsf) return cudaErrorInvalidValue;
+    if (p.dual && p.out_kind != OUT_F32) return cudaErrorInvalidValue;
+    a.KB = p.K / kNvf4StageK;
+    int bt = p.bt;
+    if (!bt) {
+        const char* env = getenv("MOE_TOKEN_TILE");
+        const int v = env ? atoi(env) : 0;
+        bt = (v == 16 || v == 32 || v == 64 || v == 128) ? v : choose_token_tile(p.M_alloc, p.G, false);
+    }
+    if (bt > 128) bt = 128;
+    if (p.dual && bt > 64) bt = 64;
+    CUtensorMap tx, tsf;
+    if (!make_map_u8(&tx, p.x, (uint64_t)p.K / 2, p.M_alloc, p.x_stride, kNvf4StageK / 2, bt,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_u8(&tsf, p.xsf, (uint64_t)p.K / 16, p.M_alloc, p.xsf_stride, kNvf4StageK / 16, bt,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    switch (bt) {
+        case 16: return dispatch_nvf4<16>(p, a, tx, tsf, st, pdl);
+        case 32: return dispatch_nvf4<32>(p, a, tx, tsf, st, pdl);
+        case 64: return dispatch_nvf4<64>(p, a, tx, tsf, st, pdl);
+        default: return dispatch_nvf4<128>(p, a, tx, tsf, st, pdl);
+    }
 }
 
 template <int BT, int WFMT>
@@ -939,6 +1240,7 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.ks1 = static_cast<const uint8_t*>(p.kscale1);
     a.zero_pad = p.zero_pad ? 1 : 0;
     a.err = p.err;
+    if (p.nvf4) return launch_nvf4(p, a, st, pdl);
     const bool wide_ok = p.wfmt == MOE_W_BF16 && !p.dual;
     int bt = p.bt;
     if (!bt) {

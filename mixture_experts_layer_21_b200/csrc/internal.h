@@ -55,8 +55,9 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, cons
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T,
                                int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
-cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes,
-                               uint8_t* sb, float* s, __half* deq, cudaStream_t st, bool pdl);
+// codes / sb rows are codes_stride / sb_stride bytes apart (K/2 and K/16 when dense).
+cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
+                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl);
 
 // ---------------------------------------------------------------- grouped GEMM
 // Output kinds of the GEMM epilogue.
@@ -90,6 +91,13 @@ struct GemmProblem {
     bool zero_pad;              // write zeros to rows [cu[G-1], M_alloc)
     int bt;                     // token tile (0 = choose)
     DevError* err;
+    // Block-scaled NVFP4 path (nvf4): x = packed e2m1 token rows (x_stride bytes apart),
+    // xsf = their e4m3 block scales (xsf_stride bytes apart), tscale = the row scales,
+    // kscale0/1 = the weights' block-scaled tiles. Needs K % kNvf4StageK == 0.
+    bool nvf4;
+    int x_stride;
+    const void* xsf;
+    int xsf_stride;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
 int choose_token_tile(long long NvS, int G, bool wide_ok);
@@ -101,6 +109,18 @@ inline int fp4_scale_bytes_per_row(int wfmt) { return wfmt == MOE_W_MXFP4 ? 2 : 
 // Prepared FP4 chunk (128 rows x 64 K): codes then scales, contiguous.
 inline int fp4_chunk_bytes(int wfmt) { return kTileN * 32 + kTileN * fp4_scale_bytes_per_row(wfmt); }
 constexpr int kFp4StageK = 128;  // K values per FP4 pipeline stage (two chunks)
+
+// Block-scaled NVFP4 tiles (weights used with NVFP4 activations): 128 weight rows x
+// 256 K values per tile, one pipeline stage. A tile is the 16384-byte image of the rows'
+// packed codes as the 128-byte swizzle lays them out in shared memory (row m at 128*m,
+// its 16-byte chunk c at chunk position c ^ (m % 8)), then four 512-byte scale blocks,
+// one per 64 K values j: byte 16*(m % 32) + 4*(m / 32) + i holds the e4m3 scale of
+// values [64j + 16i, 64j + 16i + 16) of row m (the order the scale-factor copy into
+// tensor memory reads).
+constexpr int kNvf4StageK = 256;
+constexpr int kNvf4CodeBytes = kTileN * kNvf4StageK / 2;   // 16384
+constexpr int kNvf4SfBytes = 4 * 512;
+constexpr int kNvf4TileBytes = kNvf4CodeBytes + kNvf4SfBytes;  // 18432
 
 // ---------------------------------------------------------------- device info
 int num_sms();

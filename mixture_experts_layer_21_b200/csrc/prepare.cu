@@ -7,7 +7,11 @@
 // each chunk of kFp4ChunkBytes(fmt) = 4096 + 128*S bytes holds
 //   128 rows x 32 bytes of packed e2m1 (even k in the low nibble), zero past N and K,
 //   then 128 rows x S scale bytes, S = 2 (MXFP4, two e8m0 per 64) or 4 (NVFP4, four e4m3),
-// so one stage is one contiguous copy per matrix. kdata and kscale both point at it.
+// so one stage is one contiguous copy per matrix. kdata points at it.
+//   kscale: NVFP4 with K % 256 == 0 -> the block-scaled tiles [g][nt][ks] of 128 rows x
+//           256 K values (kNvf4TileBytes each: the swizzled code image, then the scale
+//           blocks in tensor-memory copy order), read by the GEMM that takes NVFP4
+//           activations; otherwise the same address as kdata.
 //   kalpha: fp32 [G]. NVFP4: weight_scale_2 (1 if absent). MXFP4: 2^bias_g, where
 //           bias_g re-bases expert g's e8m0 exponents so its largest block scale is
 //           2^13; the GEMM stages e2m1 * 2^(e-127-bias) in f16, exact while the
@@ -24,9 +28,11 @@ constexpr int kMxTop = 140;   // re-biased exponent of the largest MXFP4 scale (
 constexpr int kMxFloor = 104; // smallest re-biased exponent staged exactly in f16
 
 struct PrepLayout {
-    int NT, KB, S;
+    int NT, KB, S, KS;
     size_t data_off, scale_off, alpha_off, scratch_off, bytes;
 };
+
+bool has_nvf4_tiles(const moe_weight_t* w) { return w->fmt == MOE_W_NVFP4 && w->K % kNvf4StageK == 0; }
 
 PrepLayout prep_layout(const moe_weight_t* w) {
     PrepLayout L{};
@@ -41,7 +47,8 @@ PrepLayout prep_layout(const moe_weight_t* w) {
         return o;
     };
     L.data_off = take(chunks * fp4_chunk_bytes(w->fmt));
-    L.scale_off = L.data_off;
+    L.KS = w->K / kNvf4StageK;
+    L.scale_off = has_nvf4_tiles(w) ? take((size_t)w->G * L.NT * L.KS * kNvf4TileBytes) : L.data_off;
     L.alpha_off = take(sizeof(float) * w->G);
     L.scratch_off = take(sizeof(int) * 2 * w->G + 16);
     L.bytes = off;
@@ -121,6 +128,38 @@ __global__ void __launch_bounds__(128) relayout_kernel(const uint8_t* __restrict
     (void)G;
 }
 
+// One block per block-scaled tile (g, nt, ks); thread m writes weight row nt*128 + m.
+// Rows past N are zero codes with zero scales.
+__global__ void __launch_bounds__(128) relayout_nvf4_kernel(const uint8_t* __restrict__ data,
+                                                            const uint8_t* __restrict__ scale, int N, int K,
+                                                            int NT, int KS, uint8_t* __restrict__ tiles) {
+    const size_t tile = blockIdx.x;
+    const int ks = (int)(tile % KS);
+    const int nt = (int)((tile / KS) % NT);
+    const size_t g = tile / ((size_t)KS * NT);
+    const int m = threadIdx.x;
+    const int n = nt * kTileN + m;
+    const bool live = n < N;
+    uint8_t* t = tiles + tile * (size_t)kNvf4TileBytes;
+    const uint4* src = reinterpret_cast<const uint4*>(data + (g * N + n) * (size_t)(K / 2) + (size_t)ks * 128);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = live ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(t + m * 128 + ((c ^ (m & 7)) << 4)) = v;
+    }
+    // 16 scales of this row for the tile's 256 values: four per 64-value block j
+    const uint8_t* srow = scale + (g * N + n) * (size_t)(K / 16) + (size_t)ks * 16;
+    uint8_t* sf = t + kNvf4CodeBytes;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t word = 0;
+        if (live)  // byte loads: the caller's scale plane need not be 4-byte aligned
+            word = (uint32_t)srow[4 * j] | (uint32_t)srow[4 * j + 1] << 8 | (uint32_t)srow[4 * j + 2] << 16 |
+                   (uint32_t)srow[4 * j + 3] << 24;
+        *reinterpret_cast<uint32_t*>(sf + j * 512 + 16 * (m & 31) + 4 * (m >> 5)) = word;
+    }
+}
+
 __global__ void alpha_kernel(const float* __restrict__ alpha, const int* __restrict__ bias, int fmt, int G,
                              float* __restrict__ kalpha) {
     for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < G; g += gridDim.x * blockDim.x) {
@@ -168,6 +207,13 @@ moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaS
         relayout_kernel<<<(unsigned)tiles, 128, 0, st>>>(static_cast<const uint8_t*>(w->data),
                                                           static_cast<const uint8_t*>(w->scale), w->fmt, w->G, w->N,
                                                           w->K, L.NT, L.KB, d_bias, kdata);
+    }
+    if (has_nvf4_tiles(w) && w->N > 0) {
+        const size_t ntiles = (size_t)w->G * L.NT * L.KS;
+        if (ntiles > 0)
+            relayout_nvf4_kernel<<<(unsigned)ntiles, 128, 0, st>>>(static_cast<const uint8_t*>(w->data),
+                                                                   static_cast<const uint8_t*>(w->scale), w->N,
+                                                                   w->K, L.NT, L.KS, kscale);
     }
     alpha_kernel<<<(w->G + 255) / 256, 256, 0, st>>>(w->alpha, d_bias, w->fmt, w->G, kalpha);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;

@@ -43,8 +43,10 @@ def test_workspace_sizes():
     a = L.moe_forward_workspace_size(64, 7168, 2048, 256, 16, 8, 0, 0)
     b = L.moe_forward_workspace_size(8192, 7168, 2048, 256, 16, 8, 0, 0)
     assert 0 < a < b
-    assert L.moe_forward_workspace_size(1024, 7168, 2048, 256, 0, 8, 2, 1) > \
-        L.moe_forward_workspace_size(1024, 7168, 2048, 256, 0, 8, 0, 0)
+    # NVFP4 activations: the fp32 gate/up and down outputs plus the quantised row records
+    nvs, H, I = 1024 * 8, 7168, 2048
+    assert L.moe_forward_workspace_size(1024, H, I, 256, 0, 8, 2, 1) >= \
+        4 * nvs * (H + I) + nvs * (H + I) * 9 // 16
     assert L.moe_forward_workspace_size(-1, 1, 1, 1, 0, 1, 0, 0) == 0
 
 
@@ -148,3 +150,26 @@ def test_grouped_gemm_and_misc_validation():
     assert L.moe_prepare_weights(ctypes.byref(wb), None, 0, None) == 0                   # BF16: no-op
     wm = _w(1, 4, 128, 48)
     assert L.moe_prepare_weights(ctypes.byref(wm), 16, 1 << 20, None) == ALIGN
+
+
+def test_grouped_gemm_nvfp4_validation():
+    f = L.moe_grouped_gemm_nvfp4
+    wn = _w(2, 4, 128, 512, kdata=16)
+    assert f(16, 16, 16, 0, ctypes.byref(wn), 16, 16, 16, 256, None) == 0            # no rows
+    assert f(16, 16, 16, 8, ctypes.byref(wn), 16, 16, 16, 100, None) == WS_SMALL
+    assert f(None, 16, 16, 8, ctypes.byref(wn), 16, 16, 16, 256, None) == INVALID
+    assert f(16, 8, 16, 8, ctypes.byref(wn), 16, 16, 16, 256, None) == ALIGN         # scales misaligned
+    assert f(16, 16, 16, 8, ctypes.byref(_w(2, 4, 128, 512)), 16, 16, 16, 256, None) == NOT_PREP
+    assert f(16, 16, 16, 8, ctypes.byref(_w(2, 4, 128, 384, kdata=16)), 16, 16, 16, 256, None) == ALIGN
+    assert f(16, 16, 16, 8, ctypes.byref(_w(1, 4, 128, 512, kdata=16)), 16, 16, 16, 256, None) == UNSUP
+    assert f(16, 16, 16, 8, ctypes.byref(_w(0, 4, 128, 512)), 16, 16, 16, 256, None) == UNSUP
+
+
+def test_nvfp4_prepared_bytes_hold_both_tile_layouts():
+    # K % 256 == 0: the f16-staging tiles plus the block-scaled tiles; otherwise the first only
+    G, N = 3, 200
+    one = L.moe_prepared_weight_bytes(ctypes.byref(_w(2, G, N, 272)))
+    both = L.moe_prepared_weight_bytes(ctypes.byref(_w(2, G, N, 512)))
+    NT = 2
+    assert one >= G * NT * 6 * (4096 + 512)
+    assert both >= G * NT * 8 * (4096 + 512) + G * NT * 2 * (16384 + 2048)

@@ -175,6 +175,38 @@ def test_grouped_gemm_fp4(lib, fmt, seg, N, K):
     check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what=fmt)
 
 
+def _nvfp4_rows(a):
+    """The oracle's NVFP4 quantisation of rows a (bf16 [M,K]): packed codes, e4m3 block
+    scales, fp32 row scales, and the exact values they stand for."""
+    codes, sb, s = O.nvfp4_quantize_rows(a.float().numpy())
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return (torch.from_numpy(packed), torch.from_numpy(sb), torch.from_numpy(s),
+            O.nvfp4_dequantize_rows(codes, sb, s))
+
+
+# K a multiple of 256 (one pipeline stage); ragged N, empty segments, padding rows, and
+# segments spanning one to three token tiles of every width
+NVF4_CASES = [([5, 40, 0, 130, 1], 256, 256, 0), ([3, 0, 130, 17], 320, 512, 3),
+              ([1, 2, 1, 3], 128, 1024, 0), ([77, 5], 208, 256, 9)]
+
+
+@pytest.mark.parametrize("seg,N,K,pad", NVF4_CASES)
+@pytest.mark.parametrize("bt", [16, 32, 64, 128])
+def test_grouped_gemm_nvfp4_block_scaled(lib, seg, N, K, pad, bt, monkeypatch):
+    monkeypatch.setenv("MOE_TOKEN_TILE", str(bt))
+    ws = _fp4_weightset("nvfp4", len(seg), N, K, seed=N + bt)
+    M = sum(seg) + pad
+    a, _, _ = W.gen_grouped_gemm_case(M, seg, 8, K, seed=K + bt)
+    codes, sb, s, deq = _nvfp4_rows(a)
+    cu = np.cumsum(seg).astype(np.int32)
+    w = lib.moe_prepare_weights(lib.Weight.from_host(ws))
+    out = lib.moe_grouped_gemm_nvfp4(to_dev(codes), to_dev(sb), to_dev(s), w, to_dev(torch.from_numpy(cu)),
+                                     out=torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    ref = O.grouped_gemm(deq, ws, cu, M_alloc=M)
+    check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what=f"nvf4 bt{bt}")
+
+
 # ------------------------------------------------------------------ S4 activation
 
 @pytest.mark.parametrize("act,sa,sb", [("silu", 1.0, 1.0), ("situ", 1.0, 1.0), ("situ", 0.7, 2.5)])
@@ -237,6 +269,10 @@ SMALL = {
     "mxfp4": W.MoEConfig("mxfp4", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4"),
     "mxfp4_silu": W.MoEConfig("mxfp4_silu", T=40, H=256, I=192, E=8, topk=2, wfmt="mxfp4"),
     "nvfp4": W.MoEConfig("nvfp4", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4", act_quant=1),
+    # gate/up K = 272 staged in f16, down K = 512 block-scaled
+    "nvfp4_mixed": W.MoEConfig("nvfp4_mixed", T=33, H=272, I=512, E=8, topk=4, wfmt="nvfp4", act_quant=1),
+    # neither K a multiple of 256: both staged in f16
+    "nvfp4_f16": W.MoEConfig("nvfp4_f16", T=40, H=272, I=304, E=8, topk=2, wfmt="nvfp4", act_quant=1),
 }
 
 
