@@ -34,6 +34,7 @@
 //   warps 6..13   (FP4 kernel) converters, two warps per TMEM lane quarter
 // Every wait is bounded; a timeout records MOE_ERR_TIMEOUT in the error word,
 // stops all roles, lets copies in flight land, frees TMEM and returns.
+#include <cmath>
 #include <mutex>
 
 #include "internal.h"
@@ -779,16 +780,16 @@ struct Nvf4Cfg {
     static constexpr int SFR_BYTES = BT * 16;
     static constexpr int SFB_OFF = SFR_OFF + (SFR_BYTES < 128 ? 128 : SFR_BYTES);  // 4 copy blocks
     static constexpr int STAGE = round1024(SFB_OFF + 4 * 512);
-    static constexpr int STAGES = cmin(kMaxStages, kSmemBudget / STAGE);
-    // TMEM: two accumulator buffers, then the scale factors of one stage (four 4-column
-    // groups per matrix, then four for the tokens)
+    // TMEM: two accumulator buffers, then one scale-factor slot per pipeline stage (four
+    // 4-column groups per matrix, then four for the tokens)
     static constexpr int ACC_COLS = NB * BT;
-    static constexpr int SFA_COL = 2 * ACC_COLS;
-    static constexpr int SFB_COL = SFA_COL + NB * 16;
-    static constexpr int TMEM_COLS = tmem_cols_pow2(SFB_COL + 16);
-    static constexpr int THREADS = 6 * 32;
+    static constexpr int SF_BASE = 2 * ACC_COLS;
+    static constexpr int SF_SLOT = NB * 16 + 16;
+    static constexpr int STAGES = cmin(cmin(kMaxStages, kSmemBudget / STAGE), (512 - SF_BASE) / SF_SLOT);
+    static constexpr int TMEM_COLS = tmem_cols_pow2(SF_BASE + STAGES * SF_SLOT);
+    static constexpr int THREADS = 7 * 32;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
-    static_assert(STAGES >= 2 && SMEM_BYTES <= kSmemLimit && SFB_COL + 16 <= 512, "NVFP4 GEMM config");
+    static_assert(STAGES >= 3 && SMEM_BYTES <= kSmemLimit && SF_BASE + STAGES * SF_SLOT <= 512, "NVFP4 GEMM config");
     static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128, "token tile");
     static_assert(B_OFF % 1024 == 0 && SFR_OFF % 128 == 0 && SFB_OFF % 128 == 0, "operand alignment");
 };
@@ -819,8 +820,10 @@ __device__ __forceinline__ void build_sfb_blocks(const uint8_t* raw, uint8_t* bl
 }
 
 // Weights in block-scaled tiles (bulk copies), tokens as packed e2m1 rows plus their
-// e4m3 scales (TMA); the tensor cores apply both scales. Warp roles as in the BF16 kernel;
-// the whole MMA warp rearranges the token scales before its lane 0 issues.
+// e4m3 scales (TMA); the tensor cores apply both scales. Warp roles: 0 producer, 1 MMA
+// issuer (one thread), 2..5 epilogue, 6 scale warp: it rearranges the token scales and
+// one of its threads copies the stage's scale factors into that stage's TMEM slot, so
+// the MMA thread issues nothing but MMAs.
 template <int BT, bool DUAL, int OUT>
 __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sf,
@@ -834,6 +837,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     auto opB = [&](int s) { return smem + s * C::STAGE + C::B_OFF; };
     auto sfRaw = [&](int s) { return smem + s * C::STAGE + C::SFR_OFF; };
     auto sfBlk = [&](int s) { return smem + s * C::STAGE + C::SFB_OFF; };
+    uint64_t* sf_full = ctl->raw_full;   // scale factors of stage s are in TMEM
     const int warp = warp_id(), lane = lane_id();
     const int G = a.G, NT = a.NT, KB = a.KB;   // KB: 256-K stages per tile
 
@@ -841,12 +845,14 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->empty[s], 1);
+            mbar_init(&sf_full[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
             mbar_init(&ctl->tempty[b], 4);
         }
         mbar_init(&ctl->drain[0], 1);
+        mbar_init(&ctl->drain[1], 1);
         ctl->abort = 0;
         fence_barrier_init();
     }
@@ -866,6 +872,8 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     pdl_launch();
     const uint32_t tmem_base = ctl->tmem_slot;
     const int total = ctl->tpre[G];
+    // scale-factor slot of stage s: matrix m's 64-K block j at + m*16 + 4j, tokens' at + NB*16 + 4j
+    auto sf_slot = [&](int s) { return tmem_base + (uint32_t)(C::SF_BASE + s * C::SF_SLOT); };
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer
@@ -904,39 +912,27 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA warp: token scales rearranged by all lanes, issue by lane 0
-        constexpr uint32_t idesc = idesc_nvf4(kTileN, BT);
-        const uint32_t sfa = tmem_base + (uint32_t)C::SFA_COL;
-        const uint32_t sfb = tmem_base + (uint32_t)C::SFB_COL;
-        int s = 0, b = 0;
-        uint32_t ph = 0, bph = 0;
-        bool ok = true, issued = false;
-        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
-            for (int kb = 0; kb < KB; ++kb) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+        if (lane == 0) {  // ---------------- MMA issuer
+            constexpr uint32_t idesc = idesc_nvf4(kTileN, BT);
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0;
+            bool ok = true, issued = false;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
-                build_sfb_blocks<BT>(sfRaw(s), sfBlk(s), lane);
-                fence_proxy_async_smem();  // the copies below read these bytes through the async proxy
-                __syncwarp();
-                if (lane == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                        for (int m = 0; m < C::NB; ++m)
-                            tmem_cp_32x128b_x4(sfa + m * 16 + 4 * j,
-                                               sf_block_desc(smem_u32(opA(s, m)) + kNvf4CodeBytes + 512 * j));
-                        tmem_cp_32x128b_x4(sfb + 4 * j, sf_block_desc(smem_u32(sfBlk(s)) + 512 * j));
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
+                for (int kb = 0; kb < KB; ++kb) {
+                    // operands landed (full) and their scale factors are in TMEM (sf_full)
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
                     const uint32_t bb = smem_u32(opB(s));
+                    const uint32_t sfs = sf_slot(s);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint64_t bdesc = sw128_kmajor_desc(bb + 32 * j);
@@ -944,9 +940,58 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
 #pragma unroll
                         for (int m = 0; m < C::NB; ++m)
                             mma_nvf4_ss(d0 + m * BT, sw128_kmajor_desc(smem_u32(opA(s, m)) + 32 * j), bdesc, idesc,
-                                        sfa + m * 16 + 4 * j, sfb + 4 * j, acc);
+                                        sfs + m * 16 + 4 * j, sfs + C::NB * 16 + 4 * j, acc);
                     }
+                    issued = true;
                     mma_commit(&ctl->empty[s]);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[b]);
+                b ^= 1;
+                if (b == 0) bph ^= 1u;
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 2);
+                ctl->abort = 1;
+                if (issued) {  // wait (bounded) for the MMAs in flight before TMEM is released
+                    int never = 0;
+                    mma_commit(&ctl->drain[0]);
+                    mbar_wait(&ctl->drain[0], 0, &never);
+                }
+            }
+        }
+    } else if (warp == 6) {
+        // ---------------- scale warp: token scales -> copy blocks (all lanes), then lane 0
+        // copies the weights' and the tokens' scale blocks into the stage's TMEM slot. The
+        // slot is free: the stage's previous MMAs completed before the producer refilled it.
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true, issued = false;
+        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                build_sfb_blocks<BT>(sfRaw(s), sfBlk(s), lane);
+                fence_proxy_async_smem();  // the copies read these bytes through the async proxy
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sfs = sf_slot(s);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                        for (int m = 0; m < C::NB; ++m)
+                            tmem_cp_32x128b_x4(sfs + m * 16 + 4 * j,
+                                               sf_block_desc(smem_u32(opA(s, m)) + kNvf4CodeBytes + 512 * j));
+                        tmem_cp_32x128b_x4(sfs + C::NB * 16 + 4 * j, sf_block_desc(smem_u32(sfBlk(s)) + 512 * j));
+                    }
+                    mma_commit(&sf_full[s]);
                 }
                 __syncwarp();
                 issued = true;
@@ -955,18 +1000,14 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                     ph ^= 1u;
                 }
             }
-            if (!ok) break;
-            if (lane == 0) mma_commit(&ctl->tfull[b]);
-            b ^= 1;
-            if (b == 0) bph ^= 1u;
         }
         if (!ok && lane == 0) {
-            report_error(a.err, MOE_ERR_TIMEOUT, 2);
+            report_error(a.err, MOE_ERR_TIMEOUT, 5);
             ctl->abort = 1;
-            if (issued) {  // wait (bounded) for the copies and MMAs in flight before TMEM is released
+            if (issued) {  // wait (bounded) for the copies in flight before TMEM is released
                 int never = 0;
-                mma_commit(&ctl->drain[0]);
-                mbar_wait(&ctl->drain[0], 0, &never);
+                mma_commit(&ctl->drain[1]);
+                mbar_wait(&ctl->drain[1], 0, &never);
             }
         }
     } else {
@@ -1149,7 +1190,17 @@ cudaError_t dispatch_nvf4(const GemmProblem& p, const GemmArgs& args, const CUte
     return run_nvf4<BT, false, OUT_BF16>(p, args, tx, tsf, st, pdl);
 }
 
-// The block-scaled NVFP4 GEMM. Token tile as for the other kernels, at most 64 for the
+// Token tile of the block-scaled GEMM. Its cost is one pipeline stage per (token tile,
+// weight tile, 256 K) whatever the tile's width, so the tile should hold a whole segment:
+// a width of at least mean + 2 sqrt(mean) covers nearly every segment once.
+int choose_token_tile_nvf4(long long NvS, int G) {
+    const long long segs = std::max<long long>(1, std::min<long long>(G, NvS));
+    const double avg = (double)NvS / (double)segs;
+    const double want = avg + 2.0 * std::sqrt(avg);
+    return want <= 16 ? 16 : want <= 32 ? 32 : want <= 64 ? 64 : 128;
+}
+
+// The block-scaled NVFP4 GEMM. Token tile as above, at most 64 for the
 // gate/up pair (two 2 x 64-column accumulator buffers plus the scale factors fill TMEM).
 cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool pdl) {
     if (p.K % kNvf4StageK || !p.kscale0 || (p.dual && !p.kscale1) || !p.xsf) return cudaErrorInvalidValue;
@@ -1159,7 +1210,7 @@ cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool
     if (!bt) {
         const char* env = getenv("MOE_TOKEN_TILE");
         const int v = env ? atoi(env) : 0;
-        bt = (v == 16 || v == 32 || v == 64 || v == 128) ? v : choose_token_tile(p.M_alloc, p.G, false);
+        bt = (v == 16 || v == 32 || v == 64 || v == 128) ? v : choose_token_tile_nvf4(p.M_alloc, p.G);
     }
     if (bt > 128) bt = 128;
     if (p.dual && bt > 64) bt = 64;
