@@ -62,7 +62,8 @@ const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? 
 // ----------------------------------------------------------------- forward workspace
 struct FwdWs {
     size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
-        xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, y, bytes;
+        xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, mx_xq, mx_xperm, mx_act, y,
+        bytes;
 };
 
 // With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
@@ -90,7 +91,7 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.perm_scratch = take(permute_ws_layout(T_max, topk, E, B).bytes);
     const bool nat1 = nvf4_k(act_quant, H), nat2 = nvf4_k(act_quant, I);
     const bool q1 = act_quant && !nat1, q2 = act_quant && !nat2;  // quantised, then staged as f16
-    L.xperm = take(nat1 ? 0 : 2 * NvS * H);
+    L.xperm = take(nat1 || wfmt == MOE_W_MXFP4 ? 0 : 2 * NvS * H);
     L.tscale = take(fp4 ? 4 * NvS : 0);
     L.xq_codes = take(q1 ? (size_t)T_max * H / 2 : 0);
     L.xq_sb = take(q1 ? (size_t)T_max * H / 16 : 0);
@@ -99,11 +100,15 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.xq_rec = take(nat1 ? (size_t)T_max * nvf4_rec_bytes(H) : 0);
     L.xperm_rec = take(nat1 ? NvS * nvf4_rec_bytes(H) : 0);
     L.act = take((fp4 ? 4 : 2) * NvS * I);  // fp32 when a row pass follows
-    L.act2 = take(fp4 && !nat2 ? 2 * NvS * I : 0);
+    L.act2 = take(fp4 && !nat2 && wfmt != MOE_W_MXFP4 ? 2 * NvS * I : 0);
     L.act2_scale = take(fp4 ? 4 * NvS : 0);
     L.act_codes = take(q2 ? NvS * I / 2 : 0);
     L.act_sb = take(q2 ? NvS * I / 16 : 0);
     L.act_rec = take(nat2 ? NvS * nvf4_rec_bytes(I) : 0);
+    const bool mx = wfmt == MOE_W_MXFP4;
+    L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H) : 0);
+    L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H) : 0);
+    L.mx_act = take(mx ? NvS * mx8_rec_bytes(I) : 0);
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
     L.bytes = off;
     return L;
@@ -171,7 +176,8 @@ moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, in
 size_t moe_grouped_gemm_workspace_size(int M_alloc, const moe_weight_t* w) {
     if (!w || M_alloc < 0) return 0;
     size_t b = kErrBytes;
-    if (w->fmt != MOE_W_BF16) b += up256(2 * (size_t)M_alloc * w->K) + up256(4 * (size_t)M_alloc);
+    if (w->fmt == MOE_W_MXFP4) b += up256((size_t)M_alloc * mx8_rec_bytes(w->K));
+    else if (w->fmt != MOE_W_BF16) b += up256(2 * (size_t)M_alloc * w->K) + up256(4 * (size_t)M_alloc);
     return b;
 }
 
@@ -205,6 +211,18 @@ moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
     if (w->fmt == MOE_W_BF16) {
         p.x = a;
         p.w0 = w->data;
+    } else if (w->fmt == MOE_W_MXFP4) {
+        // activations -> MXFP8 hi/lo records, then the block-scaled GEMM
+        uint8_t* rec = reinterpret_cast<uint8_t*>(wsb + kErrBytes);
+        const int rb = mx8_rec_bytes(w->K);
+        cudaError_t e = launch_quant_mx8(a, false, M_alloc, w->K, rec, rb, st, false);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        p.x = rec;
+        p.x_stride = rb;
+        p.mx8 = true;
+        p.kdata0 = w->kdata;
+        p.kscale0 = w->kscale;
+        pdl = true;
     } else {
         __half* a16 = reinterpret_cast<__half*>(wsb + kErrBytes);
         float* sc = reinterpret_cast<float*>(wsb + kErrBytes + up256(2 * (size_t)M_alloc * w->K));
@@ -386,6 +404,12 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     // S2 gather (+ S2q)
     if (fmt == MOE_W_BF16) {
         e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
+    } else if (fmt == MOE_W_MXFP4) {
+        // stage each token once as MXFP8 hi/lo records, then gather the records
+        const int rb = mx8_rec_bytes(H);
+        e = launch_quant_mx8(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.mx_xq), rb, st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_gather(0, w + L.mx_xq, rb / 2, perm_token, NvS, w + L.mx_xperm, nullptr, nullptr, st, pdl());
     } else if (nat1) {
         // quantise each token once into records, then gather the records into segment order
         uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.xq_rec);
@@ -434,6 +458,12 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g1.situ_b = p->act.situ_beta;
     g1.out = act;
     g1.err = err;
+    if (fmt == MOE_W_MXFP4) {
+        g1.mx8 = true;
+        g1.x = w + L.mx_xperm;
+        g1.x_stride = mx8_rec_bytes(H);
+        g1.tscale = nullptr;
+    }
     if (nat1) {
         const int rb = nvf4_rec_bytes(H);
         g1.nvf4 = true;
@@ -451,6 +481,9 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     bool row_pass = false;
     if (fmt == MOE_W_BF16) {
         g1.out_kind = OUT_BF16;
+    } else if (fmt == MOE_W_MXFP4) {
+        g1.out_kind = OUT_F32;
+        row_pass = true;
     } else if (situ && !p->act_quant) {
         // |h| <= alpha*beta*|route weight| <= alpha*beta: one fixed power of two keeps it below 2^15
         const double bound = (double)p->act.situ_alpha * p->act.situ_beta;
@@ -468,7 +501,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
     const int rb2 = nvf4_rec_bytes(I);
     if (row_pass) {
-        if (nat2) {
+        if (fmt == MOE_W_MXFP4) {
+            e = launch_quant_mx8(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.mx_act), mx8_rec_bytes(I), st,
+                                 pdl());
+        } else if (nat2) {
             uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.act_rec);
             e = launch_quant_nvfp4(act, true, NvS, I, rec, rb2, rec + I / 2, rb2, act2_scale, nullptr, st, pdl());
         } else if (p->act_quant) {
@@ -478,8 +514,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
             e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, pdl());
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        fc2_x = nat2 ? static_cast<const void*>(w + L.act_rec) : act2;
-        fc2_tscale = act2_scale;
+        fc2_x = fmt == MOE_W_MXFP4 ? static_cast<const void*>(w + L.mx_act)
+                : nat2                ? static_cast<const void*>(w + L.act_rec)
+                                      : act2;
+        fc2_tscale = fmt == MOE_W_MXFP4 ? nullptr : act2_scale;
     }
     if (!mark(4)) return MOE_ERR_CUDA;
     // S5: down grouped GEMM
@@ -501,6 +539,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.out = y;
     g2.out_kind = OUT_F32;
     g2.err = err;
+    if (fmt == MOE_W_MXFP4) {
+        g2.mx8 = true;
+        g2.x_stride = mx8_rec_bytes(I);
+    }
     if (nat2) {
         g2.nvf4 = true;
         g2.x_stride = rb2;

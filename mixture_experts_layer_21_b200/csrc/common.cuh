@@ -199,6 +199,27 @@ MOE_DEV void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T with A e2m1 held one value per byte in smem (the
+// 4-bit tensor map's 16-byte-aligned form), B e4m3, one e8m0 scale per 32 K values for
+// every row of A and of B; K = 32 per instruction. The scale of this instruction is byte
+// `id` of the 32-bit TMEM word at sfa/sfb; the id goes in the descriptor and in bits
+// 30-31 of both scale addresses.
+MOE_DEV void mma_mx8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// Its instruction descriptor: B scale id at [4,6), A e2m1 (5) at [7,10), B e4m3 (0) at
+// [10,13), N >> 3 at [17,23), scale format 1 = ue8m0 at bit 23, M >> 4 at [24,29),
+// A scale id at [29,31), dense K = 32.
+__host__ __device__ constexpr uint32_t idesc_mx8(int M, int N, uint32_t id) {
+    return (id << 4) | (5u << 7) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+           (id << 29);
+}
 // Copies 32 rows x 16 bytes of shared memory (rows 16 bytes apart) into tensor-memory
 // lanes 0..31, columns taddr..taddr+3 (bytes 4c..4c+3 of a row in column c), and the
 // same data into the other three lane quarters. Ordered with the MMAs this thread issues.

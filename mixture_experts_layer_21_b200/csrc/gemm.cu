@@ -76,7 +76,7 @@ struct GemmArgs {
 struct CtrlBlock {
     uint64_t full[kMaxStages], empty[kMaxStages];          // operand ring (smem or TMEM)
     uint64_t raw_full[kMaxStages], raw_empty[kMaxStages];  // raw ring (FP4)
-    uint64_t tfull[2], tempty[2], drain[4];
+    uint64_t tfull[2], tempty[2], drain[6];
     uint32_t tmem_slot;
     int abort;
     uint16_t lut[256];
@@ -1043,6 +1043,291 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------ MXFP4 x MXFP8 kernel
+
+template <int BT, bool DUAL>
+struct Mx8Cfg {
+    static constexpr int NB = DUAL ? 2 : 1;
+    // Narrow token tiles are issue-bound: the hi and lo terms then go to separate MMA
+    // threads with separate partial sums (added in the epilogue).
+    static constexpr int NPART = BT <= 32 ? 2 : 1;
+    static constexpr int NI = NB * NPART;                 // issuer i: matrix i % NB, term i / NB
+    static constexpr int A_BYTES = kTileN * kMx8StageK;   // 128 rows x 128 e2m1, a byte each in smem
+    static constexpr int A_TX = A_BYTES / 2;              // what the 4-bit load counts: the packed bytes
+    static constexpr int B_BYTES = BT * kMx8StageK;       // one e4m3 term
+    static constexpr int BH_OFF = NB * A_BYTES;
+    static constexpr int BL_OFF = BH_OFF + B_BYTES;
+    static constexpr int SFA_OFF = BL_OFF + B_BYTES;       // one 512-byte block per matrix
+    static constexpr int SFR_OFF = SFA_OFF + NB * 512;     // token scales as loaded: BT x 16 bytes
+    static constexpr int SFR_BYTES = BT * 16;
+    static constexpr int SFB_OFF = SFR_OFF + (SFR_BYTES < 128 ? 128 : SFR_BYTES);
+    static constexpr int STAGE = round1024(SFB_OFF + 512);
+    static constexpr int ACC_COLS = NB * NPART * BT;
+    static constexpr int SF_SLOT = 4 * NB + 4;
+    static constexpr int ACC_BUFS = 2 * ACC_COLS + 3 * SF_SLOT <= 512 ? 2 : 1;
+    static constexpr int SF_BASE = ACC_BUFS * ACC_COLS;
+    static constexpr int STAGES = cmin(cmin(kMaxStages, kSmemBudget / STAGE), (512 - SF_BASE) / SF_SLOT);
+    static constexpr int TMEM_COLS = tmem_cols_pow2(SF_BASE + STAGES * SF_SLOT);
+    static constexpr int EPI_WARP0 = 1 + NI;
+    static constexpr int SCALE_WARP = EPI_WARP0 + 4;
+    static constexpr int THREADS = (SCALE_WARP + 1) * 32;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
+    static_assert(STAGES >= 3 && SMEM_BYTES <= kSmemLimit && SF_BASE + STAGES * SF_SLOT <= 512, "MX GEMM config");
+    static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128, "token tile");
+    static_assert(BH_OFF % 1024 == 0 && BL_OFF % 1024 == 0 && SFR_OFF % 128 == 0 && SFB_OFF % 128 == 0,
+                  "operand alignment");
+};
+
+// The token tile's scales arrive as BT rows of 16 bytes covering 512 K values; word w of
+// a row holds the four scales of this stage's 128 values. The copy block wants byte
+// 16*(r % 32) + 4*(r / 32) + i = scale i of row r.
+template <int BT>
+__device__ __forceinline__ void build_sfb_block_mx8(const uint8_t* raw, uint8_t* blk, int w, int lane) {
+    if (BT < 32 && lane >= BT) return;
+    const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
+    uint8_t* d = blk + lane * 16;
+    if (BT <= 32) {
+        *reinterpret_cast<uint32_t*>(d) = rw[lane * 4 + w];
+    } else if (BT == 64) {
+        *reinterpret_cast<uint2*>(d) = make_uint2(rw[lane * 4 + w], rw[(lane + 32) * 4 + w]);
+    } else {
+        *reinterpret_cast<uint4*>(d) = make_uint4(rw[lane * 4 + w], rw[(lane + 32) * 4 + w],
+                                                  rw[(lane + 64) * 4 + w], rw[(lane + 96) * 4 + w]);
+    }
+}
+
+// MXFP4 weights (4-bit tensor map, expanded to a byte per value in smem, plus their
+// e8m0 scale blocks) against MXFP8 activations given as two e4m3 terms that share one
+// e8m0 scale per 32 values; the tensor cores apply both scales. Warp roles: 0 producer,
+// 1..NI MMA issuers, then 4 epilogue warps, then the scale warp (token scales into copy
+// blocks, scale-factor copies into the stage's TMEM slot).
+template <int BT, bool DUAL, int OUT>
+__global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
+    grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sf,
+                            const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
+                            const GemmArgs a, int Kp) {
+    using C = Mx8Cfg<BT, DUAL>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
+    volatile int* abort_flag = &ctl->abort;
+    auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
+    auto opB = [&](int s, int t) { return smem + s * C::STAGE + (t ? C::BL_OFF : C::BH_OFF); };
+    auto sfA = [&](int s, int m) { return smem + s * C::STAGE + C::SFA_OFF + m * 512; };
+    auto sfRaw = [&](int s) { return smem + s * C::STAGE + C::SFR_OFF; };
+    auto sfBlk = [&](int s) { return smem + s * C::STAGE + C::SFB_OFF; };
+    uint64_t* sf_full = ctl->raw_full;
+    const int warp = warp_id(), lane = lane_id();
+    const int G = a.G, NT = a.NT, KB = a.KB;   // KB: 128-K stages per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], C::NI);
+            mbar_init(&sf_full[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], C::NI);
+            mbar_init(&ctl->tempty[b], 4);
+        }
+        for (int i = 0; i < 6; ++i) mbar_init(&ctl->drain[i], 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_sf);
+        tma_prefetch_desc(&tm_w0);
+        if (DUAL) tma_prefetch_desc(&tm_w1);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    if (warp == 0) build_segment_table<BT>(a, ctl, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch();
+    const uint32_t tmem_base = ctl->tmem_slot;
+    const int total = ctl->tpre[G];
+    // scale-factor slot of stage s: matrix m's block at + 4m, the tokens' at + 4 NB
+    auto sf_slot = [&](int s) { return tmem_base + (uint32_t)(C::SF_BASE + s * C::SF_SLOT); };
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------- producer
+            int s = 0;
+            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            bool ok = true;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const size_t blk0 = ((size_t)g * NT + nt) * KB;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * (C::A_TX + 512) + 2 * C::B_BYTES + C::SFR_BYTES);
+                    tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g);
+                    bulk_load(sfA(s, 0), a.ks0 + (blk0 + kb) * 512, 512, &ctl->full[s]);
+                    if (DUAL) {
+                        tma_load_3d(opA(s, 1), &tm_w1, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g);
+                        bulk_load(sfA(s, 1), a.ks1 + (blk0 + kb) * 512, 512, &ctl->full[s]);
+                    }
+                    tma_load_2d(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0);
+                    tma_load_2d(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0);
+                    tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], (kb >> 2) * 16, row0);
+                    issued_mask |= 1u << s;
+                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+                int never = 0;
+                for (int q = 0; q < C::STAGES; ++q)
+                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
+            }
+        }
+    } else if (warp < C::EPI_WARP0) {
+        if (lane == 0) {  // ---------------- MMA issuers
+            const int i = warp - 1;
+            const int m = i % C::NB, p = i / C::NB;
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0;
+            bool ok = true, issued = false;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + (p * C::NB + m) * BT);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t aa = smem_u32(opA(s, m));
+                    const uint32_t sfa = sf_slot(s) + 4 * m, sfb = sf_slot(s) + 4 * C::NB;
+#pragma unroll
+                    for (int kk = 0; kk < kMx8StageK / 32; ++kk) {
+                        const uint64_t adesc = sw128_kmajor_desc(aa + 32 * kk);
+                        const uint32_t id = (uint32_t)kk, idb = id << 30;
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            if (C::NPART == 2 && t != p) continue;
+                            const uint32_t acc = (kb | kk | (C::NPART == 2 ? 0 : t)) != 0;
+                            mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, t)) + 32 * kk),
+                                       idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, acc);
+                        }
+                    }
+                    issued = true;
+                    mma_commit(&ctl->empty[s]);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&ctl->tfull[b]);
+                if (++b == C::ACC_BUFS) {
+                    b = 0;
+                    bph ^= 1u;
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 2);
+                ctl->abort = 1;
+                if (issued) {  // wait (bounded) for this issuer's MMAs before TMEM is released
+                    int never = 0;
+                    mma_commit(&ctl->drain[i]);
+                    mbar_wait(&ctl->drain[i], 0, &never);
+                }
+            }
+        }
+    } else if (warp == C::SCALE_WARP) {
+        // ---------------- scale warp (see the NVFP4 kernel); the slot of stage s is free once
+        // the producer refilled s, i.e. after the MMAs that read it completed
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true, issued = false;
+        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                build_sfb_block_mx8<BT>(sfRaw(s), sfBlk(s), kb & 3, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sfs = sf_slot(s);
+#pragma unroll
+                    for (int mm = 0; mm < C::NB; ++mm) tmem_cp_32x128b_x4(sfs + 4 * mm, sf_block_desc(smem_u32(sfA(s, mm))));
+                    tmem_cp_32x128b_x4(sfs + 4 * C::NB, sf_block_desc(smem_u32(sfBlk(s))));
+                    mma_commit(&sf_full[s]);
+                }
+                __syncwarp();
+                issued = true;
+                if (++s == C::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            report_error(a.err, MOE_ERR_TIMEOUT, 5);
+            ctl->abort = 1;
+            if (issued) {
+                int never = 0;
+                mma_commit(&ctl->drain[5]);
+                mbar_wait(&ctl->drain[5], 0, &never);
+            }
+        }
+    } else {
+        // ---------------- epilogue (4 warps)
+        const int q = warp & 3;
+        int b = 0;
+        uint32_t bph = 0;
+        for (int L = blockIdx.x; L < total; L += gridDim.x) {
+            int g, nt, row0, rows;
+            decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+                if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after();
+            epilogue_tile<BT, DUAL, OUT, C::NPART>(
+                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            if (++b == C::ACC_BUFS) {
+                b = 0;
+                bph ^= 1u;
+            }
+        }
+        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // ============================================================ host side
 
 namespace {
@@ -1121,6 +1406,21 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, 
     const cuuint32_t es[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over MXFP4 codes [G, N, Kp/2] (packed, 4-bit elements); box = 128 values x
+// 128 rows x 1, each 16 values landing in 16 bytes of shared memory (8 bytes of codes,
+// then 8 unused) with the 128-byte swizzle. Kp % 128 == 0; rows past N read as zero.
+bool make_map_w_u4(CUtensorMap* m, const void* ptr, uint64_t Kp, uint64_t N, uint64_t G) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc || Kp % 128) return false;
+    const cuuint64_t dims[3] = {Kp, N, G};
+    const cuuint64_t strides[2] = {Kp / 2, N * Kp / 2};
+    const cuuint32_t box[3] = {128, (cuuint32_t)kTileN, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1228,6 +1528,60 @@ cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool
     }
 }
 
+template <int BT, bool DUAL, int OUT>
+cudaError_t run_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
+                    const CUtensorMap& t0, const CUtensorMap& t1, int Kp, cudaStream_t st, bool pdl) {
+    using C = Mx8Cfg<BT, DUAL>;
+    auto kern = grouped_gemm_mx8_kernel<BT, DUAL, OUT>;
+    static int done[64] = {0};
+    cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, tsf, t0,
+                    t1, args, Kp);
+}
+
+template <int BT>
+cudaError_t dispatch_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
+                         const CUtensorMap& t0, const CUtensorMap& t1, int Kp, cudaStream_t st, bool pdl) {
+    if (p.dual) {
+        if (p.out_kind != OUT_F32) return cudaErrorInvalidValue;
+        return run_mx8<BT, true, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    }
+    if (p.out_kind == OUT_F32) return run_mx8<BT, false, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    return run_mx8<BT, false, OUT_BF16>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+}
+
+// The MXFP4 x MXFP8 GEMM; token tile as for the NVFP4 one.
+cudaError_t launch_mx8(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool pdl) {
+    if (!p.kdata0 || !p.kscale0 || (p.dual && (!p.kdata1 || !p.kscale1))) return cudaErrorInvalidValue;
+    const int Kp = mx8_kpad(p.K);
+    a.KB = Kp / kMx8StageK;
+    int bt = p.bt;
+    if (!bt) {
+        const char* env = getenv("MOE_TOKEN_TILE");
+        const int v = env ? atoi(env) : 0;
+        bt = (v == 16 || v == 32 || v == 64 || v == 128) ? v : choose_token_tile_nvf4(p.M_alloc, p.G);
+    }
+    if (bt > 128) bt = 128;
+    const uint8_t* rec = static_cast<const uint8_t*>(p.x);
+    CUtensorMap tx, tsf, t0, t1;
+    memset(&t1, 0, sizeof(t1));
+    if (!make_map_u8(&tx, rec, 2 * (uint64_t)Kp, p.M_alloc, p.x_stride, kMx8StageK, bt, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_u8(&tsf, rec + 2 * (size_t)Kp, mx8_scale_bytes(p.K), p.M_alloc, p.x_stride, 16, bt,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_w_u4(&t0, p.kdata0, Kp, p.N, p.G) || (p.dual && !make_map_w_u4(&t1, p.kdata1, Kp, p.N, p.G)))
+        return cudaErrorInvalidValue;
+    if (!p.dual) t1 = t0;
+    a.ks0 = static_cast<const uint8_t*>(p.kscale0);
+    a.ks1 = static_cast<const uint8_t*>(p.kscale1);
+    switch (bt) {
+        case 16: return dispatch_mx8<16>(p, a, tx, tsf, t0, t1, Kp, st, pdl);
+        case 32: return dispatch_mx8<32>(p, a, tx, tsf, t0, t1, Kp, st, pdl);
+        case 64: return dispatch_mx8<64>(p, a, tx, tsf, t0, t1, Kp, st, pdl);
+        default: return dispatch_mx8<128>(p, a, tx, tsf, t0, t1, Kp, st, pdl);
+    }
+}
+
 template <int BT, int WFMT>
 cudaError_t dispatch_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st,
                          bool pdl) {
@@ -1242,7 +1596,6 @@ cudaError_t dispatch_fp4(const GemmProblem& p, const GemmArgs& args, const CUten
 template <int BT>
 cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx,
                         const CUtensorMap& t0, const CUtensorMap& t1, cudaStream_t st, bool pdl) {
-    if (p.wfmt == MOE_W_MXFP4) return dispatch_fp4<BT, MOE_W_MXFP4>(p, args, tx, st, pdl);
     if (p.wfmt == MOE_W_NVFP4) return dispatch_fp4<BT, MOE_W_NVFP4>(p, args, tx, st, pdl);
     if (p.dual) return run_bf16<BT, true, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
     if (p.out_kind == OUT_F32) return run_bf16<BT, false, OUT_F32>(p, args, tx, t0, t1, st, pdl);
@@ -1292,6 +1645,7 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.zero_pad = p.zero_pad ? 1 : 0;
     a.err = p.err;
     if (p.nvf4) return launch_nvf4(p, a, st, pdl);
+    if (p.wfmt == MOE_W_MXFP4) return p.mx8 ? launch_mx8(p, a, st, pdl) : cudaErrorInvalidValue;
     const bool wide_ok = p.wfmt == MOE_W_BF16 && !p.dual;
     int bt = p.bt;
     if (!bt) {

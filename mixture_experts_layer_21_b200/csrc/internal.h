@@ -55,6 +55,10 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, cons
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T,
                                int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
+// Rows [R, K] (bf16 or fp32, K % 32 == 0) -> MXFP8 hi/lo records of mx8_rec_bytes(K)
+// bytes, rec_stride bytes apart.
+cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, uint8_t* rec, int rec_stride,
+                             cudaStream_t st, bool pdl);
 // codes / sb rows are codes_stride / sb_stride bytes apart (K/2 and K/16 when dense).
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
                                uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl);
@@ -98,6 +102,9 @@ struct GemmProblem {
     int x_stride;
     const void* xsf;
     int xsf_stride;
+    // MXFP4 weights (mx8): x = MXFP8 hi/lo records (x_stride bytes apart, mx8_rec_bytes(K)
+    // each), kdata0/1 = the padded codes, kscale0/1 = the scale blocks.
+    bool mx8;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
 int choose_token_tile(long long NvS, int G, bool wide_ok);
@@ -121,6 +128,17 @@ constexpr int kNvf4StageK = 256;
 constexpr int kNvf4CodeBytes = kTileN * kNvf4StageK / 2;   // 16384
 constexpr int kNvf4SfBytes = 4 * 512;
 constexpr int kNvf4TileBytes = kNvf4CodeBytes + kNvf4SfBytes;  // 18432
+
+// MXFP4 weights for the block-scaled MXFP4 x MXFP8 GEMM: kdata = packed e2m1 codes
+// [G, N, Kp/2] with K zero-padded to Kp = a multiple of 128 (what the 4-bit tensor map
+// needs), kscale = one 512-byte scale block per (g, 128-row block nt, 128-K block kb),
+// byte 16*(m % 32) + 4*(m / 32) + i = the e8m0 scale of values [128kb + 32i, +32) of
+// row m. Activations are records of Kp "hi" e4m3 codes, Kp "lo" e4m3 codes and Kp/32
+// e8m0 block scales padded to 16 bytes: value = (hi + lo) * 2^(scale - 127).
+constexpr int kMx8StageK = 128;
+inline int mx8_kpad(int K) { return (K + kMx8StageK - 1) / kMx8StageK * kMx8StageK; }
+inline int mx8_scale_bytes(int K) { return (mx8_kpad(K) / 32 + 15) / 16 * 16; }
+inline int mx8_rec_bytes(int K) { return 2 * mx8_kpad(K) + mx8_scale_bytes(K); }
 
 // ---------------------------------------------------------------- device info
 int num_sms();

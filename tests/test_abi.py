@@ -51,8 +51,9 @@ def test_workspace_sizes():
 
 
 def test_prepared_bytes():
-    w = m.moe_weight_t(1, 4, 300, 96)         # MXFP4, G=4, N=300 (3 row tiles), K=96 (2 K tiles)
-    assert L.moe_prepared_weight_bytes(ctypes.byref(w)) >= 4 * 3 * 2 * (128 * 32 + 128 * 2)
+    w = m.moe_weight_t(1, 4, 300, 96)         # MXFP4, G=4, N=300 (3 row tiles), K=96 -> padded 128
+    # codes with K padded to 128, then one 512-byte scale block per (g, row tile, 128 K)
+    assert L.moe_prepared_weight_bytes(ctypes.byref(w)) >= 4 * 300 * 64 + 4 * 3 * 1 * 512
     w.fmt = 0
     assert L.moe_prepared_weight_bytes(ctypes.byref(w)) == 0
 
