@@ -140,29 +140,31 @@ __device__ __forceinline__ void build_segment_table(const GemmArgs& a, CtrlBlock
 }
 
 // Epilogue of one tile for the warp owning TMEM lanes [32q, 32q+32). The accumulator
-// buffer at column tb holds NPART partial sums per matrix (one per MMA-issuing thread):
-// with two matrices, partial j of gate at tb + 2j*BT and of up at tb + (2j+1)*BT; with
-// one, partial j at tb + j*BT.
-template <int BT, bool DUAL, int OUT, int NPART = 1>
+// buffer at column tb holds NPART partial sums per matrix. Partial j of matrix m sits at
+// tb + (j*NB + m)*BT (partials of different issuers, PM = false), or at
+// tb + (m*NPART + j)*BT (PM = true: one MMA wrote a matrix's partials side by side).
+// With EW warps per lane quarter, warp h of a quarter takes the 16-token chunks h, h+EW, ...
+template <int BT, bool DUAL, int OUT, int NPART = 1, bool PM = false, int EW = 1>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, int g, int nt, int row0, int rows,
-                                              int q, int lane) {
+                                              int q, int lane, int h = 0) {
     const int n = nt * kTileN + q * 32 + lane;
     const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
     const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
     const float inv_sa = 1.0f / a.sa, inv_sb = 1.0f / a.sb;
-    constexpr int STRIDE = DUAL ? 2 * BT : BT;   // column distance between partials of one matrix
+    constexpr int NB = DUAL ? 2 : 1;
+    auto col = [](int m, int j) { return (PM ? m * NPART + j : j * NB + m) * BT; };
 #pragma unroll 1
-    for (int c0 = 0; c0 < BT; c0 += 16) {
+    for (int c0 = 16 * h; c0 < BT; c0 += 16 * EW) {
         if (c0 >= rows) break;
         uint32_t r0[16], r1[16];
-        tmem_ld16(tb + c0, r0);
-        if (DUAL) tmem_ld16(tb + BT + c0, r1);
+        tmem_ld16(tb + col(0, 0) + c0, r0);
+        if (DUAL) tmem_ld16(tb + col(1, 0) + c0, r1);
         tmem_ld_wait();
 #pragma unroll
         for (int pj = 1; pj < NPART; ++pj) {
             uint32_t p0[16], p1[16];
-            tmem_ld16(tb + pj * STRIDE + c0, p0);
-            if (DUAL) tmem_ld16(tb + pj * STRIDE + BT + c0, p1);
+            tmem_ld16(tb + col(0, pj) + c0, p0);
+            if (DUAL) tmem_ld16(tb + col(1, pj) + c0, p1);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -1048,10 +1050,14 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
 template <int BT, bool DUAL>
 struct Mx8Cfg {
     static constexpr int NB = DUAL ? 2 : 1;
-    // Narrow token tiles are issue-bound: the hi and lo terms then go to separate MMA
-    // threads with separate partial sums (added in the epilogue).
-    static constexpr int NPART = BT <= 32 ? 2 : 1;
-    static constexpr int NI = NB * NPART;                 // issuer i: matrix i % NB, term i / NB
+    // The hi and lo token rows sit one after the other in shared memory, so while the
+    // accumulators fit, one MMA of N = 2*BT covers both terms (MERGE): half the MMAs, and
+    // the weight tile is read once for both. Its two column halves are partial sums the
+    // epilogue adds. Otherwise (two 128-token tiles) each term is its own MMA.
+    static constexpr bool MERGE = NB * 2 * BT <= 256;
+    static constexpr int NPART = MERGE ? 2 : 1;
+    static constexpr int NI = NB;                          // MMA issuer i: matrix i
+    static constexpr int N_MMA = MERGE ? 2 * BT : BT;
     static constexpr int A_BYTES = kTileN * kMx8StageK;   // 128 rows x 128 e2m1, a byte each in smem
     static constexpr int A_TX = A_BYTES / 2;              // what the 4-bit load counts: the packed bytes
     static constexpr int B_BYTES = BT * kMx8StageK;       // one e4m3 term
@@ -1063,13 +1069,17 @@ struct Mx8Cfg {
     static constexpr int SFB_OFF = SFR_OFF + (SFR_BYTES < 128 ? 128 : SFR_BYTES);
     static constexpr int STAGE = round1024(SFB_OFF + 512);
     static constexpr int ACC_COLS = NB * NPART * BT;
-    static constexpr int SF_SLOT = 4 * NB + 4;
+    static constexpr int SFB_COLS = N_MMA > 128 ? 8 : 4;  // token scales: 4 columns per 128 MMA rows
+    static constexpr int SF_SLOT = 4 * NB + SFB_COLS;
     static constexpr int ACC_BUFS = 2 * ACC_COLS + 3 * SF_SLOT <= 512 ? 2 : 1;
     static constexpr int SF_BASE = ACC_BUFS * ACC_COLS;
     static constexpr int STAGES = cmin(cmin(kMaxStages, kSmemBudget / STAGE), (512 - SF_BASE) / SF_SLOT);
     static constexpr int TMEM_COLS = tmem_cols_pow2(SF_BASE + STAGES * SF_SLOT);
+    // Two epilogue warps per TMEM lane quarter: with one accumulator buffer the MMAs wait
+    // for the epilogue, and one warp per quarter takes about as long as the main loop.
+    static constexpr int EW = 2;
     static constexpr int EPI_WARP0 = 1 + NI;
-    static constexpr int SCALE_WARP = EPI_WARP0 + 4;
+    static constexpr int SCALE_WARP = EPI_WARP0 + 4 * EW;
     static constexpr int THREADS = (SCALE_WARP + 1) * 32;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
     static_assert(STAGES >= 3 && SMEM_BYTES <= kSmemLimit && SF_BASE + STAGES * SF_SLOT <= 512, "MX GEMM config");
@@ -1080,19 +1090,20 @@ struct Mx8Cfg {
 
 // The token tile's scales arrive as BT rows of 16 bytes covering 512 K values; word w of
 // a row holds the four scales of this stage's 128 values. The copy block wants byte
-// 16*(r % 32) + 4*(r / 32) + i = scale i of row r.
-template <int BT>
+// 16*(r % 32) + 4*(r / 32) + i = scale i of MMA row r, and MMA row r is token r % BT
+// (rows [BT, 2BT) are the lo terms of the same tokens when the terms are merged).
+template <int BT, bool MERGE>
 __device__ __forceinline__ void build_sfb_block_mx8(const uint8_t* raw, uint8_t* blk, int w, int lane) {
-    if (BT < 32 && lane >= BT) return;
+    constexpr int R = MERGE ? (2 * BT < 128 ? 2 * BT : 128) : BT;  // rows one copy block covers
     const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
+    auto word = [&](int r) { return rw[(r % BT) * 4 + w]; };
     uint8_t* d = blk + lane * 16;
-    if (BT <= 32) {
-        *reinterpret_cast<uint32_t*>(d) = rw[lane * 4 + w];
-    } else if (BT == 64) {
-        *reinterpret_cast<uint2*>(d) = make_uint2(rw[lane * 4 + w], rw[(lane + 32) * 4 + w]);
+    if (R <= 32) {
+        if (lane < R) *reinterpret_cast<uint32_t*>(d) = word(lane);
+    } else if (R == 64) {
+        *reinterpret_cast<uint2*>(d) = make_uint2(word(lane), word(lane + 32));
     } else {
-        *reinterpret_cast<uint4*>(d) = make_uint4(rw[lane * 4 + w], rw[(lane + 32) * 4 + w],
-                                                  rw[(lane + 64) * 4 + w], rw[(lane + 96) * 4 + w]);
+        *reinterpret_cast<uint4*>(d) = make_uint4(word(lane), word(lane + 32), word(lane + 64), word(lane + 96));
     }
 }
 
@@ -1128,7 +1139,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], C::NI);
-            mbar_init(&ctl->tempty[b], 4);
+            mbar_init(&ctl->tempty[b], 4 * C::EW);
         }
         for (int i = 0; i < 6; ++i) mbar_init(&ctl->drain[i], 1);
         ctl->abort = 0;
@@ -1198,7 +1209,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
     } else if (warp < C::EPI_WARP0) {
         if (lane == 0) {  // ---------------- MMA issuers
             const int i = warp - 1;
-            const int m = i % C::NB, p = i / C::NB;
+            const int m = i;
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
             bool ok = true, issued = false;
@@ -1208,7 +1219,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + (p * C::NB + m) * BT);
+                const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + m * C::NPART * BT);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
                         ok = false;
@@ -1221,12 +1232,14 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     for (int kk = 0; kk < kMx8StageK / 32; ++kk) {
                         const uint64_t adesc = sw128_kmajor_desc(aa + 32 * kk);
                         const uint32_t id = (uint32_t)kk, idb = id << 30;
+                        if (C::MERGE) {  // hi and lo rows in one MMA: partials at d and d + BT
+                            mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, 0)) + 32 * kk),
+                                       idesc_mx8(kTileN, C::N_MMA, id), sfa | idb, sfb | idb, (kb | kk) != 0);
+                        } else {
 #pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            if (C::NPART == 2 && t != p) continue;
-                            const uint32_t acc = (kb | kk | (C::NPART == 2 ? 0 : t)) != 0;
-                            mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, t)) + 32 * kk),
-                                       idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, acc);
+                            for (int t = 0; t < 2; ++t)
+                                mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, t)) + 32 * kk),
+                                           idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, (kb | kk | t) != 0);
                         }
                     }
                     issued = true;
@@ -1265,7 +1278,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     ok = false;
                     break;
                 }
-                build_sfb_block_mx8<BT>(sfRaw(s), sfBlk(s), kb & 3, lane);
+                build_sfb_block_mx8<BT, C::MERGE>(sfRaw(s), sfBlk(s), kb & 3, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -1273,7 +1286,10 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     const uint32_t sfs = sf_slot(s);
 #pragma unroll
                     for (int mm = 0; mm < C::NB; ++mm) tmem_cp_32x128b_x4(sfs + 4 * mm, sf_block_desc(smem_u32(sfA(s, mm))));
-                    tmem_cp_32x128b_x4(sfs + 4 * C::NB, sf_block_desc(smem_u32(sfBlk(s))));
+                    // MMA rows [128, 256) (the lo terms of a 128-token tile) repeat rows [0, 128)
+#pragma unroll
+                    for (int h = 0; h < C::SFB_COLS / 4; ++h)
+                        tmem_cp_32x128b_x4(sfs + 4 * C::NB + 4 * h, sf_block_desc(smem_u32(sfBlk(s))));
                     mma_commit(&sf_full[s]);
                 }
                 __syncwarp();
@@ -1294,8 +1310,8 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
             }
         }
     } else {
-        // ---------------- epilogue (4 warps)
-        const int q = warp & 3;
+        // ---------------- epilogue (4 * EW warps)
+        const int q = warp & 3, h = (warp - C::EPI_WARP0) >> 2;
         int b = 0;
         uint32_t bph = 0;
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -1307,8 +1323,9 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT, C::NPART>(
-                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane);
+            epilogue_tile<BT, DUAL, OUT, C::NPART, true, C::EW>(
+                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane,
+                h);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[b]);
@@ -1317,7 +1334,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                 bph ^= 1u;
             }
         }
-        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
+        if (a.zero_pad && OUT == OUT_BF16 && h == 0) zero_padding_rows(a, ctl, threadIdx.x - 32 * C::EPI_WARP0);
     }
 
     tc_fence_before();
