@@ -1055,8 +1055,12 @@ struct Mx8Cfg {
     // the weight tile is read once for both. Its two column halves are partial sums the
     // epilogue adds. Otherwise (two 128-token tiles) each term is its own MMA.
     static constexpr bool MERGE = NB * 2 * BT <= 256;
-    static constexpr int NPART = MERGE ? 2 : 1;
-    static constexpr int NI = NB;                          // MMA issuer i: matrix i
+    // A thread issues a block-scaled MMA about every 145 cycles, so narrow tiles split each
+    // stage's four K steps between two issuers with their own partial sums where TMEM allows.
+    static constexpr int KSPLIT = (MERGE && 2 * NB * 4 * BT <= 256) ? 2 : 1;
+    static constexpr int TERMS = MERGE ? 2 : 1;            // partials one MMA writes side by side
+    static constexpr int NPART = TERMS * KSPLIT;
+    static constexpr int NI = NB * KSPLIT;                 // issuer i: matrix i % NB, K half i / NB
     static constexpr int N_MMA = MERGE ? 2 * BT : BT;
     static constexpr int A_BYTES = kTileN * kMx8StageK;   // 128 rows x 128 e2m1, a byte each in smem
     static constexpr int A_TX = A_BYTES / 2;              // what the 4-bit load counts: the packed bytes
@@ -1209,7 +1213,8 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
     } else if (warp < C::EPI_WARP0) {
         if (lane == 0) {  // ---------------- MMA issuers
             const int i = warp - 1;
-            const int m = i;
+            const int m = i % C::NB, kh = i / C::NB;
+            constexpr int KPI = (kMx8StageK / 32) / C::KSPLIT;  // K steps per issuer and stage
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
             bool ok = true, issued = false;
@@ -1219,7 +1224,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + m * C::NPART * BT);
+                const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + (m * C::NPART + kh * C::TERMS) * BT);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
                         ok = false;
@@ -1229,17 +1234,18 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                     const uint32_t aa = smem_u32(opA(s, m));
                     const uint32_t sfa = sf_slot(s) + 4 * m, sfb = sf_slot(s) + 4 * C::NB;
 #pragma unroll
-                    for (int kk = 0; kk < kMx8StageK / 32; ++kk) {
+                    for (int j = 0; j < KPI; ++j) {
+                        const int kk = kh * KPI + j;
                         const uint64_t adesc = sw128_kmajor_desc(aa + 32 * kk);
                         const uint32_t id = (uint32_t)kk, idb = id << 30;
                         if (C::MERGE) {  // hi and lo rows in one MMA: partials at d and d + BT
                             mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, 0)) + 32 * kk),
-                                       idesc_mx8(kTileN, C::N_MMA, id), sfa | idb, sfb | idb, (kb | kk) != 0);
+                                       idesc_mx8(kTileN, C::N_MMA, id), sfa | idb, sfb | idb, (kb | j) != 0);
                         } else {
 #pragma unroll
                             for (int t = 0; t < 2; ++t)
                                 mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, t)) + 32 * kk),
-                                           idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, (kb | kk | t) != 0);
+                                           idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, (kb | j | t) != 0);
                         }
                     }
                     issued = true;
