@@ -223,10 +223,14 @@ struct Bf16Cfg {
     static constexpr int STAGE = NB * A_BYTES + B_BYTES;
     static constexpr int STAGES = cmin(kMaxStages, kSmemBudget / STAGE);
     static constexpr int ACC_COLS = NB * BT;
-    static constexpr int TMEM_COLS = tmem_cols_pow2(2 * ACC_COLS);
-    static constexpr int THREADS = 6 * 32;
+    // Two accumulator buffers when they fit; the 256-token gate/up tile has one, and two
+    // epilogue warps per lane quarter shorten the time the MMAs wait for it.
+    static constexpr int ACC_BUFS = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr int EW = ACC_BUFS == 1 ? 2 : 1;
+    static constexpr int TMEM_COLS = tmem_cols_pow2(ACC_BUFS * ACC_COLS);
+    static constexpr int THREADS = (2 + 4 * EW) * 32;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
-    static_assert(STAGES >= 2 && SMEM_BYTES <= kSmemLimit && 2 * ACC_COLS <= 512, "BF16 GEMM config");
+    static_assert(STAGES >= 2 && SMEM_BYTES <= kSmemLimit && ACC_BUFS * ACC_COLS <= 512, "BF16 GEMM config");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
 };
 
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->tfull[b], 1);
-            mbar_init(&ctl->tempty[b], 4);
+            mbar_init(&ctl->tempty[b], 4 * C::EW);
         }
         mbar_init(&ctl->drain[0], 1);
         ctl->abort = 0;
@@ -313,11 +317,15 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {  // ---------------- MMA issuer
-            constexpr uint32_t idesc = idesc_f16(1, kTileN, BT);
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
             bool ok = true, issued = false;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                // MMA width: the tile's rows rounded up to 16, so a segment's short last
+                // tile does not pay for BT columns
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const uint32_t idesc = idesc_f16(1, kTileN, cmin(BT, (rows + 15) & ~15));
                 if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -349,8 +357,10 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                 }
                 if (!ok) break;
                 mma_commit(&ctl->tfull[b]);
-                b ^= 1;
-                if (b == 0) bph ^= 1u;
+                if (++b == C::ACC_BUFS) {
+                    b = 0;
+                    bph ^= 1u;
+                }
             }
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
@@ -363,8 +373,8 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5)
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // ---------------- epilogue (warps 2 .. 2 + 4 EW)
+        const int q = warp & 3, h = (warp - 2) >> 2;  // TMEM lane quarter; chunk phase
         int b = 0;
         uint32_t bph = 0;
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -376,15 +386,17 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT>(a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g,
-                                         nt, row0, rows, q, lane);
+            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(
+                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane, h);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[b]);
-            b ^= 1;
-            if (b == 0) bph ^= 1u;
+            if (++b == C::ACC_BUFS) {
+                b = 0;
+                bph ^= 1u;
+            }
         }
-        if (a.zero_pad && OUT == OUT_BF16) zero_padding_rows(a, ctl, threadIdx.x - 64);
+        if (a.zero_pad && OUT == OUT_BF16 && h == 0) zero_padding_rows(a, ctl, threadIdx.x - 64);
     }
 
     tc_fence_before();
@@ -1627,10 +1639,12 @@ cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtens
 
 }  // namespace
 
-// Token tile from the mean segment length. 256-token tiles exist for the single-matrix
-// BF16 GEMM only: at 128 x 128 it needs about twice the shared-memory bandwidth per FLOP
-// that an SM has, and a 256-wide tile halves the weight-tile traffic per FLOP while its
-// double-buffered accumulators (2 x 256 columns) still fit in TMEM.
+// Token tile from the mean segment length. 256-token tiles exist for the BF16 GEMMs only:
+// at 128 x 128 a tile needs more shared-memory bandwidth per FLOP than an SM has, and a
+// 256-wide tile halves the weight-tile traffic per FLOP. They are chosen for the single
+// matrix (double-buffered accumulators still fit); the gate/up pair's 256-token tile has
+// one accumulator buffer and is used only when MOE_TOKEN_TILE asks for it. The MMA width
+// follows each tile's rows, so a wide tile costs a short segment little.
 int choose_token_tile(long long NvS, int G, bool wide_ok) {
     const long long segs = std::max<long long>(1, std::min<long long>(G, NvS));
     const long long avg = (NvS + segs - 1) / segs;
@@ -1669,16 +1683,20 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.err = p.err;
     if (p.nvf4) return launch_nvf4(p, a, st, pdl);
     if (p.wfmt == MOE_W_MXFP4) return p.mx8 ? launch_mx8(p, a, st, pdl) : cudaErrorInvalidValue;
+    // The gate/up pair's 256-token tile (one accumulator buffer, three pipeline stages)
+    // measured slower than two 128-token tiles; it is used only on request.
     const bool wide_ok = p.wfmt == MOE_W_BF16 && !p.dual;
+    const bool wide_req = p.wfmt == MOE_W_BF16;
     int bt = p.bt;
     if (!bt) {
         // MOE_TOKEN_TILE=16|32|64|128|256 overrides the token-tile choice (tests, tuning)
         const char* env = getenv("MOE_TOKEN_TILE");
         const int v = env ? atoi(env) : 0;
-        bt = (v == 16 || v == 32 || v == 64 || v == 128 || (v == 256 && wide_ok)) ? v
-                                                                                   : choose_token_tile(p.M_alloc, p.G, wide_ok);
+        bt = (v == 16 || v == 32 || v == 64 || v == 128 || (v == 256 && wide_req))
+                 ? v
+                 : choose_token_tile(p.M_alloc, p.G, wide_ok);
     }
-    if (bt == 256 && !wide_ok) bt = 128;
+    if (bt == 256 && !wide_req) bt = 128;
     const CUtensorMapDataType xdt =
         p.wfmt == MOE_W_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tx, t0, t1;
@@ -1700,6 +1718,7 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
         case 32: return dispatch_bt<32>(p, a, tx, t0, t1, st, pdl);
         case 64: return dispatch_bt<64>(p, a, tx, t0, t1, st, pdl);
         case 256:
+            if (p.dual) return run_bf16<256, true, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
             if (p.out_kind == OUT_F32) return run_bf16<256, false, OUT_F32>(p, a, tx, t0, t1, st, pdl);
             return run_bf16<256, false, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
         default: return dispatch_bt<128>(p, a, tx, t0, t1, st, pdl);

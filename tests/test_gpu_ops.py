@@ -312,6 +312,19 @@ def test_forward_small_matches_oracle(lib, name):
         assert r <= FP4_REL_L2, r
 
 
+def test_forward_bf16_256_token_tiles(lib, monkeypatch):
+    # the 256-token gate/up tile (one accumulator buffer, eight epilogue warps) and the
+    # per-tile MMA width: segments of about 75 rows use a fraction of each tile
+    monkeypatch.setenv("MOE_TOKEN_TILE", "256")
+    cfg = SMALL["replicas"]
+    inp = W.gen_inputs(cfg)
+    out, ids, _, _ = run_layer(lib, cfg, inp)
+    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
+                        inp.w_down)
+    assert np.array_equal(ids.cpu().numpy(), ref["ids"])
+    check_bf16(out, ref["out"], what="bt256")
+
+
 def test_forward_weight_in_combine(lib):
     cfg = SMALL["replicas"]
     inp = W.gen_inputs(cfg)
