@@ -69,10 +69,12 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt_t;
  *           epilogue_from_quant_config: finite, > 0, one per expert).
  *   kdata, kscale, kalpha : the kernel-format copy that moe_prepare_weights
  *           writes into caller memory; NULL until then. BF16 needs none.
- *           kdata: tiles of 128 rows x 64 K (codes, then scales) for the GEMM that
- *           stages FP4 weights as f16. kscale: for NVFP4 with K % 256 == 0, tiles of
- *           128 rows x 256 K for the block-scaled GEMM (moe_grouped_gemm_nvfp4);
- *           otherwise equal to kdata. kalpha: the epilogue alphas.
+ *           NVFP4 kdata: tiles of 128 rows x 64 K (codes, then scales) for the GEMM
+ *           that stages the weights as f16; kscale: for K % 256 == 0, tiles of 128
+ *           rows x 256 K for the block-scaled GEMM (moe_grouped_gemm_nvfp4), else
+ *           equal to kdata. MXFP4 kdata: the codes with K padded to a multiple of
+ *           128; kscale: the e8m0 scales in 128 x 128 blocks. kalpha: the epilogue
+ *           alphas.
  */
 typedef struct {
     int32_t fmt;            /* moe_wfmt_t */
@@ -170,9 +172,14 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w, i
  * (MoonEP page, moonep_grouped_gemm). Empty segments are skipped.
  *   a    bf16 [M_alloc, K];   out bf16 [M_alloc, N];   cu_seqlens int32 [G] on device.
  *   w    BF16 weights, or FP4 weights already prepared (else NOT_PREPARED).
- *   FP4: each row of a is converted to f16 times a power of two chosen from the
+ *   NVFP4: each row of a is converted to f16 times a power of two chosen from the
  *   row's max (exact except below 2^-30 of that max); the products with the
  *   exactly-dequantised weights accumulate in fp32 on the tensor cores.
+ *   MXFP4: each 32-value block of a row is staged as two e4m3 terms sharing one
+ *   e8m0 scale 2^e (the smallest with block max <= 448 * 2^e): hi = e4m3(v/2^e),
+ *   lo = e4m3(v/2^e - hi), within 1.07 * 2^-8 |v| + 2^(e-10) of v; the tensor cores
+ *   multiply both terms by the e2m1 weights with both block scales applied
+ *   (kind::mxf8f6f4) and accumulate in fp32.
  *   ws: at least moe_grouped_gemm_workspace_size(M_alloc, w) bytes.
  */
 size_t moe_grouped_gemm_workspace_size(int M_alloc, const moe_weight_t* w);
@@ -238,8 +245,7 @@ moe_status_t moe_quantize_nvfp4(const void* in, int in_is_f32, int R, int K,
  * finalize_weights). Untimed; synchronises `stream`.
  *   dst: caller device memory of moe_prepared_weight_bytes(w) bytes. On success
  *   w->kdata/kscale/kalpha point into dst. BF16 weights: no-op, MOE_OK.
- *   MXFP4 rows whose scales span more than 36 binades cannot be staged exactly
- *   in f16: MOE_ERR_UNSUPPORTED. Non-finite or non-positive alpha: INVALID_ARG.
+ *   An e8m0 NaN scale (255), or a non-finite or non-positive alpha: INVALID_ARG.
  */
 size_t moe_prepared_weight_bytes(const moe_weight_t* w);
 moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,

@@ -7,33 +7,37 @@
 // SITU from the TRTLLM MXFP4 page).
 //
 // Tiling ("swap AB"): one tile is 128 weight rows (the MMA M side) by BT token
-// rows (the MMA N side, 16..128) of one segment. Decode segments hold a handful
+// rows (the MMA N side, 16..256) of one segment. Decode segments hold a handful
 // of tokens, so the token side is the narrow one; the weights stream through
 // at full width. Each CTA owns one SM and walks the tile list
 // (segment, weight block, token block) with the token block fastest, so the
 // CTAs working on one weight block at the same time share it through L2.
 //
-// Two kernels share the tile schedule and the epilogue:
+// Four kernels share the tile schedule and the epilogue:
 //
 // grouped_gemm_kernel (BF16 weights): a ring of shared-memory stages
-//   {gate tile, [up tile], token tile} filled by TMA; MMA operands from smem.
+//   {gate tile, [up tile], token tile} filled by TMA; kind::f16 MMAs from smem.
 //
-// grouped_gemm_fp4_kernel (MXFP4 / NVFP4 weights): a deep shared-memory ring of
-//   small raw stages {token tile, packed e2m1 codes, block scales} filled by bulk
-//   copies and TMA; converter warps expand the codes to f16 (times the block
-//   scale, exact) straight into a ring of weight tiles in tensor memory, and the
-//   MMA reads A from TMEM and the token tile from smem. Keeping the expanded
-//   weights out of shared memory matters: with f16 weights in smem every weight
-//   costs 4 bytes of smem traffic (converter write + MMA read), which caps an FP4
-//   weight stream well below HBM bandwidth.
+// grouped_gemm_nvf4_kernel (NVFP4 weights, NVFP4 activations): block-scaled
+//   kind::mxf4nvf4 MMAs. Weights arrive as prepared 128 x 256 tiles (swizzled codes
+//   plus e4m3 scale blocks, one bulk copy each), tokens as packed e2m1 rows plus
+//   scales (TMA); a scale warp copies both scale sets into tensor memory.
 //
-// Warp roles (one CTA per SM):
-//   warp 0        producer (one thread)
-//   warp 1        MMA issuer (one thread) + TMEM owner
-//   warps 2..5    epilogue: TMEM -> registers -> alpha / activation / scales -> global
-//   warps 6..13   (FP4 kernel) converters, two warps per TMEM lane quarter
-// Every wait is bounded; a timeout records MOE_ERR_TIMEOUT in the error word,
-// stops all roles, lets copies in flight land, frees TMEM and returns.
+// grouped_gemm_mx8_kernel (MXFP4 weights, bf16 activations): block-scaled
+//   kind::mxf8f6f4 MMAs of e2m1 weights (4-bit tensor map) against the activations
+//   staged as two e4m3 terms with a shared e8m0 scale per 32 values.
+//
+// grouped_gemm_fp4_kernel (NVFP4 weights, bf16 activations): a deep ring of small
+//   raw stages {token tile, packed e2m1 codes, block scales}; converter warps expand
+//   the codes to f16 (times the block scale, exact) straight into a ring of weight
+//   tiles in tensor memory, and the MMA reads A from TMEM and the tokens from smem.
+//
+// Warp roles (one CTA per SM): a producer thread (TMA / bulk copies), one or more
+// MMA-issuing threads (the first one's warp owns TMEM), four or eight epilogue warps
+// (TMEM -> registers -> alpha / activation / scales -> global), and per kernel a
+// scale warp or converter warps. Every wait is bounded; a timeout records
+// MOE_ERR_TIMEOUT in the error word, stops all roles, lets copies in flight land,
+// frees TMEM and returns.
 #include <cmath>
 #include <mutex>
 
@@ -79,7 +83,6 @@ struct CtrlBlock {
     uint64_t tfull[2], tempty[2], drain[6];
     uint32_t tmem_slot;
     int abort;
-    uint16_t lut[256];
     int cu[kMaxG];
     int tpre[kMaxG + 1];
 };
@@ -409,13 +412,13 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 
 // ------------------------------------------------------------------ FP4 kernel
 
-template <int BT, bool DUAL, int WFMT>
+template <int BT, bool DUAL>
 struct Fp4Cfg {
     static constexpr int NB = DUAL ? 2 : 1;
     static constexpr int KS = kFp4StageK;                    // 128 K values per stage
     static constexpr int BOX_BYTES = BT * kTileK * 2;        // one 64-K token box, f16
     static constexpr int B_BYTES = 2 * BOX_BYTES;            // token tile of a stage
-    static constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;    // scale bytes per row per 64 K
+    static constexpr int S = 4;                              // e4m3 scale bytes per row per 64 K
     static constexpr int CHUNK = kTileN * 32 + kTileN * S;   // prepared 128 x 64 chunk
     static constexpr int RAW_M = 2 * CHUNK;                  // one matrix's raw bytes per stage
     static constexpr int RAW_STAGE = round1024(B_BYTES + NB * RAW_M);
@@ -464,59 +467,41 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t sc2, uint32_t
 // f16x2 holding `bits` in both halves
 __device__ __forceinline__ uint32_t dup16(uint32_t bits) { return (bits & 0xFFFFu) | (bits << 16); }
 
-// One weight row's 64 K values of one prepared chunk -> 32 f16x2 words (scale applied).
-template <int WFMT>
-__device__ __forceinline__ void convert_chunk_row(const uint8_t* chunk, int row, const uint16_t* lut,
-                                                  uint32_t (&o)[32]) {
-    constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;
+// One weight row's 64 K values of one prepared NVFP4 chunk -> 32 f16x2 words (e2m1 times
+// its e4m3 block scale; exact in f16).
+__device__ __forceinline__ void convert_chunk_row(const uint8_t* chunk, int row, uint32_t (&o)[32]) {
     const uint4 v0 = *reinterpret_cast<const uint4*>(chunk + row * 32);
     const uint4 v1 = *reinterpret_cast<const uint4*>(chunk + row * 32 + 16);
-    const uint8_t* rs = chunk + kTileN * 32 + row * S;
-    uint32_t sc[4];
-    if (WFMT == MOE_W_MXFP4) {
-        sc[0] = sc[1] = dup16(lut[rs[0]]);
-        sc[2] = sc[3] = dup16(lut[rs[1]]);
-    } else {
-        const uint32_t four = *reinterpret_cast<const uint32_t*>(rs);
-        uint32_t s01, s23;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"((uint16_t)(four & 0xFFFF)));
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s23) : "h"((uint16_t)(four >> 16)));
-        sc[0] = dup16(s01);
-        sc[1] = dup16(s01 >> 16);
-        sc[2] = dup16(s23);
-        sc[3] = dup16(s23 >> 16);
-    }
+    const uint32_t four = *reinterpret_cast<const uint32_t*>(chunk + kTileN * 32 + row * 4);
+    uint32_t s01, s23, sc[4];
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"((uint16_t)(four & 0xFFFF)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s23) : "h"((uint16_t)(four >> 16)));
+    sc[0] = dup16(s01);
+    sc[1] = dup16(s01 >> 16);
+    sc[2] = dup16(s23);
+    sc[3] = dup16(s23 >> 16);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
 }
 
 // Half of it: the 32 values [32h, 32h+32) of the chunk row -> 16 f16x2 words.
-template <int WFMT>
-__device__ __forceinline__ void convert_half_chunk_row(const uint8_t* chunk, int row, int h, const uint16_t* lut,
-                                                       uint32_t (&o)[16]) {
-    constexpr int S = WFMT == MOE_W_MXFP4 ? 2 : 4;
+__device__ __forceinline__ void convert_half_chunk_row(const uint8_t* chunk, int row, int h, uint32_t (&o)[16]) {
     const uint4 v = *reinterpret_cast<const uint4*>(chunk + row * 32 + h * 16);
-    const uint8_t* rs = chunk + kTileN * 32 + row * S;
-    uint32_t sc[2];
-    if (WFMT == MOE_W_MXFP4) {
-        sc[0] = sc[1] = dup16(lut[rs[h]]);
-    } else {
-        const uint16_t pair = *reinterpret_cast<const uint16_t*>(rs + 2 * h);
-        uint32_t s01;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"(pair));
-        sc[0] = dup16(s01);
-        sc[1] = dup16(s01 >> 16);
-    }
+    const uint16_t pair = *reinterpret_cast<const uint16_t*>(chunk + kTileN * 32 + row * 4 + 2 * h);
+    uint32_t s01, sc[2];
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s01) : "h"(pair));
+    sc[0] = dup16(s01);
+    sc[1] = dup16(s01 >> 16);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) e2m1x8_to_f16(w[i], sc[i >> 1], o + 4 * i);
 }
 
-template <int BT, bool DUAL, int WFMT, int OUT>
-__global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
+template <int BT, bool DUAL, int OUT>
+__global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
-    using C = Fp4Cfg<BT, DUAL, WFMT>;
+    using C = Fp4Cfg<BT, DUAL>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::RSTAGES * C::RAW_STAGE);
@@ -548,17 +533,6 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_slot, 512);
         tmem_relinquish();
-    }
-    if (WFMT == MOE_W_MXFP4) {
-        // e8m0 (re-biased by the weight preparation) -> f16 bits of 2^(e-127)
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-            const int e = i - 127;
-            uint16_t bits;
-            if (e >= -14 && e <= 15) bits = (uint16_t)((e + 15) << 10);
-            else if (e >= -24 && e < -14) bits = (uint16_t)(1u << (e + 24));
-            else bits = e > 15 ? (uint16_t)0x7C00 : (uint16_t)0;
-            ctl->lut[i] = bits;
-        }
     }
     pdl_wait();
     if (warp == 0) build_segment_table<BT>(a, ctl, lane);
@@ -750,12 +724,12 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL, WFMT>::THREADS, 1)
                 if (DUAL) {  // unit grp: matrix grp>>1, chunk grp&1 (64 values)
                     const int m = grp >> 1, c = grp & 1;
                     uint32_t o[32];
-                    convert_chunk_row<WFMT>(rawM(r, m) + c * C::CHUNK, row, ctl->lut, o);
+                    convert_chunk_row(rawM(r, m) + c * C::CHUNK, row, o);
                     tmem_st32(lane_base + acol + m * C::A_COLS + c * 32, o);
                 } else {     // unit grp: chunk grp>>1, half grp&1 (32 values)
                     const int c = grp >> 1, h = grp & 1;
                     uint32_t o[16];
-                    convert_half_chunk_row<WFMT>(rawM(r, 0) + c * C::CHUNK, row, h, ctl->lut, o);
+                    convert_half_chunk_row(rawM(r, 0) + c * C::CHUNK, row, h, o);
                     tmem_st16(lane_base + acol + c * 32 + h * 16, o);
                 }
                 tmem_st_wait();
@@ -1492,10 +1466,10 @@ cudaError_t run_bf16(const GemmProblem& p, const GemmArgs& args, const CUtensorM
                     args);
 }
 
-template <int BT, bool DUAL, int WFMT, int OUT>
+template <int BT, bool DUAL, int OUT>
 cudaError_t run_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st, bool pdl) {
-    using C = Fp4Cfg<BT, DUAL, WFMT>;
-    auto kern = grouped_gemm_fp4_kernel<BT, DUAL, WFMT, OUT>;
+    using C = Fp4Cfg<BT, DUAL>;
+    auto kern = grouped_gemm_fp4_kernel<BT, DUAL, OUT>;
     static int done[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
@@ -1617,21 +1591,21 @@ cudaError_t launch_mx8(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool 
     }
 }
 
-template <int BT, int WFMT>
+template <int BT>
 cudaError_t dispatch_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st,
                          bool pdl) {
     if (p.dual) {
-        if (p.out_kind == OUT_F16) return run_fp4<BT, true, WFMT, OUT_F16>(p, args, tx, st, pdl);
-        return run_fp4<BT, true, WFMT, OUT_F32>(p, args, tx, st, pdl);
+        if (p.out_kind == OUT_F16) return run_fp4<BT, true, OUT_F16>(p, args, tx, st, pdl);
+        return run_fp4<BT, true, OUT_F32>(p, args, tx, st, pdl);
     }
-    if (p.out_kind == OUT_F32) return run_fp4<BT, false, WFMT, OUT_F32>(p, args, tx, st, pdl);
-    return run_fp4<BT, false, WFMT, OUT_BF16>(p, args, tx, st, pdl);
+    if (p.out_kind == OUT_F32) return run_fp4<BT, false, OUT_F32>(p, args, tx, st, pdl);
+    return run_fp4<BT, false, OUT_BF16>(p, args, tx, st, pdl);
 }
 
 template <int BT>
 cudaError_t dispatch_bt(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx,
                         const CUtensorMap& t0, const CUtensorMap& t1, cudaStream_t st, bool pdl) {
-    if (p.wfmt == MOE_W_NVFP4) return dispatch_fp4<BT, MOE_W_NVFP4>(p, args, tx, st, pdl);
+    if (p.wfmt == MOE_W_NVFP4) return dispatch_fp4<BT>(p, args, tx, st, pdl);
     if (p.dual) return run_bf16<BT, true, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
     if (p.out_kind == OUT_F32) return run_bf16<BT, false, OUT_F32>(p, args, tx, t0, t1, st, pdl);
     return run_bf16<BT, false, OUT_BF16>(p, args, tx, t0, t1, st, pdl);
