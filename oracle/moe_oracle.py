@@ -348,6 +348,46 @@ def nvfp4_dequantize_rows(codes, sb, s):
 
 
 # --------------------------------------------------------------------------------------
+# S2q dynamic MXFP8 activation quantisation (the W4A8 mode of MXFP4 experts)
+# --------------------------------------------------------------------------------------
+
+E4M3_EMAX = 8   # exponent of e4m3's largest normal value, 448 = 1.75 * 2^8
+
+
+def mxfp8_quantize_rows(v):
+    """Dynamic MXFP8 quantisation of activation rows for MXFP4 weights.
+
+    The page lists ``(kMxfp4Static, kMxfp8Dynamic)`` as a supported weight/activation pair
+    [trtllm: _supports_quant_scheme] and says nothing more. Reading taken: the OCP MX v1.0
+    MXFP8 format with its conversion rule, per 32-value block b of a row:
+
+      X_b  = 2^(floor(log2 amax_b) - 8), the exponent clamped to e8m0's [-127, 127]
+      q    = e4m3_rne_satfinite(v / X_b)
+      value = e4m3(q) * X_b
+
+    An all-zero block takes X_b = 2^-127 and +0 codes. X_b is a power of two, so v / X_b is
+    exact and no decision depends on the arithmetic's precision. Applied, like the NVFP4
+    mode, to x in token order and to every activation row before the down GEMM.
+    Returns ``codes [R,K] uint8`` (e4m3) and ``scales [R,K/32] uint8`` (e8m0).
+    """
+    x = np.asarray(v, dtype=np.float32).astype(np.float64)
+    R, K = x.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    amax = np.abs(x).reshape(R, K // 32, 32).max(axis=2)
+    _, ex = np.frexp(amax)                       # amax = m * 2^ex, m in [0.5, 1): floor(log2) = ex - 1
+    e = np.where(amax > 0, ex - 1 - E4M3_EMAX, -127)
+    e = np.clip(e, -127, 127).astype(np.int64)
+    codes = e4m3_encode(x / np.repeat(np.ldexp(1.0, e), 32, axis=1))
+    return codes, (e + 127).astype(np.uint8)
+
+
+def mxfp8_dequantize_rows(codes, scales):
+    """Value of MXFP8 rows: e4m3(q) * 2^(s - 127), fp64 (exact)."""
+    return e4m3_decode(codes) * np.repeat(e8m0_decode(scales), 32, axis=1)
+
+
+# --------------------------------------------------------------------------------------
 # S6 combine
 # --------------------------------------------------------------------------------------
 
@@ -375,9 +415,9 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     route weight -> down grouped GEMM -> combine [moonep: module docstring and apply;
     trtllm: _invoke_kernel; fi_ep: apply].
 
-    ``cfg`` supplies E, B, topk, act, situ_alpha, situ_beta and act_quant. With act_quant, x
-    (in token order) and every activation row are NVFP4-quantised (``nvfp4_quantize_rows``)
-    before their GEMM. ``tokens`` restricts the expert maths to the rows those tokens need
+    ``cfg`` supplies E, B, topk, act, situ_alpha, situ_beta and act_quant. With act_quant = 1,
+    x (in token order) and every activation row are NVFP4-quantised (``nvfp4_quantize_rows``)
+    before their GEMM; with act_quant = 2 they are MXFP8-quantised (``mxfp8_quantize_rows``). ``tokens`` restricts the expert maths to the rows those tokens need
     (routing and permutation are always computed in full). With ``apply_topk_in_fc1`` false
     the route weight moves from the activation to the combine [fi_ep: apply_topk_in_fc1].
 
@@ -395,11 +435,16 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
 
     x64 = to_f64(x)
     res = dict(ids=ids, w=w, perm_w=perm_w, tokens=tok, **perm)
-    if cfg.act_quant:
+    if cfg.act_quant == 1:
         codes, sb, s = nvfp4_quantize_rows(np.asarray(x.float().numpy(), np.float32))
         x64 = nvfp4_dequantize_rows(codes, sb, s)
         if keep:
             res.update(xq_codes=codes, xq_sb=sb, xq_s=s)
+    elif cfg.act_quant == 2:
+        codes, sc = mxfp8_quantize_rows(np.asarray(x.float().numpy(), np.float32))
+        x64 = mxfp8_dequantize_rows(codes, sc)
+        if keep:
+            res.update(xq_codes=codes, xq_scales=sc)
 
     a_g, a_u, a_d = weight_alpha(w_gate), weight_alpha(w_up), weight_alpha(w_down)
     y = np.zeros((T * k, w_down.N), dtype=np.float64)
@@ -413,9 +458,12 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
         up = a_u[g] * (a @ weight_rows(w_up, g).T)
         h = act_and_mul(gate, up, cfg.act, cfg.situ_alpha, cfg.situ_beta,
                         perm_w[rows] if apply_topk_in_fc1 else None)
-        if cfg.act_quant:
+        if cfg.act_quant == 1:
             hc, hsb, hs = nvfp4_quantize_rows(h.astype(np.float32))
             h = nvfp4_dequantize_rows(hc, hsb, hs)
+        elif cfg.act_quant == 2:
+            hc, hsc = mxfp8_quantize_rows(h.astype(np.float32))
+            h = mxfp8_dequantize_rows(hc, hsc)
         if keep:
             h_keep[rows] = h
         y[rows] = a_d[g] * (h @ weight_rows(w_down, g).T)

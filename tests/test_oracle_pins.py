@@ -302,6 +302,56 @@ def test_nvfp4_quant_matches_bruteforce_and_bounds():
     assert np.allclose(O.nvfp4_dequantize_rows(codes2, sb2, s2), deq, rtol=1e-6, atol=0)
 
 
+def _mxfp8_brute(row):
+    """Per element: the block's power-of-two scale from a loop over exponents, then the
+    nearest point of the whole e4m3 grid times that scale (ties to the even code, beyond 448
+    clamped to 448)."""
+    grid = [float(O.e4m3_decode(np.array([c]))[0]) for c in range(127)]   # non-negative finite
+    codes, scales = [], []
+    for b in range(len(row) // 32):
+        blk = [float(v) for v in row[32 * b:32 * b + 32]]
+        amax = max(abs(v) for v in blk)
+        if amax == 0:
+            k = -127
+        else:
+            k = 0
+            while 2.0 ** k > amax:
+                k -= 1
+            while 2.0 ** (k + 1) <= amax:
+                k += 1
+            k = max(-127, min(127, k - 8))
+        scales.append(k + 127)
+        X = 2.0 ** k
+        for v in blk:
+            a = min(abs(v) / X, 448.0)
+            best = min(range(127), key=lambda c: (abs(grid[c] - a), c % 2))
+            codes.append(best | (128 if math.copysign(1.0, v) < 0 else 0))
+    return np.array(codes, np.uint8), np.array(scales, np.uint8)
+
+
+def test_mxfp8_quant_matches_bruteforce_and_special_cases():
+    x = W.gen_rows(4, 96, seed=7, dtype=torch.float32).numpy()
+    x[1, 32:64] = 0.0                                   # an all-zero block
+    x[2] *= 1e-4
+    x[3, 0:32] = np.linspace(-1.0, 1.0, 32) * 1.9 * 8.0  # amax 15.2 -> v/X reaches 486 > 448: saturates
+    codes, sc = O.mxfp8_quantize_rows(x)
+    for r in range(4):
+        bc, bs = _mxfp8_brute(x[r])
+        assert np.array_equal(codes[r], bc), r
+        assert np.array_equal(sc[r], bs), r
+    assert sc[1, 1] == 0 and np.all(codes[1, 32:64] == 0)
+    deq = O.mxfp8_dequantize_rows(codes, sc)
+    assert sc[3, 0] == 127 + 3 - 8 and deq[3, 31] == 448.0 * 2.0 ** -5 and deq[3, 0] == -448.0 * 2.0 ** -5
+    # a power of two is its block's amax exactly: scale 2^(k-8), code of 256
+    y = np.zeros((1, 32), np.float32)
+    y[0, 3] = 2.0 ** 5
+    c1, s1 = O.mxfp8_quantize_rows(y)
+    assert s1[0, 0] == 127 + 5 - 8 and O.e4m3_decode(c1[0, 3:4])[0] == 256.0
+    # values already on the grid quantise to themselves
+    c2, s2 = O.mxfp8_quantize_rows(deq.astype(np.float32))
+    assert np.array_equal(O.mxfp8_dequantize_rows(c2, s2), deq)
+
+
 # ------------------------------------------------------------------ the whole layer
 
 def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
@@ -309,9 +359,12 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
     own routing, pure-Python dot products."""
     ids, w = _route_brute(inp.logits.numpy(), cfg.topk)
     x = O.to_f64(inp.x)
-    if cfg.act_quant:
+    if cfg.act_quant == 1:
         c, sb, s = O.nvfp4_quantize_rows(inp.x.float().numpy())
         x = O.nvfp4_dequantize_rows(c, sb, s)
+    elif cfg.act_quant == 2:
+        c, sc = O.mxfp8_quantize_rows(inp.x.float().numpy())
+        x = O.mxfp8_dequantize_rows(c, sc)
     ag, au, ad = (O.weight_alpha(inp.w_gate), O.weight_alpha(inp.w_up), O.weight_alpha(inp.w_down))
     out = np.zeros((cfg.T, cfg.H))
     Wg = [O.weight_rows(inp.w_gate, e).tolist() for e in range(cfg.E)]
@@ -331,9 +384,12 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
                      for gg, uu in zip(gate, up)]
             if apply_topk_in_fc1:
                 h = [v * w[t, j] for v in h]
-            if cfg.act_quant:
+            if cfg.act_quant == 1:
                 c, sb, s = O.nvfp4_quantize_rows(np.array([h], np.float32))
                 h = O.nvfp4_dequantize_rows(c, sb, s)[0].tolist()
+            elif cfg.act_quant == 2:
+                c, sc = O.mxfp8_quantize_rows(np.array([h], np.float32))
+                h = O.mxfp8_dequantize_rows(c, sc)[0].tolist()
             y = [ad[e] * sum(a * b for a, b in zip(row, h)) for row in Wd[e]]
             wt = 1.0 if apply_topk_in_fc1 else w[t, j]
             out[t] += wt * np.array(y)
@@ -347,6 +403,8 @@ SMALL = {
                               situ_alpha=0.8, situ_beta=1.7, wfmt="mxfp4"),
     "nvfp4_quant": W.MoEConfig("nvfp4_quant", T=8, H=64, I=32, E=4, topk=2, wfmt="nvfp4",
                                act_quant=1),
+    "mxfp4_w4a8": W.MoEConfig("mxfp4_w4a8", T=8, H=64, I=64, E=4, topk=2, act="situ", wfmt="mxfp4",
+                              act_quant=2),
 }
 
 

@@ -55,7 +55,7 @@ class MoEConfig:
     situ_alpha: float = 1.0    # SITU gate cap  (activation_situ_beta)
     situ_beta: float = 1.0     # SITU up cap    (activation_situ_linear_beta)
     wfmt: str = WFMT_BF16
-    act_quant: int = 0         # 1 = dynamic NVFP4 quantisation of activations
+    act_quant: int = 0         # 1 = dynamic NVFP4, 2 = dynamic MXFP8 quantisation of activations
     x_std: float = 1.0
     logit_std: float = 1.0
     w_std: float = 0.02
@@ -95,6 +95,11 @@ CONFIGS: dict[str, MoEConfig] = {
                                act="situ", wfmt=WFMT_MXFP4),
     "nvfp4": MoEConfig("nvfp4", T=1024, H=7168, I=2048, E=256, topk=8,
                        wfmt=WFMT_NVFP4, act_quant=1),
+    # the W4A8 mode of the MXFP4 experts: the MXFP4 shapes with dynamic MXFP8 activations
+    "mxfp4_w4a8_decode": MoEConfig("mxfp4_w4a8_decode", T=32, H=2880, I=2880, E=128, topk=4,
+                                   act="situ", wfmt=WFMT_MXFP4, act_quant=2),
+    "mxfp4_w4a8_prefill": MoEConfig("mxfp4_w4a8_prefill", T=4096, H=2880, I=2880, E=128, topk=4,
+                                    act="situ", wfmt=WFMT_MXFP4, act_quant=2),
 }
 
 
