@@ -74,16 +74,43 @@ def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) 
     NvS = cfg.NvS
     wg, wu, wd = (weight_bytes_per_row(inp.w_gate), weight_bytes_per_row(inp.w_up),
                   weight_bytes_per_row(inp.w_down))
-    act_out = 2 if cfg.wfmt == "bf16" or (cfg.act == "situ" and not cfg.act_quant) else 4
+    # gate/up output: bf16 (BF16), f16 (NVFP4 weights, bf16 activations, SITU), else fp32
+    act_out = 2 if cfg.wfmt == "bf16" or (cfg.wfmt == "nvfp4" and cfg.act == "situ" and not cfg.act_quant) else 4
+    # activation operand bytes per value as the GEMMs read them
+    a_in = {0: 2.0, 1: 9.0 / 16.0, 2: 1.0 + 1.0 / 32.0}[cfg.act_quant]
+    if cfg.wfmt == "mxfp4" and not cfg.act_quant:
+        a_in = 2.0 + 1.0 / 32.0           # two e4m3 terms and a scale per 32 values
     fc1_flops = 4.0 * NvS * cfg.H * cfg.I
     fc2_flops = 2.0 * NvS * cfg.H * cfg.I
-    fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * 2 + NvS * cfg.I * act_out
-    fc2_bytes = nonempty * wd + NvS * cfg.I * 2 + NvS * cfg.H * 2
+    fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * a_in + NvS * cfg.I * act_out
+    fc2_bytes = nonempty * wd + NvS * cfg.I * a_in + NvS * cfg.H * 4
     layer_bytes = nonempty * (wg + wu + wd) + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
     return dict(nonempty=nonempty, max_seg=max_seg,
                 fc1_flops=fc1_flops, fc2_flops=fc2_flops, fc1_bytes=fc1_bytes, fc2_bytes=fc2_bytes,
                 layer_flops=fc1_flops + fc2_flops, layer_bytes=layer_bytes,
                 weight_bytes_total=nonempty * (wg + wu + wd))
+
+
+def tensor_peak_ratio(cfg) -> tuple[float, str]:
+    """Tensor peak of the path's MMA kind relative to the measured bf16 one (the nominal
+    dense ratios: fp8 2x, fp4 4x bf16)."""
+    if cfg.wfmt == "nvfp4" and cfg.act_quant == 1:
+        return 4.0, "= measured bf16 x 4 (kind::mxf4nvf4, the nominal fp4/bf16 ratio)"
+    if cfg.wfmt == "mxfp4" and cfg.act_quant == 2:
+        return 2.0, "= measured bf16 x 2 (kind::mxf8f6f4, the nominal fp8/bf16 ratio)"
+    if cfg.wfmt == "mxfp4":
+        return 1.0, ("= measured bf16 (kind::mxf8f6f4 at the fp8 rate, two e4m3 products per "
+                     "multiply-add for the hi/lo activations)")
+    return 1.0, "= measured bf16"
+
+
+def compute_dtype(cfg) -> str:
+    """The operand types the grouped GEMMs' tensor cores multiply."""
+    if cfg.wfmt == "bf16":
+        return "bf16"
+    if cfg.wfmt == "nvfp4":
+        return "nvfp4 x nvfp4 (e2m1, e4m3 block scales)" if cfg.act_quant == 1 else "f16"
+    return "mxfp4 x mxfp8 (e2m1 x e4m3, e8m0 block scales)" + ("" if cfg.act_quant else ", activations as hi+lo")
 
 
 def load_peaks() -> tuple[dict, str]:
@@ -238,8 +265,8 @@ def default_sample(cfg) -> int:
 
 def kernel_launches(cfg) -> int:
     n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
-    if cfg.act_quant:
-        n += 2                            # x quantisation, activation quantisation
+    if cfg.act_quant or cfg.wfmt == "mxfp4":
+        n += 2                            # x quantisation / staging, activation quantisation / staging
     elif cfg.wfmt != "bf16" and cfg.act != "situ":
         n += 1                            # activation row pass to f16
     return n
@@ -336,21 +363,23 @@ def run_ours(args, cfg, rank, world):
 
     peaks, peak_src = load_peaks()
     ms_step = ms_total / K
-    t_fc1_tensor = acc["fc1_flops"] / (peaks["bf16_tflops"] * 1e12)
+    tensor_mult, tensor_note = tensor_peak_ratio(cfg)
+    tensor_peak = peaks["bf16_tflops"] * tensor_mult
+    t_fc1_tensor = acc["fc1_flops"] / (tensor_peak * 1e12)
     t_fc1_hbm = acc["fc1_bytes"] / (peaks["hbm_gbs"] * 1e9)
     traffic = profiled_traffic(args.config)
     if t_fc1_tensor >= t_fc1_hbm:
         ach = acc["fc1_flops"] / (fc1_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": ach / tensor_peak}
     else:
         ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"]}
-    roof.update({"traffic": traffic, "kernel": "grouped_gemm_kernel gate+up (fused activation)",
+    roof.update({"traffic": traffic, "kernel": "grouped GEMM gate+up (fused activation)",
                  "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
-                 "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst)"})
-    t_layer_roof = max(acc["layer_flops"] / (peaks["bf16_tflops"] * 1e12),
+                 "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst); tensor peak {tensor_note}"})
+    t_layer_roof = max(acc["layer_flops"] / (tensor_peak * 1e12),
                        acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
     tok_s = job_tokens_per_s(world, cfg.T, K, ms_total)
 
@@ -366,7 +395,7 @@ def run_ours(args, cfg, rank, world):
     res = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if cfg.wfmt == "bf16" else "f16",
+        "vs_baseline": None, "dtype": compute_dtype(cfg),
         "data": "synthetic (seeded; random weights of the workload's shapes)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
                    "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant,

@@ -240,6 +240,17 @@ moe_status_t moe_quantize_nvfp4(const void* in, int in_is_f32, int R, int K,
                                 moe_stream_t stream);
 
 /*
+ * S2q — dynamic MXFP8 quantisation of activation rows, the activation side of the W4A8 mode
+ * of MXFP4 experts (TRTLLM MXFP4 page, _supports_quant_scheme: (kMxfp4Static,
+ * kMxfp8Dynamic)). The page names the mode only; the format and rule are OCP MX v1.0
+ * MXFP8: per 32 values, scale 2^e with e = floor(log2 amax) - 8 clamped to [-127, 127]
+ * (e = -127 for an all-zero block), q = e4m3_rne_satfinite(v / 2^e).
+ *   in      bf16 (in_is_f32 = 0) or fp32 (in_is_f32 = 1) [R,K], K % 32 == 0.
+ *   codes   uint8 [R,K] e4m3.   scales  uint8 [R,K/32] e8m0 (value 2^(s-127)).
+ */
+moe_status_t moe_quantize_mxfp8(const void* in, int in_is_f32, int R, int K, uint8_t* codes,
+                                uint8_t* scales, moe_stream_t stream);
+/*
  * S0 — one-time conversion of FP4 weights into the kernel's tile layout
  * (FlashInfer MoE-EP page, process_weights_after_loading; DeepSeek-V4 FI page,
  * finalize_weights). Untimed; synchronises `stream`.
@@ -262,6 +273,9 @@ moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,
  *   act_quant = 1: dynamic NVFP4 activations (NVFP4 weights only); each GEMM whose K
  *   (H for gate/up, I for down) is a multiple of 256 then runs block-scaled as in
  *   moe_grouped_gemm_nvfp4, the other one on f16-staged operands.
+ *   act_quant = 2: dynamic MXFP8 activations (MXFP4 weights only, the W4A8 mode): x and
+ *   every activation row are quantised as moe_quantize_mxfp8 does, and both GEMMs take
+ *   them as e4m3 with their e8m0 scales. Other act_quant values: INVALID_ARG.
  *   apply_topk_in_fc1 = 1 applies the route weight in the activation (default);
  *   0 applies it in the combine (FlashInfer MoE-EP page, apply_topk_in_fc1).
  *   topk_ids_out/topk_w_out: optional [T,topk] copies of the routing.

@@ -36,7 +36,7 @@ EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_wo
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
            "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc",
-           "moe_grouped_gemm_nvfp4"]
+           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8"]
 
 
 class MoEError(RuntimeError):
@@ -90,6 +90,7 @@ _sig = {
     "moe_get_device_error": (_I, [_P, _P]),
     "moe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P]),
     "moe_grouped_gemm_nvfp4": (_I, [_P, _P, _P, _I, ctypes.POINTER(moe_weight_t), _P, _P, _P, _S, _P]),
+    "moe_quantize_mxfp8": (_I, [_P, _I, _I, _I, _P, _P, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -272,6 +273,17 @@ def moe_quantize_nvfp4(x: torch.Tensor, deq: bool = True, stream=None):
     _check(_lib.moe_quantize_nvfp4(_ptr(x), 1 if x.dtype == torch.float32 else 0, R, K, _ptr(codes),
                                    _ptr(sb), _ptr(s), _ptr(d), _stream(stream)), "moe_quantize_nvfp4")
     return codes, sb, s, d
+
+
+def moe_quantize_mxfp8(x: torch.Tensor, stream=None):
+    """Dynamic MXFP8 quantisation of rows (bf16 or fp32 [R,K]): e4m3 codes [R,K] and e8m0
+    scales [R,K/32]."""
+    R, K = x.shape
+    codes = torch.empty(R, K, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(R, K // 32, dtype=torch.uint8, device=x.device)
+    _check(_lib.moe_quantize_mxfp8(_ptr(x), 1 if x.dtype == torch.float32 else 0, R, K, _ptr(codes), _ptr(scales),
+                                   _stream(stream)), "moe_quantize_mxfp8")
+    return codes, scales
 
 
 def forward_workspace(T_max, H, I, E, B, topk, wfmt="bf16", act_quant=0, device="cuda") -> torch.Tensor:

@@ -68,7 +68,9 @@ struct FwdWs {
 
 // With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
 // tensor cores; its operand rows are records of K/2 code bytes followed by K/16 scales.
-inline bool nvf4_k(int act_quant, int K) { return act_quant && K % kNvf4StageK == 0; }
+inline bool nvf4_k(int act_quant, int K) { return act_quant == 1 && K % kNvf4StageK == 0; }
+// MXFP4 weights: activations as two e4m3 terms (bf16 staged) or one (act_quant 2, MXFP8).
+inline int mx8_terms(int act_quant) { return act_quant == 2 ? 1 : 2; }
 inline int nvf4_rec_bytes(int K) { return K / 2 + K / 16; }
 
 FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
@@ -90,12 +92,12 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.inv = take(4 * NvS);
     L.perm_scratch = take(permute_ws_layout(T_max, topk, E, B).bytes);
     const bool nat1 = nvf4_k(act_quant, H), nat2 = nvf4_k(act_quant, I);
-    const bool q1 = act_quant && !nat1, q2 = act_quant && !nat2;  // quantised, then staged as f16
+    const bool q1 = act_quant == 1 && !nat1, q2 = act_quant == 1 && !nat2;  // NVFP4, then staged as f16
     L.xperm = take(nat1 || wfmt == MOE_W_MXFP4 ? 0 : 2 * NvS * H);
     L.tscale = take(fp4 ? 4 * NvS : 0);
     L.xq_codes = take(q1 ? (size_t)T_max * H / 2 : 0);
     L.xq_sb = take(q1 ? (size_t)T_max * H / 16 : 0);
-    L.xq_s = take(act_quant ? 4 * (size_t)T_max : 0);
+    L.xq_s = take(act_quant == 1 ? 4 * (size_t)T_max : 0);
     L.xq_deq = take(q1 ? 2 * (size_t)T_max * H : 0);
     L.xq_rec = take(nat1 ? (size_t)T_max * nvf4_rec_bytes(H) : 0);
     L.xperm_rec = take(nat1 ? NvS * nvf4_rec_bytes(H) : 0);
@@ -106,9 +108,10 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.act_sb = take(q2 ? NvS * I / 16 : 0);
     L.act_rec = take(nat2 ? NvS * nvf4_rec_bytes(I) : 0);
     const bool mx = wfmt == MOE_W_MXFP4;
-    L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H) : 0);
-    L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H) : 0);
-    L.mx_act = take(mx ? NvS * mx8_rec_bytes(I) : 0);
+    const int terms = mx8_terms(act_quant);
+    L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H, terms) : 0);
+    L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H, terms) : 0);
+    L.mx_act = take(mx ? NvS * mx8_rec_bytes(I, terms) : 0);
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
     L.bytes = off;
     return L;
@@ -212,14 +215,15 @@ moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
         p.x = a;
         p.w0 = w->data;
     } else if (w->fmt == MOE_W_MXFP4) {
-        // activations -> MXFP8 hi/lo records, then the block-scaled GEMM
+        // activations -> e4m3 hi/lo records, then the block-scaled GEMM
         uint8_t* rec = reinterpret_cast<uint8_t*>(wsb + kErrBytes);
-        const int rb = mx8_rec_bytes(w->K);
-        cudaError_t e = launch_quant_mx8(a, false, M_alloc, w->K, rec, rb, st, false);
+        const int rb = mx8_rec_bytes(w->K), Kp = mx8_kpad(w->K);
+        cudaError_t e = launch_quant_mx8(a, false, M_alloc, w->K, Kp, true, rec, rec + Kp, rec + 2 * Kp, rb, rb, st,
+                                         false);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         p.x = rec;
         p.x_stride = rb;
-        p.mx8 = true;
+        p.mx8 = 2;
         p.kdata0 = w->kdata;
         p.kscale0 = w->kscale;
         pdl = true;
@@ -235,6 +239,17 @@ moe_status_t moe_grouped_gemm(const void* a, int M_alloc, const moe_weight_t* w,
         pdl = true;
     }
     return cuda_status(launch_grouped_gemm(p, st, pdl));
+}
+
+moe_status_t moe_quantize_mxfp8(const void* in, int in_is_f32, int R, int K, uint8_t* codes, uint8_t* scales,
+                                moe_stream_t stream) {
+    if (R < 0 || K < 0) return MOE_ERR_INVALID_ARG;
+    if (K % 32) return MOE_ERR_ALIGNMENT;
+    if ((size_t)R * K == 0) return MOE_OK;
+    if (!in || !codes || !scales) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(in) || !aligned16(codes)) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_quant_mx8(in, in_is_f32 != 0, R, K, K, false, codes, nullptr, scales, K, K / 32,
+                                        S(stream), false));
 }
 
 moe_status_t moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sb, const float* a_s, int M_alloc,
@@ -350,7 +365,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if ((s = check_weight(p->w_gate, G, I, H)) != MOE_OK) return s;
     if ((s = check_weight(p->w_up, G, I, H)) != MOE_OK) return s;
     if ((s = check_weight(p->w_down, G, H, I)) != MOE_OK) return s;
-    if (p->act_quant && fmt != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+    // act_quant: 1 = dynamic NVFP4 (NVFP4 weights), 2 = dynamic MXFP8 (MXFP4 weights)
+    if (p->act_quant < 0 || p->act_quant > 2) return MOE_ERR_INVALID_ARG;
+    if ((p->act_quant == 1 && fmt != MOE_W_NVFP4) || (p->act_quant == 2 && fmt != MOE_W_MXFP4))
+        return MOE_ERR_UNSUPPORTED;
     if (H % 16 || I % 16) return MOE_ERR_ALIGNMENT;
     if (B > 0 && !p->replica_src) return MOE_ERR_INVALID_ARG;
     if (!ws) return MOE_ERR_INVALID_ARG;
@@ -377,6 +395,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     float* y = reinterpret_cast<float*>(w + L.y);
     const int NvS = T * k;
     const bool nat1 = nvf4_k(p->act_quant, H), nat2 = nvf4_k(p->act_quant, I);
+    const int terms = mx8_terms(p->act_quant);
     cudaStream_t st = S(stream);
     cudaError_t e;
     // Optional stage events (tracing). An event recorded between two kernels ends their
@@ -405,9 +424,11 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (fmt == MOE_W_BF16) {
         e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (fmt == MOE_W_MXFP4) {
-        // stage each token once as MXFP8 hi/lo records, then gather the records
-        const int rb = mx8_rec_bytes(H);
-        e = launch_quant_mx8(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.mx_xq), rb, st, pdl());
+        // stage each token once as e4m3 records (hi/lo, or MXFP8), then gather the records
+        const int rb = mx8_rec_bytes(H, terms), Kp = mx8_kpad(H);
+        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_xq);
+        e = launch_quant_mx8(p->x, false, T, H, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr, rec + terms * Kp,
+                             rb, rb, st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(0, w + L.mx_xq, rb / 2, perm_token, NvS, w + L.mx_xperm, nullptr, nullptr, st, pdl());
     } else if (nat1) {
@@ -459,9 +480,9 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g1.out = act;
     g1.err = err;
     if (fmt == MOE_W_MXFP4) {
-        g1.mx8 = true;
+        g1.mx8 = terms;
         g1.x = w + L.mx_xperm;
-        g1.x_stride = mx8_rec_bytes(H);
+        g1.x_stride = mx8_rec_bytes(H, terms);
         g1.tscale = nullptr;
     }
     if (nat1) {
@@ -502,8 +523,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     const int rb2 = nvf4_rec_bytes(I);
     if (row_pass) {
         if (fmt == MOE_W_MXFP4) {
-            e = launch_quant_mx8(act, true, NvS, I, reinterpret_cast<uint8_t*>(w + L.mx_act), mx8_rec_bytes(I), st,
-                                 pdl());
+            const int rb = mx8_rec_bytes(I, terms), Kp = mx8_kpad(I);
+            uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_act);
+            e = launch_quant_mx8(act, true, NvS, I, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr,
+                                 rec + terms * Kp, rb, rb, st, pdl());
         } else if (nat2) {
             uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.act_rec);
             e = launch_quant_nvfp4(act, true, NvS, I, rec, rb2, rec + I / 2, rb2, act2_scale, nullptr, st, pdl());
@@ -540,8 +563,8 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.out_kind = OUT_F32;
     g2.err = err;
     if (fmt == MOE_W_MXFP4) {
-        g2.mx8 = true;
-        g2.x_stride = mx8_rec_bytes(I);
+        g2.mx8 = terms;
+        g2.x_stride = mx8_rec_bytes(I, terms);
     }
     if (nat2) {
         g2.nvf4 = true;

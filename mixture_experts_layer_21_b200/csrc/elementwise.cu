@@ -235,30 +235,34 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
     pdl_launch();
 }
 
-// ----------------------------------------------------------------- MXFP8 hi/lo staging
-// Activation rows for the MXFP4-weight GEMM, whose tensor cores take e4m3 activations
-// with one e8m0 scale per 32 values. Each 32-value block b of a row gets the smallest
-// power of two 2^e with amax_b <= 448 * 2^e, then y = v * 2^-e (exact),
-// hi = e4m3_rne(y) and lo = e4m3_rne(y - hi) (the difference is exact in fp32), so
-// v = (hi + lo) * 2^e to within 2^-8 relative (plus 2^(e-10) absolute for values far
-// below the block's max). One warp per row, one 32-value block per lane and step;
-// blocks past K (up to the padded Kp) are zero.
-__device__ __forceinline__ int mx8_block_exp(float amax) {
+// ----------------------------------------------------------------- MXFP8 activations
+// Activation rows for the MXFP4-weight GEMM, whose tensor cores take e4m3 activations with
+// one e8m0 scale per 32 values. Two forms:
+//   hi/lo (bf16 activations): each 32-value block b gets the smallest power of two 2^e
+//     with amax_b <= 448 * 2^e, then y = v * 2^-e (exact), hi = e4m3_rne(y) and
+//     lo = e4m3_rne(y - hi) (the difference is exact in fp32), so v = (hi + lo) * 2^e to
+//     within 1.07 * 2^-8 |v| + 2^(e-10).
+//   one term (dynamic MXFP8, the OCP MX v1.0 conversion): 2^e = 2^(floor(log2 amax_b) - 8)
+//     and q = e4m3_rne_satfinite(v * 2^-e) (saturating at 448).
+// One warp per row, one 32-value block per lane and step; blocks past K (up to Kp) are zero.
+__device__ __forceinline__ int mx8_block_exp(float amax, bool two) {
     if (!(amax > 0.0f)) return -127;
     int ex;
     const float m = frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
-    const int e = m <= 0.875f ? ex - 9 : ex - 8;  // 448 * 2^(ex-9) = 0.875 * 2^ex
+    // hi/lo: 448 * 2^(ex-9) = 0.875 * 2^ex; one term: floor(log2 amax) - 8 = ex - 9
+    const int e = (two && m > 0.875f) ? ex - 8 : ex - 9;
     return max(-127, min(127, e));
 }
 
-template <bool IN_F32>
+template <bool IN_F32, bool TWO>
 __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__ in, int R, int K, int Kp,
-                                                        uint8_t* __restrict__ rec, int rec_stride) {
+                                                        uint8_t* __restrict__ hi_out, uint8_t* __restrict__ lo_out,
+                                                        uint8_t* __restrict__ sc_out, int code_stride,
+                                                        int sc_stride) {
     pdl_wait();
     const int r = blockIdx.x * 8 + warp_id();
     const int lane = lane_id();
     if (r < R) {
-        uint8_t* row = rec + (size_t)r * rec_stride;
         for (int b = lane; b < Kp / 32; b += 32) {
             uint32_t hi[8] = {0, 0, 0, 0, 0, 0, 0, 0}, lo[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             int e = -127;
@@ -269,37 +273,47 @@ __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i >> 4][i & 15]));
-                e = mx8_block_exp(amax);
+                e = mx8_block_exp(amax, TWO);
                 // 2^-e as a normal float: finite inputs give e <= 120 (amax < 2^128)
                 const float inv = __int_as_float((127 - max(e, -126)) << 23) * (e < -126 ? 2.0f : 1.0f);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float y = v[i >> 4][i & 15] * inv;
                     const uint8_t h = cvt_e4m3(y);
-                    const uint8_t l = cvt_e4m3(y - e4m3_to_f32(h));
                     hi[i >> 2] |= (uint32_t)h << (8 * (i & 3));
-                    lo[i >> 2] |= (uint32_t)l << (8 * (i & 3));
+                    if (TWO) lo[i >> 2] |= (uint32_t)cvt_e4m3(y - e4m3_to_f32(h)) << (8 * (i & 3));
                 }
             }
-            uint4* ph = reinterpret_cast<uint4*>(row + b * 32);
-            uint4* pl = reinterpret_cast<uint4*>(row + Kp + b * 32);
+            uint4* ph = reinterpret_cast<uint4*>(hi_out + (size_t)r * code_stride + b * 32);
             ph[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             ph[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-            pl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            pl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-            row[2 * Kp + b] = (uint8_t)(e + 127);
+            if (TWO) {
+                uint4* pl = reinterpret_cast<uint4*>(lo_out + (size_t)r * code_stride + b * 32);
+                pl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                pl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            }
+            sc_out[(size_t)r * sc_stride + b] = (uint8_t)(e + 127);
         }
     }
     pdl_launch();
 }
 
-cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, uint8_t* rec, int rec_stride,
-                             cudaStream_t st, bool pdl) {
+cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, int Kp, bool two, uint8_t* hi, uint8_t* lo,
+                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl) {
     if (R <= 0) return cudaSuccess;
-    const int Kp = mx8_kpad(K);
     dim3 grid((R + 7) / 8), block(256);
-    if (in_f32) return launch_k(quant_mx8_kernel<true>, grid, block, 0, st, pdl, in, R, K, Kp, rec, rec_stride);
-    return launch_k(quant_mx8_kernel<false>, grid, block, 0, st, pdl, in, R, K, Kp, rec, rec_stride);
+    if (two) {
+        if (in_f32)
+            return launch_k(quant_mx8_kernel<true, true>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
+                            code_stride, sc_stride);
+        return launch_k(quant_mx8_kernel<false, true>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
+                        code_stride, sc_stride);
+    }
+    if (in_f32)
+        return launch_k(quant_mx8_kernel<true, false>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
+                        code_stride, sc_stride);
+    return launch_k(quant_mx8_kernel<false, false>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc, code_stride,
+                    sc_stride);
 }
 
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,

@@ -1033,27 +1033,28 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
 
 // ------------------------------------------------------------------ MXFP4 x MXFP8 kernel
 
-template <int BT, bool DUAL>
+template <int BT, bool DUAL, bool TWO>
 struct Mx8Cfg {
     static constexpr int NB = DUAL ? 2 : 1;
+    // TWO: the activations are two e4m3 terms (hi/lo staging of bf16); else one (MXFP8).
     // The hi and lo token rows sit one after the other in shared memory, so while the
     // accumulators fit, one MMA of N = 2*BT covers both terms (MERGE): half the MMAs, and
     // the weight tile is read once for both. Its two column halves are partial sums the
     // epilogue adds. Otherwise (two 128-token tiles) each term is its own MMA.
-    static constexpr bool MERGE = NB * 2 * BT <= 256;
+    static constexpr bool MERGE = TWO && NB * 2 * BT <= 256;
+    static constexpr int TERMS = MERGE ? 2 : 1;            // partials one MMA writes side by side
     // A thread issues a block-scaled MMA about every 145 cycles, so narrow tiles split each
     // stage's four K steps between two issuers with their own partial sums where TMEM allows.
-    static constexpr int KSPLIT = (MERGE && 2 * NB * 4 * BT <= 256) ? 2 : 1;
-    static constexpr int TERMS = MERGE ? 2 : 1;            // partials one MMA writes side by side
+    static constexpr int KSPLIT = NB * TERMS * 2 * BT <= 128 ? 2 : 1;
     static constexpr int NPART = TERMS * KSPLIT;
     static constexpr int NI = NB * KSPLIT;                 // issuer i: matrix i % NB, K half i / NB
-    static constexpr int N_MMA = MERGE ? 2 * BT : BT;
+    static constexpr int N_MMA = TERMS * BT;
     static constexpr int A_BYTES = kTileN * kMx8StageK;   // 128 rows x 128 e2m1, a byte each in smem
     static constexpr int A_TX = A_BYTES / 2;              // what the 4-bit load counts: the packed bytes
     static constexpr int B_BYTES = BT * kMx8StageK;       // one e4m3 term
     static constexpr int BH_OFF = NB * A_BYTES;
     static constexpr int BL_OFF = BH_OFF + B_BYTES;
-    static constexpr int SFA_OFF = BL_OFF + B_BYTES;       // one 512-byte block per matrix
+    static constexpr int SFA_OFF = BH_OFF + (TWO ? 2 : 1) * B_BYTES;  // one 512-byte block per matrix
     static constexpr int SFR_OFF = SFA_OFF + NB * 512;     // token scales as loaded: BT x 16 bytes
     static constexpr int SFR_BYTES = BT * 16;
     static constexpr int SFB_OFF = SFR_OFF + (SFR_BYTES < 128 ? 128 : SFR_BYTES);
@@ -1076,6 +1077,7 @@ struct Mx8Cfg {
     static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128, "token tile");
     static_assert(BH_OFF % 1024 == 0 && BL_OFF % 1024 == 0 && SFR_OFF % 128 == 0 && SFB_OFF % 128 == 0,
                   "operand alignment");
+    static_assert(KSPLIT == 1 || MERGE || !TWO, "split K steps only with merged or single terms");
 };
 
 // The token tile's scales arrive as BT rows of 16 bytes covering 512 K values; word w of
@@ -1102,12 +1104,12 @@ __device__ __forceinline__ void build_sfb_block_mx8(const uint8_t* raw, uint8_t*
 // e8m0 scale per 32 values; the tensor cores apply both scales. Warp roles: 0 producer,
 // 1..NI MMA issuers, then 4 epilogue warps, then the scale warp (token scales into copy
 // blocks, scale-factor copies into the stage's TMEM slot).
-template <int BT, bool DUAL, int OUT>
-__global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
+template <int BT, bool DUAL, bool TWO, int OUT>
+__global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sf,
                             const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                             const GemmArgs a, int Kp) {
-    using C = Mx8Cfg<BT, DUAL>;
+    using C = Mx8Cfg<BT, DUAL, TWO>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
@@ -1170,7 +1172,8 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * (C::A_TX + 512) + 2 * C::B_BYTES + C::SFR_BYTES);
+                    mbar_arrive_expect_tx(&ctl->full[s],
+                                          C::NB * (C::A_TX + 512) + (TWO ? 2 : 1) * C::B_BYTES + C::SFR_BYTES);
                     tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g);
                     bulk_load(sfA(s, 0), a.ks0 + (blk0 + kb) * 512, 512, &ctl->full[s]);
                     if (DUAL) {
@@ -1178,7 +1181,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                         bulk_load(sfA(s, 1), a.ks1 + (blk0 + kb) * 512, 512, &ctl->full[s]);
                     }
                     tma_load_2d(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0);
-                    tma_load_2d(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0);
+                    if (TWO) tma_load_2d(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0);
                     tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], (kb >> 2) * 16, row0);
                     issued_mask |= 1u << s;
                     issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -1224,7 +1227,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL>::THREADS, 1)
                         const int kk = kh * KPI + j;
                         const uint64_t adesc = sw128_kmajor_desc(aa + 32 * kk);
                         const uint32_t id = (uint32_t)kk, idb = id << 30;
-                        if (C::MERGE) {  // hi and lo rows in one MMA: partials at d and d + BT
+                        if (C::MERGE || !TWO) {  // one MMA; merged: hi and lo partials at d and d + BT
                             mma_mx8_ss(d, adesc, sw128_kmajor_desc(smem_u32(opB(s, 0)) + 32 * kk),
                                        idesc_mx8(kTileN, C::N_MMA, id), sfa | idb, sfb | idb, (kb | j) != 0);
                         } else {
@@ -1537,11 +1540,11 @@ cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool
     }
 }
 
-template <int BT, bool DUAL, int OUT>
+template <int BT, bool DUAL, bool TWO, int OUT>
 cudaError_t run_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
                     const CUtensorMap& t0, const CUtensorMap& t1, int Kp, cudaStream_t st, bool pdl) {
-    using C = Mx8Cfg<BT, DUAL>;
-    auto kern = grouped_gemm_mx8_kernel<BT, DUAL, OUT>;
+    using C = Mx8Cfg<BT, DUAL, TWO>;
+    auto kern = grouped_gemm_mx8_kernel<BT, DUAL, TWO, OUT>;
     static int done[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
@@ -1549,15 +1552,24 @@ cudaError_t run_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMa
                     t1, args, Kp);
 }
 
+template <int BT, bool TWO>
+cudaError_t dispatch_mx8_terms(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx,
+                               const CUtensorMap& tsf, const CUtensorMap& t0, const CUtensorMap& t1, int Kp,
+                               cudaStream_t st, bool pdl) {
+    if (p.dual) {
+        if (p.out_kind != OUT_F32) return cudaErrorInvalidValue;
+        return run_mx8<BT, true, TWO, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    }
+    if (p.out_kind == OUT_F32) return run_mx8<BT, false, TWO, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    if (!TWO) return cudaErrorInvalidValue;  // the standalone bf16-output GEMM stages hi/lo
+    return run_mx8<BT, false, TWO, OUT_BF16>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+}
+
 template <int BT>
 cudaError_t dispatch_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
                          const CUtensorMap& t0, const CUtensorMap& t1, int Kp, cudaStream_t st, bool pdl) {
-    if (p.dual) {
-        if (p.out_kind != OUT_F32) return cudaErrorInvalidValue;
-        return run_mx8<BT, true, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
-    }
-    if (p.out_kind == OUT_F32) return run_mx8<BT, false, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
-    return run_mx8<BT, false, OUT_BF16>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    if (p.mx8 == 1) return dispatch_mx8_terms<BT, false>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    return dispatch_mx8_terms<BT, true>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
 }
 
 // The MXFP4 x MXFP8 GEMM; token tile as for the NVFP4 one.
@@ -1575,8 +1587,10 @@ cudaError_t launch_mx8(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool 
     const uint8_t* rec = static_cast<const uint8_t*>(p.x);
     CUtensorMap tx, tsf, t0, t1;
     memset(&t1, 0, sizeof(t1));
-    if (!make_map_u8(&tx, rec, 2 * (uint64_t)Kp, p.M_alloc, p.x_stride, kMx8StageK, bt, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_u8(&tsf, rec + 2 * (size_t)Kp, mx8_scale_bytes(p.K), p.M_alloc, p.x_stride, 16, bt,
+    const int terms = p.mx8 == 1 ? 1 : 2;
+    if (!make_map_u8(&tx, rec, (uint64_t)terms * Kp, p.M_alloc, p.x_stride, kMx8StageK, bt,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_u8(&tsf, rec + (size_t)terms * Kp, mx8_scale_bytes(p.K), p.M_alloc, p.x_stride, 16, bt,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_w_u4(&t0, p.kdata0, Kp, p.N, p.G) || (p.dual && !make_map_w_u4(&t1, p.kdata1, Kp, p.N, p.G)))
         return cudaErrorInvalidValue;

@@ -55,10 +55,12 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, cons
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T,
                                int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
-// Rows [R, K] (bf16 or fp32, K % 32 == 0) -> MXFP8 hi/lo records of mx8_rec_bytes(K)
-// bytes, rec_stride bytes apart.
-cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, uint8_t* rec, int rec_stride,
-                             cudaStream_t st, bool pdl);
+// Rows [R, K] (bf16 or fp32, K % 32 == 0) -> e4m3 codes with one e8m0 scale per 32 values,
+// Kp = mx8_kpad(K) codes per row (zero past K). two: hi and lo terms, scale chosen so the
+// block max stays <= 448 (lo != nullptr); else one term with the OCP MX MXFP8 scale.
+// Codes rows are code_stride bytes apart, scale rows sc_stride.
+cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, int Kp, bool two, uint8_t* hi, uint8_t* lo,
+                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl);
 // codes / sb rows are codes_stride / sb_stride bytes apart (K/2 and K/16 when dense).
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
                                uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl);
@@ -102,9 +104,10 @@ struct GemmProblem {
     int x_stride;
     const void* xsf;
     int xsf_stride;
-    // MXFP4 weights (mx8): x = MXFP8 hi/lo records (x_stride bytes apart, mx8_rec_bytes(K)
-    // each), kdata0/1 = the padded codes, kscale0/1 = the scale blocks.
-    bool mx8;
+    // MXFP4 weights (mx8 = number of e4m3 terms per activation: 2 = hi/lo staging of bf16,
+    // 1 = MXFP8 activations): x = records of mx8 * Kp codes then the scales (x_stride bytes
+    // apart), kdata0/1 = the padded codes, kscale0/1 = the scale blocks.
+    int mx8;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
 int choose_token_tile(long long NvS, int G, bool wide_ok);
@@ -138,7 +141,9 @@ constexpr int kNvf4TileBytes = kNvf4CodeBytes + kNvf4SfBytes;  // 18432
 constexpr int kMx8StageK = 128;
 inline int mx8_kpad(int K) { return (K + kMx8StageK - 1) / kMx8StageK * kMx8StageK; }
 inline int mx8_scale_bytes(int K) { return (mx8_kpad(K) / 32 + 15) / 16 * 16; }
-inline int mx8_rec_bytes(int K) { return 2 * mx8_kpad(K) + mx8_scale_bytes(K); }
+inline int mx8_rec_bytes(int K, int terms = 2) { return terms * mx8_kpad(K) + mx8_scale_bytes(K); }
+// W4A8 (dynamic MXFP8 activations): one e4m3 term per value instead of hi/lo, with the
+// OCP MX scale 2^(floor(log2 amax) - 8); records of mx8_rec_bytes(K, 1) bytes.
 
 // ---------------------------------------------------------------- device info
 int num_sms();

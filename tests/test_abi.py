@@ -117,6 +117,9 @@ def _fwd(**kw):
     (dict(fmt=1), NOT_PREP),                        # FP4 weights not prepared
     (dict(fmt=1, H=48, kdata=16), ALIGN),           # MXFP4 needs K % 32
     (dict(aq=1), UNSUP),                            # dynamic NVFP4 activations need NVFP4 weights
+    (dict(aq=2), UNSUP),                            # dynamic MXFP8 activations need MXFP4 weights
+    (dict(fmt=2, aq=2, kdata=16), UNSUP),
+    (dict(aq=3), INVALID),                          # no such activation quantisation
     (dict(H=72, I=128), ALIGN),                     # H % 16
     (dict(B=2), INVALID),                           # replicas without replica_src
     (dict(E=1100, topk=2), UNSUP),
@@ -151,6 +154,15 @@ def test_grouped_gemm_and_misc_validation():
     assert L.moe_prepare_weights(ctypes.byref(wb), None, 0, None) == 0                   # BF16: no-op
     wm = _w(1, 4, 128, 48)
     assert L.moe_prepare_weights(ctypes.byref(wm), 16, 1 << 20, None) == ALIGN
+
+
+def test_quantize_mxfp8_validation():
+    f = L.moe_quantize_mxfp8
+    assert f(16, 0, 4, 48, 16, 16, None) == ALIGN                 # K % 32
+    assert f(16, 0, 0, 64, 16, 16, None) == 0                     # no rows: nothing launched
+    assert f(None, 0, 4, 64, 16, 16, None) == INVALID
+    assert f(16, 0, 4, 64, 8, 16, None) == ALIGN                  # codes not 16-byte aligned
+    assert f(16, 0, -1, 64, 16, 16, None) == INVALID
 
 
 def test_grouped_gemm_nvfp4_validation():

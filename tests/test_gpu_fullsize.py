@@ -19,7 +19,8 @@ from tests.parity import FP4_REL_L2, check_bf16, rel_l2, to_dev
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-FULL = ["mixtral_prefill", "deepseek_decode", "deepseek_prefill", "mxfp4_decode", "mxfp4_prefill", "nvfp4"]
+FULL = ["mixtral_prefill", "deepseek_decode", "deepseek_prefill", "mxfp4_decode", "mxfp4_prefill", "nvfp4",
+        "mxfp4_w4a8_decode", "mxfp4_w4a8_prefill"]
 
 
 @functools.lru_cache(maxsize=2)

@@ -267,6 +267,24 @@ def test_quantize_nvfp4_bitexact(lib, dtype):
     assert np.array_equal(deq.cpu().double().numpy(), ref_deq)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantize_mxfp8_bitexact(lib, dtype):
+    R, K = 37, 2880
+    x = W.gen_rows(R, K, seed=11, dtype=torch.float32)
+    x[1] *= 1e-3
+    x[2, 64:96] = 0.0                          # a zero block
+    x[3] = 0.0                                 # a zero row
+    x[4, 100] = 75.0                           # an outlier
+    x[5, :32] = torch.linspace(-1, 1, 32) * 15.2   # saturates at 448 * 2^-5
+    x[6, :32] = 2.0 ** 5                       # a power of two
+    x = x.to(dtype)
+    codes, scales = lib.moe_quantize_mxfp8(to_dev(x))
+    torch.cuda.synchronize()
+    rc, rs = O.mxfp8_quantize_rows(x.float().numpy())
+    assert np.array_equal(scales.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
 # ------------------------------------------------------------------ the fused layer, small
 
 SMALL = {
@@ -281,6 +299,11 @@ SMALL = {
     "nvfp4_mixed": W.MoEConfig("nvfp4_mixed", T=33, H=272, I=512, E=8, topk=4, wfmt="nvfp4", act_quant=1),
     # neither K a multiple of 256: both staged in f16
     "nvfp4_f16": W.MoEConfig("nvfp4_f16", T=40, H=272, I=304, E=8, topk=2, wfmt="nvfp4", act_quant=1),
+    # W4A8: MXFP4 weights with dynamic MXFP8 activations (K padded to 128 in both GEMMs)
+    "mxfp4_w4a8": W.MoEConfig("mxfp4_w4a8", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4",
+                              act_quant=2),
+    "mxfp4_w4a8_silu": W.MoEConfig("mxfp4_w4a8_silu", T=300, H=192, I=256, E=8, topk=2, wfmt="mxfp4",
+                                   act_quant=2),
 }
 
 
