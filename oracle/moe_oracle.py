@@ -184,6 +184,60 @@ def route_topk(logits, topk: int):
     return ids.astype(np.int32), w
 
 
+def route_topk_grouped(logits, topk: int, n_group: int, topk_group: int, bias=None,
+                       routed_scaling_factor: float = 1.0):
+    """DeepSeekV3 routing: group-limited top-k on sigmoid scores with a selection bias.
+
+    The TRTLLM MXFP4 page lists ``RoutingMethodType.DeepSeekV3`` among its routing methods
+    and passes ``n_group``, ``topk_group``, ``routing_bias=e_score_correction_bias`` and
+    ``routed_scaling_factor`` to the kernel [trtllm: _supports_routing_method, apply]; it does
+    not spell the method out. Reading taken: the published DeepSeek-V3 routing.
+
+      s_e = sigmoid(l_e);  c_e = s_e + bias_e          (the bias steers selection only)
+      the E experts form n_group consecutive groups of E/n_group; a group's score is the
+      sum of its two largest c (its one c when a group has a single expert)
+      keep the topk_group groups of largest score (ties to the lower group id)
+      among their experts take the topk of largest c (ties to the lower id), in that order
+      w_j = routed_scaling_factor * s_j / sum over the chosen s
+
+    Every decision is taken in fp64 (so is the CUDA kernel's).
+    Returns ``ids [T,k] int32`` (in selection order) and ``w [T,k]`` fp64.
+    """
+    L = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    T, E = L.shape
+    if n_group < 1 or E % n_group or not (1 <= topk_group <= n_group):
+        raise ValueError("need E % n_group == 0 and 1 <= topk_group <= n_group")
+    gs = E // n_group
+    if not (1 <= topk <= topk_group * gs):
+        raise ValueError("need 1 <= topk <= topk_group * E / n_group")
+    b = np.zeros(E) if bias is None else np.asarray(bias, dtype=np.float32).astype(np.float64)
+    if T == 0:
+        return np.zeros((0, topk), np.int32), np.zeros((0, topk), np.float64)
+    s = 1.0 / (1.0 + np.exp(-L))
+    c = s + b[None, :]
+    top = -np.sort(-c.reshape(T, n_group, gs), axis=2)           # descending within each group
+    gscore = top[:, :, 0] + (top[:, :, 1] if gs >= 2 else 0.0)
+    gid = np.broadcast_to(np.arange(n_group), (T, n_group))
+    gorder = np.lexsort((gid, -gscore), axis=-1)[:, :topk_group]
+    keep = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(keep, gorder, True, axis=1)
+    allowed = np.repeat(keep, gs, axis=1)
+    eid = np.broadcast_to(np.arange(E), (T, E))
+    key = np.where(allowed, -c, np.inf)
+    ids = np.lexsort((eid, key), axis=-1)[:, :topk]
+    sel = np.take_along_axis(s, ids, axis=1)
+    w = routed_scaling_factor * sel / sel.sum(axis=1, keepdims=True)
+    return ids.astype(np.int32), w
+
+
+def route(cfg, logits, bias=None):
+    """The routing method a workload names: "renormalize" (``route_topk``) or "deepseek_v3"
+    (``route_topk_grouped`` with the workload's n_group, topk_group and scaling factor)."""
+    if getattr(cfg, "routing", "renormalize") == "deepseek_v3":
+        return route_topk_grouped(logits, cfg.topk, cfg.n_group, cfg.topk_group, bias, cfg.routed_scaling_factor)
+    return route_topk(logits, cfg.topk)
+
+
 # --------------------------------------------------------------------------------------
 # S2 permutation into expert-contiguous segments
 # --------------------------------------------------------------------------------------
@@ -410,12 +464,13 @@ def combine(y, inv_perm, topk_w=None):
 # --------------------------------------------------------------------------------------
 
 def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
-                tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False):
+                tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False, routing_bias=None):
     """The fused expert layer: route -> permute -> gate/up grouped GEMMs -> activation times
     route weight -> down grouped GEMM -> combine [moonep: module docstring and apply;
     trtllm: _invoke_kernel; fi_ep: apply].
 
-    ``cfg`` supplies E, B, topk, act, situ_alpha, situ_beta and act_quant. With act_quant = 1,
+    ``cfg`` supplies E, B, topk, act, situ_alpha, situ_beta, act_quant and the routing method
+    (``route``; ``routing_bias`` is the DeepSeekV3 method's selection bias). With act_quant = 1,
     x (in token order) and every activation row are NVFP4-quantised (``nvfp4_quantize_rows``)
     before their GEMM; with act_quant = 2 they are MXFP8-quantised (``mxfp8_quantize_rows``). ``tokens`` restricts the expert maths to the rows those tokens need
     (routing and permutation are always computed in full). With ``apply_topk_in_fc1`` false
@@ -424,7 +479,7 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     Returns a dict: ids, w, row, cu_seqlens, perm_token, perm_k, perm_w, inv_perm, tokens and
     out (fp64 ``[len(tokens), H]``); with ``keep``, also xq (codes/sb/s), h and y rows.
     """
-    ids, w = route_topk(logits, cfg.topk)
+    ids, w = route(cfg, logits, routing_bias)
     perm = assign_rows(ids, cfg.E, cfg.B, replica_src)
     T, k = ids.shape
     inv = perm["inv_perm"]

@@ -6,6 +6,7 @@ the grouped GEMM against pure-Python dot products; activations against closed fo
 limits; the whole layer against a per-token loop with no permutation and against a dense
 SwiGLU MLP; the NVFP4 activation quantiser against a brute-force nearest-grid-point search.
 """
+import itertools
 import math
 import os
 
@@ -156,6 +157,78 @@ def _perm_case(T, E, k, B, used, seed):
     if B:
         src[:used] = torch.randperm(E, generator=g)[:used].numpy()
     return ids, w, src
+
+
+def _grouped_brute(logits, bias, k, n_group, topk_group, scale):
+    """DeepSeekV3 routing by exhaustion: the group subset of size topk_group with the largest
+    total group score (ties: the lexicographically smallest ids), then repeated argmax of
+    sigmoid + bias over its experts; weights from the plain sigmoid, pure Python."""
+    L = np.asarray(logits, np.float32).astype(np.float64)
+    b = np.asarray(bias, np.float32).astype(np.float64)
+    T, E = L.shape
+    gs = E // n_group
+    ids = np.zeros((T, k), np.int64)
+    w = np.zeros((T, k))
+    for t in range(T):
+        sg = [1.0 / (1.0 + math.exp(-L[t, e])) for e in range(E)]
+        c = [sg[e] + b[e] for e in range(E)]
+        gscore = []
+        for g in range(n_group):
+            vals = sorted(c[g * gs:(g + 1) * gs], reverse=True)
+            gscore.append(vals[0] + (vals[1] if gs >= 2 else 0.0))
+        best = None
+        for sub in itertools.combinations(range(n_group), topk_group):
+            tot = sum(gscore[g] for g in sub)
+            if best is None or tot > best[0]:
+                best = (tot, sub)
+        avail = [e for g in best[1] for e in range(g * gs, (g + 1) * gs)]
+        for j in range(k):
+            pick = avail[0]
+            for e in avail[1:]:
+                if c[e] > c[pick] or (c[e] == c[pick] and e < pick):
+                    pick = e
+            ids[t, j] = pick
+            avail.remove(pick)
+        tot = sum(sg[e] for e in ids[t])
+        w[t] = [scale * sg[e] / tot for e in ids[t]]
+    return ids, w
+
+
+@pytest.mark.parametrize("E,n_group,topk_group,k,ints", [(12, 4, 2, 3, False), (16, 4, 1, 4, False),
+                                                         (24, 6, 3, 5, True), (8, 8, 3, 3, False),
+                                                         (10, 1, 1, 4, False)])
+def test_grouped_routing_matches_bruteforce(E, n_group, topk_group, k, ints):
+    g = np.random.default_rng(E + k)
+    L = g.normal(0, 2, (7, E)).astype(np.float32)
+    if ints:
+        L = np.round(L).astype(np.float32)      # many ties
+    bias = (g.normal(0, 0.05, E)).astype(np.float32)
+    ids, w = O.route_topk_grouped(L, k, n_group, topk_group, bias, 2.5)
+    bi, bw = _grouped_brute(L, bias, k, n_group, topk_group, 2.5)
+    assert np.array_equal(ids, bi)
+    assert np.allclose(w, bw, rtol=1e-12, atol=0)
+
+
+def test_grouped_routing_reductions_and_invariants():
+    g = np.random.default_rng(3)
+    L = g.normal(0, 2, (50, 64)).astype(np.float32)
+    bias = g.normal(0, 0.05, 64).astype(np.float32)
+    # one group, no bias: sigmoid is monotone, so the choice is the plain top-k of the logits
+    ids, w = O.route_topk_grouped(L, 6, 1, 1, None, 1.0)
+    ref_ids, _ = O.route_topk(L, 6)
+    assert np.array_equal(ids, ref_ids)
+    s = 1.0 / (1.0 + np.exp(-np.take_along_axis(L.astype(np.float64), ids.astype(np.int64), 1)))
+    assert np.allclose(w, s / s.sum(1, keepdims=True), rtol=1e-12)
+    # groups: every choice lies in at most topk_group groups, weights sum to the scaling factor
+    ids, w = O.route_topk_grouped(L, 8, 8, 3, bias, 2.5)
+    assert all(len(set((r // 8).tolist())) <= 3 for r in ids)
+    assert np.allclose(w.sum(1), 2.5)
+    # a constant added to every bias moves every group score alike: the choice is unchanged
+    ids2, w2 = O.route_topk_grouped(L, 8, 8, 3, bias + np.float32(0.25), 2.5)
+    assert np.array_equal(ids, ids2) and np.allclose(w, w2, rtol=1e-12)
+    # all logits equal: the lowest groups, then the lowest ids
+    ids, _ = O.route_topk_grouped(np.zeros((2, 8), np.float32), 3, 4, 2, None, 1.0)
+    assert ids.tolist() == [[0, 1, 2], [0, 1, 2]]
 
 
 @pytest.mark.parametrize("T,E,k,B,used", [(16, 8, 2, 0, 0), (50, 8, 3, 4, 2), (64, 16, 4, 6, 6),
@@ -357,7 +430,11 @@ def test_mxfp8_quant_matches_bruteforce_and_special_cases():
 def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
     """Per token, per chosen expert, the expert MLP on that token alone: no permutation,
     own routing, pure-Python dot products."""
-    ids, w = _route_brute(inp.logits.numpy(), cfg.topk)
+    if cfg.routing == "deepseek_v3":
+        ids, w = _grouped_brute(inp.logits.numpy(), inp.extra["routing_bias"].numpy(), cfg.topk, cfg.n_group,
+                                cfg.topk_group, cfg.routed_scaling_factor)
+    else:
+        ids, w = _route_brute(inp.logits.numpy(), cfg.topk)
     x = O.to_f64(inp.x)
     if cfg.act_quant == 1:
         c, sb, s = O.nvfp4_quantize_rows(inp.x.float().numpy())
@@ -405,6 +482,8 @@ SMALL = {
                                act_quant=1),
     "mxfp4_w4a8": W.MoEConfig("mxfp4_w4a8", T=8, H=64, I=64, E=4, topk=2, act="situ", wfmt="mxfp4",
                               act_quant=2),
+    "grouped_routing": W.MoEConfig("grouped_routing", T=10, H=32, I=48, E=8, topk=3, routing="deepseek_v3",
+                                   n_group=4, topk_group=2, routed_scaling_factor=2.5, logit_std=2.0),
 }
 
 
@@ -412,8 +491,9 @@ SMALL = {
 def test_layer_matches_per_token_loop(name):
     cfg = SMALL[name]
     inp = W.gen_inputs(cfg)
+    bias = inp.extra.get("routing_bias")
     res = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(),
-                        inp.w_gate, inp.w_up, inp.w_down)
+                        inp.w_gate, inp.w_up, inp.w_down, routing_bias=None if bias is None else bias.numpy())
     ref = _layer_brute(cfg, inp)
     scale = np.max(np.abs(ref))
     if cfg.act_quant:

@@ -35,6 +35,7 @@ import torch
 _S_X, _S_LOGITS, _S_GATE, _S_UP, _S_DOWN, _S_REPLICA = 1, 2, 3, 4, 5, 6
 _S_GATE_SCALE, _S_UP_SCALE, _S_DOWN_SCALE = 7, 8, 9
 _S_GATE_ALPHA, _S_UP_ALPHA, _S_DOWN_ALPHA = 10, 11, 12
+_S_BIAS = 13
 
 WFMT_BF16, WFMT_MXFP4, WFMT_NVFP4 = "bf16", "mxfp4", "nvfp4"
 
@@ -56,6 +57,10 @@ class MoEConfig:
     situ_beta: float = 1.0     # SITU up cap    (activation_situ_linear_beta)
     wfmt: str = WFMT_BF16
     act_quant: int = 0         # 1 = dynamic NVFP4, 2 = dynamic MXFP8 quantisation of activations
+    routing: str = "renormalize"   # or "deepseek_v3": grouped top-k on sigmoid scores
+    n_group: int = 1
+    topk_group: int = 1
+    routed_scaling_factor: float = 1.0
     x_std: float = 1.0
     logit_std: float = 1.0
     w_std: float = 0.02
@@ -95,6 +100,10 @@ CONFIGS: dict[str, MoEConfig] = {
                                act="situ", wfmt=WFMT_MXFP4),
     "nvfp4": MoEConfig("nvfp4", T=1024, H=7168, I=2048, E=256, topk=8,
                        wfmt=WFMT_NVFP4, act_quant=1),
+    # DeepSeekV3 routing on the DeepSeek decode shape: 8 groups of 32, 4 kept, scaling 2.5
+    "deepseek_decode_grouped": MoEConfig("deepseek_decode_grouped", T=64, H=7168, I=2048, E=256, topk=8,
+                                         B=16, B_used=8, logit_std=2.0, routing="deepseek_v3", n_group=8,
+                                         topk_group=4, routed_scaling_factor=2.5),
     # the W4A8 mode of the MXFP4 experts: the MXFP4 shapes with dynamic MXFP8 activations
     "mxfp4_w4a8_decode": MoEConfig("mxfp4_w4a8_decode", T=32, H=2880, I=2880, E=128, topk=4,
                                    act="situ", wfmt=WFMT_MXFP4, act_quant=2),
@@ -117,6 +126,14 @@ def gen_logits(cfg: MoEConfig) -> torch.Tensor:
     """Router logits ``[T,E]`` fp32, N(0, logit_std^2)."""
     g = _gen(cfg, _S_LOGITS)
     return torch.randn(cfg.T, cfg.E, generator=g) * cfg.logit_std
+
+
+def gen_routing_bias(cfg: MoEConfig) -> torch.Tensor:
+    """Selection bias of the DeepSeekV3 routing (e_score_correction_bias) ``[E]`` fp32,
+    N(0, 0.05^2): of the order of the spread of sigmoid scores near 0.5, so it reorders
+    close candidates without deciding most choices."""
+    g = _gen(cfg, _S_BIAS)
+    return torch.randn(cfg.E, generator=g) * 0.05
 
 
 def gen_replica_src(cfg: MoEConfig) -> torch.Tensor:
@@ -229,7 +246,8 @@ def gen_weights(cfg: MoEConfig) -> tuple[WeightSet, WeightSet, WeightSet, torch.
 def gen_inputs(cfg: MoEConfig) -> MoEInputs:
     """All inputs of one workload, on the CPU."""
     wg, wu, wd, src = gen_weights(cfg)
-    return MoEInputs(cfg, gen_x(cfg), gen_logits(cfg), src, wg, wu, wd)
+    extra = {"routing_bias": gen_routing_bias(cfg)} if cfg.routing == "deepseek_v3" else {}
+    return MoEInputs(cfg, gen_x(cfg), gen_logits(cfg), src, wg, wu, wd, extra)
 
 
 def gen_grouped_gemm_case(M_alloc: int, seg_lens: list[int], N: int, K: int, seed: int = 0,
