@@ -104,6 +104,14 @@ def tensor_peak_ratio(cfg) -> tuple[float, str]:
     return 1.0, "= measured bf16"
 
 
+def routing_config(cfg) -> dict:
+    """The routing method in the config record (only when it is not the default)."""
+    if cfg.routing == "renormalize":
+        return {}
+    return {"routing": cfg.routing, "n_group": cfg.n_group, "topk_group": cfg.topk_group,
+            "routed_scaling_factor": cfg.routed_scaling_factor}
+
+
 def compute_dtype(cfg) -> str:
     """The operand types the grouped GEMMs' tensor cores multiply."""
     if cfg.wfmt == "bf16":
@@ -250,8 +258,9 @@ def cpu_threads() -> int:
 def oracle_sample(cfg, inp, tokens):
     from oracle import moe_oracle as O
     t0 = time.perf_counter()
+    bias = inp.extra.get("routing_bias")
     O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                  inp.w_down, tokens=tokens)
+                  inp.w_down, tokens=tokens, routing_bias=None if bias is None else bias.numpy())
     return time.perf_counter() - t0
 
 
@@ -278,9 +287,12 @@ def run_ours(args, cfg, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = W.gen_inputs(cfg)
     ws = [m.Weight.from_host(w, dev) for w in (inp.w_gate, inp.w_up, inp.w_down)]
+    bias = inp.extra.get("routing_bias")
     layer = m.MoEForward(*ws, cfg.E, cfg.topk, cfg.B,
                          inp.replica_src.to(dev) if cfg.B else None, cfg.act, cfg.situ_alpha,
-                         cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T)
+                         cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T, routing=cfg.routing,
+                         routing_bias=None if bias is None else bias.to(dev), n_group=cfg.n_group,
+                         topk_group=cfg.topk_group, routed_scaling_factor=cfg.routed_scaling_factor)
     x_d, l_d = inp.x.to(dev), inp.logits.to(dev)
     out_d = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -399,7 +411,7 @@ def run_ours(args, cfg, rank, world):
         "vs_baseline": None, "dtype": compute_dtype(cfg),
         "data": "synthetic (seeded; random weights of the workload's shapes)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
-                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant,
+                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg),
                    "parallelism": f"replicas x{world}",
                    "l2": f"no flush: weights touched per step {acc['weight_bytes_total'] / 1e9:.2f} GB "
                          f"> L2 {L2_BYTES / 2 ** 20:.0f} MiB",
@@ -439,7 +451,7 @@ def run_reference(args, cfg):
         "steps": K, "warmup": Wm, "ms_per_step": t / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
-                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant},
+                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg)},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{S} tokens per step of {cfg.T} (routing of all), fp64 NumPy"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -116,6 +116,24 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int topk,
                             int32_t* topk_ids, float* topk_w, moe_stream_t stream);
 
 /*
+ * S1 (DeepSeekV3) — group-limited top-k on sigmoid scores, the "DeepSeekV3" routing
+ * method of the TRTLLM MXFP4 page (_supports_routing_method; apply passes n_group,
+ * topk_group, routing_bias = e_score_correction_bias and routed_scaling_factor). The
+ * page names the method only; it is taken as the published DeepSeek-V3 routing:
+ *   s_e = sigmoid(l_e), c_e = s_e + bias_e (bias may be NULL = 0; it steers selection only);
+ *   the E experts form n_group consecutive groups; a group scores the sum of its two
+ *   largest c (its one c for groups of one); the topk_group best groups are kept, ties to
+ *   the lower group; the topk largest c among their experts are chosen, ties to the lower
+ *   id, in that order; topk_w = routed_scaling_factor * s_j / sum of the chosen s.
+ *   Decisions are taken in fp64.
+ *   logits fp32 [T,E]; bias fp32 [E] or NULL; topk_ids int32 / topk_w fp32 [T,topk] out.
+ * E % n_group, 1 <= topk_group <= n_group, 1 <= topk <= topk_group*E/n_group and a finite
+ * positive scaling factor, else INVALID_ARG; E > 512, n_group > 32 or topk > 32: UNSUPPORTED.
+ */
+moe_status_t moe_route_topk_grouped(const float* logits, const float* bias, int T, int E, int topk,
+                                    int n_group, int topk_group, float routed_scaling_factor,
+                                    int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+/*
  * S2 — permute into expert-contiguous segments (MoonEP page: module docstring
  * and MoonEPExperts.apply; cu_seqlens = cumsum of per-row lengths).
  *   topk_ids/topk_w [T,topk]; replica_src int32 [B] (source expert of each
@@ -302,6 +320,12 @@ typedef struct {
     float* topk_w_out;              /* optional */
     int32_t T_max;                  /* capacity the workspace was sized for */
     void* const* stage_events;      /* optional: MOE_FWD_STAGE_EVENTS cudaEvent_t */
+    /* routing: 0 = softmax -> top-k -> renormalise (moe_route_topk), 1 = DeepSeekV3
+     * (moe_route_topk_grouped with the four fields below; other values INVALID_ARG) */
+    int32_t routing;
+    const float* routing_bias;      /* [E] or NULL */
+    int32_t n_group, topk_group;
+    float routed_scaling_factor;
 } moe_forward_args_t;
 
 size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,

@@ -36,7 +36,7 @@ EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_wo
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
            "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc",
-           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8"]
+           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8", "moe_route_topk_grouped"]
 
 
 class MoEError(RuntimeError):
@@ -66,7 +66,12 @@ class moe_forward_args_t(ctypes.Structure):
                 ("act", moe_act_params_t), ("apply_topk_in_fc1", ctypes.c_int32),
                 ("act_quant", ctypes.c_int32), ("out", ctypes.c_void_p),
                 ("topk_ids_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
-                ("T_max", ctypes.c_int32), ("stage_events", ctypes.c_void_p)]
+                ("T_max", ctypes.c_int32), ("stage_events", ctypes.c_void_p),
+                ("routing", ctypes.c_int32), ("routing_bias", ctypes.c_void_p),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float)]
+
+ROUTING = {"renormalize": 0, "deepseek_v3": 1}
 
 MOE_FWD_STAGE_EVENTS = 7
 
@@ -91,6 +96,7 @@ _sig = {
     "moe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P]),
     "moe_grouped_gemm_nvfp4": (_I, [_P, _P, _P, _I, ctypes.POINTER(moe_weight_t), _P, _P, _P, _S, _P]),
     "moe_quantize_mxfp8": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_route_topk_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -185,6 +191,18 @@ def moe_route_topk(logits: torch.Tensor, topk: int, ids=None, w=None, stream=Non
     w = w if w is not None else torch.empty(T, topk, dtype=torch.float32, device=logits.device)
     _check(_lib.moe_route_topk(_ptr(logits), T, E, topk, _ptr(ids), _ptr(w), _stream(stream)),
            "moe_route_topk")
+    return ids, w
+
+
+def moe_route_topk_grouped(logits: torch.Tensor, topk: int, n_group: int, topk_group: int, bias=None,
+                           routed_scaling_factor: float = 1.0, ids=None, w=None, stream=None):
+    """DeepSeekV3 routing (grouped top-k on sigmoid scores, bias for selection only)."""
+    T, E = logits.shape
+    ids = ids if ids is not None else torch.empty(T, topk, dtype=torch.int32, device=logits.device)
+    w = w if w is not None else torch.empty(T, topk, dtype=torch.float32, device=logits.device)
+    _check(_lib.moe_route_topk_grouped(_ptr(logits), _ptr(bias), T, E, topk, n_group, topk_group,
+                                       routed_scaling_factor, _ptr(ids), _ptr(w), _stream(stream)),
+           "moe_route_topk_grouped")
     return ids, w
 
 
@@ -297,7 +315,9 @@ class MoEForward:
 
     def __init__(self, w_gate: Weight, w_up: Weight, w_down: Weight, E: int, topk: int, B: int = 0,
                  replica_src=None, act: str = "silu", situ_alpha=1.0, situ_beta=1.0,
-                 act_quant: int = 0, apply_topk_in_fc1: bool = True, T_max: int = 1):
+                 act_quant: int = 0, apply_topk_in_fc1: bool = True, T_max: int = 1,
+                 routing: str = "renormalize", routing_bias=None, n_group: int = 1, topk_group: int = 1,
+                 routed_scaling_factor: float = 1.0):
         for w in (w_gate, w_up, w_down):
             if w.fmt != "bf16" and w.prepared is None:
                 moe_prepare_weights(w)
@@ -312,6 +332,10 @@ class MoEForward:
         self.ws = forward_workspace(T_max, self.H, self.I, E, B, topk, w_gate.fmt, act_quant,
                                     w_gate.data.device)
         self.args = moe_forward_args_t()
+        self.args.routing = ROUTING[routing]
+        self.routing_bias = routing_bias
+        self.args.n_group, self.args.topk_group = n_group, topk_group
+        self.args.routed_scaling_factor = routed_scaling_factor
 
     def __call__(self, x, router_logits, out=None, topk_ids=None, topk_w=None, stream=None,
                  stage_events=None):
@@ -339,6 +363,7 @@ class MoEForward:
         a.out = _ptr(out)
         a.topk_ids_out, a.topk_w_out = _ptr(topk_ids), _ptr(topk_w)
         a.T_max = self.T_max
+        a.routing_bias = _ptr(self.routing_bias)
         _check(_lib.moe_forward(ctypes.byref(a), _ptr(self.ws), self.ws.numel(), _stream(stream)),
                "moe_forward")
         return out

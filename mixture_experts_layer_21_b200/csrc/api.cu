@@ -8,6 +8,10 @@
 
 namespace moe {
 size_t prepared_weight_bytes(const moe_weight_t* w);
+// DeepSeekV3 routing (route_permute.cu); E <= 512, E % n_group == 0, n_group <= 32,
+// topk_group <= n_group, topk <= min(32, topk_group * E / n_group), checked here.
+cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int topk, int n_group,
+                                 int topk_group, float scale, int32_t* ids, float* w, cudaStream_t st, bool pdl);
 moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaStream_t st);
 
 int num_sms() {
@@ -146,6 +150,33 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int topk, int32_t
     if (T == 0) return MOE_OK;
     if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_route_topk(logits, T, E, topk, topk_ids, topk_w, S(stream), false));
+}
+
+}  // extern "C"
+
+namespace {
+// Arguments of the DeepSeekV3 routing; MOE_OK when the kernel supports them.
+moe_status_t check_grouped(int E, int topk, int n_group, int topk_group, float scale) {
+    if (n_group < 1 || E % n_group || topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+    if (topk < 1 || topk > topk_group * (E / n_group)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (E > 512 || n_group > 32 || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_topk_grouped(const float* logits, const float* bias, int T, int E, int topk, int n_group,
+                                    int topk_group, float routed_scaling_factor, int32_t* topk_ids, float* topk_w,
+                                    moe_stream_t stream) {
+    if (T < 0 || E < 1) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = check_grouped(E, topk, n_group, topk_group, routed_scaling_factor);
+    if (s != MOE_OK) return s;
+    if (T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_route_grouped(logits, bias, T, E, topk, n_group, topk_group, routed_scaling_factor,
+                                            topk_ids, topk_w, S(stream), false));
 }
 
 size_t moe_permute_workspace_size(int T, int topk, int E, int B) {
@@ -358,6 +389,12 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (T > p->T_max) return MOE_ERR_INVALID_ARG;  // the workspace was sized for T_max tokens
     if (E > kMaxExperts || E + B > 1024 || k > kMaxTopk) return MOE_ERR_UNSUPPORTED;
     if (!act_ok(p->act)) return MOE_ERR_INVALID_ARG;
+    // routing: 0 = softmax -> top-k -> renormalise, 1 = DeepSeekV3 grouped top-k
+    if (p->routing != 0 && p->routing != 1) return MOE_ERR_INVALID_ARG;
+    if (p->routing == 1) {
+        const moe_status_t rs = check_grouped(E, k, p->n_group, p->topk_group, p->routed_scaling_factor);
+        if (rs != MOE_OK) return rs;
+    }
     const int G = E + B;
     const int fmt = p->w_gate.fmt;
     if (p->w_up.fmt != fmt || p->w_down.fmt != fmt) return MOE_ERR_UNSUPPORTED;
@@ -414,7 +451,11 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
 
     if (!mark(0)) return MOE_ERR_CUDA;
     // S1 route
-    e = launch_route_topk(p->router_logits, T, E, k, ids, tw, st, false);
+    if (p->routing == 1)
+        e = launch_route_grouped(p->router_logits, p->routing_bias, T, E, k, p->n_group, p->topk_group,
+                                 p->routed_scaling_factor, ids, tw, st, false);
+    else
+        e = launch_route_topk(p->router_logits, T, E, k, ids, tw, st, false);
     if (e != cudaSuccess || !mark(1)) return MOE_ERR_CUDA;
     // S2 permute
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,

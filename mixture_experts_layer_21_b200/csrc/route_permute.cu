@@ -90,6 +90,142 @@ cudaError_t launch_route_topk(const float* logits, int T, int E, int topk, int32
     return launch_k(route_topk_kernel<32>, grid, block, 0, st, pdl, logits, T, E, topk, ids, w);
 }
 
+// ----------------------------------------------------------------- S1 route, DeepSeekV3
+// Grouped top-k on sigmoid scores (the "DeepSeekV3" routing method of the TRTLLM MXFP4
+// page): s = sigmoid(l), c = s + bias; groups of E/n_group consecutive experts score the
+// sum of their two largest c; the topk_group best groups are kept (ties to the lower
+// group); the topk largest c among their experts are chosen (ties to the lower id), and
+// w = scale * s / sum of the chosen s. One warp per token; every decision in fp64.
+template <int EPL>  // experts per lane (E <= 32*EPL)
+__global__ void __launch_bounds__(256) route_grouped_kernel(const float* __restrict__ logits,
+                                                            const float* __restrict__ bias, int T, int E,
+                                                            int topk, int n_group, int topk_group, float scale,
+                                                            int32_t* __restrict__ ids, float* __restrict__ w) {
+    constexpr int NONE = 0x7fffffff;
+    pdl_wait();
+    const int lane = lane_id();
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
+    if (t < T) {
+        const int gs = E / n_group;
+        const double ninf = -(double)INFINITY;
+        double sc[EPL], c[EPL];
+        const float* row = logits + (size_t)t * E;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = i * 32 + lane;
+            sc[i] = 0.0;
+            c[i] = ninf;
+            if (e < E) {
+                sc[i] = 1.0 / (1.0 + exp(-(double)row[e]));
+                c[i] = sc[i] + (bias ? (double)bias[e] : 0.0);
+            }
+        }
+        // group scores: each group's two largest c, merged across the warp; lane g keeps group g's
+        double my_gs = ninf;
+        for (int g = 0; g < n_group; ++g) {
+            double a1 = ninf, a2 = ninf;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = i * 32 + lane;
+                if (e < E && e / gs == g) {
+                    if (c[i] > a1) {
+                        a2 = a1;
+                        a1 = c[i];
+                    } else if (c[i] > a2) {
+                        a2 = c[i];
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const double b1 = __shfl_xor_sync(0xffffffffu, a1, off);
+                const double b2 = __shfl_xor_sync(0xffffffffu, a2, off);
+                const double n2 = fmax(fmin(a1, b1), fmax(a2, b2));
+                a1 = fmax(a1, b1);
+                a2 = n2;
+            }
+            if (lane == g) my_gs = a1 + (gs >= 2 ? a2 : 0.0);
+        }
+        // the topk_group best groups
+        uint32_t keep = 0;
+        for (int j = 0; j < topk_group; ++j) {
+            double bv = my_gs;
+            int bg = (lane < n_group && !(keep >> lane & 1u)) ? lane : NONE;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+                if (og != NONE && (bg == NONE || ov > bv || (ov == bv && og < bg))) {
+                    bv = ov;
+                    bg = og;
+                }
+            }
+            keep |= 1u << bg;  // bg is valid: topk_group <= n_group
+        }
+        // the topk best experts of the kept groups
+        uint32_t taken = 0;  // bit i: entry i of this lane is chosen, absent or outside the kept groups
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = i * 32 + lane;
+            if (e >= E || !(keep >> (e / gs) & 1u)) taken |= 1u << i;
+        }
+        double my_s = 0.0;
+        int my_id = 0;
+        for (int j = 0; j < topk; ++j) {
+            double bv = 0.0, bs = 0.0;
+            int bid = NONE;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                if (!(taken >> i & 1u) && (bid == NONE || c[i] > bv)) {
+                    bv = c[i];
+                    bs = sc[i];
+                    bid = i * 32 + lane;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const double os = __shfl_xor_sync(0xffffffffu, bs, off);
+                const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+                if (oid != NONE && (bid == NONE || ov > bv || (ov == bv && oid < bid))) {
+                    bv = ov;
+                    bs = os;
+                    bid = oid;
+                }
+            }
+            if (bid != NONE && (bid & 31) == lane) taken |= 1u << (bid >> 5);
+            if (lane == j) {
+                my_s = bs;
+                my_id = bid;
+            }
+        }
+        double sum = lane < topk ? my_s : 0.0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane < topk) {
+            ids[(size_t)t * topk + lane] = my_id;
+            w[(size_t)t * topk + lane] = (float)((double)scale * my_s / sum);
+        }
+    }
+    pdl_launch();
+}
+
+cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int topk, int n_group,
+                                 int topk_group, float scale, int32_t* ids, float* w, cudaStream_t st, bool pdl) {
+    const int warps = 8;
+    dim3 grid((T + warps - 1) / warps), block(32 * warps);
+    const int epl = (E + 31) / 32;
+#define MOE_ROUTE_G(N)                                                                                            \
+    return launch_k(route_grouped_kernel<N>, grid, block, 0, st, pdl, logits, bias, T, E, topk, n_group, topk_group, \
+                    scale, ids, w)
+    if (epl <= 1) MOE_ROUTE_G(1);
+    if (epl <= 2) MOE_ROUTE_G(2);
+    if (epl <= 4) MOE_ROUTE_G(4);
+    if (epl <= 8) MOE_ROUTE_G(8);
+    MOE_ROUTE_G(16);
+#undef MOE_ROUTE_G
+}
+
 // ----------------------------------------------------------------- S2 permute
 // Token blocks of 256: thread i of block b owns token b*256+i.
 constexpr int kPermBlock = 256;

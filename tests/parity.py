@@ -74,3 +74,16 @@ def check_mx8(got, ref, bound, what=""):
     assert err.size == 0 or np.all(err <= lim), \
         f"{what}: max excess {np.max(err - lim):.3e} at {worst}: got {got[worst]} ref {ref[worst]}"
     return rel_l2(got, ref)
+
+
+def routing_kwargs(cfg, inp):
+    """MoEForward's routing arguments for a workload (the DeepSeekV3 method's bias on the GPU)."""
+    bias = inp.extra.get("routing_bias")
+    return dict(routing=cfg.routing, routing_bias=None if bias is None else to_dev(bias), n_group=cfg.n_group,
+                topk_group=cfg.topk_group, routed_scaling_factor=cfg.routed_scaling_factor)
+
+
+def oracle_bias(inp):
+    """The DeepSeekV3 selection bias for the oracle, or None."""
+    bias = inp.extra.get("routing_bias")
+    return None if bias is None else bias.numpy()

@@ -103,6 +103,9 @@ def _fwd(**kw):
     p.w_down = _w(d["fmt"], G, d["H"], d["I"], kdata=kd)
     p.act = m.moe_act_params_t(d["act"], d["sa"], d["sb"])
     p.act_quant = d["aq"]
+    p.routing = kw.get("routing", 0)
+    p.n_group, p.topk_group = kw.get("n_group", 1), kw.get("topk_group", 1)
+    p.routed_scaling_factor = kw.get("scale", 1.0)
     p.apply_topk_in_fc1 = 1
     nws = L.moe_forward_workspace_size(d["T_max"], d["H"], d["I"], d["E"], d["B"], d["topk"], d["fmt"], d["aq"])
     return p, nws
@@ -123,6 +126,9 @@ def _fwd(**kw):
     (dict(H=72, I=128), ALIGN),                     # H % 16
     (dict(B=2), INVALID),                           # replicas without replica_src
     (dict(E=1100, topk=2), UNSUP),
+    (dict(routing=2), INVALID),                     # no such routing method
+    (dict(routing=1, n_group=3), INVALID),          # E % n_group
+    (dict(routing=1, n_group=2, topk_group=1, scale=0.0), INVALID),
 ])
 def test_forward_validation(kw, expect):
     p, nws = _fwd(**kw)
@@ -154,6 +160,24 @@ def test_grouped_gemm_and_misc_validation():
     assert L.moe_prepare_weights(ctypes.byref(wb), None, 0, None) == 0                   # BF16: no-op
     wm = _w(1, 4, 128, 48)
     assert L.moe_prepare_weights(ctypes.byref(wm), 16, 1 << 20, None) == ALIGN
+
+
+def test_route_grouped_validation():
+    f = L.moe_route_topk_grouped
+    ok = dict(E=256, k=8, ng=8, tg=4, sc=2.5)
+    def call(**kw):
+        d = dict(ok, **kw)
+        return f(16, None, 4, d["E"], d["k"], d["ng"], d["tg"], ctypes.c_float(d["sc"]), 16, 16, None)
+    assert f(16, None, 0, 256, 8, 8, 4, ctypes.c_float(2.5), 16, 16, None) == 0    # no tokens
+    assert call(E=250) == INVALID                 # E % n_group
+    assert call(tg=9) == INVALID                  # topk_group > n_group
+    assert call(tg=0) == INVALID
+    assert call(k=129) == INVALID                 # more than the kept groups hold
+    assert call(sc=0.0) == INVALID
+    assert call(sc=float("nan")) == INVALID
+    assert call(E=1024, ng=8) == UNSUP            # E > 512
+    assert call(E=256, ng=64, tg=4) == UNSUP      # n_group > 32
+    assert f(None, None, 4, 256, 8, 8, 4, ctypes.c_float(2.5), 16, 16, None) == INVALID
 
 
 def test_quantize_mxfp8_validation():

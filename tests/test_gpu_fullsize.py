@@ -15,12 +15,12 @@ import torch
 
 import workloads as W
 from oracle import moe_oracle as O
-from tests.parity import FP4_REL_L2, check_bf16, rel_l2, to_dev
+from tests.parity import FP4_REL_L2, check_bf16, oracle_bias, rel_l2, routing_kwargs, to_dev
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 FULL = ["mixtral_prefill", "deepseek_decode", "deepseek_prefill", "mxfp4_decode", "mxfp4_prefill", "nvfp4",
-        "mxfp4_w4a8_decode", "mxfp4_w4a8_prefill"]
+        "mxfp4_w4a8_decode", "mxfp4_w4a8_prefill", "deepseek_decode_grouped"]
 
 
 @functools.lru_cache(maxsize=2)
@@ -32,7 +32,8 @@ def _weights(E, B, B_used, H, I, wfmt, seed):
 
 def _inputs(cfg):
     wg, wu, wd, src = _weights(cfg.E, cfg.B, cfg.B_used, cfg.H, cfg.I, cfg.wfmt, cfg.seed)
-    return W.MoEInputs(cfg, W.gen_x(cfg), W.gen_logits(cfg), src, wg, wu, wd)
+    extra = {"routing_bias": W.gen_routing_bias(cfg)} if cfg.routing == "deepseek_v3" else {}
+    return W.MoEInputs(cfg, W.gen_x(cfg), W.gen_logits(cfg), src, wg, wu, wd, extra)
 
 
 def _sample_tokens(cfg, perm, n_random=192, edge=24):
@@ -53,19 +54,20 @@ def test_fullsize_forward_matches_oracle(lib, name):
     inp = _inputs(cfg)
     weights = [lib.Weight.from_host(w) for w in (inp.w_gate, inp.w_up, inp.w_down)]
     layer = lib.MoEForward(*weights, cfg.E, cfg.topk, cfg.B, to_dev(inp.replica_src) if cfg.B else None,
-                           cfg.act, cfg.situ_alpha, cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T)
+                           cfg.act, cfg.situ_alpha, cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T,
+                           **routing_kwargs(cfg, inp))
     ids = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device="cuda")
     out = layer(to_dev(inp.x), to_dev(inp.logits), topk_ids=ids)
     torch.cuda.synchronize()
     assert layer.device_error() == 0
     del layer, weights
 
-    rids, _ = O.route_topk(inp.logits.numpy(), cfg.topk)
+    rids, _ = O.route(cfg, inp.logits.numpy(), oracle_bias(inp))
     assert np.array_equal(ids.cpu().numpy(), rids)
     perm = O.assign_rows(rids, cfg.E, cfg.B, inp.replica_src.numpy())
     toks = _sample_tokens(cfg, perm)
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, tokens=toks)
+                        inp.w_down, tokens=toks, routing_bias=oracle_bias(inp))
     got = out[torch.tensor(toks, device="cuda")].float().cpu().numpy()
     if cfg.wfmt == "bf16":
         check_bf16(got, ref["out"], what=name)

@@ -6,7 +6,8 @@ import torch
 
 import workloads as W
 from oracle import moe_oracle as O
-from tests.parity import FP4_REL_L2, check_bf16, check_mx8, mx8_staging_bound, rel_l2, to_dev
+from tests.parity import (FP4_REL_L2, check_bf16, check_mx8, mx8_staging_bound, oracle_bias, rel_l2,
+                          routing_kwargs, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,6 +32,23 @@ def test_route_topk_matches_oracle(lib, T, E, k, std, ints):
 
 
 # ------------------------------------------------------------------ S2 permutation
+
+@pytest.mark.parametrize("T,E,k,n_group,topk_group,bias,ints",
+                         [(64, 256, 8, 8, 4, True, False), (300, 24, 4, 6, 2, True, True),
+                          (37, 512, 8, 16, 3, False, False), (5, 32, 32, 2, 2, True, False),
+                          (9, 64, 6, 1, 1, True, False), (17, 96, 3, 32, 3, False, True)])
+def test_route_grouped_matches_oracle(lib, T, E, k, n_group, topk_group, bias, ints):
+    g = torch.Generator().manual_seed(T + E)
+    L = torch.randn(T, E, generator=g) * 2.0
+    if ints:
+        L = torch.round(L)                      # ties between experts and between groups
+    b = (torch.randn(E, generator=g) * 0.05) if bias else None
+    ids, w = lib.moe_route_topk_grouped(to_dev(L), k, n_group, topk_group, to_dev(b), 2.5)
+    torch.cuda.synchronize()
+    rids, rw = O.route_topk_grouped(L.numpy(), k, n_group, topk_group, None if b is None else b.numpy(), 2.5)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=2e-7, atol=1e-7)
+
 
 def _perm_inputs(T, E, k, B, used, seed, skew=None):
     g = torch.Generator().manual_seed(seed)
@@ -299,6 +317,10 @@ SMALL = {
     "nvfp4_mixed": W.MoEConfig("nvfp4_mixed", T=33, H=272, I=512, E=8, topk=4, wfmt="nvfp4", act_quant=1),
     # neither K a multiple of 256: both staged in f16
     "nvfp4_f16": W.MoEConfig("nvfp4_f16", T=40, H=272, I=304, E=8, topk=2, wfmt="nvfp4", act_quant=1),
+    # DeepSeekV3 grouped routing with replicas: 6 groups of 4, 2 kept, scaling 2.5
+    "grouped_routing": W.MoEConfig("grouped_routing", T=130, H=128, I=192, E=24, topk=4, B=4, B_used=3,
+                                   logit_std=2.0, routing="deepseek_v3", n_group=6, topk_group=2,
+                                   routed_scaling_factor=2.5),
     # W4A8: MXFP4 weights with dynamic MXFP8 activations (K padded to 128 in both GEMMs)
     "mxfp4_w4a8": W.MoEConfig("mxfp4_w4a8", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4",
                               act_quant=2),
@@ -311,7 +333,8 @@ def run_layer(lib, cfg, inp, apply_topk_in_fc1=True):
     dev = lambda ws: lib.Weight.from_host(ws)
     layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, cfg.topk, cfg.B,
                            to_dev(inp.replica_src) if cfg.B else None, cfg.act, cfg.situ_alpha,
-                           cfg.situ_beta, cfg.act_quant, apply_topk_in_fc1, T_max=cfg.T)
+                           cfg.situ_beta, cfg.act_quant, apply_topk_in_fc1, T_max=cfg.T,
+                           **routing_kwargs(cfg, inp))
     ids = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device="cuda")
     tw = torch.empty(cfg.T, cfg.topk, dtype=torch.float32, device="cuda")
     out = layer(to_dev(inp.x), to_dev(inp.logits), topk_ids=ids, topk_w=tw)
@@ -326,7 +349,7 @@ def test_forward_small_matches_oracle(lib, name):
     inp = W.gen_inputs(cfg)
     out, ids, tw, _ = run_layer(lib, cfg, inp)
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down)
+                        inp.w_down, routing_bias=oracle_bias(inp))
     assert np.array_equal(ids.cpu().numpy(), ref["ids"])
     if cfg.wfmt == "bf16":
         check_bf16(out, ref["out"], what=name)
