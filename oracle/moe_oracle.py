@@ -464,7 +464,8 @@ def combine(y, inv_perm, topk_w=None):
 # --------------------------------------------------------------------------------------
 
 def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
-                tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False, routing_bias=None):
+                tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False, routing_bias=None,
+                given_topk=None, apply_router_weight_on_input: bool = False):
     """The fused expert layer: route -> permute -> gate/up grouped GEMMs -> activation times
     route weight -> down grouped GEMM -> combine [moonep: module docstring and apply;
     trtllm: _invoke_kernel; fi_ep: apply].
@@ -476,10 +477,23 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     (routing and permutation are always computed in full). With ``apply_topk_in_fc1`` false
     the route weight moves from the activation to the combine [fi_ep: apply_topk_in_fc1].
 
+    ``given_topk = (ids, w)`` skips the routing: the experts and route weights are given, as
+    in the modular and routed kernels that take a computed top-k [fi_ep: apply, topk_ids and
+    topk_weights; trtllm: _invoke_kernel]. ``apply_router_weight_on_input`` (top-1 only)
+    scales x by its route weight before the experts and leaves the activation unweighted:
+    the MoonEP experts skip their weight multiply in that case because the weighting
+    happened before dispatch [moonep: MoonEPExperts.apply].
+
     Returns a dict: ids, w, row, cu_seqlens, perm_token, perm_k, perm_w, inv_perm, tokens and
     out (fp64 ``[len(tokens), H]``); with ``keep``, also xq (codes/sb/s), h and y rows.
     """
-    ids, w = route(cfg, logits, routing_bias)
+    if given_topk is not None:
+        ids = np.asarray(given_topk[0], dtype=np.int32)
+        w = np.asarray(given_topk[1], dtype=np.float32).astype(np.float64)
+    else:
+        ids, w = route(cfg, logits, routing_bias)
+    if apply_router_weight_on_input and ids.shape[1] != 1:
+        raise ValueError("apply_router_weight_on_input needs top-1 routing")
     perm = assign_rows(ids, cfg.E, cfg.B, replica_src)
     T, k = ids.shape
     inv = perm["inv_perm"]
@@ -489,6 +503,10 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     need[inv[tok].reshape(-1)] = True
 
     x64 = to_f64(x)
+    if apply_router_weight_on_input:
+        x64 = x64 * w[:, :1]
+        apply_topk_in_fc1 = True          # the activation takes no weight (perm_w below is ignored)
+        perm_w = np.ones_like(perm_w)
     res = dict(ids=ids, w=w, perm_w=perm_w, tokens=tok, **perm)
     if cfg.act_quant == 1:
         codes, sb, s = nvfp4_quantize_rows(np.asarray(x.float().numpy(), np.float32))

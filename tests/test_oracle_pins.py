@@ -427,10 +427,13 @@ def test_mxfp8_quant_matches_bruteforce_and_special_cases():
 
 # ------------------------------------------------------------------ the whole layer
 
-def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
+def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=False):
     """Per token, per chosen expert, the expert MLP on that token alone: no permutation,
-    own routing, pure-Python dot products."""
-    if cfg.routing == "deepseek_v3":
+    own routing (or the given ids and weights), pure-Python dot products. With
+    input_weight the token is scaled by its weight before the MLP, which is then unweighted."""
+    if given is not None:
+        ids, w = np.asarray(given[0]), np.asarray(given[1], np.float32).astype(np.float64)
+    elif cfg.routing == "deepseek_v3":
         ids, w = _grouped_brute(inp.logits.numpy(), inp.extra["routing_bias"].numpy(), cfg.topk, cfg.n_group,
                                 cfg.topk_group, cfg.routed_scaling_factor)
     else:
@@ -448,8 +451,8 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
     Wu = [O.weight_rows(inp.w_up, e).tolist() for e in range(cfg.E)]
     Wd = [O.weight_rows(inp.w_down, e).tolist() for e in range(cfg.E)]
     for t in range(cfg.T):
-        xt = x[t].tolist()
         for j in range(cfg.topk):
+            xt = [v * w[t, j] for v in x[t].tolist()] if input_weight else x[t].tolist()
             e = int(ids[t, j])
             gate = [ag[e] * sum(a * b for a, b in zip(row, xt)) for row in Wg[e]]
             up = [au[e] * sum(a * b for a, b in zip(row, xt)) for row in Wu[e]]
@@ -459,7 +462,7 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
                 al, be = cfg.situ_alpha, cfg.situ_beta
                 h = [al * math.tanh(gg / al) / (1 + math.exp(-gg)) * be * math.tanh(uu / be)
                      for gg, uu in zip(gate, up)]
-            if apply_topk_in_fc1:
+            if apply_topk_in_fc1 and not input_weight:
                 h = [v * w[t, j] for v in h]
             if cfg.act_quant == 1:
                 c, sb, s = O.nvfp4_quantize_rows(np.array([h], np.float32))
@@ -468,7 +471,7 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True):
                 c, sc = O.mxfp8_quantize_rows(np.array([h], np.float32))
                 h = O.mxfp8_dequantize_rows(c, sc)[0].tolist()
             y = [ad[e] * sum(a * b for a, b in zip(row, h)) for row in Wd[e]]
-            wt = 1.0 if apply_topk_in_fc1 else w[t, j]
+            wt = 1.0 if (apply_topk_in_fc1 or input_weight) else w[t, j]
             out[t] += wt * np.array(y)
     return out
 
@@ -554,3 +557,35 @@ def test_workload_generator_is_deterministic_and_replicas_copy():
     for s in range(cfg.B):
         assert torch.equal(a.w_gate.data[cfg.E + s], a.w_gate.data[int(copy_of[s])])
     assert (src[cfg.B_used:] == -1).all() and (src[:cfg.B_used] >= 0).all()
+
+
+def test_given_topk_and_input_weighting():
+    cfg = W.MoEConfig("given", T=9, H=32, I=48, E=6, topk=2, logit_std=2.0)
+    inp = W.gen_inputs(cfg)
+    args = (cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down)
+    # the computed routing, given back, changes nothing
+    ids, w = O.route_topk(inp.logits.numpy(), cfg.topk)
+    a = O.moe_forward(*args)["out"]
+    b = O.moe_forward(*args, given_topk=(ids, w.astype(np.float32)))["out"]
+    assert np.allclose(a, b, rtol=1e-6, atol=1e-9)
+    # arbitrary given experts and weights (a repeated expert for one token included)
+    g = np.random.default_rng(5)
+    gid = g.integers(0, cfg.E, (cfg.T, cfg.topk)).astype(np.int32)
+    gw = g.uniform(0.1, 2.0, (cfg.T, cfg.topk)).astype(np.float32)
+    res = O.moe_forward(*args, given_topk=(gid, gw))["out"]
+    ref = _layer_brute(cfg, inp, given=(gid, gw))
+    assert np.allclose(res, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    # top-1 with the weight on the input: x scaled before the MLP, no weight after it
+    cfg1 = cfg.with_(topk=1)
+    args1 = (cfg1,) + args[1:]
+    w1 = g.uniform(0.2, 3.0, (cfg.T, 1)).astype(np.float32)
+    res = O.moe_forward(*args1, given_topk=(gid[:, :1], w1), apply_router_weight_on_input=True)["out"]
+    ref = _layer_brute(cfg1, inp, given=(gid[:, :1], w1), input_weight=True)
+    assert np.allclose(res, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    # unit weights: weighting the input or the output is the same
+    ones = np.ones((cfg.T, 1), np.float32)
+    u1 = O.moe_forward(*args1, given_topk=(gid[:, :1], ones), apply_router_weight_on_input=True)["out"]
+    u2 = O.moe_forward(*args1, given_topk=(gid[:, :1], ones))["out"]
+    assert np.allclose(u1, u2, rtol=1e-12)
+    with pytest.raises(ValueError):
+        O.moe_forward(*args, given_topk=(gid, gw), apply_router_weight_on_input=True)
