@@ -321,11 +321,21 @@ typedef struct {
     int32_t T_max;                  /* capacity the workspace was sized for */
     void* const* stage_events;      /* optional: MOE_FWD_STAGE_EVENTS cudaEvent_t */
     /* routing: 0 = softmax -> top-k -> renormalise (moe_route_topk), 1 = DeepSeekV3
-     * (moe_route_topk_grouped with the four fields below; other values INVALID_ARG) */
+     * (moe_route_topk_grouped with the four fields below), 2 = given: the experts and
+     * route weights of every token come in topk_ids_in / topk_w_in and router_logits may
+     * be NULL (the modular and routed kernels of the FlashInfer MoE-EP and TRTLLM MXFP4
+     * pages take a computed top-k). A token must not list an expert twice: the
+     * permutation reports that as MOE_ERR_DEVICE. Other values: INVALID_ARG. */
     int32_t routing;
     const float* routing_bias;      /* [E] or NULL */
     int32_t n_group, topk_group;
     float routed_scaling_factor;
+    const int32_t* topk_ids_in;     /* [T,topk] for routing 2 */
+    const float* topk_w_in;         /* [T,topk] for routing 2 */
+    /* 1: top-1 routing with the route weight on the input: the experts see x * w (rounded
+     * once to bf16) and the activation and the combine take no weight (MoonEP experts
+     * page, MoonEPExperts.apply). topk != 1: INVALID_ARG. */
+    int32_t apply_router_weight_on_input;
 } moe_forward_args_t;
 
 size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,

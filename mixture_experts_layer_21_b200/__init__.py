@@ -69,9 +69,11 @@ class moe_forward_args_t(ctypes.Structure):
                 ("T_max", ctypes.c_int32), ("stage_events", ctypes.c_void_p),
                 ("routing", ctypes.c_int32), ("routing_bias", ctypes.c_void_p),
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
-                ("routed_scaling_factor", ctypes.c_float)]
+                ("routed_scaling_factor", ctypes.c_float),
+                ("topk_ids_in", ctypes.c_void_p), ("topk_w_in", ctypes.c_void_p),
+                ("apply_router_weight_on_input", ctypes.c_int32)]
 
-ROUTING = {"renormalize": 0, "deepseek_v3": 1}
+ROUTING = {"renormalize": 0, "deepseek_v3": 1, "given": 2}
 
 MOE_FWD_STAGE_EVENTS = 7
 
@@ -317,7 +319,7 @@ class MoEForward:
                  replica_src=None, act: str = "silu", situ_alpha=1.0, situ_beta=1.0,
                  act_quant: int = 0, apply_topk_in_fc1: bool = True, T_max: int = 1,
                  routing: str = "renormalize", routing_bias=None, n_group: int = 1, topk_group: int = 1,
-                 routed_scaling_factor: float = 1.0):
+                 routed_scaling_factor: float = 1.0, apply_router_weight_on_input: bool = False):
         for w in (w_gate, w_up, w_down):
             if w.fmt != "bf16" and w.prepared is None:
                 moe_prepare_weights(w)
@@ -336,12 +338,13 @@ class MoEForward:
         self.routing_bias = routing_bias
         self.args.n_group, self.args.topk_group = n_group, topk_group
         self.args.routed_scaling_factor = routed_scaling_factor
+        self.args.apply_router_weight_on_input = 1 if apply_router_weight_on_input else 0
 
-    def __call__(self, x, router_logits, out=None, topk_ids=None, topk_w=None, stream=None,
-                 stage_events=None):
+    def __call__(self, x, router_logits=None, out=None, topk_ids=None, topk_w=None, stream=None,
+                 stage_events=None, topk_ids_in=None, topk_w_in=None):
         """``stage_events``: None, or a list of MOE_FWD_STAGE_EVENTS entries, each None (not
         recorded) or a torch.cuda.Event created with enable_timing and recorded once (so that
-        its handle exists)."""
+        its handle exists). ``topk_ids_in``/``topk_w_in``: the given top-k of routing "given"."""
         T = x.shape[0]
         if stage_events is not None:
             if len(stage_events) != MOE_FWD_STAGE_EVENTS:
@@ -364,6 +367,7 @@ class MoEForward:
         a.topk_ids_out, a.topk_w_out = _ptr(topk_ids), _ptr(topk_w)
         a.T_max = self.T_max
         a.routing_bias = _ptr(self.routing_bias)
+        a.topk_ids_in, a.topk_w_in = _ptr(topk_ids_in), _ptr(topk_w_in)
         _check(_lib.moe_forward(ctypes.byref(a), _ptr(self.ws), self.ws.numel(), _stream(stream)),
                "moe_forward")
         return out

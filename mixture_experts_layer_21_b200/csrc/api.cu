@@ -12,6 +12,9 @@ size_t prepared_weight_bytes(const moe_weight_t* w);
 // topk_group <= n_group, topk <= min(32, topk_group * E / n_group), checked here.
 cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int topk, int n_group,
                                  int topk_group, float scale, int32_t* ids, float* w, cudaStream_t st, bool pdl);
+// x[t,:] * w[t] rounded to bf16 (elementwise.cu); H % 8 == 0.
+cudaError_t launch_scale_rows(const __nv_bfloat16* x, const float* w, int T, int H, __nv_bfloat16* out,
+                              cudaStream_t st, bool pdl);
 moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaStream_t st);
 
 int num_sms() {
@@ -66,8 +69,8 @@ const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? 
 // ----------------------------------------------------------------- forward workspace
 struct FwdWs {
     size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
-        xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, mx_xq, mx_xperm, mx_act, y,
-        bytes;
+        xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, mx_xq, mx_xperm, mx_act,
+        x_in, y, bytes;
 };
 
 // With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
@@ -116,6 +119,7 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H, terms) : 0);
     L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H, terms) : 0);
     L.mx_act = take(mx ? NvS * mx8_rec_bytes(I, terms) : 0);
+    L.x_in = take(topk == 1 ? 2 * (size_t)T_max * H : 0);  // x times the top-1 weight (input-side weighting)
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
     L.bytes = off;
     return L;
@@ -389,8 +393,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (T > p->T_max) return MOE_ERR_INVALID_ARG;  // the workspace was sized for T_max tokens
     if (E > kMaxExperts || E + B > 1024 || k > kMaxTopk) return MOE_ERR_UNSUPPORTED;
     if (!act_ok(p->act)) return MOE_ERR_INVALID_ARG;
-    // routing: 0 = softmax -> top-k -> renormalise, 1 = DeepSeekV3 grouped top-k
-    if (p->routing != 0 && p->routing != 1) return MOE_ERR_INVALID_ARG;
+    // routing: 0 = softmax -> top-k -> renormalise, 1 = DeepSeekV3 grouped top-k, 2 = given
+    if (p->routing < 0 || p->routing > 2) return MOE_ERR_INVALID_ARG;
+    if (p->routing == 2 && (!p->topk_ids_in || !p->topk_w_in)) return MOE_ERR_INVALID_ARG;
+    if (p->apply_router_weight_on_input && k != 1) return MOE_ERR_INVALID_ARG;
     if (p->routing == 1) {
         const moe_status_t rs = check_grouped(E, k, p->n_group, p->topk_group, p->routed_scaling_factor);
         if (rs != MOE_OK) return rs;
@@ -412,14 +418,16 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (ws_bytes < moe_forward_workspace_size(p->T_max, H, I, E, B, k, fmt, p->act_quant))
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (T == 0) return MOE_OK;
-    if (!p->x || !p->router_logits || !p->out) return MOE_ERR_INVALID_ARG;
+    if (!p->x || (!p->router_logits && p->routing != 2) || !p->out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(p->x) || !aligned16(p->out) || !aligned16(ws)) return MOE_ERR_ALIGNMENT;
 
     const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant);
     char* w = static_cast<char*>(ws);
     DevError* err = reinterpret_cast<DevError*>(w);
-    int32_t* ids = p->topk_ids_out ? p->topk_ids_out : reinterpret_cast<int32_t*>(w + L.ids);
-    float* tw = p->topk_w_out ? p->topk_w_out : reinterpret_cast<float*>(w + L.w);
+    const bool given = p->routing == 2;
+    const int32_t* ids = given ? p->topk_ids_in
+                               : (p->topk_ids_out ? p->topk_ids_out : reinterpret_cast<int32_t*>(w + L.ids));
+    const float* tw = given ? p->topk_w_in : (p->topk_w_out ? p->topk_w_out : reinterpret_cast<float*>(w + L.w));
     int32_t* cu = reinterpret_cast<int32_t*>(w + L.cu);
     int32_t* perm_token = reinterpret_cast<int32_t*>(w + L.perm_token);
     float* perm_w = reinterpret_cast<float*>(w + L.perm_w);
@@ -450,25 +458,43 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     };
 
     if (!mark(0)) return MOE_ERR_CUDA;
-    // S1 route
-    if (p->routing == 1)
+    // S1 route (or the given top-k, copied to the optional outputs)
+    int32_t* ids_w = const_cast<int32_t*>(ids);
+    float* tw_w = const_cast<float*>(tw);
+    if (given) {
+        e = cudaSuccess;
+        if (p->topk_ids_out)
+            e = cudaMemcpyAsync(p->topk_ids_out, ids, sizeof(int32_t) * (size_t)T * k, cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess && p->topk_w_out)
+            e = cudaMemcpyAsync(p->topk_w_out, tw, sizeof(float) * (size_t)T * k, cudaMemcpyDeviceToDevice, st);
+    } else if (p->routing == 1) {
         e = launch_route_grouped(p->router_logits, p->routing_bias, T, E, k, p->n_group, p->topk_group,
-                                 p->routed_scaling_factor, ids, tw, st, false);
-    else
-        e = launch_route_topk(p->router_logits, T, E, k, ids, tw, st, false);
+                                 p->routed_scaling_factor, ids_w, tw_w, st, false);
+    } else {
+        e = launch_route_topk(p->router_logits, T, E, k, ids_w, tw_w, st, false);
+    }
     if (e != cudaSuccess || !mark(1)) return MOE_ERR_CUDA;
+    // top-1 weight on the input: the experts see x * w and the activation takes no weight
+    const bool in_w = p->apply_router_weight_on_input != 0;
+    const void* xin = p->x;
+    if (in_w) {
+        e = launch_scale_rows(static_cast<const __nv_bfloat16*>(p->x), tw, T, H,
+                              reinterpret_cast<__nv_bfloat16*>(w + L.x_in), st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        xin = w + L.x_in;
+    }
     // S2 permute
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
                        pdl());
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     // S2 gather (+ S2q)
     if (fmt == MOE_W_BF16) {
-        e = launch_gather(0, p->x, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
+        e = launch_gather(0, xin, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (fmt == MOE_W_MXFP4) {
         // stage each token once as e4m3 records (hi/lo, or MXFP8), then gather the records
         const int rb = mx8_rec_bytes(H, terms), Kp = mx8_kpad(H);
         uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_xq);
-        e = launch_quant_mx8(p->x, false, T, H, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr, rec + terms * Kp,
+        e = launch_quant_mx8(xin, false, T, H, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr, rec + terms * Kp,
                              rb, rb, st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(0, w + L.mx_xq, rb / 2, perm_token, NvS, w + L.mx_xperm, nullptr, nullptr, st, pdl());
@@ -476,20 +502,20 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         // quantise each token once into records, then gather the records into segment order
         uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.xq_rec);
         const int rb = nvf4_rec_bytes(H);
-        e = launch_quant_nvfp4(p->x, false, T, H, rec, rb, rec + H / 2, rb, reinterpret_cast<float*>(w + L.xq_s),
+        e = launch_quant_nvfp4(xin, false, T, H, rec, rb, rec + H / 2, rb, reinterpret_cast<float*>(w + L.xq_s),
                                nullptr, st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(1, rec, rb / 2, perm_token, NvS, w + L.xperm_rec, reinterpret_cast<float*>(w + L.xq_s),
                           tscale, st, pdl());
     } else if (p->act_quant) {
-        e = launch_quant_nvfp4(p->x, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes), H / 2,
+        e = launch_quant_nvfp4(xin, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes), H / 2,
                                reinterpret_cast<uint8_t*>(w + L.xq_sb), H / 16, reinterpret_cast<float*>(w + L.xq_s),
                                reinterpret_cast<__half*>(w + L.xq_deq), st, pdl());
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_gather(1, w + L.xq_deq, H, perm_token, NvS, xperm, reinterpret_cast<float*>(w + L.xq_s), tscale,
                           st, pdl());
     } else {
-        e = launch_gather(2, p->x, H, perm_token, NvS, xperm, nullptr, tscale, st, pdl());
+        e = launch_gather(2, xin, H, perm_token, NvS, xperm, nullptr, tscale, st, pdl());
     }
     if (e != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
 
@@ -512,7 +538,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g1.kscale1 = p->w_up.kscale;
     g1.alpha0 = weight_alpha(p->w_gate);
     g1.alpha1 = weight_alpha(p->w_up);
-    g1.perm_w = p->apply_topk_in_fc1 ? perm_w : nullptr;
+    g1.perm_w = (p->apply_topk_in_fc1 && !in_w) ? perm_w : nullptr;
     g1.tscale = fmt == MOE_W_BF16 ? nullptr : tscale;
     g1.out_scale = 1.0f;
     g1.act = p->act.act;
@@ -616,8 +642,8 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     e = launch_grouped_gemm(g2, st, pdl());
     if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
     // S6: combine
-    e = launch_combine_f32(y, inv, p->apply_topk_in_fc1 ? nullptr : tw, T, k, H, static_cast<__nv_bfloat16*>(p->out),
-                           st, pdl());
+    e = launch_combine_f32(y, inv, (p->apply_topk_in_fc1 || in_w) ? nullptr : tw, T, k, H,
+                           static_cast<__nv_bfloat16*>(p->out), st, pdl());
     if (e != cudaSuccess || !mark(6)) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -46,6 +46,39 @@ cudaError_t launch_act_and_mul(const __nv_bfloat16* gate, const __nv_bfloat16* u
                     act, sa, sb, out);
 }
 
+// ----------------------------------------------------------------- input-side route weight
+// out[t,:] = x[t,:] * w[t] (top-1 routing with the weight on the input), fp32 product,
+// one bf16 rounding. H % 8 == 0.
+__global__ void __launch_bounds__(256) scale_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const float* __restrict__ w, int T, int H,
+                                                         __nv_bfloat16* __restrict__ out) {
+    pdl_wait();
+    const long long n8 = (long long)T * H / 8;
+    for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8;
+         v += (long long)gridDim.x * blockDim.x) {
+        const float s = w[(v * 8) / H];
+        const uint4 a = reinterpret_cast<const uint4*>(x)[v];
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&a);
+        uint4 o;
+        __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            q[i] = __floats2bfloat162_rn(f.x * s, f.y * s);
+        }
+        reinterpret_cast<uint4*>(out)[v] = o;
+    }
+    pdl_launch();
+}
+
+cudaError_t launch_scale_rows(const __nv_bfloat16* x, const float* w, int T, int H, __nv_bfloat16* out,
+                              cudaStream_t st, bool pdl) {
+    const long long n8 = (long long)T * H / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int blocks = (int)std::min<long long>((n8 + 255) / 256, (long long)num_sms() * 16);
+    return launch_k(scale_rows_kernel, dim3(blocks), dim3(256), 0, st, pdl, x, w, T, H, out);
+}
+
 // ----------------------------------------------------------------- S6
 // out[t] = sum_k w[t,k] * y[inv_perm[t,k]], fp32 in k order, one bf16 rounding.
 // Grid (T, ceil(H / 1024)); each thread owns 8 contiguous columns. y is bf16 (the

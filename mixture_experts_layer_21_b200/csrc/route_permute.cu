@@ -265,7 +265,10 @@ __device__ void build_masks(uint32_t* masks, const int32_t* __restrict__ ids, in
                 report_error(err, MOE_ERR_DEVICE, t);
                 continue;
             }
-            atomicOr(&masks[e * (kPermBlock / 32) + (threadIdx.x >> 5)], 1u << (threadIdx.x & 31));
+            // a token listing one expert twice (possible only with a given top-k) is refused
+            const uint32_t bit = 1u << (threadIdx.x & 31);
+            if (atomicOr(&masks[e * (kPermBlock / 32) + (threadIdx.x >> 5)], bit) & bit)
+                report_error(err, MOE_ERR_DEVICE, t);
         }
     }
     __syncthreads();

@@ -106,6 +106,7 @@ def _fwd(**kw):
     p.routing = kw.get("routing", 0)
     p.n_group, p.topk_group = kw.get("n_group", 1), kw.get("topk_group", 1)
     p.routed_scaling_factor = kw.get("scale", 1.0)
+    p.apply_router_weight_on_input = kw.get("in_w", 0)
     p.apply_topk_in_fc1 = 1
     nws = L.moe_forward_workspace_size(d["T_max"], d["H"], d["I"], d["E"], d["B"], d["topk"], d["fmt"], d["aq"])
     return p, nws
@@ -126,7 +127,9 @@ def _fwd(**kw):
     (dict(H=72, I=128), ALIGN),                     # H % 16
     (dict(B=2), INVALID),                           # replicas without replica_src
     (dict(E=1100, topk=2), UNSUP),
-    (dict(routing=2), INVALID),                     # no such routing method
+    (dict(routing=3), INVALID),                     # no such routing method
+    (dict(routing=2), INVALID),                     # given routing without the given top-k
+    (dict(in_w=1), INVALID),                        # input-side weight needs top-1
     (dict(routing=1, n_group=3), INVALID),          # E % n_group
     (dict(routing=1, n_group=2, topk_group=1, scale=0.0), INVALID),
 ])

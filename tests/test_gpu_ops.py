@@ -371,6 +371,42 @@ def test_forward_bf16_256_token_tiles(lib, monkeypatch):
     check_bf16(out, ref["out"], what="bt256")
 
 
+def test_forward_given_topk_and_input_weight(lib):
+    # routing on a given top-k (distinct experts per token, arbitrary weights), and top-1 with
+    # the route weight on the input
+    cfg = W.MoEConfig("given", T=90, H=128, I=192, E=8, topk=2)
+    inp = W.gen_inputs(cfg)
+    g = np.random.default_rng(2)
+    gid = np.stack([g.permutation(cfg.E)[:cfg.topk] for _ in range(cfg.T)]).astype(np.int32)
+    gw = g.uniform(0.1, 2.0, (cfg.T, cfg.topk)).astype(np.float32)
+    dev = lambda ws: lib.Weight.from_host(ws)
+    for k, in_w in ((2, False), (1, True)):
+        c = cfg.with_(topk=k)
+        layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), c.E, c.topk, routing="given",
+                               apply_router_weight_on_input=in_w, T_max=c.T)
+        ids_d, w_d = to_dev(torch.from_numpy(gid[:, :k].copy())), to_dev(torch.from_numpy(gw[:, :k].copy()))
+        out = layer(to_dev(inp.x), None, topk_ids_in=ids_d, topk_w_in=w_d)
+        torch.cuda.synchronize()
+        assert layer.device_error() == 0
+        ref = O.moe_forward(c, inp.x, None, np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down,
+                            given_topk=(gid[:, :k], gw[:, :k]), apply_router_weight_on_input=in_w)
+        check_bf16(out, ref["out"], what=f"given k={k} input-weight={in_w}")
+
+
+def test_forward_given_topk_repeated_expert_is_refused(lib):
+    cfg = W.MoEConfig("given", T=20, H=128, I=192, E=8, topk=2)
+    inp = W.gen_inputs(cfg)
+    gid = np.tile(np.array([[1, 3]], np.int32), (cfg.T, 1))
+    gid[7] = [5, 5]                            # the same expert twice for token 7
+    gw = np.ones((cfg.T, 2), np.float32)
+    dev = lambda ws: lib.Weight.from_host(ws)
+    layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, cfg.topk, routing="given",
+                           T_max=cfg.T)
+    layer(to_dev(inp.x), None, topk_ids_in=to_dev(torch.from_numpy(gid)), topk_w_in=to_dev(torch.from_numpy(gw)))
+    torch.cuda.synchronize()
+    assert layer.device_error() == 6          # MOE_ERR_DEVICE
+
+
 def test_forward_weight_in_combine(lib):
     cfg = SMALL["replicas"]
     inp = W.gen_inputs(cfg)
