@@ -20,8 +20,8 @@ Page citations name the page's module and the class, method or docstring:
 * [dsv4_fi]  vllm.models.deepseek_v4.nvidia.fi_moe (DeepseekV4MegaMoEExpertsFI)
 * [trtllm]   vllm.model_executor.layers.fused_moe.experts.trtllm_mxfp4_moe
 
-Readings taken where the pages are silent are listed in the design doc and repeated
-at the function that takes them.
+Readings taken where the pages are silent are stated at the function that takes
+them.
 """
 from __future__ import annotations
 
