@@ -341,11 +341,39 @@ def situ_and_mul(gate, up, alpha: float, beta: float):
     return alpha * np.tanh(gate / alpha) * sig * (beta * np.tanh(up / beta))
 
 
+def swigluoai_and_mul(gate, up, alpha: float, beta: float, limit=None):
+    """SWIGLUOAI gated activation. The TRTLLM MXFP4 page lists SWIGLUOAI among its
+    activations and hands per-expert gemm1_alpha, gemm1_beta and gemm1_clamp_limit to the
+    kernel [trtllm: TrtLlmMxfp4ExpertsBase._supports_activation and __init__,
+    TrtLlmMxfp4ExpertsModular._invoke_kernel], without the formula. Reading taken: the
+    published GPT-OSS gated activation,
+
+      g = min(gate, limit),  u = clamp(up, -limit, limit)     (no clamp when limit is None)
+      out = g * sigmoid(alpha * g) * (u + beta)
+
+    (GPT-OSS itself uses alpha = 1.702, beta = 1, limit = 7)."""
+    g = np.asarray(gate, dtype=np.float64)
+    u = np.asarray(up, dtype=np.float64)
+    if limit is not None:
+        g = np.minimum(g, limit)
+        u = np.clip(u, -limit, limit)
+    with np.errstate(over="ignore"):
+        sig = 1.0 / (1.0 + np.exp(-alpha * g))
+    return g * sig * (u + beta)
+
+
 def act_and_mul(gate, up, act: str = "silu", situ_alpha: float = 1.0, situ_beta: float = 1.0,
-                route_w=None):
+                route_w=None, swiglu_alpha: float = 1.702, swiglu_beta: float = 1.0, swiglu_limit=7.0):
     """Gated activation times the per-row route weight (``act *= route_weight``
     [moonep: MoonEPExperts.apply])."""
-    h = silu_and_mul(gate, up) if act == "silu" else situ_and_mul(gate, up, situ_alpha, situ_beta)
+    if act == "silu":
+        h = silu_and_mul(gate, up)
+    elif act == "situ":
+        h = situ_and_mul(gate, up, situ_alpha, situ_beta)
+    elif act == "swigluoai":
+        h = swigluoai_and_mul(gate, up, swiglu_alpha, swiglu_beta, swiglu_limit)
+    else:
+        raise ValueError(act)
     if route_w is not None:
         h = h * np.asarray(route_w, dtype=np.float64)[:, None]
     return h
@@ -465,7 +493,7 @@ def combine(y, inv_perm, topk_w=None):
 
 def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
                 tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False, routing_bias=None,
-                given_topk=None, apply_router_weight_on_input: bool = False):
+                given_topk=None, apply_router_weight_on_input: bool = False, biases=None):
     """The fused expert layer: route -> permute -> gate/up grouped GEMMs -> activation times
     route weight -> down grouped GEMM -> combine [moonep: module docstring and apply;
     trtllm: _invoke_kernel; fi_ep: apply].
@@ -476,6 +504,11 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     before their GEMM; with act_quant = 2 they are MXFP8-quantised (``mxfp8_quantize_rows``). ``tokens`` restricts the expert maths to the rows those tokens need
     (routing and permutation are always computed in full). With ``apply_topk_in_fc1`` false
     the route weight moves from the activation to the combine [fi_ep: apply_topk_in_fc1].
+
+    ``biases = (b_gate [G,I], b_up [G,I], b_down [G,H])`` adds per-row biases to the GEMM
+    outputs (gemm1_bias / gemm2_bias [trtllm: TrtLlmMxfp4ExpertsModular._invoke_kernel]):
+    gate and up get theirs before the activation, and the down projection's is part of the
+    expert's output, so it is scaled by the route weight with it.
 
     ``given_topk = (ids, w)`` skips the routing: the experts and route weights are given, as
     in the modular and routed kernels that take a computed top-k [fi_ep: apply, topk_ids and
@@ -529,8 +562,12 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
         a = x64[perm["perm_token"][rows]]
         gate = a_g[g] * (a @ weight_rows(w_gate, g).T)
         up = a_u[g] * (a @ weight_rows(w_up, g).T)
+        if biases is not None:
+            gate = gate + to_f64(biases[0][g])[None, :]
+            up = up + to_f64(biases[1][g])[None, :]
         h = act_and_mul(gate, up, cfg.act, cfg.situ_alpha, cfg.situ_beta,
-                        perm_w[rows] if apply_topk_in_fc1 else None)
+                        perm_w[rows] if apply_topk_in_fc1 else None, cfg.swiglu_alpha, cfg.swiglu_beta,
+                        cfg.swiglu_limit)
         if cfg.act_quant == 1:
             hc, hsb, hs = nvfp4_quantize_rows(h.astype(np.float32))
             h = nvfp4_dequantize_rows(hc, hsb, hs)
@@ -540,6 +577,9 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
         if keep:
             h_keep[rows] = h
         y[rows] = a_d[g] * (h @ weight_rows(w_down, g).T)
+        if biases is not None:   # the expert's own bias, under the route weight when it is in h
+            wb = perm_w[rows] if apply_topk_in_fc1 else np.ones(len(rows))
+            y[rows] += wb[:, None] * to_f64(biases[2][g])[None, :]
     out = combine(y, inv[tok], None if apply_topk_in_fc1 else w[tok])
     res["out"] = out
     if keep:

@@ -427,7 +427,7 @@ def test_mxfp8_quant_matches_bruteforce_and_special_cases():
 
 # ------------------------------------------------------------------ the whole layer
 
-def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=False):
+def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=False, biases=None):
     """Per token, per chosen expert, the expert MLP on that token alone: no permutation,
     own routing (or the given ids and weights), pure-Python dot products. With
     input_weight the token is scaled by its weight before the MLP, which is then unweighted."""
@@ -456,8 +456,18 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=Fals
             e = int(ids[t, j])
             gate = [ag[e] * sum(a * b for a, b in zip(row, xt)) for row in Wg[e]]
             up = [au[e] * sum(a * b for a, b in zip(row, xt)) for row in Wu[e]]
+            if biases is not None:
+                gate = [v + float(b) for v, b in zip(gate, biases[0][e])]
+                up = [v + float(b) for v, b in zip(up, biases[1][e])]
             if cfg.act == "silu":
                 h = [gg / (1 + math.exp(-gg)) * uu for gg, uu in zip(gate, up)]
+            elif cfg.act == "swigluoai":
+                lim, al, be = cfg.swiglu_limit, cfg.swiglu_alpha, cfg.swiglu_beta
+                h = []
+                for gg, uu in zip(gate, up):
+                    if lim is not None:
+                        gg, uu = min(gg, lim), max(-lim, min(uu, lim))
+                    h.append(gg / (1 + math.exp(-al * gg)) * (uu + be))
             else:
                 al, be = cfg.situ_alpha, cfg.situ_beta
                 h = [al * math.tanh(gg / al) / (1 + math.exp(-gg)) * be * math.tanh(uu / be)
@@ -471,6 +481,9 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=Fals
                 c, sc = O.mxfp8_quantize_rows(np.array([h], np.float32))
                 h = O.mxfp8_dequantize_rows(c, sc)[0].tolist()
             y = [ad[e] * sum(a * b for a, b in zip(row, h)) for row in Wd[e]]
+            if biases is not None:   # the bias is part of the expert's output, under its weight
+                bw = w[t, j] if (apply_topk_in_fc1 and not input_weight) else 1.0
+                y = [v + bw * float(b) for v, b in zip(y, biases[2][e])]
             wt = 1.0 if (apply_topk_in_fc1 or input_weight) else w[t, j]
             out[t] += wt * np.array(y)
     return out
@@ -589,3 +602,45 @@ def test_given_topk_and_input_weighting():
     assert np.allclose(u1, u2, rtol=1e-12)
     with pytest.raises(ValueError):
         O.moe_forward(*args, given_topk=(gid, gw), apply_router_weight_on_input=True)
+
+
+def test_swigluoai_reductions_and_clamps():
+    g = np.random.default_rng(9)
+    gate, up = g.normal(0, 4, (5, 64)), g.normal(0, 4, (5, 64))
+    # no clamp, alpha 1, beta 0: silu-and-mul exactly
+    assert np.allclose(O.swigluoai_and_mul(gate, up, 1.0, 0.0, None), O.silu_and_mul(gate, up), rtol=1e-14)
+    # the clamp: a gate above the limit acts as the limit, up is clipped on both sides
+    lim = 7.0
+    assert np.allclose(O.swigluoai_and_mul(np.array([10.0]), np.array([2.0]), 1.702, 1.0, lim),
+                       O.swigluoai_and_mul(np.array([lim]), np.array([2.0]), 1.702, 1.0, lim))
+    assert np.allclose(O.swigluoai_and_mul(np.array([1.5]), np.array([-50.0]), 1.702, 1.0, lim),
+                       O.swigluoai_and_mul(np.array([1.5]), np.array([-lim]), 1.702, 1.0, lim))
+    # a gate below -limit is not clamped (the gate has an upper clamp only)
+    v = O.swigluoai_and_mul(np.array([-9.0]), np.array([0.5]), 1.0, 1.0, lim)[0]
+    assert v == -9.0 / (1.0 + math.exp(9.0)) * 1.5
+
+
+def test_biases_closed_form_and_layer_loop():
+    # all-zero weights: gate = b_gate, up = b_up, and the expert output is its down bias, so
+    # out[t] = sum_k w_k b_down[e_k] whatever the activation
+    cfg = W.MoEConfig("bias0", T=6, H=32, I=48, E=5, topk=2, act="swigluoai", bias=True, w_std=0.0)
+    inp = W.gen_inputs(cfg)
+    bg, bu, bd = inp.extra["biases"]
+    res = O.moe_forward(cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32), inp.w_gate, inp.w_up,
+                        inp.w_down, biases=(bg, bu, bd))
+    ids, w = O.route_topk(inp.logits.numpy(), cfg.topk)
+    ref = np.einsum("tk,tkh->th", w, bd.double().numpy()[ids])
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-15)
+    # random weights, SWIGLUOAI with its clamp, biases: the per-token loop
+    cfg = W.MoEConfig("bias1", T=8, H=32, I=48, E=5, topk=2, act="swigluoai", bias=True, logit_std=2.0,
+                      swiglu_limit=1.0)
+    inp = W.gen_inputs(cfg)
+    b = inp.extra["biases"]
+    res = O.moe_forward(cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32), inp.w_gate, inp.w_up,
+                        inp.w_down, biases=b)["out"]
+    ref = _layer_brute(cfg, inp, biases=b)
+    assert np.allclose(res, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    res2 = O.moe_forward(cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32), inp.w_gate, inp.w_up,
+                         inp.w_down, biases=b, apply_topk_in_fc1=False)["out"]
+    ref2 = _layer_brute(cfg, inp, apply_topk_in_fc1=False, biases=b)
+    assert np.allclose(res2, ref2, rtol=1e-9, atol=1e-12 * np.abs(ref2).max())

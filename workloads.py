@@ -58,6 +58,10 @@ class MoEConfig:
     wfmt: str = WFMT_BF16
     act_quant: int = 0         # 1 = dynamic NVFP4, 2 = dynamic MXFP8 quantisation of activations
     routing: str = "renormalize"   # or "deepseek_v3": grouped top-k on sigmoid scores
+    swiglu_alpha: float = 1.702        # SWIGLUOAI parameters (act = "swigluoai")
+    swiglu_beta: float = 1.0
+    swiglu_limit: float | None = 7.0
+    bias: bool = False                 # per-row GEMM biases (gemm1_bias, gemm2_bias)
     n_group: int = 1
     topk_group: int = 1
     routed_scaling_factor: float = 1.0
@@ -134,6 +138,17 @@ def gen_routing_bias(cfg: MoEConfig) -> torch.Tensor:
     close candidates without deciding most choices."""
     g = _gen(cfg, _S_BIAS)
     return torch.randn(cfg.E, generator=g) * 0.05
+
+
+def gen_biases(cfg: MoEConfig) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Per-row GEMM biases: gate and up ``[G,I]``, down ``[G,H]``, fp32 N(0, 0.1^2); replica
+    slots copy their source expert's (use after ``gen_replica_src``)."""
+    g = _gen(cfg, _S_BIAS + 1)
+    G = cfg.E + cfg.B
+    bg = torch.randn(G, cfg.I, generator=g) * 0.1
+    bu = torch.randn(G, cfg.I, generator=g) * 0.1
+    bd = torch.randn(G, cfg.H, generator=g) * 0.1
+    return bg, bu, bd
 
 
 def gen_replica_src(cfg: MoEConfig) -> torch.Tensor:
@@ -247,6 +262,12 @@ def gen_inputs(cfg: MoEConfig) -> MoEInputs:
     """All inputs of one workload, on the CPU."""
     wg, wu, wd, src = gen_weights(cfg)
     extra = {"routing_bias": gen_routing_bias(cfg)} if cfg.routing == "deepseek_v3" else {}
+    if cfg.bias:
+        bg, bu, bd = gen_biases(cfg)
+        for s, e in enumerate(src.tolist()):   # a replica slot holds its source expert's biases
+            if e >= 0:
+                bg[cfg.E + s], bu[cfg.E + s], bd[cfg.E + s] = bg[e], bu[e], bd[e]
+        extra["biases"] = (bg, bu, bd)
     return MoEInputs(cfg, gen_x(cfg), gen_logits(cfg), src, wg, wu, wd, extra)
 
 
