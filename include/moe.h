@@ -291,6 +291,8 @@ moe_status_t moe_prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes,
  *   act_quant = 1: dynamic NVFP4 activations (NVFP4 weights only); each GEMM whose K
  *   (H for gate/up, I for down) is a multiple of 256 then runs block-scaled as in
  *   moe_grouped_gemm_nvfp4, the other one on f16-staged operands.
+ *   MXFP4 weights with act_quant = 0 take bf16 activations, staged for the tensor cores
+ *   as two e4m3 terms as in moe_grouped_gemm.
  *   act_quant = 2: dynamic MXFP8 activations (MXFP4 weights only, the W4A8 mode): x and
  *   every activation row are quantised as moe_quantize_mxfp8 does, and both GEMMs take
  *   them as e4m3 with their e8m0 scales. Other act_quant values: INVALID_ARG.

@@ -1,0 +1,62 @@
+"""Host-side bookkeeping of bench.py (no GPU): the algorithmic FLOPs and bytes, the tensor
+peak of each path's MMA kind, the launch count and the profile-traffic lookup."""
+import numpy as np
+import torch
+
+import bench
+import workloads as W
+
+
+def _acc(cfg):
+    inp = W.gen_inputs(cfg)
+    g = torch.Generator().manual_seed(1)
+    ids = torch.stack([torch.randperm(cfg.E, generator=g)[:cfg.topk] for _ in range(cfg.T)])
+    nonempty, max_seg = bench.segment_stats(cfg, ids, inp.replica_src)
+    return inp, bench.accounting(cfg, inp, nonempty, max_seg), nonempty
+
+
+def test_flops_and_bytes_follow_the_definitions():
+    cfg = W.MoEConfig("acc", T=40, H=256, I=384, E=8, topk=2)
+    inp, a, nonempty = _acc(cfg)
+    NvS = cfg.T * cfg.topk
+    assert a["fc1_flops"] == 4.0 * NvS * cfg.H * cfg.I
+    assert a["layer_flops"] == 6.0 * NvS * cfg.H * cfg.I
+    wrow = cfg.I * cfg.H * 2                                   # one bf16 gate (or up) matrix
+    assert a["fc1_bytes"] == nonempty * 2 * wrow + NvS * cfg.H * 2 + NvS * cfg.I * 2
+    assert a["layer_bytes"] == nonempty * 3 * wrow + cfg.T * cfg.H * 4 + cfg.T * cfg.E * 4
+
+
+def test_activation_operand_bytes_per_path():
+    base = dict(T=8, H=256, I=256, E=4, topk=2)
+    NvS = 16
+    per_value = {}
+    for name, kw in {"bf16": {}, "nvfp4": dict(wfmt="nvfp4", act_quant=1), "mx_hilo": dict(wfmt="mxfp4"),
+                     "w4a8": dict(wfmt="mxfp4", act_quant=2)}.items():
+        cfg = W.MoEConfig(name, **base, **kw)
+        inp, a, nonempty = _acc(cfg)
+        wbytes = nonempty * (bench.weight_bytes_per_row(inp.w_gate) + bench.weight_bytes_per_row(inp.w_up))
+        act_out = 2 if cfg.wfmt == "bf16" else 4
+        per_value[name] = (a["fc1_bytes"] - wbytes - NvS * cfg.I * act_out) / (NvS * cfg.H)
+    assert per_value == {"bf16": 2.0, "nvfp4": 9 / 16, "mx_hilo": 2 + 1 / 32, "w4a8": 1 + 1 / 32}
+
+
+def test_tensor_peak_of_each_mma_kind():
+    assert bench.tensor_peak_ratio(W.CONFIGS["mixtral_prefill"])[0] == 1.0
+    assert bench.tensor_peak_ratio(W.CONFIGS["nvfp4"])[0] == 4.0          # kind::mxf4nvf4
+    assert bench.tensor_peak_ratio(W.CONFIGS["mxfp4_w4a8_prefill"])[0] == 2.0   # kind::mxf8f6f4, fp8 rate
+    assert bench.tensor_peak_ratio(W.CONFIGS["mxfp4_prefill"])[0] == 1.0  # two fp8 products per MAC
+
+
+def test_launch_counts_and_dtype():
+    assert bench.kernel_launches(W.CONFIGS["mixtral_prefill"]) == 8
+    assert bench.kernel_launches(W.CONFIGS["nvfp4"]) == 10
+    assert bench.kernel_launches(W.CONFIGS["mxfp4_decode"]) == 10
+    assert bench.compute_dtype(W.CONFIGS["mixtral_prefill"]) == "bf16"
+    assert bench.compute_dtype(W.CONFIGS["nvfp4"]).startswith("nvfp4")
+
+
+def test_profile_traffic_only_for_the_current_source():
+    # the committed summaries carry the hash of the GEMM sources they were taken on
+    v = bench.profiled_traffic("mixtral_prefill")
+    assert v is None or v > 0
+    assert bench.profiled_traffic("no_such_workload") is None
