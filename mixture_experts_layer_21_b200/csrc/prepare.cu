@@ -26,7 +26,7 @@ namespace moe {
 namespace {
 
 struct PrepLayout {
-    int NT, KB, S, KS;
+    int NT, KB, KS;
     size_t data_off, scale_off, alpha_off, scratch_off, bytes;
 };
 
@@ -36,7 +36,6 @@ PrepLayout prep_layout(const moe_weight_t* w) {
     PrepLayout L{};
     L.NT = (w->N + kTileN - 1) / kTileN;
     L.KB = 2 * ((w->K + 2 * kTileK - 1) / (2 * kTileK));  // padded to even
-    L.S = fp4_scale_bytes_per_row(w->fmt);
     const size_t chunks = (size_t)w->G * L.NT * L.KB;
     size_t off = 0;
     auto take = [&](size_t b) {
