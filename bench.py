@@ -70,6 +70,12 @@ def segment_stats(cfg: W.MoEConfig, topk_ids: torch.Tensor, replica_src: torch.T
     return nonempty, max_seg
 
 
+def split_fc1(cfg) -> bool:
+    """SWIGLUOAI or GEMM biases: gate and up run as two GEMMs with fp32 outputs, then a
+    bias/activation row pass; the down bias is a row pass after the down GEMM."""
+    return cfg.act == "swigluoai" or cfg.bias
+
+
 def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) -> dict:
     NvS = cfg.NvS
     wg, wu, wd = (weight_bytes_per_row(inp.w_gate), weight_bytes_per_row(inp.w_up),
@@ -84,7 +90,16 @@ def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) 
     fc2_flops = 2.0 * NvS * cfg.H * cfg.I
     fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * a_in + NvS * cfg.I * act_out
     fc2_bytes = nonempty * wd + NvS * cfg.I * a_in + NvS * cfg.H * 4
-    layer_bytes = nonempty * (wg + wu + wd) + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
+    bias_bytes = nonempty * (2 * cfg.I + cfg.H) * 4 if cfg.bias else 0
+    if split_fc1(cfg):
+        # the operand is read by both GEMMs; gate and up leave in fp32 and are read back by the
+        # row pass with the gate/up biases; h leaves in fp32 when a row pass follows (FP4)
+        act_out = 2 if cfg.wfmt == "bf16" else 4
+        fc1_bytes = (nonempty * (wg + wu) + 2 * NvS * cfg.H * a_in + 2 * 2 * NvS * cfg.I * 4
+                     + NvS * cfg.I * act_out + (nonempty * 2 * cfg.I * 4 if cfg.bias else 0))
+        if cfg.bias:
+            fc2_bytes += 2 * NvS * cfg.H * 4 + nonempty * cfg.H * 4      # the down bias pass over y
+    layer_bytes = nonempty * (wg + wu + wd) + bias_bytes + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
     return dict(nonempty=nonempty, max_seg=max_seg,
                 fc1_flops=fc1_flops, fc2_flops=fc2_flops, fc1_bytes=fc1_bytes, fc2_bytes=fc2_bytes,
                 layer_flops=fc1_flops + fc2_flops, layer_bytes=layer_bytes,
@@ -110,6 +125,16 @@ def routing_config(cfg) -> dict:
         return {}
     return {"routing": cfg.routing, "n_group": cfg.n_group, "topk_group": cfg.topk_group,
             "routed_scaling_factor": cfg.routed_scaling_factor}
+
+
+def act_config(cfg) -> dict:
+    """SWIGLUOAI's parameters and the GEMM biases in the config record, when used."""
+    d = {}
+    if cfg.act == "swigluoai":
+        d.update(swiglu_alpha=cfg.swiglu_alpha, swiglu_beta=cfg.swiglu_beta, swiglu_limit=cfg.swiglu_limit)
+    if cfg.bias:
+        d["gemm_biases"] = True
+    return d
 
 
 def compute_dtype(cfg) -> str:
@@ -260,7 +285,8 @@ def oracle_sample(cfg, inp, tokens):
     t0 = time.perf_counter()
     bias = inp.extra.get("routing_bias")
     O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                  inp.w_down, tokens=tokens, routing_bias=None if bias is None else bias.numpy())
+                  inp.w_down, tokens=tokens, routing_bias=None if bias is None else bias.numpy(),
+                  biases=inp.extra.get("biases"))
     return time.perf_counter() - t0
 
 
@@ -277,8 +303,12 @@ def kernel_launches(cfg) -> int:
     n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
     if cfg.act_quant or cfg.wfmt == "mxfp4":
         n += 2                            # x quantisation / staging, activation quantisation / staging
-    elif cfg.wfmt != "bf16" and cfg.act != "situ":
+    elif cfg.wfmt != "bf16" and (cfg.act != "situ" or split_fc1(cfg)):
         n += 1                            # activation row pass to f16
+    if split_fc1(cfg):
+        n += 2                            # gate and up as two GEMMs, the bias/activation row pass
+        if cfg.bias:
+            n += 1                        # the down bias
     return n
 
 
@@ -292,7 +322,9 @@ def run_ours(args, cfg, rank, world):
                          inp.replica_src.to(dev) if cfg.B else None, cfg.act, cfg.situ_alpha,
                          cfg.situ_beta, cfg.act_quant, True, T_max=cfg.T, routing=cfg.routing,
                          routing_bias=None if bias is None else bias.to(dev), n_group=cfg.n_group,
-                         topk_group=cfg.topk_group, routed_scaling_factor=cfg.routed_scaling_factor)
+                         topk_group=cfg.topk_group, routed_scaling_factor=cfg.routed_scaling_factor,
+                         swiglu_alpha=cfg.swiglu_alpha, swiglu_beta=cfg.swiglu_beta, swiglu_limit=cfg.swiglu_limit,
+                         biases=tuple(b.float().to(dev) for b in inp.extra["biases"]) if cfg.bias else None)
     x_d, l_d = inp.x.to(dev), inp.logits.to(dev)
     out_d = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -389,7 +421,9 @@ def run_ours(args, cfg, rank, world):
         ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"]}
-    roof.update({"traffic": traffic, "kernel": "grouped GEMM gate+up (fused activation)",
+    kname = ("grouped GEMMs gate, up (fp32 out) + bias/activation row pass" if split_fc1(cfg)
+             else "grouped GEMM gate+up (fused activation)")
+    roof.update({"traffic": traffic, "kernel": kname,
                  "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
                  "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst); tensor peak {tensor_note}"})
     t_layer_roof = max(acc["layer_flops"] / (tensor_peak * 1e12),
@@ -412,6 +446,7 @@ def run_ours(args, cfg, rank, world):
         "data": "synthetic (seeded; random weights of the workload's shapes)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
                    "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg),
+                   **act_config(cfg),
                    "parallelism": f"replicas x{world}",
                    "l2": f"no flush: weights touched per step {acc['weight_bytes_total'] / 1e9:.2f} GB "
                          f"> L2 {L2_BYTES / 2 ** 20:.0f} MiB",
@@ -451,7 +486,8 @@ def run_reference(args, cfg):
         "steps": K, "warmup": Wm, "ms_per_step": t / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
-                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg)},
+                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg),
+                   **act_config(cfg)},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{S} tokens per step of {cfg.T} (routing of all), fp64 NumPy"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -47,7 +47,7 @@ typedef enum {
     MOE_ERR_NOT_PREPARED = 8         /* FP4 weights used before moe_prepare_weights */
 } moe_status_t;
 
-typedef enum { MOE_ACT_SILU = 0, MOE_ACT_SITU = 1 } moe_act_t;
+typedef enum { MOE_ACT_SILU = 0, MOE_ACT_SITU = 1, MOE_ACT_SWIGLUOAI = 2 } moe_act_t;
 
 typedef enum { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt_t;
 
@@ -90,7 +90,8 @@ typedef struct {
 /* Gated activation. SITU (TRTLLM MXFP4 page, TrtLlmMxfp4ExpertsBase, SITU
  * comment): left = situ_alpha*tanh(g/situ_alpha)*sigmoid(g),
  * right = situ_beta*tanh(u/situ_beta); both must be > 0 (else INVALID_ARG).
- * SILU: silu(g)*u (MoonEP page, module docstring). */
+ * SILU: silu(g)*u (MoonEP page, module docstring). SWIGLUOAI takes three more
+ * parameters and is described with moe_act_ex_t. */
 typedef struct {
     int32_t act;            /* moe_act_t */
     float situ_alpha;       /* activation_situ_beta */
@@ -234,6 +235,46 @@ moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm
                              moe_stream_t stream);
 
 /*
+ * Every gated activation with its parameters. SWIGLUOAI is listed among the MXFP4
+ * experts' activations, with gemm1_alpha, gemm1_beta and gemm1_clamp_limit set to one
+ * value for every local expert (TRTLLM MXFP4 page, TrtLlmMxfp4ExpertsBase:
+ * _supports_activation and __init__). The page gives no formula; it is taken as the
+ * published GPT-OSS gated activation:
+ *   g = min(gate, swiglu_limit),  u = clamp(up, -swiglu_limit, swiglu_limit),
+ *   act = g * sigmoid(swiglu_alpha * g) * (u + swiglu_beta)
+ * with swiglu_alpha and swiglu_beta finite and swiglu_limit > 0 (+inf: no clamp), else
+ * INVALID_ARG. GPT-OSS uses alpha = 1.702, beta = 1, limit = 7.
+ */
+typedef struct {
+    int32_t act;            /* moe_act_t */
+    float situ_alpha;       /* SITU, as in moe_act_params_t */
+    float situ_beta;
+    float swiglu_alpha;     /* SWIGLUOAI: gemm1_alpha */
+    float swiglu_beta;      /* gemm1_beta */
+    float swiglu_limit;     /* gemm1_clamp_limit */
+} moe_act_ex_t;
+
+/*
+ * S4 with per-expert biases (TRTLLM MXFP4 page, TrtLlmMxfp4ExpertsModular._invoke_kernel:
+ * gemm1_bias is handed to the gate/up GEMM). For every row r of segment g
+ * (cu_seqlens[g-1] <= r < cu_seqlens[g], inclusive ends):
+ *   out[r,i] = act(gate[r,i] + bias_gate[g,i], up[r,i] + bias_up[g,i]) * perm_w[r]
+ * rows r >= cu_seqlens[G-1] are written as zero.
+ *   gate, up   [M,I] bf16 (in_is_f32 = 0) or fp32 (in_is_f32 = 1); out bf16 [M,I].
+ *   bias_gate, bias_up  fp32 [G,I], or NULL (no bias); perm_w fp32 [M] or NULL (weight 1).
+ *   cu_seqlens int32 [G] on device, non-decreasing; G >= 1.
+ *   act: any moe_act_t with its parameters (moe_act_ex_t, a HOST pointer).
+ * fp32 arithmetic, one bf16 rounding. I % 8 == 0 and 16-byte aligned gate, up, out and
+ * biases, else MOE_ERR_ALIGNMENT. moe_act_and_mul answers SWIGLUOAI with UNSUPPORTED,
+ * as moe_act_params_t has no room for its parameters.
+ */
+moe_status_t moe_bias_act_and_mul(const void* gate, const void* up, int in_is_f32,
+                                  const float* bias_gate, const float* bias_up,
+                                  const int32_t* cu_seqlens, int G, const float* perm_w,
+                                  int M, int I, const moe_act_ex_t* act, void* out,
+                                  moe_stream_t stream);
+
+/*
  * S6 — combine: out[t] = sum_k w_k * y_perm[inv_perm[t,k]], summed in fp32 in k
  * order and rounded once to bf16 (TRTLLM MXFP4 page, do_finalize). topk_w fp32
  * [T,topk], or NULL when the route weight was already applied (w_k = 1).
@@ -338,10 +379,28 @@ typedef struct {
      * once to bf16) and the activation and the combine take no weight (MoonEP experts
      * page, MoonEPExperts.apply). topk != 1: INVALID_ARG. */
     int32_t apply_router_weight_on_input;
+    /* SWIGLUOAI parameters, used when act.act == MOE_ACT_SWIGLUOAI (moe_act_ex_t). */
+    float swiglu_alpha, swiglu_beta, swiglu_limit;
+    /* Per-expert GEMM biases, fp32, each NULL or present (TRTLLM MXFP4 page,
+     * TrtLlmMxfp4ExpertsModular._invoke_kernel: gemm1_bias and gemm2_bias):
+     * bias_gate, bias_up [E+B, I] are added to the gate and up projections before the
+     * activation; bias_down [E+B, H] to the down projection, so it is scaled by the route
+     * weight with the rest of the expert's output. A redundant slot reads its own rows. */
+    const float* bias_gate;
+    const float* bias_up;
+    const float* bias_down;
 } moe_forward_args_t;
 
+/* With SWIGLUOAI or any bias the gate and up projections run as two grouped GEMMs with
+ * fp32 outputs, followed by a row pass that adds the biases and applies the activation
+ * and the route weight (moe_bias_act_and_mul), and the down bias is added to the down
+ * projection's fp32 rows before the combine. That needs 8*T_max*topk*I more workspace
+ * bytes: size it with moe_forward_workspace_size_args, which reads T_max, H, I, E, B,
+ * topk, w_gate.fmt, act_quant, act.act and the three bias pointers of `args` and
+ * otherwise equals moe_forward_workspace_size. */
 size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,
                                   int wfmt, int act_quant);
+size_t moe_forward_workspace_size_args(const moe_forward_args_t* args);
 moe_status_t moe_forward(const moe_forward_args_t* args, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 

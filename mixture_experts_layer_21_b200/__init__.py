@@ -28,7 +28,7 @@ MOE_OK = 0
 STATUS = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_ALIGNMENT",
           "MOE_ERR_WORKSPACE_TOO_SMALL", "MOE_ERR_CUDA", "MOE_ERR_DEVICE", "MOE_ERR_TIMEOUT",
           "MOE_ERR_NOT_PREPARED"]
-ACT = {"silu": 0, "situ": 1}
+ACT = {"silu": 0, "situ": 1, "swigluoai": 2}
 WFMT = {"bf16": 0, "mxfp4": 1, "nvfp4": 2}
 
 # Every symbol include/moe.h declares.
@@ -36,7 +36,8 @@ EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_wo
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
            "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc",
-           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8", "moe_route_topk_grouped"]
+           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8", "moe_route_topk_grouped",
+           "moe_bias_act_and_mul", "moe_forward_workspace_size_args"]
 
 
 class MoEError(RuntimeError):
@@ -57,6 +58,12 @@ class moe_act_params_t(ctypes.Structure):
     _fields_ = [("act", ctypes.c_int32), ("situ_alpha", ctypes.c_float), ("situ_beta", ctypes.c_float)]
 
 
+class moe_act_ex_t(ctypes.Structure):
+    _fields_ = [("act", ctypes.c_int32), ("situ_alpha", ctypes.c_float), ("situ_beta", ctypes.c_float),
+                ("swiglu_alpha", ctypes.c_float), ("swiglu_beta", ctypes.c_float),
+                ("swiglu_limit", ctypes.c_float)]
+
+
 class moe_forward_args_t(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("router_logits", ctypes.c_void_p),
                 ("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
@@ -71,7 +78,10 @@ class moe_forward_args_t(ctypes.Structure):
                 ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_float),
                 ("topk_ids_in", ctypes.c_void_p), ("topk_w_in", ctypes.c_void_p),
-                ("apply_router_weight_on_input", ctypes.c_int32)]
+                ("apply_router_weight_on_input", ctypes.c_int32),
+                ("swiglu_alpha", ctypes.c_float), ("swiglu_beta", ctypes.c_float),
+                ("swiglu_limit", ctypes.c_float),
+                ("bias_gate", ctypes.c_void_p), ("bias_up", ctypes.c_void_p), ("bias_down", ctypes.c_void_p)]
 
 ROUTING = {"renormalize": 0, "deepseek_v3": 1, "given": 2}
 
@@ -99,6 +109,8 @@ _sig = {
     "moe_grouped_gemm_nvfp4": (_I, [_P, _P, _P, _I, ctypes.POINTER(moe_weight_t), _P, _P, _P, _S, _P]),
     "moe_quantize_mxfp8": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_route_topk_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),
+    "moe_bias_act_and_mul": (_I, [_P, _P, _I, _P, _P, _P, _I, _P, _I, _I, ctypes.POINTER(moe_act_ex_t), _P, _P]),
+    "moe_forward_workspace_size_args": (_S, [ctypes.POINTER(moe_forward_args_t)]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -274,6 +286,27 @@ def moe_act_and_mul(gate, up, perm_w=None, act: str = "silu", situ_alpha=1.0, si
     return out
 
 
+def act_ex(act: str = "silu", situ_alpha: float = 1.0, situ_beta: float = 1.0, swiglu_alpha: float = 1.702,
+           swiglu_beta: float = 1.0, swiglu_limit: float | None = 7.0) -> moe_act_ex_t:
+    """Activation and parameters; ``swiglu_limit=None`` means no clamp (+inf)."""
+    lim = float("inf") if swiglu_limit is None else swiglu_limit
+    return moe_act_ex_t(ACT[act], situ_alpha, situ_beta, swiglu_alpha, swiglu_beta, lim)
+
+
+def moe_bias_act_and_mul(gate, up, cu_seqlens, bias_gate=None, bias_up=None, perm_w=None, act: str = "silu",
+                         situ_alpha=1.0, situ_beta=1.0, swiglu_alpha=1.702, swiglu_beta=1.0, swiglu_limit=7.0,
+                         out=None, stream=None):
+    """S4 with per-expert biases (fp32 [G,I]) and any activation, SWIGLUOAI included. gate/up
+    bf16 or fp32 [M,I]; bf16 out [M,I]; rows past cu_seqlens[-1] come out zero."""
+    M, I = gate.shape
+    out = out if out is not None else torch.empty(M, I, dtype=torch.bfloat16, device=gate.device)
+    a = act_ex(act, situ_alpha, situ_beta, swiglu_alpha, swiglu_beta, swiglu_limit)
+    _check(_lib.moe_bias_act_and_mul(_ptr(gate), _ptr(up), 1 if gate.dtype == torch.float32 else 0, _ptr(bias_gate),
+                                     _ptr(bias_up), _ptr(cu_seqlens), cu_seqlens.numel(), _ptr(perm_w), M, I,
+                                     ctypes.byref(a), _ptr(out), _stream(stream)), "moe_bias_act_and_mul")
+    return out
+
+
 def moe_combine(y_perm, inv_perm, topk_w=None, out=None, stream=None):
     T, k = inv_perm.shape
     H = y_perm.shape[1]
@@ -319,7 +352,12 @@ class MoEForward:
                  replica_src=None, act: str = "silu", situ_alpha=1.0, situ_beta=1.0,
                  act_quant: int = 0, apply_topk_in_fc1: bool = True, T_max: int = 1,
                  routing: str = "renormalize", routing_bias=None, n_group: int = 1, topk_group: int = 1,
-                 routed_scaling_factor: float = 1.0, apply_router_weight_on_input: bool = False):
+                 routed_scaling_factor: float = 1.0, apply_router_weight_on_input: bool = False,
+                 swiglu_alpha: float = 1.702, swiglu_beta: float = 1.0, swiglu_limit: float | None = 7.0,
+                 biases=None):
+        """``biases``: None, or (bias_gate [E+B,I], bias_up [E+B,I], bias_down [E+B,H]) fp32
+        device tensors, each of which may be None. With act "swigluoai" or any bias the layer
+        runs gate and up as two GEMMs and a bias/activation row pass."""
         for w in (w_gate, w_up, w_down):
             if w.fmt != "bf16" and w.prepared is None:
                 moe_prepare_weights(w)
@@ -331,9 +369,20 @@ class MoEForward:
         self.act_quant = act_quant
         self.apply_topk_in_fc1 = apply_topk_in_fc1
         self.T_max = T_max
-        self.ws = forward_workspace(T_max, self.H, self.I, E, B, topk, w_gate.fmt, act_quant,
-                                    w_gate.data.device)
         self.args = moe_forward_args_t()
+        a = self.args
+        a.swiglu_alpha, a.swiglu_beta = swiglu_alpha, swiglu_beta
+        a.swiglu_limit = float("inf") if swiglu_limit is None else swiglu_limit
+        self.biases = tuple(biases) if biases is not None else (None, None, None)
+        a.bias_gate, a.bias_up, a.bias_down = (_ptr(b) for b in self.biases)
+        if act == "swigluoai" or any(b is not None for b in self.biases):
+            a.T_max, a.H, a.I, a.E, a.B, a.topk = T_max, self.H, self.I, E, B, topk
+            a.w_gate, a.act, a.act_quant = w_gate.desc, self.act, act_quant
+            n = _lib.moe_forward_workspace_size_args(ctypes.byref(a))
+            self.ws = torch.zeros(n, dtype=torch.uint8, device=w_gate.data.device)
+        else:
+            self.ws = forward_workspace(T_max, self.H, self.I, E, B, topk, w_gate.fmt, act_quant,
+                                        w_gate.data.device)
         self.args.routing = ROUTING[routing]
         self.routing_bias = routing_bias
         self.args.n_group, self.args.topk_group = n_group, topk_group

@@ -16,6 +16,14 @@ cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, 
 cudaError_t launch_scale_rows(const __nv_bfloat16* x, const float* w, int T, int H, __nv_bfloat16* out,
                               cudaStream_t st, bool pdl);
 moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaStream_t st);
+// Bias and gated-activation row passes (bias_act.cu): out = act(gate + bg[seg], up + bu[seg])
+// * perm_w over [M, I] (I % 8 == 0; rows past cu[G-1] written as zero), and
+// y[r,:] += perm_w[r] * b[seg(r),:] over fp32 [M, N] (N % 8 == 0).
+cudaError_t launch_bias_act(const void* gate, const void* up, bool in_f32, const float* bg, const float* bu,
+                            const int32_t* cu, int G, const float* perm_w, int M, int I, int act, float sa, float sb,
+                            float oa, float ob, float lim, void* out, bool out_f32, cudaStream_t st, bool pdl);
+cudaError_t launch_add_row_bias(float* y, const int32_t* cu, int G, const float* b, const float* perm_w, int M, int N,
+                                cudaStream_t st, bool pdl);
 
 int num_sms() {
     static int cached[64] = {0};
@@ -49,6 +57,16 @@ bool act_ok(const moe_act_params_t& a) {
     return false;
 }
 
+// SWIGLUOAI: finite alpha and beta, a clamp limit > 0 (+inf: none; NaN fails).
+bool swiglu_ok(float alpha, float beta, float limit) {
+    return std::isfinite(alpha) && std::isfinite(beta) && limit > 0.0f;
+}
+
+bool act_ex_ok(const moe_act_ex_t& a) {
+    if (a.act == MOE_ACT_SWIGLUOAI) return swiglu_ok(a.swiglu_alpha, a.swiglu_beta, a.swiglu_limit);
+    return act_ok(moe_act_params_t{a.act, a.situ_alpha, a.situ_beta});
+}
+
 // Checks one projection's descriptor against the expected shape.
 moe_status_t check_weight(const moe_weight_t& w, int G, int N, int K) {
     if (w.G != G || w.N != N || w.K != K || !w.data) return MOE_ERR_INVALID_ARG;
@@ -70,7 +88,7 @@ const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? 
 struct FwdWs {
     size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
         xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, mx_xq, mx_xperm, mx_act,
-        x_in, y, bytes;
+        x_in, y, gu_gate, gu_up, bytes;
 };
 
 // With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
@@ -80,7 +98,9 @@ inline bool nvf4_k(int act_quant, int K) { return act_quant == 1 && K % kNvf4Sta
 inline int mx8_terms(int act_quant) { return act_quant == 2 ? 1 : 2; }
 inline int nvf4_rec_bytes(int K) { return K / 2 + K / 16; }
 
-FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
+// split: the gate and up projections run as two plain GEMMs into fp32 [NvS, I] buffers
+// (SWIGLUOAI or biases); those two buffers come last, so the other offsets do not move.
+FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant, bool split = false) {
     FwdWs L{};
     const size_t NvS = (size_t)T_max * topk;
     const int G = E + B;
@@ -121,6 +141,8 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.mx_act = take(mx ? NvS * mx8_rec_bytes(I, terms) : 0);
     L.x_in = take(topk == 1 ? 2 * (size_t)T_max * H : 0);  // x times the top-1 weight (input-side weighting)
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
+    L.gu_gate = take(split ? 4 * NvS * I : 0);
+    L.gu_up = take(split ? 4 * NvS * I : 0);
     L.bytes = off;
     return L;
 }
@@ -327,6 +349,7 @@ moe_status_t moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sb,
 
 moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm_w, int M, int I,
                              moe_act_params_t act, void* out, moe_stream_t stream) {
+    if (act.act == MOE_ACT_SWIGLUOAI) return MOE_ERR_UNSUPPORTED;  // its parameters: moe_bias_act_and_mul
     if (M < 0 || I < 0 || !act_ok(act)) return MOE_ERR_INVALID_ARG;
     if ((size_t)M * I == 0) return MOE_OK;
     if (!gate || !up || !out) return MOE_ERR_INVALID_ARG;
@@ -335,6 +358,20 @@ moe_status_t moe_act_and_mul(const void* gate, const void* up, const float* perm
                                           static_cast<const __nv_bfloat16*>(up), perm_w, M, I, act.act,
                                           act.situ_alpha, act.situ_beta, static_cast<__nv_bfloat16*>(out),
                                           S(stream), false));
+}
+
+moe_status_t moe_bias_act_and_mul(const void* gate, const void* up, int in_is_f32, const float* bias_gate,
+                                  const float* bias_up, const int32_t* cu_seqlens, int G, const float* perm_w, int M,
+                                  int I, const moe_act_ex_t* act, void* out, moe_stream_t stream) {
+    if (!act || M < 0 || I < 0 || G < 1) return MOE_ERR_INVALID_ARG;
+    if (!act_ex_ok(*act)) return MOE_ERR_INVALID_ARG;
+    if ((size_t)M * I == 0) return MOE_OK;
+    if (!gate || !up || !out || !cu_seqlens) return MOE_ERR_INVALID_ARG;
+    if (I % 8 || !aligned16(gate) || !aligned16(up) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+    if ((bias_gate && !aligned16(bias_gate)) || (bias_up && !aligned16(bias_up))) return MOE_ERR_ALIGNMENT;
+    return cuda_status(launch_bias_act(gate, up, in_is_f32 != 0, bias_gate, bias_up, cu_seqlens, G, perm_w, M, I,
+                                       act->act, act->situ_alpha, act->situ_beta, act->swiglu_alpha,
+                                       act->swiglu_beta, act->swiglu_limit, out, false, S(stream), false));
 }
 
 moe_status_t moe_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w, int T, int topk, int H,
@@ -386,13 +423,33 @@ size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int top
     return fwd_layout(T_max, H, I, E, B, topk, wfmt, act_quant).bytes;
 }
 
+}  // extern "C"
+
+namespace {
+// The layer runs gate and up as two GEMMs plus a bias/activation row pass.
+bool split_fc1(const moe_forward_args_t& a) {
+    return a.act.act == MOE_ACT_SWIGLUOAI || a.bias_gate || a.bias_up || a.bias_down;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_forward_workspace_size_args(const moe_forward_args_t* a) {
+    if (!a || a->T_max < 0 || a->H < 1 || a->I < 1 || a->E < 1 || a->B < 0 || a->topk < 1) return 0;
+    return fwd_layout(a->T_max, a->H, a->I, a->E, a->B, a->topk, a->w_gate.fmt, a->act_quant, split_fc1(*a)).bytes;
+}
+
 moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes, moe_stream_t stream) {
     if (!p) return MOE_ERR_INVALID_ARG;
     const int T = p->T, H = p->H, I = p->I, E = p->E, B = p->B, k = p->topk;
     if (T < 0 || H < 1 || I < 1 || E < 1 || B < 0 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
     if (T > p->T_max) return MOE_ERR_INVALID_ARG;  // the workspace was sized for T_max tokens
     if (E > kMaxExperts || E + B > 1024 || k > kMaxTopk) return MOE_ERR_UNSUPPORTED;
-    if (!act_ok(p->act)) return MOE_ERR_INVALID_ARG;
+    if (p->act.act == MOE_ACT_SWIGLUOAI) {
+        if (!swiglu_ok(p->swiglu_alpha, p->swiglu_beta, p->swiglu_limit)) return MOE_ERR_INVALID_ARG;
+    } else if (!act_ok(p->act)) {
+        return MOE_ERR_INVALID_ARG;
+    }
     // routing: 0 = softmax -> top-k -> renormalise, 1 = DeepSeekV3 grouped top-k, 2 = given
     if (p->routing < 0 || p->routing > 2) return MOE_ERR_INVALID_ARG;
     if (p->routing == 2 && (!p->topk_ids_in || !p->topk_w_in)) return MOE_ERR_INVALID_ARG;
@@ -415,13 +472,15 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (H % 16 || I % 16) return MOE_ERR_ALIGNMENT;
     if (B > 0 && !p->replica_src) return MOE_ERR_INVALID_ARG;
     if (!ws) return MOE_ERR_INVALID_ARG;
-    if (ws_bytes < moe_forward_workspace_size(p->T_max, H, I, E, B, k, fmt, p->act_quant))
-        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const bool split = split_fc1(*p);
+    const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant, split);
+    if (ws_bytes < L.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (T == 0) return MOE_OK;
     if (!p->x || (!p->router_logits && p->routing != 2) || !p->out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(p->x) || !aligned16(p->out) || !aligned16(ws)) return MOE_ERR_ALIGNMENT;
+    for (const float* b : {p->bias_gate, p->bias_up, p->bias_down})
+        if (b && !aligned16(b)) return MOE_ERR_ALIGNMENT;
 
-    const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant);
     char* w = static_cast<char*>(ws);
     DevError* err = reinterpret_cast<DevError*>(w);
     const bool given = p->routing == 2;
@@ -585,7 +644,38 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         g1.out_kind = OUT_F32;
         row_pass = true;
     }
-    e = launch_grouped_gemm(g1, st, pdl());
+    if (split) {
+        // SWIGLUOAI or biases: gate and up as two plain grouped GEMMs with fp32 outputs,
+        // then one row pass adds the biases and applies the activation and route weight
+        GemmProblem gg = g1;
+        gg.dual = false;
+        gg.w1 = nullptr;
+        gg.kdata1 = nullptr;
+        gg.kscale1 = nullptr;
+        gg.alpha1 = nullptr;
+        gg.perm_w = nullptr;
+        gg.act = MOE_ACT_SILU;
+        gg.out_scale = 1.0f;
+        gg.out_kind = OUT_F32;
+        gg.out = w + L.gu_gate;
+        e = launch_grouped_gemm(gg, st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        gg.w0 = p->w_up.data;
+        gg.kdata0 = p->w_up.kdata;
+        gg.kscale0 = p->w_up.kscale;
+        gg.alpha0 = weight_alpha(p->w_up);
+        gg.out = w + L.gu_up;
+        e = launch_grouped_gemm(gg, st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        // h in fp32 when a row pass quantises or stages it for FP4 weights, else bf16
+        row_pass = fmt != MOE_W_BF16;
+        fc2_out_scale = 1.0f;
+        e = launch_bias_act(w + L.gu_gate, w + L.gu_up, true, p->bias_gate, p->bias_up, cu, G, g1.perm_w, NvS, I,
+                            p->act.act, p->act.situ_alpha, p->act.situ_beta, p->swiglu_alpha, p->swiglu_beta,
+                            p->swiglu_limit, act, row_pass, st, pdl());
+    } else {
+        e = launch_grouped_gemm(g1, st, pdl());
+    }
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
     const int rb2 = nvf4_rec_bytes(I);
     if (row_pass) {
@@ -640,7 +730,13 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         g2.xsf_stride = rb2;
     }
     e = launch_grouped_gemm(g2, st, pdl());
-    if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (p->bias_down) {
+        // the expert's down bias, under the route weight when the activation carries it
+        e = launch_add_row_bias(y, cu, G, p->bias_down, g1.perm_w, NvS, H, st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (!mark(5)) return MOE_ERR_CUDA;
     // S6: combine
     e = launch_combine_f32(y, inv, (p->apply_topk_in_fc1 || in_w) ? nullptr : tw, T, k, H,
                            static_cast<__nv_bfloat16*>(p->out), st, pdl());

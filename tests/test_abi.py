@@ -108,6 +108,8 @@ def _fwd(**kw):
     p.routed_scaling_factor = kw.get("scale", 1.0)
     p.apply_router_weight_on_input = kw.get("in_w", 0)
     p.apply_topk_in_fc1 = 1
+    p.swiglu_alpha, p.swiglu_beta, p.swiglu_limit = kw.get("oa", 1.702), kw.get("ob", 1.0), kw.get("lim", 7.0)
+    p.bias_gate, p.bias_up, p.bias_down = kw.get("bias_gate"), kw.get("bias_up"), kw.get("bias_down")
     nws = L.moe_forward_workspace_size(d["T_max"], d["H"], d["I"], d["E"], d["B"], d["topk"], d["fmt"], d["aq"])
     return p, nws
 
@@ -132,6 +134,12 @@ def _fwd(**kw):
     (dict(in_w=1), INVALID),                        # input-side weight needs top-1
     (dict(routing=1, n_group=3), INVALID),          # E % n_group
     (dict(routing=1, n_group=2, topk_group=1, scale=0.0), INVALID),
+    (dict(act=2, oa=float("nan")), INVALID),        # SWIGLUOAI: finite alpha and beta,
+    (dict(act=2, ob=float("inf")), INVALID),
+    (dict(act=2, lim=0.0), INVALID),                # a clamp limit > 0
+    (dict(act=2, lim=float("nan")), INVALID),
+    (dict(bias_gate=8), ALIGN),                     # biases 16-byte aligned
+    (dict(bias_down=24), ALIGN),
 ])
 def test_forward_validation(kw, expect):
     p, nws = _fwd(**kw)
@@ -213,3 +221,95 @@ def test_nvfp4_prepared_bytes_hold_both_tile_layouts():
     NT = 2
     assert one >= G * NT * 6 * (4096 + 512)
     assert both >= G * NT * 8 * (4096 + 512) + G * NT * 2 * (16384 + 2048)
+
+
+def _c_struct(name):
+    """(field, kind) of a typedef struct in moe.h, in declaration order; kind is i32, f32, ptr
+    or the name of a nested struct."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r"\s*;", src).group(1)
+    out = []
+    for decl in filter(None, (d.strip() for d in body.split(";"))):
+        first, *rest = decl.split(",")
+        fname = re.findall(r"\w+", first)[-1]
+        base = first[: first.rindex(fname)]
+        btype = [t for t in re.findall(r"\w+", base) if t != "const"][0]
+        for d, nm in [(first, fname)] + [(r, re.findall(r"\w+", r)[-1]) for r in rest]:
+            ptr = "*" in base or "*" in d[len(base):]
+            out.append((nm, "ptr" if ptr else {"int32_t": "i32", "float": "f32"}.get(btype, btype)))
+    return out
+
+
+def _ctypes_struct(cls):
+    kinds = {ctypes.c_int32: "i32", ctypes.c_float: "f32", ctypes.c_void_p: "ptr"}
+    return [(n, kinds.get(t, t.__name__)) for n, t in cls._fields_]
+
+
+@pytest.mark.parametrize("name", ["moe_weight_t", "moe_act_params_t", "moe_act_ex_t", "moe_forward_args_t"])
+def test_binding_structs_match_the_header(name):
+    # the ctypes mirrors must list the header's fields in its order with the same kinds,
+    # so that both compilers lay them out alike
+    assert _ctypes_struct(getattr(m, name)) == _c_struct(name)
+
+
+def test_forward_workspace_with_biases_or_swigluoai():
+    p, nws = _fwd()
+    assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == nws      # fused gate/up: the same size
+    p, _ = _fwd(act=2)
+    n2 = L.moe_forward_workspace_size_args(ctypes.byref(p))
+    assert n2 >= nws + 8 * (8 * 2) * 128                                  # two fp32 [T_max*topk, I] buffers
+    assert L.moe_forward(ctypes.byref(p), 16, nws, None) == WS_SMALL
+    for b in ("bias_gate", "bias_up", "bias_down"):
+        p, _ = _fwd(**{b: 16})
+        assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == n2
+        p.T = 0
+        assert L.moe_forward(ctypes.byref(p), 16, n2, None) == 0           # no tokens: nothing launched
+    assert L.moe_forward_workspace_size_args(None) == 0
+
+
+def test_bias_act_validation():
+    f = L.moe_bias_act_and_mul
+
+    def call(act, M=4, I=16, G=2, gate=16, bg=None, cu=16):
+        return f(gate, 16, 0, bg, None, cu, G, None, M, I, ctypes.byref(act), 16, None)
+
+    ok = m.act_ex()
+    assert call(m.act_ex("swigluoai", swiglu_limit=0.0)) == INVALID
+    assert call(m.act_ex("swigluoai", swiglu_alpha=float("inf"))) == INVALID
+    assert call(m.act_ex("situ", situ_alpha=-1.0)) == INVALID
+    assert call(m.moe_act_ex_t(7, 1.0, 1.0, 1.0, 1.0, 1.0)) == INVALID
+    assert call(ok, G=0) == INVALID
+    assert call(ok, M=0) == 0                                     # no rows: nothing launched
+    assert call(ok, I=12) == ALIGN                                # I % 8
+    assert call(ok, bg=8) == ALIGN                                # bias not 16-byte aligned
+    assert call(ok, gate=None) == INVALID
+    assert call(ok, cu=None) == INVALID
+    assert f(16, 16, 0, None, None, 16, 2, None, 4, 16, None, 16, None) == INVALID   # no activation
+    # moe_act_params_t has no room for SWIGLUOAI's parameters
+    assert L.moe_act_and_mul(16, 16, None, 4, 16, m.moe_act_params_t(2, 1.0, 1.0), 16, None) == UNSUP
+
+
+def test_binding_struct_offsets_match_gcc(tmp_path):
+    # the header compiled by the host C compiler: every field's offset and every struct's
+    # size equal the ctypes mirror's
+    names = ["moe_weight_t", "moe_act_params_t", "moe_act_ex_t", "moe_forward_args_t"]
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "moe.h"', "int main(void) {"]
+    for n in names:
+        lines.append(f'printf("{n} sizeof %zu\\n", sizeof({n}));')
+        for f, _ in _c_struct(n):
+            lines.append(f'printf("{n} {f} %zu\\n", offsetof({n}, {f}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        n, f, v = line.split()
+        got[(n, f)] = int(v)
+    for n in names:
+        cls = getattr(m, n)
+        assert got[(n, "sizeof")] == ctypes.sizeof(cls), n
+        for f, _ in cls._fields_:
+            assert got[(n, f)] == getattr(cls, f).offset, (n, f)

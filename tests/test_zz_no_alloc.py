@@ -7,8 +7,8 @@ inside the library; this checks, through the C ABI, that two calls in a row give
 same results as the workspace-taking entry point. Indices and gathered rows are
 integer/byte data, so the comparison is bit-exact.
 
-The file name sorts last so that a run stopping at the first failure has run every
-other test first.
+The file name sorts late so that a run stopping at the first failure has run the
+other tests first.
 """
 import numpy as np
 import pytest

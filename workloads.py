@@ -62,6 +62,8 @@ class MoEConfig:
     swiglu_beta: float = 1.0
     swiglu_limit: float | None = 7.0
     bias: bool = False                 # per-row GEMM biases (gemm1_bias, gemm2_bias)
+    bias_std: float = 0.1              # their spread: gate and up, and down
+    bias_down_std: float = 0.1
     n_group: int = 1
     topk_group: int = 1
     routed_scaling_factor: float = 1.0
@@ -109,6 +111,14 @@ CONFIGS: dict[str, MoEConfig] = {
                                          B=16, B_used=8, logit_std=2.0, routing="deepseek_v3", n_group=8,
                                          topk_group=4, routed_scaling_factor=2.5),
     # the W4A8 mode of the MXFP4 experts: the MXFP4 shapes with dynamic MXFP8 activations
+    # the MXFP4 shapes with SWIGLUOAI (GPT-OSS constants) and per-expert GEMM biases, spread
+    # near the projections' own magnitudes (gate/up ~18, down ~400 with these weights)
+    "mxfp4_swiglu_bias_decode": MoEConfig("mxfp4_swiglu_bias_decode", T=32, H=2880, I=2880, E=128, topk=4,
+                                          act="swigluoai", wfmt=WFMT_MXFP4, bias=True, bias_std=10.0,
+                                          bias_down_std=400.0),
+    "mxfp4_swiglu_bias_prefill": MoEConfig("mxfp4_swiglu_bias_prefill", T=4096, H=2880, I=2880, E=128, topk=4,
+                                           act="swigluoai", wfmt=WFMT_MXFP4, bias=True, bias_std=10.0,
+                                           bias_down_std=400.0),
     "mxfp4_w4a8_decode": MoEConfig("mxfp4_w4a8_decode", T=32, H=2880, I=2880, E=128, topk=4,
                                    act="situ", wfmt=WFMT_MXFP4, act_quant=2),
     "mxfp4_w4a8_prefill": MoEConfig("mxfp4_w4a8_prefill", T=4096, H=2880, I=2880, E=128, topk=4,
@@ -141,13 +151,13 @@ def gen_routing_bias(cfg: MoEConfig) -> torch.Tensor:
 
 
 def gen_biases(cfg: MoEConfig) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Per-row GEMM biases: gate and up ``[G,I]``, down ``[G,H]``, fp32 N(0, 0.1^2); replica
-    slots copy their source expert's (use after ``gen_replica_src``)."""
+    """Per-row GEMM biases: gate and up ``[G,I]`` fp32 N(0, bias_std^2), down ``[G,H]`` fp32
+    N(0, bias_down_std^2); ``gen_inputs`` makes replica slots copy their source expert's."""
     g = _gen(cfg, _S_BIAS + 1)
     G = cfg.E + cfg.B
-    bg = torch.randn(G, cfg.I, generator=g) * 0.1
-    bu = torch.randn(G, cfg.I, generator=g) * 0.1
-    bd = torch.randn(G, cfg.H, generator=g) * 0.1
+    bg = torch.randn(G, cfg.I, generator=g) * cfg.bias_std
+    bu = torch.randn(G, cfg.I, generator=g) * cfg.bias_std
+    bd = torch.randn(G, cfg.H, generator=g) * cfg.bias_down_std
     return bg, bu, bd
 
 
