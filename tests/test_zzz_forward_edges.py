@@ -1,0 +1,70 @@
+"""GPU parity of the fused layer at the edges of its argument ranges: one token, one expert
+(a dense SwiGLU MLP), every expert chosen by every token, the largest top-k, the largest number
+of weight rows (E + B = 1024) and every token sending its first choice to one expert.
+
+Routing ids are compared bit-exactly and outputs with the BF16 tolerance of tests/parity.py
+(|d| <= 2e-2 + 2^-8 |ref| elementwise, rel-L2 <= 1e-2); the FP4 case with rel-L2 <= 3e-2.
+The file name sorts after the GPU files whose kernels these cases reuse, so a run that stops at
+its first failure has run those first.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import moe_oracle as O
+from tests.parity import FP4_REL_L2, check_bf16, rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+EDGES = {
+    "one_token": W.MoEConfig("one_token", T=1, H=128, I=256, E=8, topk=2),
+    "one_token_mxfp4": W.MoEConfig("one_token_mxfp4", T=1, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4"),
+    "one_token_nvfp4": W.MoEConfig("one_token_nvfp4", T=1, H=512, I=256, E=16, topk=8, wfmt="nvfp4",
+                                   act_quant=1),
+    "dense": W.MoEConfig("dense", T=77, H=128, I=192, E=1, topk=1),
+    "topk_is_E": W.MoEConfig("topk_is_E", T=50, H=128, I=128, E=4, topk=4),
+    "topk_32": W.MoEConfig("topk_32", T=20, H=128, I=128, E=64, topk=32),
+    "max_rows": W.MoEConfig("max_rows", T=64, H=128, I=128, E=1000, topk=8, B=24, B_used=12, logit_std=2.0),
+}
+
+
+def _run(lib, cfg, inp, logits):
+    dev = lambda ws: lib.Weight.from_host(ws)
+    layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, cfg.topk, cfg.B,
+                           to_dev(inp.replica_src) if cfg.B else None, cfg.act, cfg.situ_alpha, cfg.situ_beta,
+                           cfg.act_quant, True, T_max=cfg.T)
+    ids = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device="cuda")
+    out = layer(to_dev(inp.x), to_dev(logits), topk_ids=ids)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    ref = O.moe_forward(cfg, inp.x, logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down)
+    assert np.array_equal(ids.cpu().numpy(), ref["ids"])
+    if cfg.wfmt == "bf16":
+        check_bf16(out, ref["out"], what=cfg.name)
+    else:
+        r = rel_l2(out.float().cpu().numpy(), ref["out"])
+        assert r <= FP4_REL_L2, f"{cfg.name}: rel-L2 {r:.3e}"
+    return ref
+
+
+@pytest.mark.parametrize("name", list(EDGES))
+def test_forward_edges_match_oracle(lib, name):
+    cfg = EDGES[name]
+    inp = W.gen_inputs(cfg)
+    ref = _run(lib, cfg, inp, inp.logits)
+    if name == "max_rows":       # the replica slots are used and the last weight rows are reached
+        cu = ref["cu_seqlens"]
+        assert np.count_nonzero(np.diff(np.concatenate([[0], cu]))[cfg.E:]) > 0
+
+
+def test_forward_one_expert_takes_every_first_choice(lib):
+    # expert 3's logit is raised for every token: its segment holds all T rows (three token
+    # tiles, the last with one row) while the second choices spread over the rest
+    cfg = W.MoEConfig("skew", T=257, H=128, I=256, E=8, topk=2)
+    inp = W.gen_inputs(cfg)
+    logits = inp.logits.clone()
+    logits[:, 3] += 100.0
+    ref = _run(lib, cfg, inp, logits)
+    assert np.all(ref["ids"][:, 0] == 3)
+    assert int(ref["cu_seqlens"][3] - ref["cu_seqlens"][2]) == cfg.T
