@@ -149,7 +149,10 @@ moe_status_t moe_route_topk_grouped(const float* logits, const float* bias, int 
  *   A replicated expert's n assignments (ascending token) are cut into
  *   contiguous chunks over [e, its slots ascending], chunk i holding
  *   n/R + (i < n%R) rows. Indices are bit-exact with the oracle.
- *   An expert id outside [0,E) sets MOE_ERR_DEVICE in the workspace error word.
+ *   An expert id outside [0,E), or one expert listed twice by a token, sets MOE_ERR_DEVICE
+ *   in the workspace error word; the out-of-range assignment gets inv_perm = -1, and the
+ *   rows then left without an assignment (from cu_seqlens[E+B-1] to NvS) get token 0 and
+ *   weight 0, so that x_perm reads only rows of x.
  *   ws: at least moe_permute_workspace_size(T, topk, E, B) bytes.
  */
 size_t moe_permute_workspace_size(int T, int topk, int E, int B);
@@ -278,7 +281,8 @@ moe_status_t moe_bias_act_and_mul(const void* gate, const void* up, int in_is_f3
  * S6 — combine: out[t] = sum_k w_k * y_perm[inv_perm[t,k]], summed in fp32 in k
  * order and rounded once to bf16 (TRTLLM MXFP4 page, do_finalize). topk_w fp32
  * [T,topk], or NULL when the route weight was already applied (w_k = 1).
- * y_perm bf16 [>= T*topk, H]; out bf16 [T,H].
+ * y_perm bf16 [>= T*topk, H]; out bf16 [T,H]. A negative inv_perm entry (an assignment
+ * the permutation refused) contributes nothing.
  */
 moe_status_t moe_combine(const void* y_perm, const int32_t* inv_perm, const float* topk_w,
                          int T, int topk, int H, void* out, moe_stream_t stream);

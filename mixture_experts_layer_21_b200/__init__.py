@@ -226,21 +226,31 @@ def permute_workspace(T: int, topk: int, E: int, B: int, device="cuda") -> torch
 
 
 def moe_permute(topk_ids, topk_w, E: int, B: int = 0, replica_src=None, x=None, M_alloc=None,
-                ws=None, stream=None):
+                ws=None, stream=None, out=None):
+    """``out``: optional dict of caller-allocated outputs (any of cu_seqlens, perm_token,
+    perm_w, inv_perm, x_perm [M_alloc,H]); the others are allocated here."""
     T, k = topk_ids.shape
     dev = topk_ids.device
     NvS = T * k
+    out = out or {}
     M_alloc = NvS if M_alloc is None else M_alloc
     ws = ws if ws is not None else permute_workspace(T, k, E, B, dev)
-    cu = torch.empty(E + B, dtype=torch.int32, device=dev)
-    perm_token = torch.empty(NvS, dtype=torch.int32, device=dev)
-    perm_w = torch.empty(NvS, dtype=torch.float32, device=dev)
-    inv = torch.empty(T, k, dtype=torch.int32, device=dev)
+    def buf(name, shape, dtype):
+        t = out.get(name)
+        return t if t is not None else torch.empty(shape, dtype=dtype, device=dev)
+
+    cu = buf("cu_seqlens", (E + B,), torch.int32)
+    perm_token = buf("perm_token", (NvS,), torch.int32)
+    perm_w = buf("perm_w", (NvS,), torch.float32)
+    inv = buf("inv_perm", (T, k), torch.int32)
     x_perm = None
     H = 0
     if x is not None:
         H = x.shape[1]
-        x_perm = torch.zeros(M_alloc, H, dtype=x.dtype, device=dev)
+        x_perm = out.get("x_perm")
+        if x_perm is None:
+            x_perm = torch.zeros(M_alloc, H, dtype=x.dtype, device=dev)
+        M_alloc = x_perm.shape[0]
     _check(_lib.moe_permute(_ptr(topk_ids), _ptr(topk_w), T, k, E, B, _ptr(replica_src), _ptr(x), H,
                             _ptr(cu), _ptr(perm_token), _ptr(perm_w), _ptr(inv), _ptr(x_perm), M_alloc,
                             _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const YT* __restrict__ y,
         for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
         for (int j = 0; j < topk; ++j) {
             const int r = inv_perm[(size_t)t * topk + j];
+            if (r < 0) continue;  // an assignment the permutation refused (bad expert id)
             const float wj = topk_w ? topk_w[(size_t)t * topk + j] : 1.0f;
             float f[8];
             load8(y, (size_t)r, H, c8, f);

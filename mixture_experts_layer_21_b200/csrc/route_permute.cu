@@ -291,12 +291,16 @@ __global__ void __launch_bounds__(kPermBlock) permute_count_kernel(const int32_t
 }
 
 // One block: per-expert running sums over token blocks, the replica split and the
-// inclusive scan of segment lengths over the G = E + B weight rows.
+// inclusive scan of segment lengths over the G = E + B weight rows. Rows from the last
+// segment end up to NvS receive no assignment unless an id was bad (out of range, or an
+// expert listed twice by one token; both reported): they get token 0 and weight 0, so that
+// a gather over all NvS rows reads only rows of x.
 __global__ void __launch_bounds__(1024) permute_scan_kernel(
     const int* __restrict__ blkcnt, int nblk, int E, int B, const int32_t* __restrict__ replica_src,
     int* __restrict__ blkoff, int* __restrict__ total, int* __restrict__ nrep,
     int* __restrict__ rep_ptr, int* __restrict__ rep_rows, int* __restrict__ rowstart,
-    int32_t* __restrict__ cu_seqlens, DevError* err) {
+    int32_t* __restrict__ cu_seqlens, int NvS, int32_t* __restrict__ perm_token, float* __restrict__ perm_w,
+    DevError* err) {
     extern __shared__ int sm[];  // [G] segment sizes, then [1024] scan scratch
     const int G = E + B;
     int* seg = sm;
@@ -365,8 +369,12 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(
         }
     }
     __syncthreads();
-    block_exclusive_scan(seg, G, rowstart);
+    const int filled = block_exclusive_scan(seg, G, rowstart);
     for (int g = threadIdx.x; g < G; g += blockDim.x) cu_seqlens[g] = rowstart[g] + seg[g];
+    for (int r = filled + threadIdx.x; r < NvS; r += blockDim.x) {
+        perm_token[r] = 0;
+        perm_w[r] = 0.0f;
+    }
     pdl_launch();
 }
 
@@ -438,7 +446,7 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
     // the scan and scatter follow this function's own kernels: they always overlap with them
     e = launch_k(permute_scan_kernel, dim3(1), dim3(1024), scan_smem, st, L.nblk > 0 ? true : pdl,
                  (const int*)blkcnt, L.nblk, E, B, replica_src, blkoff, total, nrep, rep_ptr, rep_rows,
-                 rowstart, cu_seqlens, err);
+                 rowstart, cu_seqlens, T * topk, perm_token, perm_w, err);
     if (e != cudaSuccess) return e;
     if (L.nblk > 0) {
         e = launch_k(permute_scatter_kernel, dim3(L.nblk), dim3(kPermBlock), mask_smem, st, true, ids,

@@ -68,3 +68,61 @@ def test_forward_one_expert_takes_every_first_choice(lib):
     ref = _run(lib, cfg, inp, logits)
     assert np.all(ref["ids"][:, 0] == 3)
     assert int(ref["cu_seqlens"][3] - ref["cu_seqlens"][2]) == cfg.T
+
+
+# ------------------------------------------------------------------ bad ids and output margins
+# Set up so that every access stays in bounds whatever the kernels do with the bad rows:
+# perm_token starts at 0 (a valid token), and the combine's y_perm is a view that starts
+# inside a larger buffer.
+
+def test_permute_bad_ids_fill_unassigned_rows(lib):
+    # token 2 names expert 9 (E = 4) and token 5 names expert 1 twice: both are reported, the
+    # out-of-range assignment gets inv_perm = -1, and the two rows no assignment reaches get
+    # token 0 and weight 0; x_perm rows past M_alloc's NvS keep their canary
+    T, k, E, H = 8, 2, 4, 64
+    ids = torch.tensor([[0, 1], [2, 3], [9, 0], [1, 2], [3, 0], [1, 1], [2, 0], [3, 1]], dtype=torch.int32)
+    w = torch.full((T, k), 0.5)
+    x = W.gen_rows(T, H, seed=5)
+    canary_w = 7.0
+    canary_x = torch.full((T * k + 4, H), -3.0, dtype=torch.bfloat16)
+    out = dict(perm_token=torch.zeros(T * k, dtype=torch.int32, device="cuda"),
+               perm_w=torch.full((T * k,), canary_w, device="cuda"), x_perm=canary_x.cuda())
+    r = lib.moe_permute(to_dev(ids), to_dev(w), E, 0, x=to_dev(x), out=out)
+    assert lib.moe_get_device_error(r["ws"]) == 6             # MOE_ERR_DEVICE
+    cu = r["cu_seqlens"].cpu().numpy()
+    assert cu[-1] == T * k - 2
+    inv = r["inv_perm"].cpu().numpy()
+    assert inv[2, 0] == -1 and inv[5, 0] == inv[5, 1] >= 0
+    pt, pw = r["perm_token"].cpu().numpy(), r["perm_w"].cpu().numpy()
+    assert np.all(pt[cu[-1]:] == 0) and np.all(pw[cu[-1]:] == 0.0)
+    xp = r["x_perm"].cpu()
+    assert torch.equal(xp[cu[-1]:T * k], x[:1].expand(int(T * k - cu[-1]), H))
+    assert torch.equal(xp[T * k:], canary_x[T * k:])
+    # every valid assignment still lands on a row of its expert holding its token
+    for t in range(T):
+        for j in range(k):
+            e = int(ids[t, j])
+            if 0 <= e < E:
+                row = int(inv[t, j])
+                assert (cu[e - 1] if e else 0) <= row < cu[e] and pt[row] == t
+
+
+def test_combine_skips_refused_assignments(lib):
+    T, k, H = 5, 3, 64
+    rows = T * k
+    big = W.gen_rows(rows + 8, H, seed=9)
+    big[:8] = 1000.0                                          # canary rows before y_perm
+    y = big.cuda()[8:]
+    inv = torch.arange(rows, dtype=torch.int32).reshape(T, k)
+    inv[1, 2] = -1
+    inv[4, 0] = -1
+    tw = W.gen_rows(T, k, seed=10, dtype=torch.float32)
+    out = lib.moe_combine(y, to_dev(inv), to_dev(tw))
+    torch.cuda.synchronize()
+    yk = big[8:].double().numpy()
+    ref = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            if inv[t, j] >= 0:
+                ref[t] += float(tw[t, j]) * yk[int(inv[t, j])]
+    check_bf16(out, ref, what="combine with refused rows")
