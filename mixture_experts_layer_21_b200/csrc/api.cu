@@ -4,6 +4,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 namespace moe {
@@ -46,6 +48,28 @@ inline cudaStream_t S(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s)
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 inline size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Host-timeline ranges for profilers (NVTX): one around a whole call and one nested range
+// per stage, so that e.g. `ncu --nvtx --nvtx-include "moe_forward/gate_up/"` picks out one
+// stage's kernels. Without an attached tool each call is a branch.
+class Trace {
+  public:
+    explicit Trace(const char* name) { nvtxRangePushA(name); }
+    ~Trace() {
+        if (stage_) nvtxRangePop();
+        nvtxRangePop();
+    }
+    Trace(const Trace&) = delete;
+    Trace& operator=(const Trace&) = delete;
+    void stage(const char* name) {
+        if (stage_) nvtxRangePop();
+        nvtxRangePushA(name);
+        stage_ = true;
+    }
+
+  private:
+    bool stage_ = false;
+};
 
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopk = 32;
@@ -516,6 +540,8 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         return r;
     };
 
+    Trace trace("moe_forward");
+    trace.stage("route");
     if (!mark(0)) return MOE_ERR_CUDA;
     // S1 route (or the given top-k, copied to the optional outputs)
     int32_t* ids_w = const_cast<int32_t*>(ids);
@@ -543,6 +569,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         xin = w + L.x_in;
     }
     // S2 permute
+    trace.stage("permute");
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
                        pdl());
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -579,6 +606,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (e != cudaSuccess || !mark(2)) return MOE_ERR_CUDA;
 
     // S3 + S4: gate/up grouped GEMM with the activation epilogue
+    trace.stage("gate_up");
     const bool situ = p->act.act == MOE_ACT_SITU;
     GemmProblem g1{};
     g1.x = xperm;
@@ -678,6 +706,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     }
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
     const int rb2 = nvf4_rec_bytes(I);
+    trace.stage("act_row_pass");
     if (row_pass) {
         if (fmt == MOE_W_MXFP4) {
             const int rb = mx8_rec_bytes(I, terms), Kp = mx8_kpad(I);
@@ -701,6 +730,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     }
     if (!mark(4)) return MOE_ERR_CUDA;
     // S5: down grouped GEMM
+    trace.stage("down");
     GemmProblem g2{};
     g2.x = fc2_x;
     g2.M_alloc = NvS;
@@ -738,6 +768,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     }
     if (!mark(5)) return MOE_ERR_CUDA;
     // S6: combine
+    trace.stage("combine");
     e = launch_combine_f32(y, inv, (p->apply_topk_in_fc1 || in_w) ? nullptr : tw, T, k, H,
                            static_cast<__nv_bfloat16*>(p->out), st, pdl());
     if (e != cudaSuccess || !mark(6)) return MOE_ERR_CUDA;
