@@ -161,15 +161,20 @@ def test_forward_bias_weight_in_combine(lib):
 
 
 def test_forward_bias_input_weight_top1(lib):
-    # top-1 with the route weight on the input: no weight on the biases either
-    cfg = W.MoEConfig("bias_top1", T=90, H=128, I=192, E=8, topk=1, act="swigluoai", swiglu_limit=0.3, bias=True)
+    # a given top-1 with weights in [0.1, 2] on the input: the experts see x * w, and neither
+    # the activation nor the biases take the weight again
+    cfg = W.MoEConfig("bias_top1", T=90, H=128, I=192, E=8, topk=1, act="swigluoai", swiglu_limit=0.3, bias=True,
+                      bias_down_std=0.03)
     inp = W.gen_inputs(cfg)
-    layer = _layer(lib, cfg, inp, apply_router_weight_on_input=True)
-    out = layer(to_dev(inp.x), to_dev(inp.logits))
+    g = np.random.default_rng(3)
+    gid = g.integers(0, cfg.E, (cfg.T, 1)).astype(np.int32)
+    gw = g.uniform(0.1, 2.0, (cfg.T, 1)).astype(np.float32)
+    layer = _layer(lib, cfg, inp, routing="given", apply_router_weight_on_input=True)
+    out = layer(to_dev(inp.x), None, topk_ids_in=to_dev(torch.from_numpy(gid)), topk_w_in=to_dev(torch.from_numpy(gw)))
     torch.cuda.synchronize()
     assert layer.device_error() == 0
-    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, apply_router_weight_on_input=True, biases=inp.extra["biases"])
+    ref = O.moe_forward(cfg, inp.x, None, inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down,
+                        given_topk=(gid, gw), apply_router_weight_on_input=True, biases=inp.extra["biases"])
     check_bf16(out, ref["out"], what="bias, input weight")
 
 
