@@ -1,6 +1,9 @@
 """GPU parity of the fused layer at the edges of its argument ranges: one token, one expert
 (a dense SwiGLU MLP), every expert chosen by every token, the largest top-k, the largest number
-of weight rows (E + B = 1024) and every token sending its first choice to one expert.
+of weight rows (E + B = 1024) and every token sending its first choice to one expert. Also the
+NVFP4-weight layer with bf16 activations (act_quant = 0), whose f16 staging of x (a gather
+with a per-row power-of-two scale) and of h (a row pass, or SITU's fixed-scale f16 epilogue)
+no other forward case takes.
 
 Routing ids are compared bit-exactly and outputs with the BF16 tolerance of tests/parity.py
 (|d| <= 2e-2 + 2^-8 |ref| elementwise, rel-L2 <= 1e-2); the FP4 case with rel-L2 <= 3e-2.
@@ -26,6 +29,10 @@ EDGES = {
     "topk_is_E": W.MoEConfig("topk_is_E", T=50, H=128, I=128, E=4, topk=4),
     "topk_32": W.MoEConfig("topk_32", T=20, H=128, I=128, E=64, topk=32),
     "max_rows": W.MoEConfig("max_rows", T=64, H=128, I=128, E=1000, topk=8, B=24, B_used=12, logit_std=2.0),
+    "nvfp4_w4a16_silu": W.MoEConfig("nvfp4_w4a16_silu", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4"),
+    # K = 272 and 304: neither a multiple of the 64-value chunk, so x and h take 2-D tensor maps
+    "nvfp4_w4a16_situ": W.MoEConfig("nvfp4_w4a16_situ", T=40, H=272, I=304, E=8, topk=2, wfmt="nvfp4", act="situ",
+                                    situ_alpha=0.8, situ_beta=1.7),
 }
 
 
