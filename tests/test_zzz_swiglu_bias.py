@@ -191,3 +191,26 @@ def test_fullsize_swiglu_bias_decode(lib):
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
                         inp.w_down, biases=inp.extra["biases"])
     _check(cfg, out, ref["out"], cfg.name)
+
+
+@pytest.mark.slow
+def test_fullsize_swiglu_bias_prefill(lib):
+    # the MXFP4 prefill workload (T=4096) with SWIGLUOAI and biases as bench.py times it;
+    # ids for every token, outputs on the full-size tests' token sample
+    from tests.test_gpu_fullsize import _sample_tokens
+
+    cfg = W.CONFIGS["mxfp4_swiglu_bias_prefill"]
+    inp = W.gen_inputs(cfg)
+    layer = _layer(lib, cfg, inp)
+    ids = torch.empty(cfg.T, cfg.topk, dtype=torch.int32, device="cuda")
+    out = layer(to_dev(inp.x), to_dev(inp.logits), topk_ids=ids)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    rids, _ = O.route(cfg, inp.logits.numpy())
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    toks = _sample_tokens(cfg, O.assign_rows(rids, cfg.E, cfg.B, inp.replica_src.numpy()))
+    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
+                        inp.w_down, tokens=toks, biases=inp.extra["biases"])
+    got = out[torch.tensor(toks, device="cuda")].float().cpu().numpy()
+    r = rel_l2(got, ref["out"])
+    assert r <= FP4_REL_L2, f"{cfg.name}: rel-L2 {r:.3e}"
