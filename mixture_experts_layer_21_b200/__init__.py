@@ -434,6 +434,25 @@ class MoEForward:
     def device_error(self, stream=None) -> int:
         return _lib.moe_get_device_error(_ptr(self.ws), _stream(stream))
 
+    def graph(self, x, router_logits=None, out=None, warmup: int = 1, **kw):
+        """One forward on these buffers captured into a CUDA graph; ``graph.replay()`` reruns the
+        layer on whatever x / router_logits (and the given top-k, if any) then hold and writes
+        ``out``. ``warmup`` eager calls on a side stream come first: they also set the library's
+        one-time host state (kernel attributes, the SM count), which must not be set up during
+        capture. Returns ``(graph, out)``."""
+        T = x.shape[0]
+        out = out if out is not None else torch.empty(T, self.H, dtype=torch.bfloat16, device=x.device)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                self(x, router_logits, out=out, **kw)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(x, router_logits, out=out, **kw)
+        return g, out
+
 
 def moe_forward(x, router_logits, w_gate: Weight, w_up: Weight, w_down: Weight, E: int, topk: int,
                 B: int = 0, replica_src=None, act="silu", situ_alpha=1.0, situ_beta=1.0, act_quant=0,

@@ -133,3 +133,35 @@ def test_combine_skips_refused_assignments(lib):
             if inv[t, j] >= 0:
                 ref[t] += float(tw[t, j]) * yk[int(inv[t, j])]
     check_bf16(out, ref, what="combine with refused rows")
+
+
+# ------------------------------------------------------------------ CUDA graph capture
+
+@pytest.mark.parametrize("name", ["replicas_bf16", "mxfp4", "nvfp4"])
+def test_forward_graph_replay_matches_eager(lib, name):
+    # the forward (programmatic dependent launches, no host sync, no allocation) captured once
+    # and replayed: bitwise the eager result, also after new inputs are copied into the
+    # captured buffers
+    cfg = {"replicas_bf16": W.MoEConfig("g_bf16", T=300, H=128, I=256, E=16, topk=4, B=6, B_used=4),
+           "mxfp4": W.MoEConfig("g_mxfp4", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4"),
+           "nvfp4": W.MoEConfig("g_nvfp4", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4", act_quant=1)}[name]
+    inp = W.gen_inputs(cfg)
+    inp2 = W.gen_inputs(cfg.with_(seed=1))
+    dev = lambda ws: lib.Weight.from_host(ws)
+    layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, cfg.topk, cfg.B,
+                           to_dev(inp.replica_src) if cfg.B else None, cfg.act, cfg.situ_alpha, cfg.situ_beta,
+                           cfg.act_quant, True, T_max=cfg.T)
+    x, logits = to_dev(inp.x), to_dev(inp.logits)
+    eager1 = layer(x, logits).clone()
+    eager2 = layer(to_dev(inp2.x), to_dev(inp2.logits)).clone()
+    g, out = layer.graph(x, logits)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager1)
+    x.copy_(to_dev(inp2.x))
+    logits.copy_(to_dev(inp2.logits))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager2)
+    assert layer.device_error() == 0
+    del g
