@@ -618,6 +618,9 @@ def test_swigluoai_reductions_and_clamps():
     # a gate below -limit is not clamped (the gate has an upper clamp only)
     v = O.swigluoai_and_mul(np.array([-9.0]), np.array([0.5]), 1.0, 1.0, lim)[0]
     assert v == -9.0 / (1.0 + math.exp(9.0)) * 1.5
+    # an infinite limit (the C ABI's "no clamp") is no clamp
+    assert np.array_equal(O.swigluoai_and_mul(gate, up, 1.702, 1.0, np.inf),
+                          O.swigluoai_and_mul(gate, up, 1.702, 1.0, None))
 
 
 def test_biases_closed_form_and_layer_loop():
