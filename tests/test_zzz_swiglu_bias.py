@@ -3,8 +3,9 @@ the bias/activation row pass alone (moe_bias_act_and_mul), and the layer, which 
 up as two grouped GEMMs with fp32 outputs when either is asked for.
 
 Tolerances: the row pass computes in fp32 and rounds once to bf16, so each output lies within
-half a bf16 ulp (<= 2^-8 |ref|) of the fp64 oracle plus the fp32 arithmetic's error
-(<= 1e-5 at these magnitudes); padding rows are exactly zero. Layers: as in tests/parity.py
+half a bf16 ulp (<= 2^-8 |ref|) of the fp64 oracle plus the fp32 arithmetic's error (a few
+fp32 ulps: <= 1e-6 |ref| + 1e-5, the absolute part for outputs that cancel); padding rows
+are exactly zero. Layers: as in tests/parity.py
 (BF16 |d| <= 2e-2 + 2^-8 |ref| and rel-L2 <= 1e-2; FP4 weights rel-L2 <= 3e-2).
 
 The file name sorts after every other test file: these kernels are the newest, so a run that
@@ -64,7 +65,7 @@ def test_bias_act_matches_oracle(lib, act, in_f32, biases, weighted):
         ref[s:e] = _oracle_act(gg, uu, None if pw is None else O.to_f64(pw[s:e]), p)
     assert np.all(got[M - PAD:] == 0.0)
     err = np.abs(got - ref)
-    lim = 2.0 ** -8 * np.abs(ref) + 1e-5
+    lim = (2.0 ** -8 + 1e-6) * np.abs(ref) + 1e-5
     worst = np.unravel_index(np.argmax(err - lim), err.shape)
     assert np.all(err <= lim), f"max excess {np.max(err - lim):.3e} at {worst}: got {got[worst]} ref {ref[worst]}"
     if act == "swigluoai":     # the clamp was reached on both inputs
