@@ -1,6 +1,5 @@
 """Host-side bookkeeping of bench.py (no GPU): the algorithmic FLOPs and bytes, the tensor
 peak of each path's MMA kind, the launch count and the profile-traffic lookup."""
-import numpy as np
 import torch
 
 import bench
