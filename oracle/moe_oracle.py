@@ -491,6 +491,21 @@ def combine(y, inv_perm, topk_w=None):
 # The whole layer
 # --------------------------------------------------------------------------------------
 
+def weighted_input(x, w_top1):
+    """The experts' input when the top-1 route weight is applied on the input side.
+
+    With ``apply_router_weight_on_input`` the MoonEP experts skip their own weight multiply
+    because the weighting already happened before dispatch [moonep: MoonEPExperts.apply], so
+    what the experts receive is an activation tensor in the model's dtype: x scaled by its
+    weight. Reading taken: the product of the bf16 x and the fp32 weight is formed in fp32 and
+    rounded once to bf16 (RNE). The dynamic activation quantisation of the experts' input
+    [fi_ep: FlashInferMoeEpExperts docstring; dsv4_fi: forward, quantize_input] then applies
+    to this tensor, like to any other input of the experts. Returns bf16 ``[T,H]``.
+    """
+    wt = torch.from_numpy(np.asarray(w_top1, dtype=np.float32).reshape(-1, 1))
+    return (x.float() * wt).to(torch.bfloat16)
+
+
 def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
                 tokens=None, apply_topk_in_fc1: bool = True, keep: bool = False, routing_bias=None,
                 given_topk=None, apply_router_weight_on_input: bool = False, biases=None):
@@ -518,7 +533,9 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     happened before dispatch [moonep: MoonEPExperts.apply].
 
     Returns a dict: ids, w, row, cu_seqlens, perm_token, perm_k, perm_w, inv_perm, tokens and
-    out (fp64 ``[len(tokens), H]``); with ``keep``, also xq (codes/sb/s), h and y rows.
+    out (fp64 ``[len(tokens), H]``); with ``keep``, also xq (codes/sb/s), the experts' input
+    x_exp (token order, after any input weighting and quantisation), the activation rows
+    h_pre (before their quantisation) and h (as the down GEMM takes them), and y rows.
     """
     if given_topk is not None:
         ids = np.asarray(given_topk[0], dtype=np.int32)
@@ -535,19 +552,21 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     need = np.zeros(T * k, dtype=bool)
     need[inv[tok].reshape(-1)] = True
 
-    x64 = to_f64(x)
+    x_in = x
     if apply_router_weight_on_input:
-        x64 = x64 * w[:, :1]
+        x_in = weighted_input(x, w[:, 0])
         apply_topk_in_fc1 = True          # the activation takes no weight (perm_w below is ignored)
         perm_w = np.ones_like(perm_w)
+    x64 = to_f64(x_in)
     res = dict(ids=ids, w=w, perm_w=perm_w, tokens=tok, **perm)
+    # the dynamic activation quantisers see what the experts see: x, or x times its weight
     if cfg.act_quant == 1:
-        codes, sb, s = nvfp4_quantize_rows(np.asarray(x.float().numpy(), np.float32))
+        codes, sb, s = nvfp4_quantize_rows(np.asarray(x_in.float().numpy(), np.float32))
         x64 = nvfp4_dequantize_rows(codes, sb, s)
         if keep:
             res.update(xq_codes=codes, xq_sb=sb, xq_s=s)
     elif cfg.act_quant == 2:
-        codes, sc = mxfp8_quantize_rows(np.asarray(x.float().numpy(), np.float32))
+        codes, sc = mxfp8_quantize_rows(np.asarray(x_in.float().numpy(), np.float32))
         x64 = mxfp8_dequantize_rows(codes, sc)
         if keep:
             res.update(xq_codes=codes, xq_scales=sc)
@@ -555,6 +574,7 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
     a_g, a_u, a_d = weight_alpha(w_gate), weight_alpha(w_up), weight_alpha(w_down)
     y = np.zeros((T * k, w_down.N), dtype=np.float64)
     h_keep = np.zeros((T * k, w_gate.N), dtype=np.float64) if keep else None
+    h_pre_keep = np.zeros((T * k, w_gate.N), dtype=np.float64) if keep else None
     for g, (s0, s1) in enumerate(segment_bounds(perm["cu_seqlens"])):
         rows = np.nonzero(need[s0:s1])[0] + s0
         if len(rows) == 0:
@@ -568,6 +588,8 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
         h = act_and_mul(gate, up, cfg.act, cfg.situ_alpha, cfg.situ_beta,
                         perm_w[rows] if apply_topk_in_fc1 else None, cfg.swiglu_alpha, cfg.swiglu_beta,
                         cfg.swiglu_limit)
+        if keep:
+            h_pre_keep[rows] = h
         if cfg.act_quant == 1:
             hc, hsb, hs = nvfp4_quantize_rows(h.astype(np.float32))
             h = nvfp4_dequantize_rows(hc, hsb, hs)
@@ -582,6 +604,7 @@ def moe_forward(cfg, x, logits, replica_src, w_gate, w_up, w_down, *,
             y[rows] += wb[:, None] * to_f64(biases[2][g])[None, :]
     out = combine(y, inv[tok], None if apply_topk_in_fc1 else w[tok])
     res["out"] = out
+    res["apply_topk_in_fc1"] = apply_topk_in_fc1
     if keep:
-        res.update(h=h_keep, y=y)
+        res.update(h=h_keep, h_pre=h_pre_keep, y=y, x_exp=x64)
     return res

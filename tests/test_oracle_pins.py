@@ -438,13 +438,22 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=Fals
                                 cfg.topk_group, cfg.routed_scaling_factor)
     else:
         ids, w = _route_brute(inp.logits.numpy(), cfg.topk)
-    x = O.to_f64(inp.x)
-    if cfg.act_quant == 1:
-        c, sb, s = O.nvfp4_quantize_rows(inp.x.float().numpy())
-        x = O.nvfp4_dequantize_rows(c, sb, s)
-    elif cfg.act_quant == 2:
-        c, sc = O.mxfp8_quantize_rows(inp.x.float().numpy())
-        x = O.mxfp8_dequantize_rows(c, sc)
+    def expert_input(t, j):
+        # with the weight on the input: bf16 x times the fp32 weight in fp32, rounded to
+        # bf16, and only then quantised, one token row at a time
+        row = inp.x[t:t + 1].float()
+        if input_weight:
+            row = torch.tensor([[float(np.float32(v) * np.float32(w[t, j])) for v in row[0].tolist()]],
+                               dtype=torch.float32).to(torch.bfloat16).float()
+        r = row.numpy()
+        if cfg.act_quant == 1:
+            c, sb, s = O.nvfp4_quantize_rows(r)
+            return O.nvfp4_dequantize_rows(c, sb, s)[0].tolist()
+        if cfg.act_quant == 2:
+            c, sc = O.mxfp8_quantize_rows(r)
+            return O.mxfp8_dequantize_rows(c, sc)[0].tolist()
+        return r[0].astype(np.float64).tolist()
+
     ag, au, ad = (O.weight_alpha(inp.w_gate), O.weight_alpha(inp.w_up), O.weight_alpha(inp.w_down))
     out = np.zeros((cfg.T, cfg.H))
     Wg = [O.weight_rows(inp.w_gate, e).tolist() for e in range(cfg.E)]
@@ -452,7 +461,7 @@ def _layer_brute(cfg, inp, apply_topk_in_fc1=True, given=None, input_weight=Fals
     Wd = [O.weight_rows(inp.w_down, e).tolist() for e in range(cfg.E)]
     for t in range(cfg.T):
         for j in range(cfg.topk):
-            xt = [v * w[t, j] for v in x[t].tolist()] if input_weight else x[t].tolist()
+            xt = expert_input(t, j)
             e = int(ids[t, j])
             gate = [ag[e] * sum(a * b for a, b in zip(row, xt)) for row in Wg[e]]
             up = [au[e] * sum(a * b for a, b in zip(row, xt)) for row in Wu[e]]
@@ -604,6 +613,40 @@ def test_given_topk_and_input_weighting():
         O.moe_forward(*args, given_topk=(gid, gw), apply_router_weight_on_input=True)
 
 
+@pytest.mark.parametrize("wfmt,aq", [("nvfp4", 1), ("mxfp4", 2)])
+def test_input_weighting_reaches_the_activation_quantiser(wfmt, aq):
+    """Top-1 weight on the input with dynamic activation quantisation: the quantiser sees the
+    weighted input (what the experts receive when the weighting happens before dispatch)."""
+    cfg = W.MoEConfig("given_q", T=8, H=64, I=64, E=4, topk=1, wfmt=wfmt, act_quant=aq)
+    inp = W.gen_inputs(cfg)
+    args = (cfg, inp.x, inp.logits.numpy(), np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down)
+    g = np.random.default_rng(11)
+    gid = g.integers(0, cfg.E, (cfg.T, 1)).astype(np.int32)
+    ones = np.ones((cfg.T, 1), np.float32)
+    outs = {}
+    for v in (0.25, 4.0):
+        full = np.full((cfg.T, 1), v, np.float32)
+        outs[v] = O.moe_forward(*args, given_topk=(gid, full), apply_router_weight_on_input=True)["out"]
+        # a power of two scales x exactly in bf16 and moves both quantisers' scales by the same
+        # power, so this is the unweighted layer on the input x * v
+        xs = inp.x * v
+        assert torch.equal(xs.float(), inp.x.float() * v)
+        ref = O.moe_forward(cfg, xs, *args[2:], given_topk=(gid, ones))["out"]
+        assert np.array_equal(outs[v], ref)
+    # the weight is not dropped: the layer is nonlinear, so the two differ
+    assert np.linalg.norm(outs[0.25] - outs[4.0]) > 0.5 * np.linalg.norm(outs[4.0])
+    # other weights: the codes are those of bf16(x * w), not of x
+    w1 = g.uniform(0.2, 3.0, (cfg.T, 1)).astype(np.float32)
+    res = O.moe_forward(*args, given_topk=(gid, w1), apply_router_weight_on_input=True, keep=True)
+    xw = torch.tensor(inp.x.float().numpy() * w1, dtype=torch.float32).to(torch.bfloat16).float().numpy()
+    quant = O.nvfp4_quantize_rows if aq == 1 else O.mxfp8_quantize_rows
+    assert np.array_equal(res["xq_codes"], quant(xw)[0])
+    assert not np.array_equal(res["xq_codes"], quant(inp.x.float().numpy())[0])
+    # and the per-token loop, which weights, rounds and then quantises each token by itself
+    ref = _layer_brute(cfg, inp, given=(gid, w1), input_weight=True)
+    assert np.linalg.norm(res["out"] - ref) <= 1e-3 * np.linalg.norm(ref)
+
+
 def test_swigluoai_reductions_and_clamps():
     g = np.random.default_rng(9)
     gate, up = g.normal(0, 4, (5, 64)), g.normal(0, 4, (5, 64))
@@ -647,3 +690,26 @@ def test_biases_closed_form_and_layer_loop():
                          inp.w_down, biases=b, apply_topk_in_fc1=False)["out"]
     ref2 = _layer_brute(cfg, inp, apply_topk_in_fc1=False, biases=b)
     assert np.allclose(res2, ref2, rtol=1e-9, atol=1e-12 * np.abs(ref2).max())
+
+
+# ------------------------------------------------------------------ the FP4 parity bound itself
+
+@pytest.mark.parametrize("name", ["nvfp4_quant", "mxfp4_situ", "mxfp4_w4a8"])
+def test_fp4_layer_bound_passes_rounding_and_catches_a_wrong_block(name):
+    """The element-wise FP4 bound of the GPU tests admits the oracle's own output rounded to
+    bf16 (RNE, as the combine rounds) and rejects one token's 16 outputs off by 30 %."""
+    from tests.parity import check_fp4_layer, fp4_layer_bound
+
+    cfg = SMALL[name].with_(T=24, H=128, I=128)
+    inp = W.gen_inputs(cfg)
+    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
+                        inp.w_down, keep=True)
+    rounded = torch.from_numpy(ref["out"]).float().to(torch.bfloat16)
+    check_fp4_layer(rounded, ref, cfg, inp, what=name)
+    bad = ref["out"].copy()
+    bad[5, 16:32] *= 0.7
+    with pytest.raises(AssertionError):
+        check_fp4_layer(torch.from_numpy(bad).float().to(torch.bfloat16), ref, cfg, inp, what=name)
+    # and it is not vacuous: typically a few percent of the output's mean magnitude
+    b = fp4_layer_bound(cfg, inp, ref)
+    assert np.median(b) < 0.2 * np.abs(ref["out"]).mean()
