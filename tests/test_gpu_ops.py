@@ -6,7 +6,7 @@ import torch
 
 import workloads as W
 from oracle import moe_oracle as O
-from tests.parity import (FP4_REL_L2, check_bf16, check_mx8, mx8_staging_bound, oracle_bias, rel_l2,
+from tests.parity import (FP4_REL_L2, check_bf16, check_fp4_layer, check_mx8, mx8_staging_bound, oracle_bias, rel_l2,
                           routing_kwargs, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -349,13 +349,12 @@ def test_forward_small_matches_oracle(lib, name):
     inp = W.gen_inputs(cfg)
     out, ids, tw, _ = run_layer(lib, cfg, inp)
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, routing_bias=oracle_bias(inp))
+                        inp.w_down, routing_bias=oracle_bias(inp), keep=cfg.wfmt != "bf16")
     assert np.array_equal(ids.cpu().numpy(), ref["ids"])
     if cfg.wfmt == "bf16":
         check_bf16(out, ref["out"], what=name)
     else:
-        r = rel_l2(out.float().cpu().numpy(), ref["out"])
-        assert r <= FP4_REL_L2, r
+        check_fp4_layer(out, ref, cfg, inp, what=name)
 
 
 def test_forward_bf16_256_token_tiles(lib, monkeypatch):
@@ -391,6 +390,34 @@ def test_forward_given_topk_and_input_weight(lib):
         ref = O.moe_forward(c, inp.x, None, np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down,
                             given_topk=(gid[:, :k], gw[:, :k]), apply_router_weight_on_input=in_w)
         check_bf16(out, ref["out"], what=f"given k={k} input-weight={in_w}")
+
+
+@pytest.mark.parametrize("wfmt,aq,H,I", [("nvfp4", 1, 512, 256), ("nvfp4", 1, 160, 96), ("mxfp4", 2, 256, 320)])
+def test_forward_input_weight_with_activation_quant(lib, wfmt, aq, H, I):
+    # top-1 weight on the input with dynamic activation quantisation: the quantiser sees x
+    # times the weight, rounded to bf16 (both the block-scaled NVFP4 path, K % 256 == 0, and
+    # its f16-staged fallback, and the W4A8 path)
+    cfg = W.MoEConfig("given_q", T=70, H=H, I=I, E=8, topk=1, wfmt=wfmt, act_quant=aq)
+    inp = W.gen_inputs(cfg)
+    g = np.random.default_rng(3)
+    gid = g.integers(0, cfg.E, (cfg.T, 1)).astype(np.int32)
+    dev = lambda ws: lib.Weight.from_host(ws)
+    layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, 1, routing="given",
+                           act_quant=aq, apply_router_weight_on_input=True, T_max=cfg.T)
+    outs = {}
+    for name, gw in (("uniform", g.uniform(0.2, 3.0, (cfg.T, 1))), ("x0.25", np.full((cfg.T, 1), 0.25)),
+                     ("x4", np.full((cfg.T, 1), 4.0))):
+        gw = gw.astype(np.float32)
+        out = layer(to_dev(inp.x), None, topk_ids_in=to_dev(torch.from_numpy(gid)),
+                    topk_w_in=to_dev(torch.from_numpy(gw)))
+        torch.cuda.synchronize()
+        assert layer.device_error() == 0
+        ref = O.moe_forward(cfg, inp.x, None, np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down,
+                            given_topk=(gid, gw), apply_router_weight_on_input=True, keep=True)
+        check_fp4_layer(out, ref, cfg, inp, what=f"{wfmt} input weight {name}")
+        outs[name] = out.float().cpu().numpy()
+    # the weight reached the experts' quantised input
+    assert rel_l2(outs["x0.25"], outs["x4"]) > 0.5
 
 
 def test_forward_given_topk_repeated_expert_is_refused(lib):

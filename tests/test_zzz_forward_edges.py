@@ -16,7 +16,7 @@ import torch
 
 import workloads as W
 from oracle import moe_oracle as O
-from tests.parity import FP4_REL_L2, check_bf16, rel_l2, to_dev
+from tests.parity import check_bf16, check_fp4_layer, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -45,13 +45,13 @@ def _run(lib, cfg, inp, logits):
     out = layer(to_dev(inp.x), to_dev(logits), topk_ids=ids)
     torch.cuda.synchronize()
     assert layer.device_error() == 0
-    ref = O.moe_forward(cfg, inp.x, logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down)
+    ref = O.moe_forward(cfg, inp.x, logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down,
+                        keep=cfg.wfmt != "bf16")
     assert np.array_equal(ids.cpu().numpy(), ref["ids"])
     if cfg.wfmt == "bf16":
         check_bf16(out, ref["out"], what=cfg.name)
     else:
-        r = rel_l2(out.float().cpu().numpy(), ref["out"])
-        assert r <= FP4_REL_L2, f"{cfg.name}: rel-L2 {r:.3e}"
+        check_fp4_layer(out, ref, cfg, inp, what=cfg.name)
     return ref
 
 

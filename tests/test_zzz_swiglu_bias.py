@@ -17,7 +17,7 @@ import torch
 
 import workloads as W
 from oracle import moe_oracle as O
-from tests.parity import FP4_REL_L2, check_bf16, rel_l2, to_dev
+from tests.parity import check_bf16, check_fp4_layer, rel_l2, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -119,12 +119,11 @@ def _layer(lib, cfg, inp, **kw):
                           swiglu_limit=cfg.swiglu_limit, biases=_biases(inp), **kw)
 
 
-def _check(cfg, out, ref, what):
+def _check(cfg, inp, out, ref, what):
     if cfg.wfmt == "bf16":
-        check_bf16(out, ref, what=what)
+        check_bf16(out, ref["out"], what=what)
     else:
-        r = rel_l2(out.float().cpu().numpy(), ref)
-        assert r <= FP4_REL_L2, f"{what}: rel-L2 {r:.3e}"
+        check_fp4_layer(out, ref, cfg, inp, what=what)
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -137,9 +136,9 @@ def test_forward_swiglu_bias_matches_oracle(lib, name):
     torch.cuda.synchronize()
     assert layer.device_error() == 0
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, biases=inp.extra.get("biases"))
+                        inp.w_down, biases=inp.extra.get("biases"), keep=cfg.wfmt != "bf16")
     assert np.array_equal(ids.cpu().numpy(), ref["ids"])
-    _check(cfg, out, ref["out"], name)
+    _check(cfg, inp, out, ref, name)
     b = inp.extra.get("biases")
     if b is not None:
         for part, bb in (("gate/up", (0 * b[0], 0 * b[1], b[2])), ("down", (b[0], b[1], 0 * b[2]))):
@@ -190,8 +189,8 @@ def test_fullsize_swiglu_bias_decode(lib):
     torch.cuda.synchronize()
     assert layer.device_error() == 0
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, biases=inp.extra["biases"])
-    _check(cfg, out, ref["out"], cfg.name)
+                        inp.w_down, biases=inp.extra["biases"], keep=True)
+    _check(cfg, inp, out, ref, cfg.name)
 
 
 @pytest.mark.slow
@@ -211,7 +210,6 @@ def test_fullsize_swiglu_bias_prefill(lib):
     assert np.array_equal(ids.cpu().numpy(), rids)
     toks = _sample_tokens(cfg, O.assign_rows(rids, cfg.E, cfg.B, inp.replica_src.numpy()))
     ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
-                        inp.w_down, tokens=toks, biases=inp.extra["biases"])
+                        inp.w_down, tokens=toks, biases=inp.extra["biases"], keep=True)
     got = out[torch.tensor(toks, device="cuda")].float().cpu().numpy()
-    r = rel_l2(got, ref["out"])
-    assert r <= FP4_REL_L2, f"{cfg.name}: rel-L2 {r:.3e}"
+    check_fp4_layer(got, ref, cfg, inp, what=cfg.name)
