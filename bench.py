@@ -4,14 +4,17 @@
 
 A step is one full forward of the layer (route -> permute -> gate/up GEMM with the
 activation -> down GEMM -> combine) over one batch of seeded synthetic inputs. The
-default workload is the Mixtral-shaped BF16 prefill (T=4096, H=4096, I=14336, E=8,
-top-2). With N GPUs (torchrun, one process per GPU) every rank runs its own replica of
-the layer on its own batch: there is no data-path collective ("weak" scaling); the time
-is the max over ranks of the device time.
+default workload is the largest one-GPU workload, the DeepSeek-shaped BF16 prefill
+(T=8192, H=7168, I=2048, E=256 plus 16 redundant slots, top-8). With N GPUs (torchrun,
+one process per GPU; `--gpus N` alone relaunches itself that way) every rank runs its
+own replica of the layer on its own batch: there is no data-path collective ("weak"
+scaling); the time is the max over ranks of the device time.
 
 value   tokens/s over all ranks, inputs resident in HBM, CUDA events on the stream.
-e2e     the same through the public call with pinned host buffers: the H2D copy of x
-        and the router logits and the D2H copy of the output are inside the timed region.
+e2e     the same through the public call with pinned host buffers: every step copies x
+        and the router logits host -> device and the output device -> host inside the
+        timed region, double-buffered on two copy streams so that the copies of one step
+        overlap the layer of the previous one.
 roofline  the dominant kernel (the gate/up grouped GEMM), algorithmic FLOPs or bytes per
         launch over its event-timed duration, against MEASURED_PEAKS.json.
 cpu_baseline  the CPU oracle on a bounded token sample, rank 0, N = 1 only.
@@ -180,6 +183,23 @@ def profiled_traffic(workload: str) -> float | None:
         return float(vals["dram_bytes_per_launch_full"])
     except (KeyError, ValueError):
         return None
+
+
+def needs_l2_flush(weight_bytes_touched: float) -> bool:
+    """A step whose weights fit in L2 would find them there on the next step."""
+    return weight_bytes_touched <= L2_BYTES
+
+
+def config_record(cfg, weight_bytes_touched: float) -> dict:
+    """The workload's record, the same in both arms: its shapes and modes, and how the L2 is
+    handled between timed steps (not flushed when the weights a step touches exceed it, else
+    flushed by a 2 x L2 write between individually timed steps)."""
+    l2 = (f"flushed between steps: weights touched per step {weight_bytes_touched / 1e6:.1f} MB "
+          f"<= L2 {L2_BYTES / 2 ** 20:.0f} MiB" if needs_l2_flush(weight_bytes_touched) else
+          f"no flush: weights touched per step {weight_bytes_touched / 1e9:.2f} GB > L2 {L2_BYTES / 2 ** 20:.0f} MiB")
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
+            "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant,
+            **routing_config(cfg), **act_config(cfg), "l2": l2}
 
 
 # ---------------------------------------------------------------------------- ranks
@@ -357,17 +377,28 @@ def run_ours(args, cfg, rank, world):
         return row
 
     fc1_evs = [new_events() for _ in range(K)]
+    flush = needs_l2_flush(acc["weight_bytes_total"])
+    scrub = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier()
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0.record(stream)
         for i in range(K):
             ev = fc1_evs[i]
+            if flush:                     # outside the step's own events
+                scrub.fill_(float(i))
+                step_evs[i][0].record(stream)
             layer(x_d, l_d, out=out_d, stage_events=[None, None, ev[2], ev[3], None, None, None])
+            if flush:
+                step_evs[i][1].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    if flush:
+        ms_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_evs))
+    else:
+        ms_total = max_over_ranks(t0.elapsed_time(t1))
     fc1_ms = float(np.mean([fc1_evs[i][2].elapsed_time(fc1_evs[i][3]) for i in range(K)]))
     assert layer.device_error() == 0, "device error in timed region"
 
@@ -381,30 +412,58 @@ def run_ours(args, cfg, rank, world):
     # ---- end to end through the public call, host buffers
     e2e = None
     if not args.no_e2e:
+        # Two device buffer sets: step i copies its inputs into set i % 2 on the H2D stream
+        # while the layer of step i - 1 runs, and its output leaves on the D2H stream while
+        # step i + 1 runs. Events order each buffer's reuse.
         x_h = inp.x.pin_memory()
         l_h = inp.logits.pin_memory()
-        o_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+        o_h = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        xs = [x_d, torch.empty_like(x_d)]
+        ls = [l_d, torch.empty_like(l_d)]
+        outs = [out_d, torch.empty_like(out_d)]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        loaded, computed, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        used = [False, False]
 
-        def e2e_step():
-            x_d.copy_(x_h, non_blocking=True)
-            l_d.copy_(l_h, non_blocking=True)
-            layer(x_d, l_d, out=out_d)
-            o_h.copy_(out_d, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if used[b]:
+                    h2d.wait_event(computed[b])           # the layer of step i-2 read this set
+                xs[b].copy_(x_h, non_blocking=True)
+                ls[b].copy_(l_h, non_blocking=True)
+                loaded[b].record(h2d)
+            stream.wait_event(loaded[b])
+            if used[b]:
+                stream.wait_event(drained[b])             # step i-2's output has left
+            layer(xs[b], ls[b], out=outs[b])
+            computed[b].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(computed[b])
+                o_h[b].copy_(outs[b], non_blocking=True)
+                drained[b].record(d2h)
+            used[b] = True
 
-        for _ in range(Wm):
-            e2e_step()
+        for i in range(Wm):
+            e2e_step(i)
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(K):
-            e2e_step()
+        h2d.wait_event(a0)
+        for i in range(Wm, Wm + K):
+            e2e_step(i)
+        for b in range(2):
+            stream.wait_event(drained[b])
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(a0.elapsed_time(a1))
+        assert layer.device_error() == 0, "device error in the end-to-end pass"
         e2e = {"value": job_tokens_per_s(world, cfg.T, K, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 4),
-               "d2h_bytes_per_step": int(o_h.numel() * 2)}
+               "d2h_bytes_per_step": int(o_h[0].numel() * 2),
+               "overlap": "double-buffered: H2D and D2H on their own streams overlap the layer"}
 
     peaks, peak_src = load_peaks()
     ms_step = ms_total / K
@@ -444,13 +503,9 @@ def run_ours(args, cfg, rank, world):
         "warmup": Wm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": compute_dtype(cfg),
         "data": "synthetic (seeded; random weights of the workload's shapes)",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
-                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg),
-                   **act_config(cfg),
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: weights touched per step {acc['weight_bytes_total'] / 1e9:.2f} GB "
-                         f"> L2 {L2_BYTES / 2 ** 20:.0f} MiB",
-                   "nonempty_segments": acc["nonempty"], "max_segment": acc["max_seg"]},
+        "config": config_record(cfg, acc["weight_bytes_total"]),
+        "parallelism": f"replicas x{world} (one process per GPU, no data-path collective)",
+        "workload_stats": {"nonempty_segments": acc["nonempty"], "max_segment": acc["max_seg"]},
         "roofline": roof,
         "layer_roofline": {"t_roof_ms": t_layer_roof * 1e3, "frac": t_layer_roof * 1e3 / ms_step,
                            "flops": acc["layer_flops"], "bytes": acc["layer_bytes"],
@@ -466,7 +521,12 @@ def run_ours(args, cfg, rank, world):
 
 def run_reference(args, cfg):
     """The CPU oracle on the host cores, each step a bounded token sample."""
+    from oracle import moe_oracle as O
+
     inp = W.gen_inputs(cfg)
+    bias = inp.extra.get("routing_bias")
+    ids, _ = O.route(cfg, inp.logits.numpy(), None if bias is None else bias.numpy())
+    acc = accounting(cfg, inp, *segment_stats(cfg, torch.from_numpy(ids), inp.replica_src))
     S = max(1, default_sample(cfg) // 4)
     K, Wm = args.steps, args.warmup
     # keep the whole run within a few minutes: shrink the sample if a calibration step is slow
@@ -485,9 +545,8 @@ def run_reference(args, cfg):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 1,
         "steps": K, "warmup": Wm, "ms_per_step": t / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "B": cfg.B,
-                   "topk": cfg.topk, "act": cfg.act, "weights": cfg.wfmt, "act_quant": cfg.act_quant, **routing_config(cfg),
-                   **act_config(cfg)},
+        "config": config_record(cfg, acc["weight_bytes_total"]),
+        "workload_stats": {"nonempty_segments": acc["nonempty"], "max_segment": acc["max_seg"]},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{S} tokens per step of {cfg.T} (routing of all), fp64 NumPy"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -499,7 +558,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="mixtral_prefill", choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default="deepseek_prefill", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -513,6 +572,17 @@ def main(argv=None):
         cfg = cfg.with_(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: relaunch under the torch launcher on this node
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr=127.0.0.1", f"--master-port={29500 + os.getpid() % 1000}",
+               os.path.abspath(__file__), *(argv if argv is not None else sys.argv[1:])]
+        os.execv(sys.executable, cmd)
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
 
     if args.impl == "reference":
         if rank != 0:

@@ -52,8 +52,19 @@ def test_reference_arm_only_rank0_runs():
     # a rank other than 0 exits 0 without work and prints nothing
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
-                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+                        "--gpus", "2", "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
+                       timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_gpus_must_match_the_launched_world():
+    # a world of 2 ranks launched for --gpus 4 (or --gpus left at 1) is refused, not mislabelled
+    for gpus in ("4", "1"):
+        env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                            "tiny", "--gpus", gpus, "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                           text=True, timeout=300)
+        assert r.returncode == 2 and r.stdout.strip() == "" and "WORLD_SIZE=2" in r.stderr
 
 
 def test_reference_arm_rank0_prints_one_line():
