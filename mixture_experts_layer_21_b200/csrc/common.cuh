@@ -28,7 +28,9 @@ MOE_DEV void report_error(DevError* e, int code, int detail) {
     if (e && atomicCAS(&e->code, 0, code) == 0) atomicExch(&e->detail, detail);
 }
 
-// Upper bound for any single pipeline wait, in SM clock cycles (~1 s at 2 GHz).
+// Default upper bound for any single wait, in SM clock cycles (~1 s at 2 GHz). Pipeline
+// waits take the launch's own limit (GemmArgs::wait_limit, this by default); the waits that
+// let copies and MMAs in flight finish after an abort always take this one.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
 // ---------------------------------------------------------------- PDL
@@ -66,16 +68,16 @@ MOE_DEV bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits until the phase with the given parity has completed. Gives up after
-// kWaitLimitCycles or when *abort becomes non-zero; returns false then.
-MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Waits until the phase with the given parity has completed. Gives up after `limit`
+// cycles or when *abort becomes non-zero; returns false then.
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long limit = kWaitLimitCycles) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
 }
 

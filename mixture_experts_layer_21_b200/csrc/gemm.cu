@@ -75,6 +75,7 @@ struct GemmArgs {
     int zero_pad;
     int x3d;          // FP4: the token map is 3-D {64, rows, K/64}: one copy per 128-K stage
     DevError* err;
+    long long wait_limit;  // cycles a pipeline wait may take before the kernel gives up
 };
 
 struct CtrlBlock {
@@ -140,6 +141,27 @@ __device__ __forceinline__ void build_segment_table(const GemmArgs& a, CtrlBlock
         prev_chunk_end = __shfl_sync(0xffffffffu, eff, 31);
     }
     if (lane == 0) ctl->tpre[0] = 0;
+}
+
+// What one thread has in flight: the producer's stages (and the parity of each one's last
+// issue), or whether a tcgen05 issuer (MMA or scale copies) issued anything.
+struct Issued {
+    uint32_t mask = 0, par = 0;
+    bool tc = false;
+};
+
+// After an abort, before the CTA's shared and tensor memory are released: the producer
+// waits for its copies to land, a tcgen05 issuer commits to its own drain barrier and waits
+// for it. An abort can come after a role left its loop normally, so this runs for every
+// role once all have stopped. These waits take the default limit; nothing aborts them.
+__device__ __forceinline__ void drain_in_flight(const Issued& is, uint64_t* full, int stages, uint64_t* drain) {
+    int never = 0;
+    for (int q = 0; q < stages; ++q)
+        if (is.mask >> q & 1u) mbar_wait(&full[q], is.par >> q & 1u, &never);
+    if (is.tc && drain) {
+        mma_commit(drain);
+        mbar_wait(drain, 0, &never);
+    }
 }
 
 // Epilogue of one tile for the warp owning TMEM lanes [32q, 32q+32). The accumulator
@@ -249,6 +271,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
     volatile int* abort_flag = &ctl->abort;
+    Issued is;  // this thread's copies or tcgen05 operations in flight
     auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
     auto opB = [&](int s) { return smem + s * C::STAGE + C::NB * C::A_BYTES; };
     const int warp = warp_id(), lane = lane_id();
@@ -288,13 +311,13 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {  // ---------------- TMA producer
             int s = 0;
-            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -302,8 +325,8 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                     tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g);
                     if (DUAL) tma_load_3d(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g);
                     tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * kTileK, row0);
-                    issued_mask |= 1u << s;
-                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -313,30 +336,27 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 1);
                 ctl->abort = 1;
-                int never = 0;  // let every copy this thread issued land before the CTA exits
-                for (int q = 0; q < C::STAGES; ++q)
-                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {  // ---------------- MMA issuer
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 // MMA width: the tile's rows rounded up to 16, so a segment's short last
                 // tile does not pay for BT columns
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 const uint32_t idesc = idesc_f16(1, kTileN, cmin(BT, (rows + 15) & ~15));
-                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag, a.wait_limit)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag)) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -351,7 +371,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                         mma_f16_ss(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, acc);
                         if (DUAL) mma_f16_ss(d0 + BT, sw128_kmajor_desc(a1 + kk * 32), bdesc, idesc, acc);
                     }
-                    issued = true;
+                    is.tc = true;
                     mma_commit(&ctl->empty[s]);
                     if (++s == C::STAGES) {
                         s = 0;
@@ -368,11 +388,6 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {  // wait (bounded) for the MMAs in flight before TMEM is released
-                    int never = 0;
-                    mma_commit(&ctl->drain[0]);
-                    mbar_wait(&ctl->drain[0], 0, &never);
-                }
             }
         }
     } else {
@@ -383,7 +398,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
             int g, nt, row0, rows;
             decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag, a.wait_limit)) {
                 if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
                 ctl->abort = 1;
                 break;
@@ -404,6 +419,11 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        drain_in_flight(is, ctl->full, C::STAGES, warp == 1 && lane == 0 ? &ctl->drain[0] : nullptr);
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -506,6 +526,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::RSTAGES * C::RAW_STAGE);
     volatile int* abort_flag = &ctl->abort;
+    Issued is;  // this thread's copies or tcgen05 operations in flight
     // raw stage r: [token box 0][token box 1][matrix 0: chunk kb, chunk kb+1][matrix 1: ...]
     auto rawB = [&](int r) { return smem + r * C::RAW_STAGE; };
     auto rawM = [&](int r, int m) { return smem + r * C::RAW_STAGE + C::B_BYTES + m * C::RAW_M; };
@@ -546,14 +567,14 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer: two token boxes (TMA) + one copy per matrix
             int r = 0;
-            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 const size_t chunk0 = ((size_t)g * NT + nt) * (2 * KB);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->raw_empty[r], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&ctl->raw_empty[r], ph ^ 1u, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -567,8 +588,8 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
                         tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0);
                         tma_load_2d(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0);
                     }
-                    issued_mask |= 1u << r;
-                    issued_par = (issued_par & ~(1u << r)) | (ph << r);
+                    is.mask |= 1u << r;
+                    is.par = (is.par & ~(1u << r)) | (ph << r);
                     if (++r == C::RSTAGES) {
                         r = 0;
                         ph ^= 1u;
@@ -578,9 +599,6 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 1);
                 ctl->abort = 1;
-                int never = 0;
-                for (int q = 0; q < C::RSTAGES; ++q)
-                    if (issued_mask >> q & 1u) mbar_wait(&ctl->raw_full[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp < C::EPI_WARP0) {
@@ -599,9 +617,9 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
             const int kk0 = p_i * KPI;
             int s = 0, r = 0, b = 0;
             uint32_t ph = 0, rph = 0, bph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag, a.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -610,7 +628,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
                 for (int kb = 0; kb < KB; ++kb) {
                     // the converters arrive on full[s] only after they saw raw stage r land, so
                     // this one wait also orders the token tile before the MMA
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag)) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -636,7 +654,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
                                        (kb > 0 || j > 0) ? 1u : 0u);
                         }
                     }
-                    issued = true;
+                    is.tc = true;
                     // one commit per stage: it frees raw stage r and, for the converters, the
                     // TMEM weight slot of this stage
                     mma_commit(&ctl->raw_empty[r]);
@@ -659,11 +677,6 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {  // wait (bounded) for this issuer's MMAs before TMEM is released
-                    int never = 0;
-                    mma_commit(&ctl->drain[i]);
-                    mbar_wait(&ctl->drain[i], 0, &never);
-                }
             }
         }
     } else if (warp < C::CONV_WARP0) {
@@ -674,7 +687,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
             int g, nt, row0, rows;
             decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag, a.wait_limit)) {
                 if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
                 ctl->abort = 1;
                 break;
@@ -708,10 +721,10 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
                 // The TMEM weight slot s is free once the MMAs of stage it - A_STAGES are done,
                 // which the issuers' commit on that stage's raw barrier records. That barrier
                 // cannot run a phase ahead: it would need stage it - A_STAGES + RSTAGES > it.
-                bool got = mbar_wait(&ctl->raw_full[r], rph, abort_flag);
+                bool got = mbar_wait(&ctl->raw_full[r], rph, abort_flag, a.wait_limit);
                 if (got && it >= C::A_STAGES) {
                     const long long j = it - C::A_STAGES;
-                    got = mbar_wait(&ctl->raw_empty[j % C::RSTAGES], (uint32_t)((j / C::RSTAGES) & 1), abort_flag);
+                    got = mbar_wait(&ctl->raw_empty[j % C::RSTAGES], (uint32_t)((j / C::RSTAGES) & 1), abort_flag, a.wait_limit);
                 }
                 if (!got) {
                     if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 4);
@@ -750,6 +763,12 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        drain_in_flight(is, ctl->raw_full, C::RSTAGES,
+                        warp >= 1 && warp < C::EPI_WARP0 && lane == 0 ? &ctl->drain[warp - 1] : nullptr);
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
@@ -821,6 +840,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
     volatile int* abort_flag = &ctl->abort;
+    Issued is;  // this thread's copies or tcgen05 operations in flight
     auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
     auto opB = [&](int s) { return smem + s * C::STAGE + C::B_OFF; };
     auto sfRaw = [&](int s) { return smem + s * C::STAGE + C::SFR_OFF; };
@@ -866,14 +886,14 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer
             int s = 0;
-            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 const size_t tile0 = ((size_t)g * NT + nt) * KB;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -883,8 +903,8 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                     if (DUAL) bulk_load(opA(s, 1), a.ks1 + off, kNvf4TileBytes, &ctl->full[s]);
                     tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * (kNvf4StageK / 2), row0);
                     tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], kb * (kNvf4StageK / 16), row0);
-                    issued_mask |= 1u << s;
-                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -894,9 +914,6 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 1);
                 ctl->abort = 1;
-                int never = 0;
-                for (int q = 0; q < C::STAGES; ++q)
-                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp == 1) {
@@ -904,9 +921,9 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
             constexpr uint32_t idesc = idesc_nvf4(kTileN, BT);
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag, a.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -914,7 +931,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
                 for (int kb = 0; kb < KB; ++kb) {
                     // operands landed (full) and their scale factors are in TMEM (sf_full)
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit) || !mbar_wait(&sf_full[s], ph, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -930,7 +947,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                             mma_nvf4_ss(d0 + m * BT, sw128_kmajor_desc(smem_u32(opA(s, m)) + 32 * j), bdesc, idesc,
                                         sfs + m * 16 + 4 * j, sfs + C::NB * 16 + 4 * j, acc);
                     }
-                    issued = true;
+                    is.tc = true;
                     mma_commit(&ctl->empty[s]);
                     if (++s == C::STAGES) {
                         s = 0;
@@ -945,11 +962,6 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {  // wait (bounded) for the MMAs in flight before TMEM is released
-                    int never = 0;
-                    mma_commit(&ctl->drain[0]);
-                    mbar_wait(&ctl->drain[0], 0, &never);
-                }
             }
         }
     } else if (warp == 6) {
@@ -958,10 +970,10 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
         // slot is free: the stage's previous MMAs completed before the producer refilled it.
         int s = 0;
         uint32_t ph = 0;
-        bool ok = true, issued = false;
+        bool ok = true;
         for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit))) {
                     ok = false;
                     break;
                 }
@@ -982,7 +994,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                     mma_commit(&sf_full[s]);
                 }
                 __syncwarp();
-                issued = true;
+                is.tc = true;
                 if (++s == C::STAGES) {
                     s = 0;
                     ph ^= 1u;
@@ -992,11 +1004,6 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
         if (!ok && lane == 0) {
             report_error(a.err, MOE_ERR_TIMEOUT, 5);
             ctl->abort = 1;
-            if (issued) {  // wait (bounded) for the copies in flight before TMEM is released
-                int never = 0;
-                mma_commit(&ctl->drain[1]);
-                mbar_wait(&ctl->drain[1], 0, &never);
-            }
         }
     } else {
         // ---------------- epilogue (warps 2..5)
@@ -1006,7 +1013,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
             int g, nt, row0, rows;
             decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag, a.wait_limit)) {
                 if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
                 ctl->abort = 1;
                 break;
@@ -1025,6 +1032,12 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        drain_in_flight(is, ctl->full, C::STAGES,
+                        lane != 0 ? nullptr : warp == 1 ? &ctl->drain[0] : warp == 6 ? &ctl->drain[1] : nullptr);
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -1114,6 +1127,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
     volatile int* abort_flag = &ctl->abort;
+    Issued is;  // this thread's copies or tcgen05 operations in flight
     auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
     auto opB = [&](int s, int t) { return smem + s * C::STAGE + (t ? C::BL_OFF : C::BH_OFF); };
     auto sfA = [&](int s, int m) { return smem + s * C::STAGE + C::SFA_OFF + m * 512; };
@@ -1161,14 +1175,14 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer
             int s = 0;
-            uint32_t ph = 0, issued_mask = 0, issued_par = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 const size_t blk0 = ((size_t)g * NT + nt) * KB;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -1183,8 +1197,8 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                     tma_load_2d(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0);
                     if (TWO) tma_load_2d(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0);
                     tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], (kb >> 2) * 16, row0);
-                    issued_mask |= 1u << s;
-                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -1194,9 +1208,6 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 1);
                 ctl->abort = 1;
-                int never = 0;
-                for (int q = 0; q < C::STAGES; ++q)
-                    if (issued_mask >> q & 1u) mbar_wait(&ctl->full[q], issued_par >> q & 1u, &never);
             }
         }
     } else if (warp < C::EPI_WARP0) {
@@ -1206,16 +1217,16 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
             constexpr int KPI = (kMx8StageK / 32) / C::KSPLIT;  // K steps per issuer and stage
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag)) {
+                if (!mbar_wait(&ctl->tempty[b], bph ^ 1u, abort_flag, a.wait_limit)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(b * C::ACC_COLS + (m * C::NPART + kh * C::TERMS) * BT);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag) || !mbar_wait(&sf_full[s], ph, abort_flag)) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit) || !mbar_wait(&sf_full[s], ph, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -1237,7 +1248,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                                            idesc_mx8(kTileN, BT, id), sfa | idb, sfb | idb, (kb | j | t) != 0);
                         }
                     }
-                    issued = true;
+                    is.tc = true;
                     mma_commit(&ctl->empty[s]);
                     if (++s == C::STAGES) {
                         s = 0;
@@ -1254,11 +1265,6 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
             if (!ok) {
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
-                if (issued) {  // wait (bounded) for this issuer's MMAs before TMEM is released
-                    int never = 0;
-                    mma_commit(&ctl->drain[i]);
-                    mbar_wait(&ctl->drain[i], 0, &never);
-                }
             }
         }
     } else if (warp == C::SCALE_WARP) {
@@ -1266,10 +1272,10 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
         // the producer refilled s, i.e. after the MMAs that read it completed
         int s = 0;
         uint32_t ph = 0;
-        bool ok = true, issued = false;
+        bool ok = true;
         for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit))) {
                     ok = false;
                     break;
                 }
@@ -1288,7 +1294,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                     mma_commit(&sf_full[s]);
                 }
                 __syncwarp();
-                issued = true;
+                is.tc = true;
                 if (++s == C::STAGES) {
                     s = 0;
                     ph ^= 1u;
@@ -1298,11 +1304,6 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
         if (!ok && lane == 0) {
             report_error(a.err, MOE_ERR_TIMEOUT, 5);
             ctl->abort = 1;
-            if (issued) {
-                int never = 0;
-                mma_commit(&ctl->drain[5]);
-                mbar_wait(&ctl->drain[5], 0, &never);
-            }
         }
     } else {
         // ---------------- epilogue (4 * EW warps)
@@ -1312,7 +1313,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
             int g, nt, row0, rows;
             decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag)) {
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag, a.wait_limit)) {
                 if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
                 ctl->abort = 1;
                 break;
@@ -1334,6 +1335,15 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        drain_in_flight(is, ctl->full, C::STAGES,
+                        lane != 0                         ? nullptr
+                        : warp >= 1 && warp < C::EPI_WARP0 ? &ctl->drain[warp - 1]
+                        : warp == C::SCALE_WARP           ? &ctl->drain[5]
+                                                          : nullptr);
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -1643,9 +1653,23 @@ int choose_token_tile(long long NvS, int G, bool wide_ok) {
     return 256;
 }
 
+// The pipeline-wait limit of a launch: MOE_WAIT_LIMIT_CYCLES (a positive integer, read at
+// every launch) or the default of about one second. A shorter limit is for tests of the
+// timeout path; the waits for copies and MMAs in flight after an abort keep the default.
+long long wait_limit_cycles() {
+    const char* env = getenv("MOE_WAIT_LIMIT_CYCLES");
+    if (env) {
+        char* end = nullptr;
+        const long long v = strtoll(env, &end, 10);
+        if (end != env && *end == '\0' && v > 0) return std::min(v, kWaitLimitCycles);
+    }
+    return kWaitLimitCycles;
+}
+
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl) {
     if (p.G > kMaxG) return cudaErrorInvalidValue;
     GemmArgs a{};
+    a.wait_limit = wait_limit_cycles();
     a.cu = p.cu_seqlens;
     a.G = p.G;
     a.N = p.N;
