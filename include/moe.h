@@ -177,9 +177,12 @@ moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, in
  *   The first call on a device looks up that array's device address (with that
  *   device current); make that first call before any stream capture.
  *   All calls share the one array: calls that overlap on the GPU (two streams,
- *   two host threads) race and must be serialised by the caller. An expert id
- *   outside [0,E) is skipped (its inv_perm entry is -1); unlike moe_permute the
- *   error word is internal and cleared at every call.
+ *   two host threads) race and must be serialised by the caller.
+ *   Bad data is handled as in moe_permute: an expert id outside [0,E), or a token
+ *   listing one expert twice, is skipped (its inv_perm entry is -1, and the rows
+ *   no assignment reaches get token 0 and weight 0); a replica_src entry outside
+ *   [-1,E) is ignored. Each sets the call's error word, which lives in the array,
+ *   starts at zero at every call and is read by moe_permute_noalloc_status.
  */
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w, int T, int topk,
                                  int E, int B, const int32_t* replica_src,
@@ -187,6 +190,14 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float* topk_w, i
                                  int32_t* cu_seqlens, int32_t* perm_token, float* perm_w,
                                  int32_t* inv_perm, void* x_perm, int M_alloc,
                                  moe_stream_t stream);
+
+/*
+ * The device-detected status of the last moe_permute_noalloc call on the current
+ * device: synchronises `stream`, returns MOE_OK or the code the kernels recorded
+ * (MOE_ERR_DEVICE for the bad data above) and clears it. Allocates nothing. Like the
+ * call itself it shares the one array: read it before the next call on the device.
+ */
+moe_status_t moe_permute_noalloc_status(moe_stream_t stream);
 
 /*
  * S3/S5 — grouped GEMM: out[seg_g] = alpha_g * a[seg_g] @ W[g]^T for every

@@ -36,7 +36,7 @@ EXPORTS = ["moe_status_string", "moe_version", "moe_route_topk", "moe_permute_wo
            "moe_permute", "moe_grouped_gemm_workspace_size", "moe_grouped_gemm", "moe_act_and_mul",
            "moe_combine", "moe_quantize_nvfp4", "moe_prepared_weight_bytes", "moe_prepare_weights",
            "moe_forward_workspace_size", "moe_forward", "moe_get_device_error", "moe_permute_noalloc",
-           "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8", "moe_route_topk_grouped",
+           "moe_permute_noalloc_status", "moe_grouped_gemm_nvfp4", "moe_quantize_mxfp8", "moe_route_topk_grouped",
            "moe_bias_act_and_mul", "moe_forward_workspace_size_args"]
 
 
@@ -106,6 +106,7 @@ _sig = {
     "moe_forward": (_I, [ctypes.POINTER(moe_forward_args_t), _P, _S, _P]),
     "moe_get_device_error": (_I, [_P, _P]),
     "moe_permute_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P]),
+    "moe_permute_noalloc_status": (_I, [_P]),
     "moe_grouped_gemm_nvfp4": (_I, [_P, _P, _P, _I, ctypes.POINTER(moe_weight_t), _P, _P, _P, _S, _P]),
     "moe_quantize_mxfp8": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_route_topk_grouped": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _P]),

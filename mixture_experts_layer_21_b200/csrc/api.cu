@@ -71,9 +71,6 @@ class Trace {
     bool stage_ = false;
 };
 
-constexpr int kMaxExperts = 1024;
-constexpr int kMaxTopk = 32;
-
 bool act_ok(const moe_act_params_t& a) {
     if (a.act == MOE_ACT_SILU) return true;
     if (a.act == MOE_ACT_SITU)
@@ -239,7 +236,7 @@ moe_status_t moe_permute(const int32_t* topk_ids, const float* topk_w, int T, in
                          float* perm_w, int32_t* inv_perm, void* x_perm, int M_alloc, void* ws, size_t ws_bytes,
                          moe_stream_t stream) {
     if (T < 0 || topk < 1 || E < 1 || B < 0 || topk > E) return MOE_ERR_INVALID_ARG;
-    if (E > kMaxExperts || E + B > 2 * kMaxExperts || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
+    if (E > kMaxExperts || E + B > kMaxRows || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
     if (B > 0 && !replica_src) return MOE_ERR_INVALID_ARG;
     if (!cu_seqlens || !ws) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_permute_workspace_size(T, topk, E, B)) return MOE_ERR_WORKSPACE_TOO_SMALL;

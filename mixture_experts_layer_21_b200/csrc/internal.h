@@ -29,6 +29,12 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 // ---------------------------------------------------------------- S1/S2
+// Limits of the routing and permutation kernels (the scan's shared-memory tables are sized
+// for these): experts E, experts plus redundant slots E + B, and top-k.
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxRows = 2 * kMaxExperts;
+constexpr int kMaxTopk = 32;
+
 cudaError_t launch_route_topk(const float* logits, int T, int E, int topk, int32_t* ids, float* w,
                               cudaStream_t st, bool pdl);
 

@@ -56,7 +56,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float
                                             int32_t* inv_perm, void* x_perm, int M_alloc,
                                             moe_stream_t stream) {
     if (T < 0 || topk < 1 || E < 1 || B < 0 || topk > E) return MOE_ERR_INVALID_ARG;
-    if (E > 1024 || E + B > 2048 || topk > 32) return MOE_ERR_UNSUPPORTED;
+    if (E > kMaxExperts || E + B > kMaxRows || topk > kMaxTopk) return MOE_ERR_UNSUPPORTED;
     if (B > 0 && !replica_src) return MOE_ERR_INVALID_ARG;
     if (!cu_seqlens) return MOE_ERR_INVALID_ARG;
     // the scratch these sizes need must fit in the fixed array
@@ -79,4 +79,20 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, const float
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (x_perm) e = launch_gather(0, x, H, perm_token, T * topk, x_perm, nullptr, nullptr, st, true);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// The device-detected status of the last moe_permute_noalloc call on the current device
+// (its error word lives in the scratch array): waits for the stream, reads the word and
+// clears it. Allocates nothing.
+extern "C" moe_status_t moe_permute_noalloc_status(moe_stream_t stream) {
+    void* base = nullptr;
+    if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    DevError h{0, 0};
+    if (cudaMemcpy(&h, base, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (h.code != 0) {
+        if (cudaMemset(base, 0, sizeof(h)) != cudaSuccess) return MOE_ERR_CUDA;
+        return static_cast<moe_status_t>(h.code);
+    }
+    return MOE_OK;
 }
