@@ -104,6 +104,37 @@ MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, 
         "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
+// The same two loads with an L2 cache policy (a createpolicy value; see l2_policy).
+MOE_DEV void tma_load_2d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+MOE_DEV void tma_load_3d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// L2 cache policies: 0 = none (plain loads), 1 = evict first (data read once), 2 = evict last
+// (data many CTAs re-read). Returns 0 for "none", which no createpolicy value equals.
+MOE_DEV uint64_t l2_policy(int kind) {
+    uint64_t p = 0;
+    if (kind == 1) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, %1;" : "=l"(p) : "f"(1.0f));
+    else if (kind == 2) asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, %1;" : "=l"(p) : "f"(1.0f));
+    return p;
+}
+MOE_DEV void tma_load_2d_p(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, uint64_t pol) {
+    if (pol) tma_load_2d_hint(dst, m, bar, x, y, pol);
+    else tma_load_2d(dst, m, bar, x, y);
+}
+MOE_DEV void tma_load_3d_p(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z, uint64_t pol) {
+    if (pol) tma_load_3d_hint(dst, m, bar, x, y, z, pol);
+    else tma_load_3d(dst, m, bar, x, y, z);
+}
 // Untiled bulk copy global -> shared; both addresses 16-byte aligned, bytes % 16 == 0.
 MOE_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
@@ -111,6 +142,16 @@ MOE_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+MOE_DEV void bulk_load_p(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+    if (pol)
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+                smem_u32(dst)),
+            "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+            : "memory");
+    else
+        bulk_load(dst, src, bytes, bar);
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -271,6 +312,85 @@ MOE_DEV void tmem_st16(uint32_t taddr, const uint32_t* r) {
         : "memory");
 }
 MOE_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// A cluster of two CTAs on two SMs runs one MMA stream: the CTA of rank 0 (the leader) issues
+// tcgen05.mma.cta_group::2, whose A operand is 128 rows from each CTA's shared memory, whose B
+// operand is N/2 rows from each, and whose accumulator is 128 rows x N columns in each CTA's
+// tensor memory (its own A rows). Both CTAs allocate tensor memory together; every tcgen05
+// instruction of such a kernel takes cta_group::2.
+MOE_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of both CTAs: release what this thread wrote, wait for all, acquire.
+MOE_DEV void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// The address of the same shared-memory location in the CTA of cluster rank `rank`.
+MOE_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier given by its cluster address (mapa), with cluster-scope release.
+MOE_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+MOE_DEV bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// mbar_wait for a barrier that the other CTA of the pair arrives on (cluster-scope acquire).
+MOE_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, long long limit) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_cluster(a, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+// Tensor memory of the pair: the same warp of both CTAs, the same destination slot.
+MOE_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+MOE_DEV void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A * B^T over the pair (M = 256: 128 rows of A per CTA; B: N/2 rows per CTA).
+MOE_DEV void mma_f16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on the mbarrier at this offset in each CTA of `mask` when the pair MMAs this
+// thread issued so far complete.
+MOE_DEV void mma_commit_pair(uint64_t* bar, uint16_t mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(mask)
+        : "memory");
+}
 
 // ---------------------------------------------------------------- misc
 MOE_DEV int warp_id() { return threadIdx.x >> 5; }

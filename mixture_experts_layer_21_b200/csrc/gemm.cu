@@ -76,6 +76,7 @@ struct GemmArgs {
     int x3d;          // FP4: the token map is 3-D {64, rows, K/64}: one copy per 128-K stage
     DevError* err;
     long long wait_limit;  // cycles a pipeline wait may take before the kernel gives up
+    int l2_w, l2_t;        // L2 policy of the weight and of the token copies (see l2_policy)
 };
 
 struct CtrlBlock {
@@ -106,8 +107,13 @@ __device__ __forceinline__ void decode_tile(int L, const CtrlBlock* c, int G, in
     nt = r / mcount;
     const int mt = r - nt * mcount;
     const int start = g ? c->cu[g - 1] : 0;
-    row0 = start + mt * BT;
-    rows = min(BT, c->cu[g] - row0);
+    // the segment's mcount = ceil(len / BT) token tiles share its rows evenly (in multiples of
+    // 16, at most BT each), so that the tiles of one weight block take about the same time and
+    // read the weight tile from L2 together; (mcount - 1) * rs < len keeps every tile non-empty
+    const int len = c->cu[g] - start;
+    const int rs = min(BT, ((len + mcount - 1) / mcount + 15) & ~15);
+    row0 = start + mt * rs;
+    rows = min(rs, c->cu[g] - row0);
 }
 
 // One warp: the segment table (cu, clamped, and the running tile count tpre).
@@ -310,6 +316,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------- TMA producer
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -322,9 +329,9 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
-                    tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g);
-                    if (DUAL) tma_load_3d(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g);
-                    tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * kTileK, row0);
+                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
+                    if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
+                    tma_load_2d_p(opB(s), &tm_x, &ctl->full[s], kb * kTileK, row0, pol_t);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
@@ -427,6 +434,249 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ BF16 kernel on CTA pairs
+
+// The BF16 GEMM with two SMs per tile (a cluster of two CTAs, cta_group::2 MMAs). A pair tile
+// is 256 weight rows (128 from each CTA's shared memory) by up to BT tokens (BT/2 rows in each
+// CTA), so each SM moves half the token operand per FLOP of a one-SM tile of the same width.
+// The leader (rank 0) issues the MMAs; both CTAs produce their own operands and run the
+// epilogue of their own 128 weight rows. Barriers:
+//   full[s]   each CTA: its own copies of stage s landed (the leader's MMA thread waits on
+//             its own; in the peer, warp 1 waits and forwards to the leader's pfull[s])
+//   pfull[s]  leader: the peer's stage s landed
+//   empty[s]  each CTA: the MMAs that read stage s completed (commit multicast to both)
+//   tfull[b]  each CTA: accumulator buffer b holds a finished tile (commit multicast)
+//   tempty[b] leader: both CTAs' epilogue warps have drained buffer b
+template <int BT, bool DUAL>
+struct PairCfg {
+    static constexpr int NB = DUAL ? 2 : 1;
+    static constexpr int A_BYTES = kTileN * kTileK * 2;   // this CTA's 128 weight rows x 64 K
+    static constexpr int B_ROWS = BT / 2;                 // this CTA's half of the token tile
+    static constexpr int B_BYTES = B_ROWS * kTileK * 2;
+    static constexpr int STAGE = NB * A_BYTES + B_BYTES;
+    static constexpr int STAGES = cmin(kMaxStages, kSmemBudget / STAGE);
+    static constexpr int ACC_COLS = NB * BT;
+    static constexpr int ACC_BUFS = 2 * ACC_COLS <= 512 ? 2 : 1;
+    // with one accumulator buffer the MMAs wait for the epilogue: two warps per lane quarter
+    static constexpr int EW = ACC_BUFS == 1 ? 2 : 1;
+    static constexpr int EPI_WARPS = 4 * EW;
+    static constexpr int TMEM_COLS = tmem_cols_pow2(ACC_BUFS * ACC_COLS);
+    static constexpr int THREADS = (2 + EPI_WARPS) * 32;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + kCtrlBytes;
+    static_assert(STAGES >= 3 && SMEM_BYTES <= kSmemLimit && ACC_BUFS * ACC_COLS <= 512, "pair GEMM config");
+    static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "pair MMA N: a multiple of 32 (16 per CTA) up to 256");
+    static_assert(B_BYTES % 1024 == 0, "operands stay 1024-byte aligned");
+};
+
+// MMA width of a pair tile: its rows rounded up to 32 (each CTA's half a multiple of 16).
+__device__ __forceinline__ int pair_mma_n(int rows, int bt) { return min(bt, (rows + 31) & ~31); }
+
+template <int BT, bool DUAL, int OUT>
+__global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
+                             const __grid_constant__ CUtensorMap tm_w1, const GemmArgs a) {
+    using C = PairCfg<BT, DUAL>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
+    volatile int* abort_flag = &ctl->abort;
+    Issued is;  // this thread's copies or tcgen05 operations in flight
+    uint64_t* pfull = ctl->raw_full;
+    auto opA = [&](int s, int m) { return smem + s * C::STAGE + m * C::A_BYTES; };
+    auto opB = [&](int s) { return smem + s * C::STAGE + C::NB * C::A_BYTES; };
+    const int warp = warp_id(), lane = lane_id();
+    const int G = a.G, NT = a.NT, KB = a.KB;     // NT: blocks of 256 weight rows
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+            mbar_init(&pfull[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], 2 * C::EPI_WARPS);
+        }
+        mbar_init(&ctl->drain[0], 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w0);
+        if (DUAL) tma_prefetch_desc(&tm_w1);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&ctl->tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    pdl_wait();
+    if (warp == 0) build_segment_table<BT>(a, ctl, lane);
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
+    tc_fence_after();
+    pdl_launch();
+    const uint32_t tmem_base = ctl->tmem_slot;
+    const int total = ctl->tpre[G];
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------- producer: this CTA's weight rows and token half
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int L = pair; L < total && ok; L += npairs) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const int trow = row0 + (int)rank * (pair_mma_n(rows, BT) / 2);
+                const int wrow = (2 * nt + (int)rank) * kTileN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
+                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                    if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                    tma_load_2d_p(opB(s), &tm_x, &ctl->full[s], kb * kTileK, trow, pol_t);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {  // ---------------- MMA issuer of the pair
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0;
+            bool ok = true;
+            for (int L = pair; L < total && ok; L += npairs) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const uint32_t idesc = idesc_f16(1, 2 * kTileN, pair_mma_n(rows, BT));
+                if (!mbar_wait_cluster(&ctl->tempty[b], bph ^ 1u, abort_flag, a.wait_limit)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit) ||
+                        !mbar_wait_cluster(&pfull[s], ph, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(opA(s, 0));
+                    const uint32_t a1 = smem_u32(opA(s, DUAL ? 1 : 0));
+                    const uint32_t bb = smem_u32(opB(s));
+#pragma unroll
+                    for (int kk = 0; kk < kTileK / 16; ++kk) {
+                        const uint64_t bdesc = sw128_kmajor_desc(bb + kk * 32);
+                        const uint32_t acc = (kb | kk) != 0;
+                        mma_f16_ss_pair(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, acc);
+                        if (DUAL) mma_f16_ss_pair(d0 + BT, sw128_kmajor_desc(a1 + kk * 32), bdesc, idesc, acc);
+                    }
+                    is.tc = true;
+                    mma_commit_pair(&ctl->empty[s], 0x3);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair(&ctl->tfull[b], 0x3);
+                if (++b == C::ACC_BUFS) {
+                    b = 0;
+                    bph ^= 1u;
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 2);
+                ctl->abort = 1;
+            }
+        } else if (lane == 0) {  // ---------------- peer: tells the leader each stage landed
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int L = pair; L < total && ok; L += npairs) {
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&pfull[s]), 0));
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 6);
+                ctl->abort = 1;
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2 .. 2 + 4 EW) of this CTA's 128 weight rows
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        int b = 0;
+        uint32_t bph = 0;
+        for (int L = pair; L < total; L += npairs) {
+            int g, nt, row0, rows;
+            decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+            if (!mbar_wait(&ctl->tfull[b], bph, abort_flag, a.wait_limit)) {
+                if (lane == 0) report_error(a.err, MOE_ERR_TIMEOUT, 3);
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after();
+            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(
+                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, 2 * nt + (int)rank, row0,
+                rows, q, lane, h);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
+            if (++b == C::ACC_BUFS) {
+                b = 0;
+                bph ^= 1u;
+            }
+        }
+        if (a.zero_pad && OUT == OUT_BF16 && h == 0) zero_padding_rows(a, ctl, threadIdx.x - 64);
+    }
+
+    // Every CTA lets what it has in flight finish whether or not anything aborted (in a normal
+    // run these waits return at once): the producer's copies, and in the leader the pair's MMAs.
+    // Then neither CTA's shared or tensor memory is in use by the other, and both free it.
+    tc_fence_before();
+    __syncthreads();
+    {
+        int never = 0;
+        for (int q = 0; q < C::STAGES; ++q)
+            if (is.mask >> q & 1u) mbar_wait(&ctl->full[q], is.par >> q & 1u, &never);
+        if (is.tc) {
+            mma_commit_pair(&ctl->drain[0], 0x1);
+            mbar_wait(&ctl->drain[0], 0, &never);
+        }
+    }
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -566,6 +816,7 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer: two token boxes (TMA) + one copy per matrix
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int r = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -580,13 +831,13 @@ __global__ void __launch_bounds__(Fp4Cfg<BT, DUAL>::THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&ctl->raw_full[r], C::B_BYTES + C::NB * C::RAW_M);
                     const size_t off = (chunk0 + 2 * kb) * C::CHUNK;
-                    bulk_load(rawM(r, 0), a.kd0 + off, C::RAW_M, &ctl->raw_full[r]);
-                    if (DUAL) bulk_load(rawM(r, 1), a.kd1 + off, C::RAW_M, &ctl->raw_full[r]);
+                    bulk_load_p(rawM(r, 0), a.kd0 + off, C::RAW_M, &ctl->raw_full[r], pol_w);
+                    if (DUAL) bulk_load_p(rawM(r, 1), a.kd1 + off, C::RAW_M, &ctl->raw_full[r], pol_w);
                     if (a.x3d) {  // both 64-K boxes of the token tile in one copy: {64, rows, chunks}
-                        tma_load_3d(rawB(r), &tm_x, &ctl->raw_full[r], 0, row0, 2 * kb);
+                        tma_load_3d_p(rawB(r), &tm_x, &ctl->raw_full[r], 0, row0, 2 * kb, pol_t);
                     } else {
-                        tma_load_2d(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0);
-                        tma_load_2d(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0);
+                        tma_load_2d_p(rawB(r), &tm_x, &ctl->raw_full[r], kb * C::KS, row0, pol_t);
+                        tma_load_2d_p(rawB(r) + C::BOX_BYTES, &tm_x, &ctl->raw_full[r], kb * C::KS + kTileK, row0, pol_t);
                     }
                     is.mask |= 1u << r;
                     is.par = (is.par & ~(1u << r)) | (ph << r);
@@ -885,6 +1136,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -899,10 +1151,10 @@ __global__ void __launch_bounds__(Nvf4Cfg<BT, DUAL>::THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES + C::SFR_BYTES);
                     const size_t off = (tile0 + kb) * (size_t)kNvf4TileBytes;
-                    bulk_load(opA(s, 0), a.ks0 + off, kNvf4TileBytes, &ctl->full[s]);
-                    if (DUAL) bulk_load(opA(s, 1), a.ks1 + off, kNvf4TileBytes, &ctl->full[s]);
-                    tma_load_2d(opB(s), &tm_x, &ctl->full[s], kb * (kNvf4StageK / 2), row0);
-                    tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], kb * (kNvf4StageK / 16), row0);
+                    bulk_load_p(opA(s, 0), a.ks0 + off, kNvf4TileBytes, &ctl->full[s], pol_w);
+                    if (DUAL) bulk_load_p(opA(s, 1), a.ks1 + off, kNvf4TileBytes, &ctl->full[s], pol_w);
+                    tma_load_2d_p(opB(s), &tm_x, &ctl->full[s], kb * (kNvf4StageK / 2), row0, pol_t);
+                    tma_load_2d_p(sfRaw(s), &tm_sf, &ctl->full[s], kb * (kNvf4StageK / 16), row0, pol_t);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
@@ -1174,6 +1426,7 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------- producer
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -1188,15 +1441,15 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&ctl->full[s],
                                           C::NB * (C::A_TX + 512) + (TWO ? 2 : 1) * C::B_BYTES + C::SFR_BYTES);
-                    tma_load_3d(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g);
-                    bulk_load(sfA(s, 0), a.ks0 + (blk0 + kb) * 512, 512, &ctl->full[s]);
+                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g, pol_w);
+                    bulk_load_p(sfA(s, 0), a.ks0 + (blk0 + kb) * 512, 512, &ctl->full[s], pol_w);
                     if (DUAL) {
-                        tma_load_3d(opA(s, 1), &tm_w1, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g);
-                        bulk_load(sfA(s, 1), a.ks1 + (blk0 + kb) * 512, 512, &ctl->full[s]);
+                        tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g, pol_w);
+                        bulk_load_p(sfA(s, 1), a.ks1 + (blk0 + kb) * 512, 512, &ctl->full[s], pol_w);
                     }
-                    tma_load_2d(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0);
-                    if (TWO) tma_load_2d(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0);
-                    tma_load_2d(sfRaw(s), &tm_sf, &ctl->full[s], (kb >> 2) * 16, row0);
+                    tma_load_2d_p(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0, pol_t);
+                    if (TWO) tma_load_2d_p(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0, pol_t);
+                    tma_load_2d_p(sfRaw(s), &tm_sf, &ctl->full[s], (kb >> 2) * 16, row0, pol_t);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
@@ -1479,6 +1732,48 @@ cudaError_t run_bf16(const GemmProblem& p, const GemmArgs& args, const CUtensorM
                     args);
 }
 
+// Pairs that can be resident at once (clusters of two CTAs, one CTA per SM), per device.
+template <typename Kern>
+int max_pairs_once(Kern kern, int smem, int threads, int (&cache)[64]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cache[dev]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms() / 2));
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return 0;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <int BT, bool DUAL, int OUT>
+cudaError_t run_pair(const GemmProblem& p, GemmArgs args, const CUtensorMap& tx, const CUtensorMap& t0,
+                     const CUtensorMap& t1, cudaStream_t st, bool pdl) {
+    using C = PairCfg<BT, DUAL>;
+    auto kern = grouped_gemm_pair_kernel<BT, DUAL, OUT>;
+    static int done[64] = {0};
+    static int pairs_cache[64] = {0};
+    cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+    const int maxp = max_pairs_once(kern, C::SMEM_BYTES, C::THREADS, pairs_cache);
+    if (maxp < 1) return cudaErrorInvalidConfiguration;
+    args.NT = (p.N + 2 * kTileN - 1) / (2 * kTileN);
+    const long long tiles_ub = ((long long)(p.M_alloc + BT - 1) / BT + p.G) * args.NT;
+    const int pairs = (int)std::max<long long>(1, std::min<long long>(maxp, tiles_ub));
+    return launch_k_pairs(kern, dim3(2 * pairs), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, t0, t1,
+                          args);
+}
+
 template <int BT, bool DUAL, int OUT>
 cudaError_t run_fp4(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, cudaStream_t st, bool pdl) {
     using C = Fp4Cfg<BT, DUAL>;
@@ -1666,10 +1961,33 @@ long long wait_limit_cycles() {
     return kWaitLimitCycles;
 }
 
+// The BF16 GEMM runs on CTA pairs when segments average more than 96 rows (a pair tile is
+// up to 256 tokens wide) and no token tile was forced. MOE_GEMM_PAIRS=0 turns this off, =1
+// forces it for any segment size.
+bool use_pairs(const GemmProblem& p) {
+    const char* env = getenv("MOE_GEMM_PAIRS");
+    if (env && env[0] == '0' && env[1] == '\0') return false;
+    if (env && env[0] == '1' && env[1] == '\0') return true;
+    if (p.bt || getenv("MOE_TOKEN_TILE")) return false;
+    const long long segs = std::max<long long>(1, std::min<long long>(p.G, p.M_alloc));
+    return p.M_alloc > 96 * segs;
+}
+
+// L2 policies of the copies: MOE_L2_HINTS = 0 none, 1 token rows evict-last, 2 also the
+// weights evict-first (default 1). Token rows are re-read by every weight block of their
+// segment; weight tiles by the few token tiles of a segment, close together in time.
+void l2_policies(int* w, int* t) {
+    const char* env = getenv("MOE_L2_HINTS");
+    const int m = env && env[0] >= '0' && env[0] <= '2' && env[1] == '\0' ? env[0] - '0' : 1;
+    *t = m >= 1 ? 2 : 0;
+    *w = m >= 2 ? 1 : 0;
+}
+
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl) {
     if (p.G > kMaxG) return cudaErrorInvalidValue;
     GemmArgs a{};
     a.wait_limit = wait_limit_cycles();
+    l2_policies(&a.l2_w, &a.l2_t);
     a.cu = p.cu_seqlens;
     a.G = p.G;
     a.N = p.N;
@@ -1709,6 +2027,20 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
                  : choose_token_tile(p.M_alloc, p.G, wide_ok);
     }
     if (bt == 256 && !wide_req) bt = 128;
+    // BF16 prefill shapes run on CTA pairs: 256 weight rows x up to 256 tokens per pair tile
+    // (MOE_GEMM_PAIRS=0 keeps the one-SM kernel, e.g. to compare the two)
+    if (p.wfmt == MOE_W_BF16 && use_pairs(p)) {
+        CUtensorMap tx, t0, t1;
+        memset(&t1, 0, sizeof(t1));
+        if (!make_map_2d(&tx, p.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.M_alloc, 128) ||
+            !make_map_3d(&t0, p.w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G) ||
+            (p.dual && !make_map_3d(&t1, p.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G)))
+            return cudaErrorInvalidValue;
+        if (!p.dual) t1 = t0;
+        if (p.dual) return run_pair<256, true, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
+        if (p.out_kind == OUT_F32) return run_pair<256, false, OUT_F32>(p, a, tx, t0, t1, st, pdl);
+        return run_pair<256, false, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
+    }
     const CUtensorMapDataType xdt =
         p.wfmt == MOE_W_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tx, t0, t1;

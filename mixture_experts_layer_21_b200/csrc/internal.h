@@ -57,6 +57,27 @@ cudaError_t launch_rows_to_f16(const void* src, bool in_f32, int R, int K, __hal
 cudaError_t launch_act_and_mul(const __nv_bfloat16* gate, const __nv_bfloat16* up,
                                const float* perm_w, int M, int I, int act, float sa, float sb,
                                __nv_bfloat16* out, cudaStream_t st, bool pdl);
+// The same for a grid of CTA pairs (clusters of two CTAs; grid.x even).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv_perm, const float* topk_w,
                            int T, int topk, int H, __nv_bfloat16* out, cudaStream_t st, bool pdl);
 cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const float* topk_w, int T,

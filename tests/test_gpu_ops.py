@@ -159,6 +159,44 @@ def test_grouped_gemm_bf16_256_token_tile(lib, monkeypatch):
     check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what="bt256")
 
 
+def test_grouped_gemm_bf16_pairs_ragged(lib, monkeypatch):
+    # the CTA-pair kernel on segments of every awkward length (1, one under and over a tile of
+    # 256, several tiles, empty), N not a multiple of the 256-row pair block, K not of 64,
+    # padding rows after the last segment
+    monkeypatch.setenv("MOE_GEMM_PAIRS", "1")
+    seg = [1, 17, 0, 33, 100, 255, 256, 257, 600, 31]
+    M, N, K = sum(seg) + 5, 200, 136
+    a, wt, _ = W.gen_grouped_gemm_case(M, seg, N, K, seed=77)
+    cu = np.cumsum(seg).astype(np.int32)
+    w = lib.Weight("bf16", to_dev(wt))
+    out = lib.moe_grouped_gemm(to_dev(a), w, to_dev(torch.from_numpy(cu)),
+                               out=torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    ref = O.grouped_gemm(O.to_f64(a), W.WeightSet("bf16", wt), cu, M_alloc=M)
+    check_bf16(out, ref, atol=1e-5 * max(1.0, np.abs(ref).max()), rtol=2.0 ** -8, rel=4e-3, what="pairs")
+
+
+def test_forward_bf16_pairs_ragged(lib, monkeypatch):
+    # the fused layer with both GEMMs on CTA pairs: a given top-1 routing that gives the
+    # experts 0, 1, 17, 33, 100, 255, 256, 257 and 300 tokens; I = 384 leaves the second pair
+    # block of the gate/up GEMM half empty, H = 208 is not a multiple of 64
+    monkeypatch.setenv("MOE_GEMM_PAIRS", "1")
+    lens = [0, 1, 17, 33, 100, 255, 256, 257, 300]
+    cfg = W.MoEConfig("pairs", T=sum(lens), H=208, I=384, E=len(lens), topk=1)
+    inp = W.gen_inputs(cfg)
+    gid = np.concatenate([np.full(n, e, np.int32) for e, n in enumerate(lens)])
+    gid = np.random.default_rng(4).permutation(gid).reshape(-1, 1)
+    gw = np.random.default_rng(5).uniform(0.2, 1.0, (cfg.T, 1)).astype(np.float32)
+    dev = lambda ws: lib.Weight.from_host(ws)
+    layer = lib.MoEForward(dev(inp.w_gate), dev(inp.w_up), dev(inp.w_down), cfg.E, 1, routing="given", T_max=cfg.T)
+    out = layer(to_dev(inp.x), None, topk_ids_in=to_dev(torch.from_numpy(gid)), topk_w_in=to_dev(torch.from_numpy(gw)))
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    ref = O.moe_forward(cfg, inp.x, None, np.zeros(0, np.int32), inp.w_gate, inp.w_up, inp.w_down,
+                        given_topk=(gid, gw))
+    check_bf16(out, ref["out"], what="pairs forward")
+
+
 def test_grouped_gemm_bf16_matches_torch_grouped_mm(lib):
     if not hasattr(torch, "_grouped_mm"):
         pytest.skip("torch._grouped_mm unavailable")

@@ -22,12 +22,14 @@ pytestmark = pytest.mark.gpu
 MOE_ERR_TIMEOUT = 7
 
 CASES = {
-    # one per GEMM kernel: BF16; NVFP4 x NVFP4 block-scaled; MXFP4 x e4m3 hi/lo; NVFP4 weights
-    # with bf16 activations (converter warps into tensor memory)
+    # one per GEMM kernel: BF16 on one SM; NVFP4 x NVFP4 block-scaled; MXFP4 x e4m3 hi/lo;
+    # NVFP4 weights with bf16 activations (converter warps into tensor memory)
     "bf16": W.MoEConfig("t_bf16", T=300, H=512, I=256, E=8, topk=2),
     "nvfp4": W.MoEConfig("t_nvfp4", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4", act_quant=1),
     "mxfp4": W.MoEConfig("t_mxfp4", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4"),
     "nvfp4_a16": W.MoEConfig("t_nvfp4_a16", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4"),
+    # BF16 on CTA pairs (segments of about 150 rows)
+    "bf16_pairs": W.MoEConfig("t_bf16_pairs", T=600, H=256, I=256, E=8, topk=2),
 }
 
 
@@ -40,6 +42,7 @@ def test_wait_timeout_is_reported_and_the_next_call_is_correct(lib, name, monkey
                            situ_alpha=cfg.situ_alpha, situ_beta=cfg.situ_beta, act_quant=cfg.act_quant,
                            T_max=cfg.T)
     x, logits = to_dev(inp.x), to_dev(inp.logits)
+    monkeypatch.setenv("MOE_GEMM_PAIRS", "1" if name == "bf16_pairs" else "0")
     monkeypatch.setenv("MOE_WAIT_LIMIT_CYCLES", "1")
     layer(x, logits)
     torch.cuda.synchronize()                       # the kernels returned
