@@ -73,12 +73,6 @@ def segment_stats(cfg: W.MoEConfig, topk_ids: torch.Tensor, replica_src: torch.T
     return nonempty, max_seg
 
 
-def split_fc1(cfg) -> bool:
-    """SWIGLUOAI or GEMM biases: gate and up run as two GEMMs with fp32 outputs, then a
-    bias/activation row pass; the down bias is a row pass after the down GEMM."""
-    return cfg.act == "swigluoai" or cfg.bias
-
-
 def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) -> dict:
     NvS = cfg.NvS
     wg, wu, wd = (weight_bytes_per_row(inp.w_gate), weight_bytes_per_row(inp.w_up),
@@ -94,14 +88,10 @@ def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) 
     fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * a_in + NvS * cfg.I * act_out
     fc2_bytes = nonempty * wd + NvS * cfg.I * a_in + NvS * cfg.H * 4
     bias_bytes = nonempty * (2 * cfg.I + cfg.H) * 4 if cfg.bias else 0
-    if split_fc1(cfg):
-        # the operand is read by both GEMMs; gate and up leave in fp32 and are read back by the
-        # row pass with the gate/up biases; h leaves in fp32 when a row pass follows (FP4)
-        act_out = 2 if cfg.wfmt == "bf16" else 4
-        fc1_bytes = (nonempty * (wg + wu) + 2 * NvS * cfg.H * a_in + 2 * 2 * NvS * cfg.I * 4
-                     + NvS * cfg.I * act_out + (nonempty * 2 * cfg.I * 4 if cfg.bias else 0))
-        if cfg.bias:
-            fc2_bytes += 2 * NvS * cfg.H * 4 + nonempty * cfg.H * 4      # the down bias pass over y
+    if cfg.bias:
+        # the epilogues read each non-empty expert's bias rows: gate and up, then down
+        fc1_bytes += nonempty * 2 * cfg.I * 4
+        fc2_bytes += nonempty * cfg.H * 4
     layer_bytes = nonempty * (wg + wu + wd) + bias_bytes + cfg.T * cfg.H * 2 * 2 + cfg.T * cfg.E * 4
     return dict(nonempty=nonempty, max_seg=max_seg,
                 fc1_flops=fc1_flops, fc2_flops=fc2_flops, fc1_bytes=fc1_bytes, fc2_bytes=fc2_bytes,
@@ -323,12 +313,8 @@ def kernel_launches(cfg) -> int:
     n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
     if cfg.act_quant or cfg.wfmt == "mxfp4":
         n += 2                            # x quantisation / staging, activation quantisation / staging
-    elif cfg.wfmt != "bf16" and (cfg.act != "situ" or split_fc1(cfg)):
+    elif cfg.wfmt != "bf16" and cfg.act != "situ":
         n += 1                            # activation row pass to f16
-    if split_fc1(cfg):
-        n += 2                            # gate and up as two GEMMs, the bias/activation row pass
-        if cfg.bias:
-            n += 1                        # the down bias
     return n
 
 
@@ -480,8 +466,7 @@ def run_ours(args, cfg, rank, world):
         ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"]}
-    kname = ("grouped GEMMs gate, up (fp32 out) + bias/activation row pass" if split_fc1(cfg)
-             else "grouped GEMM gate+up (fused activation)")
+    kname = "grouped GEMM gate+up (fused activation" + (", biases)" if cfg.bias else ")")
     roof.update({"traffic": traffic, "kernel": kname,
                  "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
                  "kernel_ms": fc1_ms, "peak_source": f"{peak_src} (burst); tensor peak {tensor_note}"})

@@ -406,13 +406,12 @@ typedef struct {
     const float* bias_down;
 } moe_forward_args_t;
 
-/* With SWIGLUOAI or any bias the gate and up projections run as two grouped GEMMs with
- * fp32 outputs, followed by a row pass that adds the biases and applies the activation
- * and the route weight (moe_bias_act_and_mul), and the down bias is added to the down
- * projection's fp32 rows before the combine. That needs 8*T_max*topk*I more workspace
- * bytes: size it with moe_forward_workspace_size_args, which reads T_max, H, I, E, B,
- * topk, w_gate.fmt, act_quant, act.act and the three bias pointers of `args` and
- * otherwise equals moe_forward_workspace_size. */
+/* SWIGLUOAI and the biases run inside the grouped GEMMs: the gate/up GEMM's epilogue adds
+ * the gate and up biases, applies the activation and the route weight; the down GEMM's
+ * epilogue adds the down bias (times the route weight when the activation carries it) to
+ * the fp32 rows the combine sums. They need no workspace of their own:
+ * moe_forward_workspace_size_args (which reads T_max, H, I, E, B, topk, w_gate.fmt and
+ * act_quant of `args`) equals moe_forward_workspace_size. */
 size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int topk,
                                   int wfmt, int act_quant);
 size_t moe_forward_workspace_size_args(const moe_forward_args_t* args);

@@ -367,8 +367,7 @@ class MoEForward:
                  swiglu_alpha: float = 1.702, swiglu_beta: float = 1.0, swiglu_limit: float | None = 7.0,
                  biases=None):
         """``biases``: None, or (bias_gate [E+B,I], bias_up [E+B,I], bias_down [E+B,H]) fp32
-        device tensors, each of which may be None. With act "swigluoai" or any bias the layer
-        runs gate and up as two GEMMs and a bias/activation row pass."""
+        device tensors, each of which may be None; the GEMMs' epilogues apply them."""
         for w in (w_gate, w_up, w_down):
             if w.fmt != "bf16" and w.prepared is None:
                 moe_prepare_weights(w)

@@ -18,14 +18,11 @@ cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, 
 cudaError_t launch_scale_rows(const __nv_bfloat16* x, const float* w, int T, int H, __nv_bfloat16* out,
                               cudaStream_t st, bool pdl);
 moe_status_t prepare_weights(moe_weight_t* w, void* dst, size_t dst_bytes, cudaStream_t st);
-// Bias and gated-activation row passes (bias_act.cu): out = act(gate + bg[seg], up + bu[seg])
-// * perm_w over [M, I] (I % 8 == 0; rows past cu[G-1] written as zero), and
-// y[r,:] += perm_w[r] * b[seg(r),:] over fp32 [M, N] (N % 8 == 0).
+// The bias and gated-activation row pass (bias_act.cu): out = act(gate + bg[seg], up + bu[seg])
+// * perm_w over [M, I] (I % 8 == 0; rows past cu[G-1] written as zero).
 cudaError_t launch_bias_act(const void* gate, const void* up, bool in_f32, const float* bg, const float* bu,
                             const int32_t* cu, int G, const float* perm_w, int M, int I, int act, float sa, float sb,
                             float oa, float ob, float lim, void* out, bool out_f32, cudaStream_t st, bool pdl);
-cudaError_t launch_add_row_bias(float* y, const int32_t* cu, int G, const float* b, const float* perm_w, int M, int N,
-                                cudaStream_t st, bool pdl);
 
 int num_sms() {
     static int cached[64] = {0};
@@ -109,7 +106,7 @@ const float* weight_alpha(const moe_weight_t& w) { return w.fmt == MOE_W_BF16 ? 
 struct FwdWs {
     size_t ids, w, cu, perm_token, perm_w, inv, perm_scratch, xperm, tscale, xq_codes, xq_sb, xq_s,
         xq_deq, xq_rec, xperm_rec, act, act2, act2_scale, act_codes, act_sb, act_rec, mx_xq, mx_xperm, mx_act,
-        x_in, y, gu_gate, gu_up, bytes;
+        x_in, y, bytes;
 };
 
 // With NVFP4 activations a GEMM whose K is a multiple of 256 runs block-scaled on the
@@ -119,9 +116,7 @@ inline bool nvf4_k(int act_quant, int K) { return act_quant == 1 && K % kNvf4Sta
 inline int mx8_terms(int act_quant) { return act_quant == 2 ? 1 : 2; }
 inline int nvf4_rec_bytes(int K) { return K / 2 + K / 16; }
 
-// split: the gate and up projections run as two plain GEMMs into fp32 [NvS, I] buffers
-// (SWIGLUOAI or biases); those two buffers come last, so the other offsets do not move.
-FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant, bool split = false) {
+FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int act_quant) {
     FwdWs L{};
     const size_t NvS = (size_t)T_max * topk;
     const int G = E + B;
@@ -162,8 +157,6 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.mx_act = take(mx ? NvS * mx8_rec_bytes(I, terms) : 0);
     L.x_in = take(topk == 1 ? 2 * (size_t)T_max * H : 0);  // x times the top-1 weight (input-side weighting)
     L.y = take(4 * NvS * H);  // fp32: the output is rounded to bf16 once, in the combine
-    L.gu_gate = take(split ? 4 * NvS * I : 0);
-    L.gu_up = take(split ? 4 * NvS * I : 0);
     L.bytes = off;
     return L;
 }
@@ -446,18 +439,13 @@ size_t moe_forward_workspace_size(int T_max, int H, int I, int E, int B, int top
 
 }  // extern "C"
 
-namespace {
-// The layer runs gate and up as two GEMMs plus a bias/activation row pass.
-bool split_fc1(const moe_forward_args_t& a) {
-    return a.act.act == MOE_ACT_SWIGLUOAI || a.bias_gate || a.bias_up || a.bias_down;
-}
-}  // namespace
-
 extern "C" {
 
+// The workspace of a given argument set. SWIGLUOAI and the GEMM biases run in the GEMMs'
+// epilogues and need nothing extra, so this equals moe_forward_workspace_size.
 size_t moe_forward_workspace_size_args(const moe_forward_args_t* a) {
     if (!a || a->T_max < 0 || a->H < 1 || a->I < 1 || a->E < 1 || a->B < 0 || a->topk < 1) return 0;
-    return fwd_layout(a->T_max, a->H, a->I, a->E, a->B, a->topk, a->w_gate.fmt, a->act_quant, split_fc1(*a)).bytes;
+    return fwd_layout(a->T_max, a->H, a->I, a->E, a->B, a->topk, a->w_gate.fmt, a->act_quant).bytes;
 }
 
 moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -493,8 +481,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (H % 16 || I % 16) return MOE_ERR_ALIGNMENT;
     if (B > 0 && !p->replica_src) return MOE_ERR_INVALID_ARG;
     if (!ws) return MOE_ERR_INVALID_ARG;
-    const bool split = split_fc1(*p);
-    const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant, split);
+    const FwdWs L = fwd_layout(p->T_max, H, I, E, B, k, fmt, p->act_quant);
     if (ws_bytes < L.bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (T == 0) return MOE_OK;
     if (!p->x || (!p->router_logits && p->routing != 2) || !p->out) return MOE_ERR_INVALID_ARG;
@@ -628,6 +615,11 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g1.act = p->act.act;
     g1.situ_a = p->act.situ_alpha;
     g1.situ_b = p->act.situ_beta;
+    g1.sw_alpha = p->swiglu_alpha;
+    g1.sw_beta = p->swiglu_beta;
+    g1.sw_limit = p->swiglu_limit;
+    g1.bias0 = p->bias_gate;
+    g1.bias1 = p->bias_up;
     g1.out = act;
     g1.err = err;
     if (fmt == MOE_W_MXFP4) {
@@ -669,38 +661,9 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         g1.out_kind = OUT_F32;
         row_pass = true;
     }
-    if (split) {
-        // SWIGLUOAI or biases: gate and up as two plain grouped GEMMs with fp32 outputs,
-        // then one row pass adds the biases and applies the activation and route weight
-        GemmProblem gg = g1;
-        gg.dual = false;
-        gg.w1 = nullptr;
-        gg.kdata1 = nullptr;
-        gg.kscale1 = nullptr;
-        gg.alpha1 = nullptr;
-        gg.perm_w = nullptr;
-        gg.act = MOE_ACT_SILU;
-        gg.out_scale = 1.0f;
-        gg.out_kind = OUT_F32;
-        gg.out = w + L.gu_gate;
-        e = launch_grouped_gemm(gg, st, pdl());
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        gg.w0 = p->w_up.data;
-        gg.kdata0 = p->w_up.kdata;
-        gg.kscale0 = p->w_up.kscale;
-        gg.alpha0 = weight_alpha(p->w_up);
-        gg.out = w + L.gu_up;
-        e = launch_grouped_gemm(gg, st, pdl());
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        // h in fp32 when a row pass quantises or stages it for FP4 weights, else bf16
-        row_pass = fmt != MOE_W_BF16;
-        fc2_out_scale = 1.0f;
-        e = launch_bias_act(w + L.gu_gate, w + L.gu_up, true, p->bias_gate, p->bias_up, cu, G, g1.perm_w, NvS, I,
-                            p->act.act, p->act.situ_alpha, p->act.situ_beta, p->swiglu_alpha, p->swiglu_beta,
-                            p->swiglu_limit, act, row_pass, st, pdl());
-    } else {
-        e = launch_grouped_gemm(g1, st, pdl());
-    }
+    // S3 + S4 in one launch: gate and up, their biases, the activation (SWIGLUOAI included)
+    // and the route weight in the epilogue
+    e = launch_grouped_gemm(g1, st, pdl());
     if (e != cudaSuccess || !mark(3)) return MOE_ERR_CUDA;
     const int rb2 = nvf4_rec_bytes(I);
     trace.stage("act_row_pass");
@@ -746,6 +709,10 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     g2.out = y;
     g2.out_kind = OUT_F32;
     g2.err = err;
+    // the expert's down bias is part of its output: under the route weight when the
+    // activation carries the weight, else the combine weights it with the rest
+    g2.bias0 = p->bias_down;
+    g2.bias_rw = g1.perm_w;
     if (fmt == MOE_W_MXFP4) {
         g2.mx8 = terms;
         g2.x_stride = mx8_rec_bytes(I, terms);
@@ -757,13 +724,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
         g2.xsf_stride = rb2;
     }
     e = launch_grouped_gemm(g2, st, pdl());
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (p->bias_down) {
-        // the expert's down bias, under the route weight when the activation carries it
-        e = launch_add_row_bias(y, cu, G, p->bias_down, g1.perm_w, NvS, H, st, pdl());
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-    }
-    if (!mark(5)) return MOE_ERR_CUDA;
+    if (e != cudaSuccess || !mark(5)) return MOE_ERR_CUDA;
     // S6: combine
     trace.stage("combine");
     e = launch_combine_f32(y, inv, (p->apply_topk_in_fc1 || in_w) ? nullptr : tw, T, k, H,

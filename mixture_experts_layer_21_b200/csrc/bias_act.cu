@@ -1,13 +1,12 @@
-// Row passes of the layer with per-expert GEMM biases and the SWIGLUOAI activation
-// (TRTLLM MXFP4 experts page: SWIGLUOAI among the supported activations, gemm1_alpha,
-// gemm1_beta and gemm1_clamp_limit broadcast to every local expert in __init__, and
-// gemm1_bias / gemm2_bias handed to the kernel in _invoke_kernel).
+// The standalone bias/activation row pass (moe_bias_act_and_mul): per-expert gate/up
+// biases and every gated activation, SWIGLUOAI included (TRTLLM MXFP4 experts page:
+// SWIGLUOAI among the supported activations, gemm1_alpha, gemm1_beta and
+// gemm1_clamp_limit broadcast to every local expert in __init__, gemm1_bias handed to the
+// kernel in _invoke_kernel). The fused layer does the same in the gate/up GEMM's epilogue.
 //
-// With these, the gate and up projections come out of two plain grouped GEMMs in fp32;
 // bias_act_kernel adds each row's expert bias, applies the gated activation and the route
-// weight; after the down GEMM, add_row_bias_kernel adds the down projection's bias under
-// the same route weight. The expert of a segment row is found from cu_seqlens (inclusive
-// segment ends) by binary search, so redundant slots use their own bias rows.
+// weight. The expert of a segment row is found from cu_seqlens (inclusive segment ends) by
+// binary search, so redundant slots use their own bias rows.
 #include "internal.h"
 
 namespace moe {
@@ -124,33 +123,6 @@ __global__ void __launch_bounds__(256) bias_act_kernel(const void* __restrict__ 
     pdl_launch();
 }
 
-// y[r,n] += perm_w[r] * b[g,n] (perm_w NULL: weight 1) for the rows of segment g < G;
-// rows at or past cu[G-1] are left as they are. y fp32 [M, N], b fp32 [G, N], N % 8 == 0.
-__global__ void __launch_bounds__(256) add_row_bias_kernel(float* __restrict__ y, const int32_t* __restrict__ cu,
-                                                           int G, const float* __restrict__ b,
-                                                           const float* __restrict__ perm_w, int M, int N) {
-    pdl_wait();
-    const int c8n = N / 8;
-    const long long n8 = (long long)M * c8n;
-    for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8;
-         v += (long long)gridDim.x * blockDim.x) {
-        const int r = (int)(v / c8n);
-        const int c = (int)(v - (long long)r * c8n) * 8;
-        const int g = segment_of(cu, G, r);
-        if (g < G) {
-            const size_t i = (size_t)r * N + c;
-            const float w = perm_w ? perm_w[r] : 1.0f;
-            float yv[8], bv[8];
-            ld8<true>(y, i, yv);
-            ld8<true>(b, (size_t)g * N + c, bv);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) yv[q] = fmaf(w, bv[q], yv[q]);
-            st8<true>(y, i, yv);
-        }
-    }
-    pdl_launch();
-}
-
 namespace {
 inline int row_pass_blocks(long long n8) {
     return (int)std::min<long long>((n8 + 255) / 256, (long long)num_sms() * 16);
@@ -176,13 +148,6 @@ cudaError_t launch_bias_act(const void* gate, const void* up, bool in_f32, const
                         a, out);
     return launch_k(bias_act_kernel<false, false>, grid, block, 0, st, pdl, gate, up, bg, bu, cu, G, perm_w, M, I, a,
                     out);
-}
-
-cudaError_t launch_add_row_bias(float* y, const int32_t* cu, int G, const float* b, const float* perm_w, int M, int N,
-                                cudaStream_t st, bool pdl) {
-    const long long n8 = (long long)M * (N / 8);
-    if (n8 == 0) return cudaSuccess;
-    return launch_k(add_row_bias_kernel, dim3(row_pass_blocks(n8)), dim3(256), 0, st, pdl, y, cu, G, b, perm_w, M, N);
 }
 
 }  // namespace moe

@@ -415,5 +415,12 @@ MOE_DEV float act_apply_fast(int act, float g, float u, float a, float b, float 
     if (act == MOE_ACT_SITU) return a * fast_tanh(g * inv_a) * fast_sigmoid(g) * (b * fast_tanh(u * inv_b));
     return g * fast_sigmoid(g) * u;
 }
+// SWIGLUOAI (the GPT-OSS gated activation): g = min(gate, lim), u = clamp(up, -lim, lim),
+// g * sigmoid(alpha * g) * (u + beta); lim = +inf is no clamp.
+MOE_DEV float swigluoai_fast(float g, float u, float alpha, float beta, float lim) {
+    const float gc = fminf(g, lim);
+    const float uc = fminf(fmaxf(u, -lim), lim);
+    return gc * fast_sigmoid(alpha * gc) * (uc + beta);
+}
 
 }  // namespace moe

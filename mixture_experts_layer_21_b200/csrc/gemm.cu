@@ -77,6 +77,12 @@ struct GemmArgs {
     DevError* err;
     long long wait_limit;  // cycles a pipeline wait may take before the kernel gives up
     int l2_w, l2_t;        // L2 policy of the weight and of the token copies (see l2_policy)
+    // Per-expert fp32 biases [G, N] (or NULL): the gate/up pair adds bias0 / bias1 before the
+    // activation; a single GEMM adds bias_rw[row] * bias0 to its output (bias_rw NULL: 1).
+    const float* bias0;
+    const float* bias1;
+    const float* bias_rw;
+    float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI
 };
 
 struct CtrlBlock {
@@ -181,6 +187,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
     const int n = nt * kTileN + q * 32 + lane;
     const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
     const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
+    const float bn0 = (a.bias0 && n < a.N) ? a.bias0[(size_t)g * a.N + n] : 0.0f;
+    const float bn1 = (DUAL && a.bias1 && n < a.N) ? a.bias1[(size_t)g * a.N + n] : 0.0f;
     const float inv_sa = 1.0f / a.sa, inv_sb = 1.0f / a.sb;
     constexpr int NB = DUAL ? 2 : 1;
     auto col = [](int m, int j) { return (PM ? m * NPART + j : j * NB + m) * BT; };
@@ -207,7 +215,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
         const int my_row = row0 + c0 + (lane & 15);
         const bool row_ok = c0 + (lane & 15) < rows;
         const float my_ts = (a.tscale && row_ok) ? a.tscale[my_row] : 1.0f;
-        const float my_pw = (DUAL && a.perm_w && row_ok) ? a.perm_w[my_row] : 1.0f;
+        // the dual GEMM's route weight; a single GEMM's weight of its bias
+        const float* rw = DUAL ? a.perm_w : a.bias_rw;
+        const float my_pw = (rw && row_ok) ? rw[my_row] : 1.0f;
         {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -218,13 +228,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
                     const int row = row0 + c0 + j;
                     float v;
                     if (DUAL) {
-                        const float gv = __uint_as_float(r0[j]) * al0 * ts;
-                        const float uv = __uint_as_float(r1[j]) * al1 * ts;
-                        v = act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb) * pw;
+                        const float gv = __uint_as_float(r0[j]) * al0 * ts + bn0;
+                        const float uv = __uint_as_float(r1[j]) * al1 * ts + bn1;
+                        v = (a.act == MOE_ACT_SWIGLUOAI
+                                 ? swigluoai_fast(gv, uv, a.sw_alpha, a.sw_beta, a.sw_limit)
+                                 : act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb)) *
+                            pw;
+                        v *= a.out_scale;
                     } else {
-                        v = __uint_as_float(r0[j]) * al0 * ts;
+                        v = __uint_as_float(r0[j]) * al0 * ts * a.out_scale + pw * bn0;
                     }
-                    v *= a.out_scale;
                     const size_t idx = (size_t)row * a.N + n;
                     if (OUT == OUT_BF16) reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
                     else if (OUT == OUT_F16) reinterpret_cast<__half*>(a.out)[idx] = __float2half_rn(v);
@@ -2002,6 +2015,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.perm_w = p.perm_w;
     a.tscale = p.tscale;
     a.out_scale = p.out_scale;
+    a.bias0 = p.bias0;
+    a.bias1 = p.bias1;
+    a.bias_rw = p.bias_rw;
+    a.sw_alpha = p.sw_alpha;
+    a.sw_beta = p.sw_beta;
+    a.sw_limit = p.sw_limit;
     a.act = p.act;
     a.sa = p.situ_a;
     a.sb = p.situ_b;

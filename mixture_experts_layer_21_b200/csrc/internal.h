@@ -135,6 +135,13 @@ struct GemmProblem {
     // 1 = MXFP8 activations): x = records of mx8 * Kp codes then the scales (x_stride bytes
     // apart), kdata0/1 = the padded codes, kscale0/1 = the scale blocks.
     int mx8;
+    // Per-expert fp32 biases [G, N] or NULL (gemm1_bias / gemm2_bias): the dual GEMM adds
+    // bias0 to gate and bias1 to up before the activation; a single GEMM adds
+    // bias_rw[row] * bias0 to its (scaled) output, bias_rw NULL meaning 1.
+    const float* bias0;
+    const float* bias1;
+    const float* bias_rw;
+    float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI (act == MOE_ACT_SWIGLUOAI)
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
 int choose_token_tile(long long NvS, int G, bool wide_ok);

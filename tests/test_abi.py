@@ -254,17 +254,17 @@ def test_binding_structs_match_the_header(name):
 
 
 def test_forward_workspace_with_biases_or_swigluoai():
+    # SWIGLUOAI and the biases run in the GEMM epilogues: no workspace of their own
     p, nws = _fwd()
-    assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == nws      # fused gate/up: the same size
+    assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == nws
     p, _ = _fwd(act=2)
-    n2 = L.moe_forward_workspace_size_args(ctypes.byref(p))
-    assert n2 >= nws + 8 * (8 * 2) * 128                                  # two fp32 [T_max*topk, I] buffers
-    assert L.moe_forward(ctypes.byref(p), 16, nws, None) == WS_SMALL
+    assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == nws
+    assert L.moe_forward(ctypes.byref(p), 16, nws - 1, None) == WS_SMALL
     for b in ("bias_gate", "bias_up", "bias_down"):
         p, _ = _fwd(**{b: 16})
-        assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == n2
+        assert L.moe_forward_workspace_size_args(ctypes.byref(p)) == nws
         p.T = 0
-        assert L.moe_forward(ctypes.byref(p), 16, n2, None) == 0           # no tokens: nothing launched
+        assert L.moe_forward(ctypes.byref(p), 16, nws, None) == 0          # no tokens: nothing launched
     assert L.moe_forward_workspace_size_args(None) == 0
 
 

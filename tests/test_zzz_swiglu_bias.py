@@ -1,12 +1,13 @@
 """GPU parity of the per-expert GEMM biases and the SWIGLUOAI activation against the oracle:
-the bias/activation row pass alone (moe_bias_act_and_mul), and the layer, which runs gate and
-up as two grouped GEMMs with fp32 outputs when either is asked for.
+the bias/activation row pass alone (moe_bias_act_and_mul), and the layer, which applies both
+in the grouped GEMMs' epilogues.
 
 Tolerances: the row pass computes in fp32 and rounds once to bf16, so each output lies within
 half a bf16 ulp (<= 2^-8 |ref|) of the fp64 oracle plus the fp32 arithmetic's error (a few
 fp32 ulps: <= 1e-6 |ref| + 1e-5, the absolute part for outputs that cancel); padding rows
 are exactly zero. Layers: as in tests/parity.py
-(BF16 |d| <= 2e-2 + 2^-8 |ref| and rel-L2 <= 1e-2; FP4 weights rel-L2 <= 3e-2).
+(BF16 |d| <= 2e-2 + 2^-8 |ref| and rel-L2 <= 1e-2; FP4 weights the element-wise bound derived
+from the layer's arithmetic and rel-L2 <= 3e-2).
 
 The file name sorts after every other test file: these kernels are the newest, so a run that
 stops at its first failure has run all the others first.
@@ -83,7 +84,7 @@ SMALL = {
     # replicas and empty slots: every slot reads its own bias rows
     "bf16_silu_bias_replicas": W.MoEConfig("bf16_silu_bias_replicas", T=300, H=128, I=256, E=16, topk=4, B=6,
                                            B_used=4, logit_std=2.0, bias=True, bias_down_std=0.03),
-    # SWIGLUOAI without biases (the split path taken for the activation alone)
+    # SWIGLUOAI without biases
     "bf16_swiglu_nobias": W.MoEConfig("bf16_swiglu_nobias", T=40, H=128, I=192, E=8, topk=2, act="swigluoai",
                                       swiglu_alpha=1.2, swiglu_limit=None),
     # MXFP4 weights with bf16 activations, the GPT-OSS activation constants
