@@ -77,12 +77,15 @@ def accounting(cfg: W.MoEConfig, inp: W.MoEInputs, nonempty: int, max_seg: int) 
     NvS = cfg.NvS
     wg, wu, wd = (weight_bytes_per_row(inp.w_gate), weight_bytes_per_row(inp.w_up),
                   weight_bytes_per_row(inp.w_down))
-    # gate/up output: bf16 (BF16), f16 (NVFP4 weights, bf16 activations, SITU), else fp32
-    act_out = 2 if cfg.wfmt == "bf16" or (cfg.wfmt == "nvfp4" and cfg.act == "situ" and not cfg.act_quant) else 4
     # activation operand bytes per value as the GEMMs read them
     a_in = {0: 2.0, 1: 9.0 / 16.0, 2: 1.0 + 1.0 / 32.0}[cfg.act_quant]
     if cfg.wfmt == "mxfp4" and not cfg.act_quant:
         a_in = 2.0 + 1.0 / 32.0           # two e4m3 terms and a scale per 32 values
+    # gate/up output: bf16 (BF16), f16 (NVFP4 weights, bf16 activations, SITU), the down
+    # GEMM's e4m3 records (MXFP4), else fp32
+    act_out = 2 if cfg.wfmt == "bf16" or (cfg.wfmt == "nvfp4" and cfg.act == "situ" and not cfg.act_quant) else 4
+    if cfg.wfmt == "mxfp4":
+        act_out = a_in
     fc1_flops = 4.0 * NvS * cfg.H * cfg.I
     fc2_flops = 2.0 * NvS * cfg.H * cfg.I
     fc1_bytes = nonempty * (wg + wu) + NvS * cfg.H * a_in + NvS * cfg.I * act_out
@@ -311,8 +314,10 @@ def default_sample(cfg) -> int:
 
 def kernel_launches(cfg) -> int:
     n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
-    if cfg.act_quant or cfg.wfmt == "mxfp4":
-        n += 2                            # x quantisation / staging, activation quantisation / staging
+    if cfg.wfmt == "mxfp4":
+        n += 1                            # x staging (the gate/up epilogue stages the activations)
+    elif cfg.act_quant:
+        n += 2                            # x quantisation, activation quantisation
     elif cfg.wfmt != "bf16" and cfg.act != "situ":
         n += 1                            # activation row pass to f16
     return n

@@ -144,13 +144,15 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.xq_deq = take(q1 ? 2 * (size_t)T_max * H : 0);
     L.xq_rec = take(nat1 ? (size_t)T_max * nvf4_rec_bytes(H) : 0);
     L.xperm_rec = take(nat1 ? NvS * nvf4_rec_bytes(H) : 0);
-    L.act = take((fp4 ? 4 : 2) * NvS * I);  // fp32 when a row pass follows
+    const bool mx = wfmt == MOE_W_MXFP4;
+    // h: bf16 (BF16 weights), fp32 when a row pass follows (NVFP4 weights); the MXFP4 gate/up
+    // epilogue writes the down GEMM's records directly
+    L.act = take(mx ? 0 : (fp4 ? 4 : 2) * NvS * I);
     L.act2 = take(fp4 && !nat2 && wfmt != MOE_W_MXFP4 ? 2 * NvS * I : 0);
     L.act2_scale = take(fp4 ? 4 * NvS : 0);
     L.act_codes = take(q2 ? NvS * I / 2 : 0);
     L.act_sb = take(q2 ? NvS * I / 16 : 0);
     L.act_rec = take(nat2 ? NvS * nvf4_rec_bytes(I) : 0);
-    const bool mx = wfmt == MOE_W_MXFP4;
     const int terms = mx8_terms(act_quant);
     L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H, terms) : 0);
     L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H, terms) : 0);
@@ -646,8 +648,12 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (fmt == MOE_W_BF16) {
         g1.out_kind = OUT_BF16;
     } else if (fmt == MOE_W_MXFP4) {
-        g1.out_kind = OUT_F32;
-        row_pass = true;
+        // the epilogue writes h straight as the down GEMM's e4m3 records and e8m0 scales
+        g1.out_kind = OUT_MX8;
+        g1.out = w + L.mx_act;
+        g1.out_terms = terms;
+        g1.out_stride = mx8_rec_bytes(I, terms);
+        fc2_x = w + L.mx_act;
     } else if (situ && !p->act_quant) {
         // |h| <= alpha*beta*|route weight| <= alpha*beta: one fixed power of two keeps it below 2^15
         const double bound = (double)p->act.situ_alpha * p->act.situ_beta;
@@ -668,12 +674,7 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     const int rb2 = nvf4_rec_bytes(I);
     trace.stage("act_row_pass");
     if (row_pass) {
-        if (fmt == MOE_W_MXFP4) {
-            const int rb = mx8_rec_bytes(I, terms), Kp = mx8_kpad(I);
-            uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_act);
-            e = launch_quant_mx8(act, true, NvS, I, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr,
-                                 rec + terms * Kp, rb, rb, st, pdl());
-        } else if (nat2) {
+        if (nat2) {
             uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.act_rec);
             e = launch_quant_nvfp4(act, true, NvS, I, rec, rb2, rec + I / 2, rb2, act2_scale, nullptr, st, pdl());
         } else if (p->act_quant) {
@@ -683,10 +684,8 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
             e = launch_rows_to_f16(act, true, NvS, I, act2, act2_scale, st, pdl());
         }
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        fc2_x = fmt == MOE_W_MXFP4 ? static_cast<const void*>(w + L.mx_act)
-                : nat2                ? static_cast<const void*>(w + L.act_rec)
-                                      : act2;
-        fc2_tscale = fmt == MOE_W_MXFP4 ? nullptr : act2_scale;
+        fc2_x = nat2 ? static_cast<const void*>(w + L.act_rec) : act2;
+        fc2_tscale = act2_scale;
     }
     if (!mark(4)) return MOE_ERR_CUDA;
     // S5: down grouped GEMM

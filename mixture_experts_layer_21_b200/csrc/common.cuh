@@ -392,6 +392,35 @@ MOE_DEV void mma_commit_pair(uint64_t* bar, uint16_t mask) {
         : "memory");
 }
 
+// ---------------------------------------------------------------- e4m3 / MX staging
+// fp32 -> e4m3 (round to nearest even, saturating at +-448) and back.
+MOE_DEV uint8_t cvt_e4m3(float x) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return (uint8_t)(r & 0xFF);
+}
+MOE_DEV float e4m3_to_f32(uint8_t c) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)c));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
+}
+// Exponent e of the e8m0 scale 2^e of a 32-value block with largest magnitude amax, for the
+// MXFP4 GEMM's activations: two terms (hi/lo staging of bf16): the smallest e with
+// amax <= 448 * 2^e; one term (MXFP8, the OCP MX v1.0 rule): floor(log2 amax) - 8. A zero
+// block takes -127. Clamped to e8m0's [-127, 127].
+MOE_DEV int mx8_block_exp(float amax, bool two) {
+    if (!(amax > 0.0f)) return -127;
+    int ex;
+    const float m = frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
+    // hi/lo: 448 * 2^(ex-9) = 0.875 * 2^ex; one term: floor(log2 amax) - 8 = ex - 9
+    const int e = (two && m > 0.875f) ? ex - 8 : ex - 9;
+    return max(-127, min(127, e));
+}
+// 2^-e as a normal float for the e of mx8_block_exp (finite inputs give e <= 120).
+MOE_DEV float mx8_inv_scale(int e) {
+    return __int_as_float((127 - max(e, -126)) << 23) * (e < -126 ? 2.0f : 1.0f);
+}
+
 // ---------------------------------------------------------------- misc
 MOE_DEV int warp_id() { return threadIdx.x >> 5; }
 MOE_DEV int lane_id() { return threadIdx.x & 31; }

@@ -155,11 +155,6 @@ cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const fl
 //   sb   = e4m3_rne_satfinite(amax_b / (6 s_r))   per 16 values
 //   q    = e2m1_rne_satfinite(v / (sb s_r))
 // A zero row or a block scale that rounds to zero gives +0 codes.
-__device__ __forceinline__ uint8_t cvt_e4m3(float x) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
-    return (uint8_t)(r & 0xFF);
-}
 // Two values -> one byte: `lo` in the low nibble.
 __device__ __forceinline__ uint8_t cvt_e2m1x2(float lo, float hi) {
     uint16_t r;
@@ -167,11 +162,6 @@ __device__ __forceinline__ uint8_t cvt_e2m1x2(float lo, float hi) {
         : "=h"(r)
         : "f"(hi), "f"(lo));
     return (uint8_t)r;
-}
-__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
-    uint32_t h2;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)c));
-    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
 }
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint8_t b) {
     uint32_t r;
@@ -269,6 +259,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
     pdl_launch();
 }
 
+
 // ----------------------------------------------------------------- MXFP8 activations
 // Activation rows for the MXFP4-weight GEMM, whose tensor cores take e4m3 activations with
 // one e8m0 scale per 32 values. Two forms:
@@ -279,15 +270,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
 //   one term (dynamic MXFP8, the OCP MX v1.0 conversion): 2^e = 2^(floor(log2 amax_b) - 8)
 //     and q = e4m3_rne_satfinite(v * 2^-e) (saturating at 448).
 // One warp per row, one 32-value block per lane and step; blocks past K (up to Kp) are zero.
-__device__ __forceinline__ int mx8_block_exp(float amax, bool two) {
-    if (!(amax > 0.0f)) return -127;
-    int ex;
-    const float m = frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
-    // hi/lo: 448 * 2^(ex-9) = 0.875 * 2^ex; one term: floor(log2 amax) - 8 = ex - 9
-    const int e = (two && m > 0.875f) ? ex - 8 : ex - 9;
-    return max(-127, min(127, e));
-}
-
+// (mx8_block_exp, in common.cuh, picks e.)
 template <bool IN_F32, bool TWO>
 __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__ in, int R, int K, int Kp,
                                                         uint8_t* __restrict__ hi_out, uint8_t* __restrict__ lo_out,
@@ -308,8 +291,7 @@ __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__
 #pragma unroll
                 for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i >> 4][i & 15]));
                 e = mx8_block_exp(amax, TWO);
-                // 2^-e as a normal float: finite inputs give e <= 120 (amax < 2^128)
-                const float inv = __int_as_float((127 - max(e, -126)) << 23) * (e < -126 ? 2.0f : 1.0f);
+                const float inv = mx8_inv_scale(e);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float y = v[i >> 4][i & 15] * inv;

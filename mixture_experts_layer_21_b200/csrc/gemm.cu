@@ -83,6 +83,7 @@ struct GemmArgs {
     const float* bias1;
     const float* bias_rw;
     float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI
+    int out_terms, out_stride, out_kpad;  // OUT_MX8 records: terms, row stride, codes per term
 };
 
 struct CtrlBlock {
@@ -224,7 +225,31 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, in
                 // every lane takes part in the shuffles; only in-range outputs are stored
                 const float ts = __shfl_sync(0xffffffffu, my_ts, j);
                 const float pw = __shfl_sync(0xffffffffu, my_pw, j);
-                if (n < a.N && c0 + j < rows) {
+                if constexpr (OUT == OUT_MX8) {
+                    // the warp's 32 lanes are one 32-value block of the down GEMM's K: its
+                    // scale is a warp max; lanes past N (up to the padded K) write zeros
+                    float v = 0.0f;
+                    if (DUAL && n < a.N && c0 + j < rows) {
+                        const float gv = __uint_as_float(r0[j]) * al0 * ts + bn0;
+                        const float uv = __uint_as_float(r1[j]) * al1 * ts + bn1;
+                        v = (a.act == MOE_ACT_SWIGLUOAI
+                                 ? swigluoai_fast(gv, uv, a.sw_alpha, a.sw_beta, a.sw_limit)
+                                 : act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb)) *
+                            pw;
+                    }
+                    float am = fabsf(v);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+                    if (c0 + j < rows) {
+                        const int e = mx8_block_exp(am, a.out_terms == 2);
+                        const float y = v * mx8_inv_scale(e);
+                        uint8_t* rec = reinterpret_cast<uint8_t*>(a.out) + (size_t)(row0 + c0 + j) * a.out_stride;
+                        const uint8_t hi = cvt_e4m3(y);
+                        rec[n] = hi;
+                        if (a.out_terms == 2) rec[a.out_kpad + n] = cvt_e4m3(y - e4m3_to_f32(hi));
+                        if (lane == 0) rec[a.out_terms * a.out_kpad + n / 32] = (uint8_t)(e + 127);
+                    }
+                } else if (n < a.N && c0 + j < rows) {
                     const int row = row0 + c0 + j;
                     float v;
                     if (DUAL) {
@@ -1875,6 +1900,7 @@ cudaError_t dispatch_mx8_terms(const GemmProblem& p, const GemmArgs& args, const
                                const CUtensorMap& tsf, const CUtensorMap& t0, const CUtensorMap& t1, int Kp,
                                cudaStream_t st, bool pdl) {
     if (p.dual) {
+        if (p.out_kind == OUT_MX8) return run_mx8<BT, true, TWO, OUT_MX8>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
         if (p.out_kind != OUT_F32) return cudaErrorInvalidValue;
         return run_mx8<BT, true, TWO, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
     }
@@ -2021,6 +2047,13 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     a.sw_alpha = p.sw_alpha;
     a.sw_beta = p.sw_beta;
     a.sw_limit = p.sw_limit;
+    a.out_terms = p.out_terms;
+    a.out_stride = p.out_stride;
+    a.out_kpad = p.out_kind == OUT_MX8 ? mx8_kpad(p.N) : 0;
+    // the records cover the padded K of the down GEMM: N_tiles * 128 = mx8_kpad(N)
+    if (p.out_kind == OUT_MX8 && (p.wfmt != MOE_W_MXFP4 || !p.dual || p.N % 32 ||
+                                  (p.out_terms != 1 && p.out_terms != 2)))
+        return cudaErrorInvalidValue;
     a.act = p.act;
     a.sa = p.situ_a;
     a.sb = p.situ_b;

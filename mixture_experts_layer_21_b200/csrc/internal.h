@@ -94,7 +94,10 @@ cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_
 
 // ---------------------------------------------------------------- grouped GEMM
 // Output kinds of the GEMM epilogue.
-enum OutKind { OUT_BF16 = 0, OUT_F16 = 1, OUT_F32 = 2 };
+// OUT_MX8: the activation rows as the MXFP4 GEMM's operand records (see kMx8StageK below):
+// e4m3 codes (hi and lo, or one term) and one e8m0 scale per 32 values, straight from the
+// gate/up epilogue.
+enum OutKind { OUT_BF16 = 0, OUT_F16 = 1, OUT_F32 = 2, OUT_MX8 = 3 };
 
 struct GemmProblem {
     // tokens: [M_alloc, K] bf16 (BF16 weights) or f16 (FP4 weights), row-major
@@ -142,6 +145,8 @@ struct GemmProblem {
     const float* bias1;
     const float* bias_rw;
     float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI (act == MOE_ACT_SWIGLUOAI)
+    // OUT_MX8: records of out_terms e4m3 terms (2: hi/lo, 1: MXFP8), out_stride bytes apart
+    int out_terms, out_stride;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
 int choose_token_tile(long long NvS, int G, bool wide_ok);
