@@ -1407,12 +1407,16 @@ __device__ __forceinline__ void build_sfb_block_mx8(const uint8_t* raw, uint8_t*
 // e8m0 scale per 32 values; the tensor cores apply both scales. Warp roles: 0 producer,
 // 1..NI MMA issuers, then 4 epilogue warps, then the scale warp (token scales into copy
 // blocks, scale-factor copies into the stage's TMEM slot).
-template <int BT, bool DUAL, bool TWO, int OUT>
-__global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
+// WIDE (single matrix): a tile is two consecutive 128-row weight blocks, handled like the
+// gate/up pair (two weight tiles per stage), so a stage of a decode tile streams as many
+// weight bytes per fixed per-stage cost as the pair does; the epilogue writes both blocks.
+template <int BT, bool DUAL, bool TWO, int OUT, bool WIDE = false>
+__global__ void __launch_bounds__(Mx8Cfg<BT, DUAL || WIDE, TWO>::THREADS, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_sf,
                             const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                             const GemmArgs a, int Kp) {
-    using C = Mx8Cfg<BT, DUAL, TWO>;
+    static_assert(!(DUAL && WIDE), "WIDE is a single-matrix mode");
+    using C = Mx8Cfg<BT, DUAL || WIDE, TWO>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
@@ -1471,7 +1475,13 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-                const size_t blk0 = ((size_t)g * NT + nt) * KB;
+                // 128-row weight blocks of this tile: nt (and nt for up), or 2nt and 2nt + 1.
+                // A second block past the last one is zero-filled by the tensor map; its
+                // scale copy repeats the last block's (times zero weights: no effect).
+                const int NT1 = WIDE ? (a.N + kTileN - 1) / kTileN : NT;
+                const int wb0 = WIDE ? 2 * nt : nt, wb1 = WIDE ? 2 * nt + 1 : nt;
+                const size_t blk0 = ((size_t)g * NT1 + wb0) * KB;
+                const size_t blk1 = ((size_t)g * NT1 + min(wb1, NT1 - 1)) * KB;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit)) {
                         ok = false;
@@ -1479,11 +1489,11 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&ctl->full[s],
                                           C::NB * (C::A_TX + 512) + (TWO ? 2 : 1) * C::B_BYTES + C::SFR_BYTES);
-                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g, pol_w);
+                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kMx8StageK, wb0 * kTileN, g, pol_w);
                     bulk_load_p(sfA(s, 0), a.ks0 + (blk0 + kb) * 512, 512, &ctl->full[s], pol_w);
-                    if (DUAL) {
-                        tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kMx8StageK, nt * kTileN, g, pol_w);
-                        bulk_load_p(sfA(s, 1), a.ks1 + (blk0 + kb) * 512, 512, &ctl->full[s], pol_w);
+                    if (DUAL || WIDE) {
+                        tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kMx8StageK, wb1 * kTileN, g, pol_w);
+                        bulk_load_p(sfA(s, 1), a.ks1 + (blk1 + kb) * 512, 512, &ctl->full[s], pol_w);
                     }
                     tma_load_2d_p(opB(s, 0), &tm_x, &ctl->full[s], kb * kMx8StageK, row0, pol_t);
                     if (TWO) tma_load_2d_p(opB(s, 1), &tm_x, &ctl->full[s], Kp + kb * kMx8StageK, row0, pol_t);
@@ -1610,9 +1620,14 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL, TWO>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT, C::NPART, true, C::EW>(
-                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane,
-                h);
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS);
+            if constexpr (WIDE) {  // block 2nt, then block 2nt + 1 (its partials NPART * BT columns on)
+                epilogue_tile<BT, false, OUT, C::NPART, true, C::EW>(a, tb, g, 2 * nt, row0, rows, q, lane, h);
+                epilogue_tile<BT, false, OUT, C::NPART, true, C::EW>(a, tb + C::NPART * BT, g, 2 * nt + 1, row0, rows,
+                                                                     q, lane, h);
+            } else {
+                epilogue_tile<BT, DUAL, OUT, C::NPART, true, C::EW>(a, tb, g, nt, row0, rows, q, lane, h);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[b]);
@@ -1883,16 +1898,28 @@ cudaError_t launch_nvf4(const GemmProblem& p, GemmArgs& a, cudaStream_t st, bool
     }
 }
 
-template <int BT, bool DUAL, bool TWO, int OUT>
-cudaError_t run_mx8(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& tsf,
+template <int BT, bool DUAL, bool TWO, int OUT, bool WIDE = false>
+cudaError_t run_mx8(const GemmProblem& p, GemmArgs args, const CUtensorMap& tx, const CUtensorMap& tsf,
                     const CUtensorMap& t0, const CUtensorMap& t1, int Kp, cudaStream_t st, bool pdl) {
-    using C = Mx8Cfg<BT, DUAL, TWO>;
-    auto kern = grouped_gemm_mx8_kernel<BT, DUAL, TWO, OUT>;
+    using C = Mx8Cfg<BT, DUAL || WIDE, TWO>;
+    auto kern = grouped_gemm_mx8_kernel<BT, DUAL, TWO, OUT, WIDE>;
     static int done[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
+    if (WIDE) {  // tiles of two 128-row blocks of the one matrix
+        args.NT = (p.N + 2 * kTileN - 1) / (2 * kTileN);
+        args.ks1 = args.ks0;
+    }
     return launch_k(kern, dim3(grid_for(p, args, BT)), dim3(C::THREADS), (size_t)C::SMEM_BYTES, st, pdl, tx, tsf, t0,
                     t1, args, Kp);
+}
+
+// The single-matrix MXFP4 GEMM streams two weight blocks per stage for decode-sized token
+// tiles (MOE_MX8_WIDE=0 keeps one).
+bool mx8_wide(int bt) {
+    const char* env = getenv("MOE_MX8_WIDE");
+    if (env && env[0] == '0' && env[1] == '\0') return false;
+    return bt <= 32;
 }
 
 template <int BT, bool TWO>
@@ -1903,6 +1930,13 @@ cudaError_t dispatch_mx8_terms(const GemmProblem& p, const GemmArgs& args, const
         if (p.out_kind == OUT_MX8) return run_mx8<BT, true, TWO, OUT_MX8>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
         if (p.out_kind != OUT_F32) return cudaErrorInvalidValue;
         return run_mx8<BT, true, TWO, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+    }
+    if constexpr (BT <= 32) {
+        if (mx8_wide(BT)) {
+            if (p.out_kind == OUT_F32) return run_mx8<BT, false, TWO, OUT_F32, true>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+            if (!TWO) return cudaErrorInvalidValue;
+            return run_mx8<BT, false, TWO, OUT_BF16, true>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
+        }
     }
     if (p.out_kind == OUT_F32) return run_mx8<BT, false, TWO, OUT_F32>(p, args, tx, tsf, t0, t1, Kp, st, pdl);
     if (!TWO) return cudaErrorInvalidValue;  // the standalone bf16-output GEMM stages hi/lo

@@ -239,6 +239,29 @@ def test_grouped_gemm_fp4(lib, fmt, seg, N, K):
         check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what=fmt)
 
 
+@pytest.mark.parametrize("bt", [16, 32])
+def test_grouped_gemm_mxfp4_wide_matches_narrow(lib, bt, monkeypatch):
+    # the single-matrix MXFP4 GEMM with two weight blocks per tile (the decode form): N = 384
+    # is three 128-row blocks, so the second wide tile is half past the end; against the
+    # staging bound and bit for bit against one block per tile
+    monkeypatch.setenv("MOE_TOKEN_TILE", str(bt))
+    seg, N, K = [3, 0, 20, 1, 37], 384, 256
+    ws = _fp4_weightset("mxfp4", len(seg), N, K, seed=bt + 1)
+    M = sum(seg) + 3
+    a, _, _ = W.gen_grouped_gemm_case(M, seg, 8, K, seed=bt)
+    cu = np.cumsum(seg).astype(np.int32)
+    w = lib.moe_prepare_weights(lib.Weight.from_host(ws))
+    outs = {}
+    for wide in ("1", "0"):
+        monkeypatch.setenv("MOE_MX8_WIDE", wide)
+        outs[wide] = lib.moe_grouped_gemm(to_dev(a), w, to_dev(torch.from_numpy(cu)))
+        torch.cuda.synchronize()
+    ref = O.grouped_gemm(O.to_f64(a), ws, cu, M_alloc=M)
+    r = check_mx8(outs["1"], ref, mx8_staging_bound(O.to_f64(a), ws, cu, M), what=f"wide bt{bt}")
+    assert r <= 4e-3, r
+    assert torch.equal(outs["1"], outs["0"])
+
+
 def _nvfp4_rows(a):
     """The oracle's NVFP4 quantisation of rows a (bf16 [M,K]): packed codes, e4m3 block
     scales, fp32 row scales, and the exact values they stand for."""
