@@ -233,10 +233,11 @@ def fp4_layer_bound(cfg, inp, ref, gamma=GAMMA, tail=TAIL):
     y_abs = np.zeros((len(perm_token), wd.N))
     biases = inp.extra.get("biases") if getattr(cfg, "bias", False) else None
     dq = [_Dequant(w) for w in (wg, wu, wd)]
-    for g, (s0, s1) in enumerate(O.segment_bounds(cu)):
+
+    def segment(g, s0, s1):
         rows = np.nonzero(need[s0:s1])[0] + s0
         if len(rows) == 0:
-            continue
+            return
         a1 = x_exp[perm_token[rows]].astype(np.float32)
         if cfg.wfmt == "mxfp4" and cfg.act_quant == 0:
             sd_a1 = r3 * _hilo_err(a1)
@@ -306,6 +307,12 @@ def fp4_layer_bound(cfg, inp, ref, gamma=GAMMA, tail=TAIL):
         if np.any(flips):
             fl_y[rows] = ad[g] * np.minimum(flips @ np.abs(Wd).T, tail * _sd(flips, Wd2))
         y_abs[rows] = np.abs(ref["y"][rows])
+
+    # segments write disjoint rows; numpy releases the GIL in the matmuls and large array ops
+    import concurrent.futures as cf
+    import os
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda t: segment(t[0], *t[1]), enumerate(O.segment_bounds(cu))))
     wt = np.ones((len(tok), k)) if in_fc1 else np.abs(np.asarray(ref["w"], np.float64)[tok])
     var = np.zeros((len(tok), wd.N))
     fl = np.zeros((len(tok), wd.N))
