@@ -554,12 +554,16 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases for profiling; not a bench line)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E, with no redundant slots (smaller cases for profiling; not a bench line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     cfg = W.CONFIGS[args.config]
     if args.tokens:
         cfg = cfg.with_(T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
+    if args.experts:
+        cfg = cfg.with_(E=args.experts, B=0, B_used=0, name=f"{cfg.name}_E{args.experts}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.gpus < 1:
