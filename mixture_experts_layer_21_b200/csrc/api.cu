@@ -559,9 +559,16 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
                        pdl());
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    // S2 gather (+ S2q)
+    // S2 gather (+ S2q). BF16 gate/up on CTA pairs can read the token rows of x by perm_token
+    // itself (MOE_FUSED_GATHER=1), which saves writing and re-reading x_perm.
+    GemmProblem probe{};
+    probe.wfmt = fmt;
+    probe.M_alloc = NvS;
+    probe.G = G;
+    const char* fg = getenv("MOE_FUSED_GATHER");
+    const bool fused_gather = fmt == MOE_W_BF16 && fg && fg[0] == '1' && fg[1] == '\0' && gemm_uses_pairs(probe);
     if (fmt == MOE_W_BF16) {
-        e = launch_gather(0, xin, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
+        e = fused_gather ? cudaSuccess : launch_gather(0, xin, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (fmt == MOE_W_MXFP4) {
         // stage each token once as e4m3 records (hi/lo, or MXFP8), then gather the records
         const int rb = mx8_rec_bytes(H, terms), Kp = mx8_kpad(H);
@@ -595,7 +602,9 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     trace.stage("gate_up");
     const bool situ = p->act.act == MOE_ACT_SITU;
     GemmProblem g1{};
-    g1.x = xperm;
+    g1.x = fused_gather ? xin : xperm;
+    g1.gather_idx = fused_gather ? perm_token : nullptr;
+    g1.gather_rows = T;
     g1.M_alloc = NvS;
     g1.cu_seqlens = cu;
     g1.G = G;

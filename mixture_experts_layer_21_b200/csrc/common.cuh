@@ -154,6 +154,15 @@ MOE_DEV void bulk_load_p(void* dst, const void* src, uint32_t bytes, uint64_t* b
         bulk_load(dst, src, bytes, bar);
 }
 
+// 16 bytes global -> shared through L2 (cp.async, LSU path); src_bytes < 16 zero-fills the rest.
+MOE_DEV void cp_async16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+// Arrive on an mbarrier (counted in its expected arrivals) once this thread's cp.asyncs land.
+MOE_DEV void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 // ---------------------------------------------------------------- tcgen05
 MOE_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -84,6 +84,10 @@ struct GemmArgs {
     const float* bias_rw;
     float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI
     int out_terms, out_stride, out_kpad;  // OUT_MX8 records: terms, row stride, codes per term
+    // fused gather (CTA pairs): token row r of the GEMM is row gather_idx[r] of gx [gather_rows, K]
+    const int32_t* gather_idx;
+    const __nv_bfloat16* gx;
+    int gather_rows;
 };
 
 struct CtrlBlock {
@@ -512,11 +516,16 @@ struct PairCfg {
 // MMA width of a pair tile: its rows rounded up to 32 (each CTA's half a multiple of 16).
 __device__ __forceinline__ int pair_mma_n(int rows, int bt) { return min(bt, (rows + 31) & ~31); }
 
-template <int BT, bool DUAL, int OUT>
+// GATHER: the token half of each stage is gathered from gx by gather_idx (the permutation's
+// perm_token) by the producer warp's 32 lanes with cp.async, in the 128-byte-swizzled layout
+// the MMA reads, instead of a TMA box of pre-gathered rows; stage s is full after lane 0's
+// weight copies and 32 cp.async arrivals.
+template <int BT, bool DUAL, int OUT, bool GATHER = false>
 __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                              const __grid_constant__ CUtensorMap tm_w1, const GemmArgs a) {
     using C = PairCfg<BT, DUAL>;
+    static_assert(!GATHER || C::B_ROWS == 128, "the gather maps 4 rows per lane");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
@@ -533,7 +542,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->full[s], GATHER ? 33 : 1);
             mbar_init(&ctl->empty[s], 1);
             mbar_init(&pfull[s], 1);
         }
@@ -564,7 +573,62 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
     const int total = ctl->tpre[G];
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- producer: this CTA's weight rows and token half
+        if (GATHER) {  // ---------------- producer warp: weights by TMA (lane 0), tokens gathered
+            const uint64_t pol_w = l2_policy(a.l2_w);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            const int K = a.K;
+            for (int L = pair; L < total && ok; L += npairs) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                const int trow = row0 + (int)rank * (pair_mma_n(rows, BT) / 2);
+                const int wrow = (2 * nt + (int)rank) * kTileN;
+                // this lane's rows of the half: lane + 32 i; rows past the GEMM's rows read a
+                // valid token (their products are discarded), ids outside [0, gather_rows) too
+                const __nv_bfloat16* src[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = min(trow + lane + 32 * i, a.M_alloc - 1);
+                    const int t = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
+                    src[i] = a.gx + (size_t)t * K;
+                }
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit))) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES);
+                        tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                        if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                    }
+                    const uint32_t bb = smem_u32(opB(s));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = lane + 32 * i;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int k = kb * kTileK + c * 8;
+                            // 16 bytes of row `row`, chunk c, at chunk position c ^ (row % 8)
+                            cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), k < K ? src[i] + k : a.gx,
+                                       k < K ? 16u : 0u);
+                        }
+                    }
+                    cp_async_arrive_noinc(&ctl->full[s]);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok && lane == 0) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+            }
+        } else if (lane == 0) {  // ---------------- producer: this CTA's weight rows and token half
             const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
@@ -617,6 +681,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if (GATHER) fence_proxy_async_smem();  // the gathered rows came by the generic proxy
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(opA(s, 0));
                     const uint32_t a1 = smem_u32(opA(s, DUAL ? 1 : 0));
@@ -656,6 +721,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if (GATHER) fence_proxy_async_smem();
                     mbar_arrive_cluster(mapa_shared(smem_u32(&pfull[s]), 0));
                     if (++s == C::STAGES) {
                         s = 0;
@@ -1809,11 +1875,11 @@ int max_pairs_once(Kern kern, int smem, int threads, int (&cache)[64]) {
     return cache[dev];
 }
 
-template <int BT, bool DUAL, int OUT>
+template <int BT, bool DUAL, int OUT, bool GATHER = false>
 cudaError_t run_pair(const GemmProblem& p, GemmArgs args, const CUtensorMap& tx, const CUtensorMap& t0,
                      const CUtensorMap& t1, cudaStream_t st, bool pdl) {
     using C = PairCfg<BT, DUAL>;
-    auto kern = grouped_gemm_pair_kernel<BT, DUAL, OUT>;
+    auto kern = grouped_gemm_pair_kernel<BT, DUAL, OUT, GATHER>;
     static int done[64] = {0};
     static int pairs_cache[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
@@ -2046,6 +2112,10 @@ bool use_pairs(const GemmProblem& p) {
     return p.M_alloc > 96 * segs;
 }
 
+// Whether launch_grouped_gemm runs this problem on CTA pairs (the caller may then let it
+// gather token rows itself).
+bool gemm_uses_pairs(const GemmProblem& p) { return p.wfmt == MOE_W_BF16 && use_pairs(p); }
+
 // L2 policies of the copies: MOE_L2_HINTS = 0 none, 1 token rows evict-last, 2 also the
 // weights evict-first (default 1). Token rows are re-read by every weight block of their
 // segment; weight tiles by the few token tiles of a segment, close together in time.
@@ -2118,11 +2188,20 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     if (p.wfmt == MOE_W_BF16 && use_pairs(p)) {
         CUtensorMap tx, t0, t1;
         memset(&t1, 0, sizeof(t1));
-        if (!make_map_2d(&tx, p.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.M_alloc, 128) ||
+        if (!make_map_2d(&tx, p.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.gather_idx ? p.gather_rows : p.M_alloc,
+                         128) ||
             !make_map_3d(&t0, p.w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G) ||
             (p.dual && !make_map_3d(&t1, p.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G)))
             return cudaErrorInvalidValue;
         if (!p.dual) t1 = t0;
+        if (p.gather_idx) {
+            // token rows straight from x: K % 8 == 0 keeps each 16-byte chunk inside a row
+            if (!p.dual || p.K % 8 || p.gather_rows < 1) return cudaErrorInvalidValue;
+            a.gather_idx = p.gather_idx;
+            a.gx = static_cast<const __nv_bfloat16*>(p.x);
+            a.gather_rows = p.gather_rows;
+            return run_pair<256, true, OUT_BF16, true>(p, a, tx, t0, t1, st, pdl);
+        }
         if (p.dual) return run_pair<256, true, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
         if (p.out_kind == OUT_F32) return run_pair<256, false, OUT_F32>(p, a, tx, t0, t1, st, pdl);
         return run_pair<256, false, OUT_BF16>(p, a, tx, t0, t1, st, pdl);

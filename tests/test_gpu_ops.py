@@ -176,11 +176,14 @@ def test_grouped_gemm_bf16_pairs_ragged(lib, monkeypatch):
     check_bf16(out, ref, atol=1e-5 * max(1.0, np.abs(ref).max()), rtol=2.0 ** -8, rel=4e-3, what="pairs")
 
 
-def test_forward_bf16_pairs_ragged(lib, monkeypatch):
+@pytest.mark.parametrize("fused_gather", ["0", "1"])
+def test_forward_bf16_pairs_ragged(lib, fused_gather, monkeypatch):
     # the fused layer with both GEMMs on CTA pairs: a given top-1 routing that gives the
     # experts 0, 1, 17, 33, 100, 255, 256, 257 and 300 tokens; I = 384 leaves the second pair
-    # block of the gate/up GEMM half empty, H = 208 is not a multiple of 64
+    # block of the gate/up GEMM half empty, H = 208 is not a multiple of 64. With the fused
+    # gather the gate/up GEMM reads the token rows of x by the permutation itself.
     monkeypatch.setenv("MOE_GEMM_PAIRS", "1")
+    monkeypatch.setenv("MOE_FUSED_GATHER", fused_gather)
     lens = [0, 1, 17, 33, 100, 255, 256, 257, 300]
     cfg = W.MoEConfig("pairs", T=sum(lens), H=208, I=384, E=len(lens), topk=1)
     inp = W.gen_inputs(cfg)

@@ -28,8 +28,10 @@ CASES = {
     "nvfp4": W.MoEConfig("t_nvfp4", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4", act_quant=1),
     "mxfp4": W.MoEConfig("t_mxfp4", T=40, H=256, I=320, E=8, topk=4, act="situ", wfmt="mxfp4"),
     "nvfp4_a16": W.MoEConfig("t_nvfp4_a16", T=50, H=512, I=256, E=16, topk=8, wfmt="nvfp4"),
-    # BF16 on CTA pairs (segments of about 150 rows)
+    # BF16 on CTA pairs (segments of about 150 rows), with the token rows pre-gathered or
+    # gathered by the GEMM's producer warp
     "bf16_pairs": W.MoEConfig("t_bf16_pairs", T=600, H=256, I=256, E=8, topk=2),
+    "bf16_pairs_gather": W.MoEConfig("t_bf16_pairs_gather", T=600, H=256, I=256, E=8, topk=2),
 }
 
 
@@ -42,7 +44,8 @@ def test_wait_timeout_is_reported_and_the_next_call_is_correct(lib, name, monkey
                            situ_alpha=cfg.situ_alpha, situ_beta=cfg.situ_beta, act_quant=cfg.act_quant,
                            T_max=cfg.T)
     x, logits = to_dev(inp.x), to_dev(inp.logits)
-    monkeypatch.setenv("MOE_GEMM_PAIRS", "1" if name == "bf16_pairs" else "0")
+    monkeypatch.setenv("MOE_GEMM_PAIRS", "1" if name.startswith("bf16_pairs") else "0")
+    monkeypatch.setenv("MOE_FUSED_GATHER", "1" if name == "bf16_pairs_gather" else "0")
     monkeypatch.setenv("MOE_WAIT_LIMIT_CYCLES", "1")
     layer(x, logits)
     torch.cuda.synchronize()                       # the kernels returned
