@@ -2100,14 +2100,14 @@ long long wait_limit_cycles() {
     return kWaitLimitCycles;
 }
 
-// The BF16 GEMM runs on CTA pairs when segments average more than 96 rows (a pair tile is
-// up to 256 tokens wide) and no token tile was forced. MOE_GEMM_PAIRS=0 turns this off, =1
-// forces it for any segment size.
+// The BF16 GEMM runs on CTA pairs on request: MOE_GEMM_PAIRS=1 for any segment size, =2 when
+// segments average more than 96 rows (a pair tile is up to 256 tokens wide) and no token tile
+// was forced. Off by default: the one-SM kernel measured faster on B200.
 bool use_pairs(const GemmProblem& p) {
     const char* env = getenv("MOE_GEMM_PAIRS");
-    if (env && env[0] == '0' && env[1] == '\0') return false;
-    if (env && env[0] == '1' && env[1] == '\0') return true;
-    if (p.bt || getenv("MOE_TOKEN_TILE")) return false;
+    if (!env || env[1] != '\0') return false;
+    if (env[0] == '1') return true;
+    if (env[0] != '2' || p.bt || getenv("MOE_TOKEN_TILE")) return false;
     const long long segs = std::max<long long>(1, std::min<long long>(p.G, p.M_alloc));
     return p.M_alloc > 96 * segs;
 }
