@@ -520,12 +520,17 @@ __device__ __forceinline__ int pair_mma_n(int rows, int bt) { return min(bt, (ro
 // perm_token) by the producer warp's 32 lanes with cp.async, in the 128-byte-swizzled layout
 // the MMA reads, instead of a TMA box of pre-gathered rows; stage s is full after lane 0's
 // weight copies and 32 cp.async arrivals.
-template <int BT, bool DUAL, int OUT, bool GATHER = false>
+// FWD = false (without GATHER): both CTAs' copies of stage s complete on the leader's full[s]
+// (cta_group::2 TMA loads), whose expected bytes the leader's producer sets for both, so the
+// MMA waits on one local barrier and no stage takes a forwarding hop. The peer cannot watch
+// its own copies then; after an abort it lets them settle (a bounded pause) before exiting.
+template <int BT, bool DUAL, int OUT, bool GATHER = false, bool FWD = true>
 __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w0,
                              const __grid_constant__ CUtensorMap tm_w1, const GemmArgs a) {
     using C = PairCfg<BT, DUAL>;
     static_assert(!GATHER || C::B_ROWS == 128, "the gather maps 4 rows per lane");
+    static_assert(FWD || !GATHER, "the gather completes on each CTA's own barriers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     CtrlBlock* ctl = reinterpret_cast<CtrlBlock*>(smem + C::STAGES * C::STAGE);
@@ -643,10 +648,18 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
-                    tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
-                    if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
-                    tma_load_2d_p(opB(s), &tm_x, &ctl->full[s], kb * kTileK, trow, pol_t);
+                    if (FWD) {
+                        mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES + C::B_BYTES);
+                        tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                        if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
+                        tma_load_2d_p(opB(s), &tm_x, &ctl->full[s], kb * kTileK, trow, pol_t);
+                    } else {
+                        const uint32_t bar = mapa_shared(smem_u32(&ctl->full[s]), 0);  // the leader's
+                        if (leader) mbar_arrive_expect_tx(&ctl->full[s], 2 * (C::NB * C::A_BYTES + C::B_BYTES));
+                        tma_load_3d_pair(opA(s, 0), &tm_w0, bar, kb * kTileK, wrow, g);
+                        if (DUAL) tma_load_3d_pair(opA(s, 1), &tm_w1, bar, kb * kTileK, wrow, g);
+                        tma_load_2d_pair(opB(s), &tm_x, bar, kb * kTileK, trow);
+                    }
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
                     if (++s == C::STAGES) {
@@ -676,8 +689,8 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(b * C::ACC_COLS);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ctl->full[s], ph, abort_flag, a.wait_limit) ||
-                        !mbar_wait_cluster(&pfull[s], ph, abort_flag, a.wait_limit)) {
+                    if (!mbar_wait_cluster(&ctl->full[s], ph, abort_flag, a.wait_limit) ||
+                        (FWD && !mbar_wait_cluster(&pfull[s], ph, abort_flag, a.wait_limit))) {
                         ok = false;
                         break;
                     }
@@ -711,7 +724,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                 report_error(a.err, MOE_ERR_TIMEOUT, 2);
                 ctl->abort = 1;
             }
-        } else if (lane == 0) {  // ---------------- peer: tells the leader each stage landed
+        } else if (FWD && lane == 0) {  // ---------------- peer: tells the leader each stage landed
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -769,8 +782,17 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
     __syncthreads();
     {
         int never = 0;
-        for (int q = 0; q < C::STAGES; ++q)
-            if (is.mask >> q & 1u) mbar_wait(&ctl->full[q], is.par >> q & 1u, &never);
+        // FWD = false: only the leader's full barriers track copies (both CTAs'); the peer's
+        // copies of a stage the leader never armed are not tracked: after an abort the peer
+        // waits about 100 microseconds, far longer than a copy takes, before it can exit
+        if (FWD || leader) {
+            for (int q = 0; q < C::STAGES; ++q)
+                if (is.mask >> q & 1u) mbar_wait(&ctl->full[q], is.par >> q & 1u, &never);
+        } else if (is.mask && *abort_flag) {
+            const long long t0 = clock64();
+            while (clock64() - t0 < 200000) {
+            }
+        }
         if (is.tc) {
             mma_commit_pair(&ctl->drain[0], 0x1);
             mbar_wait(&ctl->drain[0], 0, &never);
@@ -1875,11 +1897,11 @@ int max_pairs_once(Kern kern, int smem, int threads, int (&cache)[64]) {
     return cache[dev];
 }
 
-template <int BT, bool DUAL, int OUT, bool GATHER = false>
+template <int BT, bool DUAL, int OUT, bool GATHER = false, bool FWD = true>
 cudaError_t run_pair(const GemmProblem& p, GemmArgs args, const CUtensorMap& tx, const CUtensorMap& t0,
                      const CUtensorMap& t1, cudaStream_t st, bool pdl) {
     using C = PairCfg<BT, DUAL>;
-    auto kern = grouped_gemm_pair_kernel<BT, DUAL, OUT, GATHER>;
+    auto kern = grouped_gemm_pair_kernel<BT, DUAL, OUT, GATHER, FWD>;
     static int done[64] = {0};
     static int pairs_cache[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
@@ -2200,11 +2222,18 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
             a.gather_idx = p.gather_idx;
             a.gx = static_cast<const __nv_bfloat16*>(p.x);
             a.gather_rows = p.gather_rows;
-            return run_pair<256, true, OUT_BF16, true>(p, a, tx, t0, t1, st, pdl);
+            return run_pair<256, true, OUT_BF16, true, true>(p, a, tx, t0, t1, st, pdl);
         }
-        if (p.dual) return run_pair<256, true, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
-        if (p.out_kind == OUT_F32) return run_pair<256, false, OUT_F32>(p, a, tx, t0, t1, st, pdl);
-        return run_pair<256, false, OUT_BF16>(p, a, tx, t0, t1, st, pdl);
+        // MOE_PAIR_FWD=1: the peer forwards each stage instead of completing the leader's barrier
+        const char* fwd = getenv("MOE_PAIR_FWD");
+        if (fwd && fwd[0] == '1' && fwd[1] == '\0') {
+            if (p.dual) return run_pair<256, true, OUT_BF16, false, true>(p, a, tx, t0, t1, st, pdl);
+            if (p.out_kind == OUT_F32) return run_pair<256, false, OUT_F32, false, true>(p, a, tx, t0, t1, st, pdl);
+            return run_pair<256, false, OUT_BF16, false, true>(p, a, tx, t0, t1, st, pdl);
+        }
+        if (p.dual) return run_pair<256, true, OUT_BF16, false, false>(p, a, tx, t0, t1, st, pdl);
+        if (p.out_kind == OUT_F32) return run_pair<256, false, OUT_F32, false, false>(p, a, tx, t0, t1, st, pdl);
+        return run_pair<256, false, OUT_BF16, false, false>(p, a, tx, t0, t1, st, pdl);
     }
     const CUtensorMapDataType xdt =
         p.wfmt == MOE_W_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;

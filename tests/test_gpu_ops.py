@@ -159,11 +159,14 @@ def test_grouped_gemm_bf16_256_token_tile(lib, monkeypatch):
     check_bf16(out, ref, atol=1e-4 * np.abs(ref).max(), rtol=2.0 ** -8, rel=4e-3, what="bt256")
 
 
-def test_grouped_gemm_bf16_pairs_ragged(lib, monkeypatch):
+@pytest.mark.parametrize("fwd", ["0", "1"])
+def test_grouped_gemm_bf16_pairs_ragged(lib, fwd, monkeypatch):
     # the CTA-pair kernel on segments of every awkward length (1, one under and over a tile of
     # 256, several tiles, empty), N not a multiple of the 256-row pair block, K not of 64,
-    # padding rows after the last segment
+    # padding rows after the last segment; both ways of completing a stage (on the leader's
+    # barrier, or forwarded by the peer)
     monkeypatch.setenv("MOE_GEMM_PAIRS", "1")
+    monkeypatch.setenv("MOE_PAIR_FWD", fwd)
     seg = [1, 17, 0, 33, 100, 255, 256, 257, 600, 31]
     M, N, K = sum(seg) + 5, 200, 136
     a, wt, _ = W.gen_grouped_gemm_case(M, seg, N, K, seed=77)
