@@ -559,14 +559,16 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
                        pdl());
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    // S2 gather (+ S2q). BF16 gate/up on CTA pairs can read the token rows of x by perm_token
-    // itself (MOE_FUSED_GATHER=1), which saves writing and re-reading x_perm.
+    // S2 gather (+ S2q). The BF16 gate/up GEMM with 128-token tiles (or on CTA pairs) can read
+    // the token rows of x by perm_token itself (MOE_FUSED_GATHER=1), which saves writing and
+    // re-reading x_perm.
     GemmProblem probe{};
     probe.wfmt = fmt;
+    probe.dual = true;
     probe.M_alloc = NvS;
     probe.G = G;
     const char* fg = getenv("MOE_FUSED_GATHER");
-    const bool fused_gather = fmt == MOE_W_BF16 && fg && fg[0] == '1' && fg[1] == '\0' && gemm_uses_pairs(probe);
+    const bool fused_gather = fmt == MOE_W_BF16 && fg && fg[0] == '1' && fg[1] == '\0' && gemm_can_gather(probe);
     if (fmt == MOE_W_BF16) {
         e = fused_gather ? cudaSuccess : launch_gather(0, xin, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (fmt == MOE_W_MXFP4) {

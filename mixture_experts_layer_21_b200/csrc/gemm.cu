@@ -307,12 +307,17 @@ struct Bf16Cfg {
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
 };
 
-template <int BT, bool DUAL, int OUT>
+// GATHER (the 128-token gate/up tile): the token tile of each stage is gathered from gx by
+// gather_idx (the permutation's perm_token) by the producer warp's 32 lanes with cp.async, in
+// the 128-byte-swizzled layout the MMA reads; stage s is full after lane 0's weight copies and
+// 32 cp.async arrivals.
+template <int BT, bool DUAL, int OUT, bool GATHER = false>
 __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_w0,
                         const __grid_constant__ CUtensorMap tm_w1, const GemmArgs a) {
     using C = Bf16Cfg<BT, DUAL>;
+    static_assert(!GATHER || BT == 128, "the gather maps 4 rows per lane");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment by offsetting the shared array itself (no integer round trip),
     // so that every access below stays a shared-memory access
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->full[s], GATHER ? 33 : 1);
             mbar_init(&ctl->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -357,7 +362,60 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
     const int total = ctl->tpre[G];
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- TMA producer
+        if (GATHER) {  // ---------------- producer warp: weights by TMA (lane 0), tokens gathered
+            const uint64_t pol_w = l2_policy(a.l2_w);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            const int K = a.K;
+            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
+                int g, nt, row0, rows;
+                decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
+                // this lane's tile rows lane + 32 i; rows past the GEMM's rows read a valid token
+                // (their products are discarded), ids outside [0, gather_rows) too
+                const __nv_bfloat16* src[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = min(row0 + lane + 32 * i, a.M_alloc - 1);
+                    const int t = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
+                    src[i] = a.gx + (size_t)t * K;
+                }
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit))) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&ctl->full[s], C::NB * C::A_BYTES);
+                        tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
+                        if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
+                    }
+                    const uint32_t bb = smem_u32(opB(s));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = lane + 32 * i;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int k = kb * kTileK + c * 8;
+                            // 16 bytes of row `row`, chunk c, at chunk position c ^ (row % 8)
+                            cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), k < K ? src[i] + k : a.gx,
+                                       k < K ? 16u : 0u);
+                        }
+                    }
+                    cp_async_arrive_noinc(&ctl->full[s]);
+                    is.mask |= 1u << s;
+                    is.par = (is.par & ~(1u << s)) | (ph << s);
+                    if (++s == C::STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok && lane == 0) {
+                report_error(a.err, MOE_ERR_TIMEOUT, 1);
+                ctl->abort = 1;
+            }
+        } else if (lane == 0) {  // ---------------- TMA producer
             const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
@@ -409,6 +467,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if (GATHER) fence_proxy_async_smem();  // the gathered rows came by the generic proxy
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(opA(s, 0));
                     const uint32_t a1 = smem_u32(opA(s, DUAL ? 1 : 0));
@@ -1861,11 +1920,11 @@ int grid_for(const GemmProblem& p, const GemmArgs& args, int bt) {
     return (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles_ub));
 }
 
-template <int BT, bool DUAL, int OUT>
+template <int BT, bool DUAL, int OUT, bool GATHER = false>
 cudaError_t run_bf16(const GemmProblem& p, const GemmArgs& args, const CUtensorMap& tx, const CUtensorMap& t0,
                      const CUtensorMap& t1, cudaStream_t st, bool pdl) {
     using C = Bf16Cfg<BT, DUAL>;
-    auto kern = grouped_gemm_kernel<BT, DUAL, OUT>;
+    auto kern = grouped_gemm_kernel<BT, DUAL, OUT, GATHER>;
     static int done[64] = {0};
     cudaError_t e = set_smem_once(kern, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
@@ -2134,9 +2193,16 @@ bool use_pairs(const GemmProblem& p) {
     return p.M_alloc > 96 * segs;
 }
 
-// Whether launch_grouped_gemm runs this problem on CTA pairs (the caller may then let it
-// gather token rows itself).
-bool gemm_uses_pairs(const GemmProblem& p) { return p.wfmt == MOE_W_BF16 && use_pairs(p); }
+// Whether launch_grouped_gemm can gather this problem's token rows itself (BF16 gate/up with
+// 128-token tiles on one SM, or on CTA pairs).
+bool gemm_can_gather(const GemmProblem& p) {
+    if (p.wfmt != MOE_W_BF16 || !p.dual) return false;
+    if (use_pairs(p)) return true;
+    const char* env = getenv("MOE_TOKEN_TILE");
+    const int v = env ? atoi(env) : 0;
+    const int bt = p.bt ? p.bt : (v ? v : choose_token_tile(p.M_alloc, p.G, false));
+    return bt == 128;
+}
 
 // L2 policies of the copies: MOE_L2_HINTS = 0 none, 1 token rows evict-last, 2 also the
 // weights evict-first (default 1). Token rows are re-read by every weight block of their
@@ -2207,6 +2273,19 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl)
     if (bt == 256 && !wide_req) bt = 128;
     // BF16 prefill shapes run on CTA pairs: 256 weight rows x up to 256 tokens per pair tile
     // (MOE_GEMM_PAIRS=0 keeps the one-SM kernel, e.g. to compare the two)
+    if (p.wfmt == MOE_W_BF16 && p.gather_idx && !use_pairs(p)) {
+        // the 128-token gate/up tile gathering its own token rows from x
+        if (!p.dual || p.K % 8 || p.gather_rows < 1) return cudaErrorInvalidValue;
+        CUtensorMap tx, t0, t1;
+        if (!make_map_2d(&tx, p.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.gather_rows, 128) ||
+            !make_map_3d(&t0, p.w0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G) ||
+            !make_map_3d(&t1, p.w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.K, p.N, p.G))
+            return cudaErrorInvalidValue;
+        a.gather_idx = p.gather_idx;
+        a.gx = static_cast<const __nv_bfloat16*>(p.x);
+        a.gather_rows = p.gather_rows;
+        return run_bf16<128, true, OUT_BF16, true>(p, a, tx, t0, t1, st, pdl);
+    }
     if (p.wfmt == MOE_W_BF16 && use_pairs(p)) {
         CUtensorMap tx, t0, t1;
         memset(&t1, 0, sizeof(t1));

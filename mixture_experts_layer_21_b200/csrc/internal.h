@@ -147,13 +147,13 @@ struct GemmProblem {
     float sw_alpha, sw_beta, sw_limit;  // SWIGLUOAI (act == MOE_ACT_SWIGLUOAI)
     // OUT_MX8: records of out_terms e4m3 terms (2: hi/lo, 1: MXFP8), out_stride bytes apart
     int out_terms, out_stride;
-    // BF16 gate/up on CTA pairs only: token row r is row gather_idx[r] of x [gather_rows, K]
-    // (the permutation's perm_token), so no pre-gathered copy is needed
+    // BF16 gate/up (128-token tiles, or CTA pairs): token row r is row gather_idx[r] of
+    // x [gather_rows, K] (the permutation's perm_token), so no pre-gathered copy is needed
     const int32_t* gather_idx;
     int gather_rows;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t st, bool pdl);
-bool gemm_uses_pairs(const GemmProblem& p);
+bool gemm_can_gather(const GemmProblem& p);
 int choose_token_tile(long long NvS, int G, bool wide_ok);
 
 // FP4 kernel layout: tiles of 128 weight rows x 64 K values.

@@ -203,6 +203,21 @@ def test_forward_bf16_pairs_ragged(lib, fused_gather, monkeypatch):
     check_bf16(out, ref["out"], what="pairs forward")
 
 
+def test_forward_bf16_fused_gather_one_sm(lib, monkeypatch):
+    # the one-SM gate/up GEMM with 128-token tiles reading its token rows of x by the
+    # permutation (segments of about 150 rows, H = 208 not a multiple of 64): the oracle's
+    # output, and the same bits as the pre-gathered form
+    cfg = W.MoEConfig("gather1", T=600, H=208, I=256, E=8, topk=2, B=3, B_used=2)
+    inp = W.gen_inputs(cfg)
+    outs = {}
+    for fg in ("1", "0"):
+        monkeypatch.setenv("MOE_FUSED_GATHER", fg)
+        outs[fg], _, _, _ = run_layer(lib, cfg, inp)
+    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up, inp.w_down)
+    check_bf16(outs["1"], ref["out"], what="fused gather")
+    assert torch.equal(outs["1"], outs["0"])
+
+
 def test_grouped_gemm_bf16_matches_torch_grouped_mm(lib):
     if not hasattr(torch, "_grouped_mm"):
         pytest.skip("torch._grouped_mm unavailable")
