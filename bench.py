@@ -313,13 +313,15 @@ def default_sample(cfg) -> int:
 # ---------------------------------------------------------------------------- arms
 
 def kernel_launches(cfg) -> int:
-    n = 1 + 3 + 1 + 1 + 1 + 1            # route, permute x3, gather, fc1, fc2, combine
-    if cfg.wfmt == "mxfp4":
-        n += 1                            # x staging (the gate/up epilogue stages the activations)
-    elif cfg.act_quant:
-        n += 2                            # x quantisation, activation quantisation
-    elif cfg.wfmt != "bf16" and cfg.act != "situ":
-        n += 1                            # activation row pass to f16
+    n = 1 + 3 + 1 + 1 + 1                 # route, permute x3, gate/up GEMM, down GEMM, combine
+    # the gate/up operand in segment order: a gather (BF16; NVFP4 weights with bf16
+    # activations, as f16) or one staging / quantisation pass over the gathered rows (MXFP4;
+    # NVFP4 activations when H % 256 == 0, else quantisation then a gather)
+    n += 2 if (cfg.wfmt == "nvfp4" and cfg.act_quant == 1 and cfg.H % 256) else 1
+    # the down operand: a row pass for NVFP4 weights (NVFP4 quantisation, or f16 staging
+    # unless SITU bounds h); the MXFP4 gate/up epilogue writes its records itself
+    if cfg.wfmt == "nvfp4" and (cfg.act_quant == 1 or cfg.act != "situ"):
+        n += 1
     return n
 
 

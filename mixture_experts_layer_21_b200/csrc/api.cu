@@ -140,9 +140,9 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.tscale = take(fp4 ? 4 * NvS : 0);
     L.xq_codes = take(q1 ? (size_t)T_max * H / 2 : 0);
     L.xq_sb = take(q1 ? (size_t)T_max * H / 16 : 0);
-    L.xq_s = take(act_quant == 1 ? 4 * (size_t)T_max : 0);
+    L.xq_s = take(q1 ? 4 * (size_t)T_max : 0);
     L.xq_deq = take(q1 ? 2 * (size_t)T_max * H : 0);
-    L.xq_rec = take(nat1 ? (size_t)T_max * nvf4_rec_bytes(H) : 0);
+    L.xq_rec = 0;
     L.xperm_rec = take(nat1 ? NvS * nvf4_rec_bytes(H) : 0);
     const bool mx = wfmt == MOE_W_MXFP4;
     // h: bf16 (BF16 weights), fp32 when a row pass follows (NVFP4 weights); the MXFP4 gate/up
@@ -154,7 +154,7 @@ FwdWs fwd_layout(int T_max, int H, int I, int E, int B, int topk, int wfmt, int 
     L.act_sb = take(q2 ? NvS * I / 16 : 0);
     L.act_rec = take(nat2 ? NvS * nvf4_rec_bytes(I) : 0);
     const int terms = mx8_terms(act_quant);
-    L.mx_xq = take(mx ? (size_t)T_max * mx8_rec_bytes(H, terms) : 0);
+    L.mx_xq = 0;
     L.mx_xperm = take(mx ? NvS * mx8_rec_bytes(H, terms) : 0);
     L.mx_act = take(mx ? NvS * mx8_rec_bytes(I, terms) : 0);
     L.x_in = take(topk == 1 ? 2 * (size_t)T_max * H : 0);  // x times the top-1 weight (input-side weighting)
@@ -572,22 +572,18 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     if (fmt == MOE_W_BF16) {
         e = fused_gather ? cudaSuccess : launch_gather(0, xin, H, perm_token, NvS, xperm, nullptr, nullptr, st, pdl());
     } else if (fmt == MOE_W_MXFP4) {
-        // stage each token once as e4m3 records (hi/lo, or MXFP8), then gather the records
+        // stage the gathered rows as e4m3 records (hi/lo, or MXFP8) in segment order, one pass
         const int rb = mx8_rec_bytes(H, terms), Kp = mx8_kpad(H);
-        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_xq);
-        e = launch_quant_mx8(xin, false, T, H, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr, rec + terms * Kp,
-                             rb, rb, st, pdl());
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        e = launch_gather(0, w + L.mx_xq, rb / 2, perm_token, NvS, w + L.mx_xperm, nullptr, nullptr, st, pdl());
+        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.mx_xperm);
+        e = launch_quant_mx8(xin, false, NvS, H, Kp, terms == 2, rec, terms == 2 ? rec + Kp : nullptr,
+                             rec + terms * Kp, rb, rb, st, pdl(), perm_token, T);
     } else if (nat1) {
-        // quantise each token once into records, then gather the records into segment order
-        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.xq_rec);
+        // quantise the gathered rows into records in segment order, one pass (a row's codes
+        // depend on that row alone, so a token quantised twice gives the same bits)
+        uint8_t* rec = reinterpret_cast<uint8_t*>(w + L.xperm_rec);
         const int rb = nvf4_rec_bytes(H);
-        e = launch_quant_nvfp4(xin, false, T, H, rec, rb, rec + H / 2, rb, reinterpret_cast<float*>(w + L.xq_s),
-                               nullptr, st, pdl());
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-        e = launch_gather(1, rec, rb / 2, perm_token, NvS, w + L.xperm_rec, reinterpret_cast<float*>(w + L.xq_s),
-                          tscale, st, pdl());
+        e = launch_quant_nvfp4(xin, false, NvS, H, rec, rb, rec + H / 2, rb, tscale, nullptr, st, pdl(), perm_token,
+                               T);
     } else if (p->act_quant) {
         e = launch_quant_nvfp4(xin, false, T, H, reinterpret_cast<uint8_t*>(w + L.xq_codes), H / 2,
                                reinterpret_cast<uint8_t*>(w + L.xq_sb), H / 16, reinterpret_cast<float*>(w + L.xq_s),

@@ -202,16 +202,19 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
                                                           uint8_t* __restrict__ codes, int cstride,
                                                           uint8_t* __restrict__ sbo, int sstride,
                                                           float* __restrict__ so,
-                                                          __half* __restrict__ deq) {
+                                                          __half* __restrict__ deq,
+                                                          const int32_t* __restrict__ row_idx, int in_rows) {
     pdl_wait();
     const int r = blockIdx.x * 8 + warp_id();
     const int lane = lane_id();
     if (r < R) {
         const int nb = K / 16;
+        // output row r quantises input row r, or row_idx[r] (clamped into the input)
+        const size_t ri = row_idx ? (size_t)min(max(row_idx[r], 0), in_rows - 1) : (size_t)r;
         float amax = 0.0f;
         for (int b = lane; b < nb; b += 32) {
             float v[16];
-            load16<IN_F32>(in, (size_t)r * K + b * 16, v);
+            load16<IN_F32>(in, ri * K + b * 16, v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
         }
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const void* __restrict
         const float six_s = __fmul_rn(6.0f, s);
         for (int b = lane; b < nb; b += 32) {
             float v[16];
-            load16<IN_F32>(in, (size_t)r * K + b * 16, v);
+            load16<IN_F32>(in, ri * K + b * 16, v);
             float bmax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
@@ -275,18 +278,21 @@ template <bool IN_F32, bool TWO>
 __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__ in, int R, int K, int Kp,
                                                         uint8_t* __restrict__ hi_out, uint8_t* __restrict__ lo_out,
                                                         uint8_t* __restrict__ sc_out, int code_stride,
-                                                        int sc_stride) {
+                                                        int sc_stride, const int32_t* __restrict__ row_idx,
+                                                        int in_rows) {
     pdl_wait();
     const int r = blockIdx.x * 8 + warp_id();
     const int lane = lane_id();
     if (r < R) {
+        // output row r stages input row r, or row_idx[r] (clamped into the input)
+        const size_t ri = row_idx ? (size_t)min(max(row_idx[r], 0), in_rows - 1) : (size_t)r;
         for (int b = lane; b < Kp / 32; b += 32) {
             uint32_t hi[8] = {0, 0, 0, 0, 0, 0, 0, 0}, lo[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             int e = -127;
             if (b * 32 < K) {
                 float v[2][16];
-                load16<IN_F32>(in, (size_t)r * K + b * 32, v[0]);
-                load16<IN_F32>(in, (size_t)r * K + b * 32 + 16, v[1]);
+                load16<IN_F32>(in, ri * K + b * 32, v[0]);
+                load16<IN_F32>(in, ri * K + b * 32 + 16, v[1]);
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i >> 4][i & 15]));
@@ -315,32 +321,34 @@ __global__ void __launch_bounds__(256) quant_mx8_kernel(const void* __restrict__
 }
 
 cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, int Kp, bool two, uint8_t* hi, uint8_t* lo,
-                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl) {
+                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl,
+                             const int32_t* row_idx, int in_rows) {
     if (R <= 0) return cudaSuccess;
     dim3 grid((R + 7) / 8), block(256);
     if (two) {
         if (in_f32)
             return launch_k(quant_mx8_kernel<true, true>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
-                            code_stride, sc_stride);
+                            code_stride, sc_stride, row_idx, in_rows);
         return launch_k(quant_mx8_kernel<false, true>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
-                        code_stride, sc_stride);
+                        code_stride, sc_stride, row_idx, in_rows);
     }
     if (in_f32)
         return launch_k(quant_mx8_kernel<true, false>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc,
-                        code_stride, sc_stride);
+                        code_stride, sc_stride, row_idx, in_rows);
     return launch_k(quant_mx8_kernel<false, false>, grid, block, 0, st, pdl, in, R, K, Kp, hi, lo, sc, code_stride,
-                    sc_stride);
+                    sc_stride, row_idx, in_rows);
 }
 
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
-                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl) {
+                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl,
+                               const int32_t* row_idx, int in_rows) {
     if (R <= 0) return cudaSuccess;
     dim3 grid((R + 7) / 8), block(256);
     if (in_f32)
         return launch_k(quant_nvfp4_kernel<true>, grid, block, 0, st, pdl, in, R, K, codes, codes_stride, sb,
-                        sb_stride, s, deq);
+                        sb_stride, s, deq, row_idx, in_rows);
     return launch_k(quant_nvfp4_kernel<false>, grid, block, 0, st, pdl, in, R, K, codes, codes_stride, sb, sb_stride,
-                    s, deq);
+                    s, deq, row_idx, in_rows);
 }
 
 }  // namespace moe

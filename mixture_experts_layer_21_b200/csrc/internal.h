@@ -86,11 +86,16 @@ cudaError_t launch_combine_f32(const float* y, const int32_t* inv_perm, const fl
 // Kp = mx8_kpad(K) codes per row (zero past K). two: hi and lo terms, scale chosen so the
 // block max stays <= 448 (lo != nullptr); else one term with the OCP MX MXFP8 scale.
 // Codes rows are code_stride bytes apart, scale rows sc_stride.
+// With row_idx, output row r is taken from input row row_idx[r] (of in_rows): the staging of
+// gathered rows in one pass.
 cudaError_t launch_quant_mx8(const void* in, bool in_f32, int R, int K, int Kp, bool two, uint8_t* hi, uint8_t* lo,
-                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl);
-// codes / sb rows are codes_stride / sb_stride bytes apart (K/2 and K/16 when dense).
+                             uint8_t* sc, int code_stride, int sc_stride, cudaStream_t st, bool pdl,
+                             const int32_t* row_idx = nullptr, int in_rows = 0);
+// codes / sb rows are codes_stride / sb_stride bytes apart (K/2 and K/16 when dense); row_idx
+// as for launch_quant_mx8.
 cudaError_t launch_quant_nvfp4(const void* in, bool in_f32, int R, int K, uint8_t* codes, int codes_stride,
-                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl);
+                               uint8_t* sb, int sb_stride, float* s, __half* deq, cudaStream_t st, bool pdl,
+                               const int32_t* row_idx = nullptr, int in_rows = 0);
 
 // ---------------------------------------------------------------- grouped GEMM
 // Output kinds of the GEMM epilogue.
