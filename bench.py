@@ -313,7 +313,9 @@ def default_sample(cfg) -> int:
 # ---------------------------------------------------------------------------- arms
 
 def kernel_launches(cfg) -> int:
-    n = 1 + 3 + 1 + 1 + 1                 # route, permute x3, gate/up GEMM, down GEMM, combine
+    # route, the permutation (one kernel for at most 256 tokens, else count, scan, scatter),
+    # gate/up GEMM, down GEMM, combine
+    n = 1 + (1 if cfg.T <= 256 else 3) + 1 + 1 + 1
     # the gate/up operand in segment order: a gather (BF16; NVFP4 weights with bf16
     # activations, as f16) or one staging / quantisation pass over the gathered rows (MXFP4;
     # NVFP4 activations when H % 256 == 0, else quantisation then a gather)

@@ -258,7 +258,7 @@ __device__ void build_masks(uint32_t* masks, const int32_t* __restrict__ ids, in
     for (int i = threadIdx.x; i < E * (kPermBlock / 32); i += blockDim.x) masks[i] = 0u;
     __syncthreads();
     const int t = t0 + threadIdx.x;
-    if (t < T) {
+    if (threadIdx.x < kPermBlock && t < T) {
         for (int j = 0; j < topk; ++j) {
             const int e = ids[(size_t)t * topk + j];
             if (e < 0 || e >= E) {
@@ -295,17 +295,17 @@ __global__ void __launch_bounds__(kPermBlock) permute_count_kernel(const int32_t
 // segment end up to NvS receive no assignment unless an id was bad (out of range, or an
 // expert listed twice by one token; both reported): they get token 0 and weight 0, so that
 // a gather over all NvS rows reads only rows of x.
-__global__ void __launch_bounds__(1024) permute_scan_kernel(
-    const int* __restrict__ blkcnt, int nblk, int E, int B, const int32_t* __restrict__ replica_src,
+// The scan's work for one block of 1024 threads; sm holds [G] segment sizes, then [1024]
+// scan scratch.
+__device__ void permute_scan_body(
+    int* sm, const int* __restrict__ blkcnt, int nblk, int E, int B, const int32_t* __restrict__ replica_src,
     int* __restrict__ blkoff, int* __restrict__ total, int* __restrict__ nrep,
     int* __restrict__ rep_ptr, int* __restrict__ rep_rows, int* __restrict__ rowstart,
     int32_t* __restrict__ cu_seqlens, int NvS, int32_t* __restrict__ perm_token, float* __restrict__ perm_w,
     DevError* err) {
-    extern __shared__ int sm[];  // [G] segment sizes, then [1024] scan scratch
     const int G = E + B;
     int* seg = sm;
     int* scratch = sm + G;
-    pdl_wait();
     // per-expert totals and block offsets; replica counts
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
@@ -375,21 +375,30 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(
         perm_token[r] = 0;
         perm_w[r] = 0.0f;
     }
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(
+    const int* __restrict__ blkcnt, int nblk, int E, int B, const int32_t* __restrict__ replica_src,
+    int* __restrict__ blkoff, int* __restrict__ total, int* __restrict__ nrep,
+    int* __restrict__ rep_ptr, int* __restrict__ rep_rows, int* __restrict__ rowstart,
+    int32_t* __restrict__ cu_seqlens, int NvS, int32_t* __restrict__ perm_token, float* __restrict__ perm_w,
+    DevError* err) {
+    extern __shared__ int sm[];  // [G] segment sizes, then [1024] scan scratch
+    pdl_wait();
+    permute_scan_body(sm, blkcnt, nblk, E, B, replica_src, blkoff, total, nrep, rep_ptr, rep_rows, rowstart,
+                      cu_seqlens, NvS, perm_token, perm_w, err);
     pdl_launch();
 }
 
-__global__ void __launch_bounds__(kPermBlock) permute_scatter_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int topk, int E,
-    const int* __restrict__ blkoff, const int* __restrict__ total, const int* __restrict__ nrep,
-    const int* __restrict__ rep_ptr, const int* __restrict__ rep_rows,
-    const int* __restrict__ rowstart, int32_t* __restrict__ perm_token, float* __restrict__ perm_w,
-    int32_t* __restrict__ inv_perm, DevError* err) {
-    extern __shared__ uint32_t masks[];
-    pdl_wait();
-    const int t0 = blockIdx.x * kPermBlock;
-    build_masks(masks, ids, T, topk, E, t0, nullptr);
-    const int t = t0 + threadIdx.x;
-    if (t < T) {
+// Token block `blk`'s assignments to their rows, from the block's masks (threads 0..255
+// own the block's tokens).
+__device__ void permute_scatter_body(
+    const uint32_t* masks, int blk, const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T,
+    int topk, int E, const int* __restrict__ blkoff, const int* __restrict__ total, const int* __restrict__ nrep,
+    const int* __restrict__ rep_ptr, const int* __restrict__ rep_rows, const int* __restrict__ rowstart,
+    int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_perm) {
+    const int t = blk * kPermBlock + threadIdx.x;
+    if (threadIdx.x < kPermBlock && t < T) {
         const int word = threadIdx.x >> 5;
         const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
         for (int j = 0; j < topk; ++j) {
@@ -401,7 +410,7 @@ __global__ void __launch_bounds__(kPermBlock) permute_scatter_kernel(
             const uint32_t* m = masks + e * (kPermBlock / 32);
             int rank = __popc(m[word] & below);
             for (int q = 0; q < word; ++q) rank += __popc(m[q]);
-            const int r = blkoff[(size_t)blockIdx.x * E + e] + rank;
+            const int r = blkoff[(size_t)blk * E + e] + rank;
             const int n = total[e], R = nrep[e];
             const int q = n / R, rem = n % R, big = rem * (q + 1);
             int chunk, pos;
@@ -419,7 +428,48 @@ __global__ void __launch_bounds__(kPermBlock) permute_scatter_kernel(
             inv_perm[(size_t)t * topk + j] = dst;
         }
     }
-    (void)err;
+}
+
+__global__ void __launch_bounds__(kPermBlock) permute_scatter_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int topk, int E,
+    const int* __restrict__ blkoff, const int* __restrict__ total, const int* __restrict__ nrep,
+    const int* __restrict__ rep_ptr, const int* __restrict__ rep_rows,
+    const int* __restrict__ rowstart, int32_t* __restrict__ perm_token, float* __restrict__ perm_w,
+    int32_t* __restrict__ inv_perm) {
+    extern __shared__ uint32_t masks[];
+    pdl_wait();
+    build_masks(masks, ids, T, topk, E, blockIdx.x * kPermBlock, nullptr);
+    permute_scatter_body(masks, blockIdx.x, ids, topk_w, T, topk, E, blkoff, total, nrep, rep_ptr, rep_rows,
+                         rowstart, perm_token, perm_w, inv_perm);
+    pdl_launch();
+}
+
+// At most one token block: the count, the scan and the scatter in one CTA of 1024 threads
+// (three launches fewer for decode batches). Shared memory: the block's masks [E * 8], then
+// the scan's [G + 1024].
+__global__ void __launch_bounds__(1024) permute_one_block_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int topk, int E, int B,
+    const int32_t* __restrict__ replica_src, int* __restrict__ blkcnt, int* __restrict__ blkoff,
+    int* __restrict__ total, int* __restrict__ nrep, int* __restrict__ rep_ptr, int* __restrict__ rep_rows,
+    int* __restrict__ rowstart, int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ perm_token,
+    float* __restrict__ perm_w, int32_t* __restrict__ inv_perm, DevError* err) {
+    extern __shared__ uint32_t smem_u[];
+    uint32_t* masks = smem_u;
+    int* sm = reinterpret_cast<int*>(smem_u + (size_t)E * (kPermBlock / 32));
+    pdl_wait();
+    build_masks(masks, ids, T, topk, E, 0, err);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int q = 0; q < kPermBlock / 32; ++q) c += __popc(masks[e * (kPermBlock / 32) + q]);
+        blkcnt[e] = c;
+    }
+    __syncthreads();
+    permute_scan_body(sm, blkcnt, 1, E, B, replica_src, blkoff, total, nrep, rep_ptr, rep_rows, rowstart,
+                      cu_seqlens, T * topk, perm_token, perm_w, err);
+    __syncthreads();
+    permute_scatter_body(masks, 0, ids, topk_w, T, topk, E, blkoff, total, nrep, rep_ptr, rep_rows, rowstart,
+                         perm_token, perm_w, inv_perm);
     pdl_launch();
 }
 
@@ -437,6 +487,25 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
     int* rowstart = reinterpret_cast<int*>(ws + L.rowstart);
     const size_t mask_smem = sizeof(uint32_t) * E * (kPermBlock / 32);
     cudaError_t e;
+    if (L.nblk == 1) {
+        const size_t smem = mask_smem + sizeof(int) * (E + B + 1024);
+        if (smem > 48 * 1024) {
+            static int done[64] = {0};
+            int dev = 0;
+            e = cudaGetDevice(&dev);
+            if (e != cudaSuccess) return e;
+            if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+            if (!done[dev]) {
+                e = cudaFuncSetAttribute(permute_one_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+                if (e != cudaSuccess) return e;
+                done[dev] = 1;
+            }
+        }
+        return launch_k(permute_one_block_kernel, dim3(1), dim3(1024), smem, st, pdl, ids, topk_w, T, topk, E, B,
+                        replica_src, blkcnt, blkoff, total, nrep, rep_ptr, rep_rows, rowstart, cu_seqlens,
+                        perm_token, perm_w, inv_perm, err);
+    }
     if (L.nblk > 0) {
         e = launch_k(permute_count_kernel, dim3(L.nblk), dim3(kPermBlock), mask_smem, st, pdl, ids, T,
                      topk, E, blkcnt, err);
@@ -452,7 +521,7 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
         e = launch_k(permute_scatter_kernel, dim3(L.nblk), dim3(kPermBlock), mask_smem, st, true, ids,
                      topk_w, T, topk, E, (const int*)blkoff, (const int*)total, (const int*)nrep,
                      (const int*)rep_ptr, (const int*)rep_rows, (const int*)rowstart, perm_token,
-                     perm_w, inv_perm, err);
+                     perm_w, inv_perm);
     }
     return e;
 }
