@@ -313,9 +313,13 @@ def default_sample(cfg) -> int:
 # ---------------------------------------------------------------------------- arms
 
 def kernel_launches(cfg) -> int:
-    # route, the permutation (one kernel for at most 256 tokens, else count, scan, scatter),
+    # route and permutation (one kernel for at most 256 tokens with the default routing; else
+    # the routing, then the count, scan and scatter, or one kernel for at most 256 tokens),
     # gate/up GEMM, down GEMM, combine
-    n = 1 + (1 if cfg.T <= 256 else 3) + 1 + 1 + 1
+    if cfg.T <= 256:
+        n = (1 if cfg.routing == "renormalize" else 2) + 1 + 1 + 1
+    else:
+        n = 1 + 3 + 1 + 1 + 1
     # the gate/up operand in segment order: a gather (BF16; NVFP4 weights with bf16
     # activations, as f16) or one staging / quantisation pass over the gathered rows (MXFP4;
     # NVFP4 activations when H % 256 == 0, else quantisation then a gather)

@@ -541,9 +541,14 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     } else if (p->routing == 1) {
         e = launch_route_grouped(p->router_logits, p->routing_bias, T, E, k, p->n_group, p->topk_group,
                                  p->routed_scaling_factor, ids_w, tw_w, st, false);
+    } else if (T <= 256) {
+        // decode batches: the routing and the permutation in one launch
+        e = launch_route_permute_one_block(p->router_logits, T, E, k, ids_w, tw_w, B, p->replica_src, cu, perm_token,
+                                           perm_w, inv, err, w + L.perm_scratch, st, false);
     } else {
         e = launch_route_topk(p->router_logits, T, E, k, ids_w, tw_w, st, false);
     }
+    const bool permuted = !given && p->routing == 0 && T <= 256;
     if (e != cudaSuccess || !mark(1)) return MOE_ERR_CUDA;
     // top-1 weight on the input: the experts see x * w and the activation takes no weight
     const bool in_w = p->apply_router_weight_on_input != 0;
@@ -556,9 +561,11 @@ moe_status_t moe_forward(const moe_forward_args_t* p, void* ws, size_t ws_bytes,
     }
     // S2 permute
     trace.stage("permute");
-    e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch, st,
-                       pdl());
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!permuted) {
+        e = launch_permute(ids, tw, T, k, E, B, p->replica_src, cu, perm_token, perm_w, inv, err, w + L.perm_scratch,
+                           st, pdl());
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
     // S2 gather (+ S2q). The BF16 gate/up GEMM with 128-token tiles (or on CTA pairs) can read
     // the token rows of x by perm_token itself (MOE_FUSED_GATHER=1), which saves writing and
     // re-reading x_perm.

@@ -47,6 +47,12 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
                            const int32_t* replica_src, int32_t* cu_seqlens, int32_t* perm_token,
                            float* perm_w, int32_t* inv_perm, DevError* err, char* scratch,
                            cudaStream_t st, bool pdl);
+// Routing (softmax -> top-k -> renormalise) and the permutation of 1 <= T <= 256 tokens in one
+// launch; the same outputs as launch_route_topk followed by launch_permute.
+cudaError_t launch_route_permute_one_block(const float* logits, int T, int E, int topk, int32_t* ids, float* w,
+                                          int B, const int32_t* replica_src, int32_t* cu_seqlens,
+                                          int32_t* perm_token, float* perm_w, int32_t* inv_perm, DevError* err,
+                                          char* ws, cudaStream_t st, bool pdl);
 cudaError_t launch_gather(int mode, const void* src, int H, const int32_t* perm_token, int NvS,
                           void* dst, const float* src_scale, float* dst_scale, cudaStream_t st,
                           bool pdl);

@@ -12,15 +12,12 @@
 namespace moe {
 
 // ----------------------------------------------------------------- S1 route
+// Token t's top-k by one warp (all 32 lanes): ids and renormalised weights, in selection order.
 template <int EPL>  // logits per lane (E <= 32*EPL)
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
-                                                         int E, int topk,
-                                                         int32_t* __restrict__ ids,
-                                                         float* __restrict__ w) {
-    pdl_wait();
+__device__ __forceinline__ void route_token(const float* __restrict__ logits, int t, int E, int topk,
+                                            int32_t* __restrict__ ids, float* __restrict__ w) {
     const int lane = lane_id();
-    const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
-    if (t < T) {
+    {
         float v[EPL];
         const float* row = logits + (size_t)t * E;
 #pragma unroll
@@ -74,6 +71,16 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
             w[(size_t)t * topk + lane] = z / sum;
         }
     }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T,
+                                                         int E, int topk,
+                                                         int32_t* __restrict__ ids,
+                                                         float* __restrict__ w) {
+    pdl_wait();
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp_id();
+    if (t < T) route_token<EPL>(logits, t, E, topk, ids, w);
     pdl_launch();
 }
 
@@ -444,6 +451,13 @@ __global__ void __launch_bounds__(kPermBlock) permute_scatter_kernel(
     pdl_launch();
 }
 
+__device__ void permute_one_block_body(
+    uint32_t* smem_u, const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int topk, int E,
+    int B, const int32_t* __restrict__ replica_src, int* __restrict__ blkcnt, int* __restrict__ blkoff,
+    int* __restrict__ total, int* __restrict__ nrep, int* __restrict__ rep_ptr, int* __restrict__ rep_rows,
+    int* __restrict__ rowstart, int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ perm_token,
+    float* __restrict__ perm_w, int32_t* __restrict__ inv_perm, DevError* err);
+
 // At most one token block: the count, the scan and the scatter in one CTA of 1024 threads
 // (three launches fewer for decode batches). Shared memory: the block's masks [E * 8], then
 // the scan's [G + 1024].
@@ -454,9 +468,38 @@ __global__ void __launch_bounds__(1024) permute_one_block_kernel(
     int* __restrict__ rowstart, int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ perm_token,
     float* __restrict__ perm_w, int32_t* __restrict__ inv_perm, DevError* err) {
     extern __shared__ uint32_t smem_u[];
+    pdl_wait();
+    permute_one_block_body(smem_u, ids, topk_w, T, topk, E, B, replica_src, blkcnt, blkoff, total, nrep, rep_ptr,
+                           rep_rows, rowstart, cu_seqlens, perm_token, perm_w, inv_perm, err);
+    pdl_launch();
+}
+
+// Softmax -> top-k -> renormalise for at most 256 tokens (32 warps) and their permutation,
+// one CTA: two launches fewer than the routing plus the permutation for decode batches.
+template <int EPL>
+__global__ void __launch_bounds__(1024) route_permute_one_block_kernel(
+    const float* __restrict__ logits, int T, int E, int topk, int32_t* __restrict__ ids, float* __restrict__ topk_w,
+    int B, const int32_t* __restrict__ replica_src, int* __restrict__ blkcnt, int* __restrict__ blkoff,
+    int* __restrict__ total, int* __restrict__ nrep, int* __restrict__ rep_ptr, int* __restrict__ rep_rows,
+    int* __restrict__ rowstart, int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ perm_token,
+    float* __restrict__ perm_w, int32_t* __restrict__ inv_perm, DevError* err) {
+    extern __shared__ uint32_t smem_u[];
+    pdl_wait();
+    for (int t = warp_id(); t < T; t += blockDim.x >> 5) route_token<EPL>(logits, t, E, topk, ids, topk_w);
+    __syncthreads();
+    permute_one_block_body(smem_u, ids, topk_w, T, topk, E, B, replica_src, blkcnt, blkoff, total, nrep, rep_ptr,
+                           rep_rows, rowstart, cu_seqlens, perm_token, perm_w, inv_perm, err);
+    pdl_launch();
+}
+
+__device__ void permute_one_block_body(
+    uint32_t* smem_u, const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T, int topk, int E,
+    int B, const int32_t* __restrict__ replica_src, int* __restrict__ blkcnt, int* __restrict__ blkoff,
+    int* __restrict__ total, int* __restrict__ nrep, int* __restrict__ rep_ptr, int* __restrict__ rep_rows,
+    int* __restrict__ rowstart, int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ perm_token,
+    float* __restrict__ perm_w, int32_t* __restrict__ inv_perm, DevError* err) {
     uint32_t* masks = smem_u;
     int* sm = reinterpret_cast<int*>(smem_u + (size_t)E * (kPermBlock / 32));
-    pdl_wait();
     build_masks(masks, ids, T, topk, E, 0, err);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int c = 0;
@@ -470,7 +513,6 @@ __global__ void __launch_bounds__(1024) permute_one_block_kernel(
     __syncthreads();
     permute_scatter_body(masks, 0, ids, topk_w, T, topk, E, blkoff, total, nrep, rep_ptr, rep_rows, rowstart,
                          perm_token, perm_w, inv_perm);
-    pdl_launch();
 }
 
 cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int topk, int E, int B,
@@ -524,6 +566,50 @@ cudaError_t launch_permute(const int32_t* ids, const float* topk_w, int T, int t
                      perm_w, inv_perm);
     }
     return e;
+}
+
+cudaError_t launch_route_permute_one_block(const float* logits, int T, int E, int topk, int32_t* ids, float* w,
+                                          int B, const int32_t* replica_src, int32_t* cu_seqlens,
+                                          int32_t* perm_token, float* perm_w, int32_t* inv_perm, DevError* err,
+                                          char* ws, cudaStream_t st, bool pdl) {
+    if (T < 1 || T > kPermBlock) return cudaErrorInvalidValue;
+    const PermuteWs L = permute_ws_layout(T, topk, E, B);
+    int* blkcnt = reinterpret_cast<int*>(ws + L.blkcnt);
+    int* blkoff = reinterpret_cast<int*>(ws + L.blkoff);
+    int* total = reinterpret_cast<int*>(ws + L.total);
+    int* nrep = reinterpret_cast<int*>(ws + L.nrep);
+    int* rep_ptr = reinterpret_cast<int*>(ws + L.rep_ptr);
+    int* rep_rows = reinterpret_cast<int*>(ws + L.rep_rows);
+    int* rowstart = reinterpret_cast<int*>(ws + L.rowstart);
+    const size_t smem = sizeof(uint32_t) * E * (kPermBlock / 32) + sizeof(int) * (E + B + 1024);
+    const int epl = (E + 31) / 32;
+    cudaError_t e = cudaSuccess;
+#define MOE_RP(N)                                                                                                  \
+    {                                                                                                              \
+        auto k = route_permute_one_block_kernel<N>;                                                                \
+        if (smem > 48 * 1024) {                                                                                    \
+            static int done[64] = {0};                                                                             \
+            int dev = 0;                                                                                           \
+            if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;                                                \
+            if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;                                               \
+            if (!done[dev]) {                                                                                      \
+                if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=       \
+                    cudaSuccess)                                                                                   \
+                    return e;                                                                                      \
+                done[dev] = 1;                                                                                     \
+            }                                                                                                      \
+        }                                                                                                          \
+        return launch_k(k, dim3(1), dim3(1024), smem, st, pdl, logits, T, E, topk, ids, w, B, replica_src, blkcnt, \
+                        blkoff, total, nrep, rep_ptr, rep_rows, rowstart, cu_seqlens, perm_token, perm_w, inv_perm, \
+                        err);                                                                                      \
+    }
+    if (epl <= 1) MOE_RP(1);
+    if (epl <= 2) MOE_RP(2);
+    if (epl <= 4) MOE_RP(4);
+    if (epl <= 8) MOE_RP(8);
+    if (epl <= 16) MOE_RP(16);
+    MOE_RP(32);
+#undef MOE_RP
 }
 
 // ----------------------------------------------------------------- row gathers

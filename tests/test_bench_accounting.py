@@ -51,7 +51,7 @@ def test_tensor_peak_of_each_mma_kind():
 def test_launch_counts_and_dtype():
     assert bench.kernel_launches(W.CONFIGS["mixtral_prefill"]) == 8
     assert bench.kernel_launches(W.CONFIGS["nvfp4"]) == 9
-    assert bench.kernel_launches(W.CONFIGS["mxfp4_decode"]) == 6
+    assert bench.kernel_launches(W.CONFIGS["mxfp4_decode"]) == 5
     assert bench.compute_dtype(W.CONFIGS["mixtral_prefill"]) == "bf16"
     assert bench.compute_dtype(W.CONFIGS["nvfp4"]).startswith("nvfp4")
 
@@ -75,16 +75,17 @@ def test_bias_and_swigluoai_accounting():
     assert a["fc2_bytes"] == nonempty * wrow + NvS * cfg.I * 2 + NvS * cfg.H * 4 + nonempty * cfg.H * 4
     assert a["layer_bytes"] == (nonempty * 3 * wrow + nonempty * (2 * cfg.I + cfg.H) * 4
                                 + cfg.T * cfg.H * 4 + cfg.T * cfg.E * 4)
-    # (T <= 256: the permutation is one kernel)
-    assert bench.kernel_launches(cfg) == 6
-    assert bench.kernel_launches(cfg.with_(bias=False)) == 6
+    # (T <= 256: routing and permutation are one kernel)
+    assert bench.kernel_launches(cfg) == 5
+    assert bench.kernel_launches(cfg.with_(bias=False)) == 5
     assert bench.kernel_launches(cfg.with_(T=300)) == 8
-    assert bench.kernel_launches(W.CONFIGS["mxfp4_swiglu_bias_decode"]) == 6
+    assert bench.kernel_launches(W.CONFIGS["mxfp4_swiglu_bias_decode"]) == 5
+    assert bench.kernel_launches(W.CONFIGS["deepseek_decode_grouped"]) == 6
     # NVFP4 weights, bf16 activations, SITU: the epilogue stores f16 directly, with or without
     # biases (SITU bounds h either way)
     nv = W.MoEConfig("nv", T=8, H=256, I=256, E=4, topk=2, act="situ", wfmt="nvfp4")
-    assert bench.kernel_launches(nv) == 6
-    assert bench.kernel_launches(nv.with_(bias=True)) == 6
+    assert bench.kernel_launches(nv) == 5
+    assert bench.kernel_launches(nv.with_(bias=True)) == 5
     assert bench.act_config(W.CONFIGS["mxfp4_swiglu_bias_decode"]) == dict(
         swiglu_alpha=1.702, swiglu_beta=1.0, swiglu_limit=7.0, gemm_biases=True)
     assert bench.act_config(W.CONFIGS["mixtral_prefill"]) == {}
