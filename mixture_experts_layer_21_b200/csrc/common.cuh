@@ -436,10 +436,21 @@ MOE_DEV float e4m3_to_f32(uint8_t c) {
 // block takes -127. Clamped to e8m0's [-127, 127].
 MOE_DEV int mx8_block_exp(float amax, bool two) {
     if (!(amax > 0.0f)) return -127;
+    // amax = m * 2^ex with m in [0.5, 1). For a normal amax = (1 + f) 2^(E - 127) that is
+    // ex = E - 126 and m = (1 + f) / 2, so m > 0.875 exactly when f > 0.75, i.e. when the
+    // fraction field exceeds 0x600000; subnormals and infinities take frexpf.
+    const uint32_t bits = __float_as_uint(amax);
+    const int E = (int)(bits >> 23);
     int ex;
-    const float m = frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
+    bool big;
+    if (E > 0 && E < 255) {
+        ex = E - 126;
+        big = (bits & 0x7FFFFFu) > 0x600000u;
+    } else {
+        big = frexpf(amax, &ex) > 0.875f;
+    }
     // hi/lo: 448 * 2^(ex-9) = 0.875 * 2^ex; one term: floor(log2 amax) - 8 = ex - 9
-    const int e = (two && m > 0.875f) ? ex - 8 : ex - 9;
+    const int e = (two && big) ? ex - 8 : ex - 9;
     return max(-127, min(127, e));
 }
 // 2^-e as a normal float for the e of mx8_block_exp (finite inputs give e <= 120).

@@ -186,94 +186,184 @@ __device__ __forceinline__ void drain_in_flight(const Issued& is, uint64_t* full
 // tb + (j*NB + m)*BT (partials of different issuers, PM = false), or at
 // tb + (m*NPART + j)*BT (PM = true: one MMA wrote a matrix's partials side by side).
 // With EW warps per lane quarter, warp h of a quarter takes the 16-token chunks h, h+EW, ...
+
+// Tokens c0 .. c0+15 of this lane's row, partial sums added: matrix 0 in r0, matrix 1 in r1.
+template <int BT, bool DUAL, int NPART, bool PM>
+__device__ __forceinline__ void epi_load16(uint32_t tb, int c0, uint32_t (&r0)[16], uint32_t (&r1)[16]) {
+    constexpr int NB = DUAL ? 2 : 1;
+    auto col = [](int m, int j) { return (PM ? m * NPART + j : j * NB + m) * BT; };
+    tmem_ld16(tb + col(0, 0) + c0, r0);
+    if (DUAL) tmem_ld16(tb + col(1, 0) + c0, r1);
+    tmem_ld_wait();
+#pragma unroll
+    for (int pj = 1; pj < NPART; ++pj) {
+        uint32_t p0[16], p1[16];
+        tmem_ld16(tb + col(0, pj) + c0, p0);
+        if (DUAL) tmem_ld16(tb + col(1, pj) + c0, p1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            r0[j] = __float_as_uint(__uint_as_float(r0[j]) + __uint_as_float(p0[j]));
+            if (DUAL) r1[j] = __float_as_uint(__uint_as_float(r1[j]) + __uint_as_float(p1[j]));
+        }
+    }
+}
+
+// What a lane's output column n needs for every token of a tile.
+struct EpiCol {
+    int n;
+    float al0, al1, bn0, bn1, inv_sa, inv_sb;
+};
+
+template <bool DUAL>
+__device__ __forceinline__ EpiCol epi_col(const GemmArgs& a, int g, int nt, int q, int lane) {
+    EpiCol c;
+    c.n = nt * kTileN + q * 32 + lane;
+    c.al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
+    c.al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
+    c.bn0 = (a.bias0 && c.n < a.N) ? a.bias0[(size_t)g * a.N + c.n] : 0.0f;
+    c.bn1 = (DUAL && a.bias1 && c.n < a.N) ? a.bias1[(size_t)g * a.N + c.n] : 0.0f;
+    c.inv_sa = 1.0f / a.sa;
+    c.inv_sb = 1.0f / a.sb;
+    return c;
+}
+
+// Per-token factors of a 16-token chunk, loaded by lane (token % 16) and broadcast later:
+// the token's activation row scale and the dual GEMM's route weight (a single GEMM's: the
+// weight of its bias).
+template <bool DUAL>
+__device__ __forceinline__ void epi_token_factors(const GemmArgs& a, int row0, int c0, int rows, int lane, float& ts,
+                                                  float& pw) {
+    const int my_row = row0 + c0 + (lane & 15);
+    const bool row_ok = c0 + (lane & 15) < rows;
+    ts = (a.tscale && row_ok) ? a.tscale[my_row] : 1.0f;
+    const float* rw = DUAL ? a.perm_w : a.bias_rw;
+    pw = (rw && row_ok) ? rw[my_row] : 1.0f;
+}
+
+// The gated activation of one token (the dual GEMM) times its route weight.
+__device__ __forceinline__ float epi_gated(const GemmArgs& a, const EpiCol& c, uint32_t x0, uint32_t x1, float ts,
+                                           float pw) {
+    const float gv = __uint_as_float(x0) * c.al0 * ts + c.bn0;
+    const float uv = __uint_as_float(x1) * c.al1 * ts + c.bn1;
+    return (a.act == MOE_ACT_SWIGLUOAI ? swigluoai_fast(gv, uv, a.sw_alpha, a.sw_beta, a.sw_limit)
+                                       : act_apply_fast(a.act, gv, uv, a.sa, a.sb, c.inv_sa, c.inv_sb)) *
+           pw;
+}
+
+// One token's 32-value block of the down GEMM's K (this warp's 32 lanes): its e8m0 scale,
+// then the e4m3 code (and the lo term's) of each lane's value. Lanes past N (up to the padded
+// K) hold zeros. All lanes take part. For finite values the block exponent is a
+// non-decreasing function of the block's largest magnitude, so it is the warp max of the
+// lanes' own exponents: one integer reduction instead of a shuffle tree over floats. An
+// infinite value makes the block's largest magnitude infinite (key 255), and the block takes
+// that magnitude's exponent; NaNs do not count, as in a max over floats.
+__device__ __forceinline__ void epi_store_mx8(const GemmArgs& a, int row, int n, int lane, float v) {
+    const bool two = a.out_terms == 2;
+    const float av = fabsf(v);
+    const unsigned key = isinf(av) ? 255u : (unsigned)(mx8_block_exp(av, two) + 127);
+    const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+    const int e = kmax == 255u ? mx8_block_exp(__int_as_float(0x7f800000), two) : (int)kmax - 127;
+    const float y = v * mx8_inv_scale(e);
+    uint8_t* rec = reinterpret_cast<uint8_t*>(a.out) + (size_t)row * a.out_stride;
+    const uint8_t hi = cvt_e4m3(y);
+    rec[n] = hi;
+    if (two) rec[a.out_kpad + n] = cvt_e4m3(y - e4m3_to_f32(hi));
+    if (lane == 0) rec[a.out_terms * a.out_kpad + n / 32] = (uint8_t)(e + 127);
+}
+
+template <int OUT>
+__device__ __forceinline__ void epi_store(const GemmArgs& a, int row, int n, float v) {
+    const size_t idx = (size_t)row * a.N + n;
+    if (OUT == OUT_BF16) reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
+    else if (OUT == OUT_F16) reinterpret_cast<__half*>(a.out)[idx] = __float2half_rn(v);
+    else reinterpret_cast<float*>(a.out)[idx] = v;
+}
+
 template <int BT, bool DUAL, int OUT, int NPART = 1, bool PM = false, int EW = 1>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tb, int g, int nt, int row0, int rows,
                                               int q, int lane, int h = 0) {
-    const int n = nt * kTileN + q * 32 + lane;
-    const float al0 = a.alpha0 ? a.alpha0[g] : 1.0f;
-    const float al1 = a.alpha1 ? a.alpha1[g] : 1.0f;
-    const float bn0 = (a.bias0 && n < a.N) ? a.bias0[(size_t)g * a.N + n] : 0.0f;
-    const float bn1 = (DUAL && a.bias1 && n < a.N) ? a.bias1[(size_t)g * a.N + n] : 0.0f;
-    const float inv_sa = 1.0f / a.sa, inv_sb = 1.0f / a.sb;
-    constexpr int NB = DUAL ? 2 : 1;
-    auto col = [](int m, int j) { return (PM ? m * NPART + j : j * NB + m) * BT; };
+    const EpiCol c = epi_col<DUAL>(a, g, nt, q, lane);
+    const int n = c.n;
 #pragma unroll 1
     for (int c0 = 16 * h; c0 < BT; c0 += 16 * EW) {
         if (c0 >= rows) break;
         uint32_t r0[16], r1[16];
-        tmem_ld16(tb + col(0, 0) + c0, r0);
-        if (DUAL) tmem_ld16(tb + col(1, 0) + c0, r1);
-        tmem_ld_wait();
+        epi_load16<BT, DUAL, NPART, PM>(tb, c0, r0, r1);
+        float my_ts, my_pw;
+        epi_token_factors<DUAL>(a, row0, c0, rows, lane, my_ts, my_pw);
 #pragma unroll
-        for (int pj = 1; pj < NPART; ++pj) {
-            uint32_t p0[16], p1[16];
-            tmem_ld16(tb + col(0, pj) + c0, p0);
-            if (DUAL) tmem_ld16(tb + col(1, pj) + c0, p1);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                r0[j] = __float_as_uint(__uint_as_float(r0[j]) + __uint_as_float(p0[j]));
-                if (DUAL) r1[j] = __float_as_uint(__uint_as_float(r1[j]) + __uint_as_float(p1[j]));
+        for (int j = 0; j < 16; ++j) {
+            // every lane takes part in the shuffles; only in-range outputs are stored
+            const float ts = __shfl_sync(0xffffffffu, my_ts, j);
+            const float pw = __shfl_sync(0xffffffffu, my_pw, j);
+            const int row = row0 + c0 + j;
+            if constexpr (OUT == OUT_MX8) {
+                // rows, c0 and j are the same in every lane, so the warp stays whole
+                if (c0 + j < rows)
+                    epi_store_mx8(a, row, n, lane, DUAL && n < a.N ? epi_gated(a, c, r0[j], r1[j], ts, pw) : 0.0f);
+            } else if (n < a.N && c0 + j < rows) {
+                const float v = DUAL ? epi_gated(a, c, r0[j], r1[j], ts, pw) * a.out_scale
+                                     : __uint_as_float(r0[j]) * c.al0 * ts * a.out_scale + pw * c.bn0;
+                epi_store<OUT>(a, row, n, v);
             }
         }
-        // per-token factors of this 16-token chunk: one coalesced load, then broadcasts
-        const int my_row = row0 + c0 + (lane & 15);
-        const bool row_ok = c0 + (lane & 15) < rows;
-        const float my_ts = (a.tscale && row_ok) ? a.tscale[my_row] : 1.0f;
-        // the dual GEMM's route weight; a single GEMM's weight of its bias
-        const float* rw = DUAL ? a.perm_w : a.bias_rw;
-        const float my_pw = (rw && row_ok) ? rw[my_row] : 1.0f;
-        {
+    }
+}
+
+// The epilogue of a single-buffered accumulator whose output is the down GEMM's e4m3
+// records (the MXFP4 gate/up tile). The next tile's MMAs wait for it, so phase 1 only reads
+// this warp's chunks out of tensor memory and applies the activation into registers; then
+// `release()` frees the accumulator, and phase 2 encodes and stores while the next tile's
+// MMAs run. The values are those of epilogue_tile.
+template <int BT, int NPART, bool PM, int EW, typename Rel>
+__device__ __forceinline__ void epilogue_tile_mx8_staged(const GemmArgs& a, uint32_t tb, int g, int nt, int row0,
+                                                         int rows, int q, int lane, int h, Rel release) {
+    constexpr int NCH = BT / (16 * EW);  // this warp's chunks
+    const EpiCol c = epi_col<true>(a, g, nt, q, lane);
+    const int n = c.n;
+    float vals[NCH][16];
+#pragma unroll
+    for (int ci = 0; ci < NCH; ++ci) {
+        const int c0 = 16 * (h + ci * EW);
+        if (c0 < rows) {
+            uint32_t r0[16], r1[16];
+            epi_load16<BT, true, NPART, PM>(tb, c0, r0, r1);
+            float my_ts, my_pw;
+            epi_token_factors<true>(a, row0, c0, rows, lane, my_ts, my_pw);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                // every lane takes part in the shuffles; only in-range outputs are stored
                 const float ts = __shfl_sync(0xffffffffu, my_ts, j);
                 const float pw = __shfl_sync(0xffffffffu, my_pw, j);
-                if constexpr (OUT == OUT_MX8) {
-                    // the warp's 32 lanes are one 32-value block of the down GEMM's K: its
-                    // scale is a warp max; lanes past N (up to the padded K) write zeros
-                    float v = 0.0f;
-                    if (DUAL && n < a.N && c0 + j < rows) {
-                        const float gv = __uint_as_float(r0[j]) * al0 * ts + bn0;
-                        const float uv = __uint_as_float(r1[j]) * al1 * ts + bn1;
-                        v = (a.act == MOE_ACT_SWIGLUOAI
-                                 ? swigluoai_fast(gv, uv, a.sw_alpha, a.sw_beta, a.sw_limit)
-                                 : act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb)) *
-                            pw;
-                    }
-                    float am = fabsf(v);
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-                    if (c0 + j < rows) {
-                        const int e = mx8_block_exp(am, a.out_terms == 2);
-                        const float y = v * mx8_inv_scale(e);
-                        uint8_t* rec = reinterpret_cast<uint8_t*>(a.out) + (size_t)(row0 + c0 + j) * a.out_stride;
-                        const uint8_t hi = cvt_e4m3(y);
-                        rec[n] = hi;
-                        if (a.out_terms == 2) rec[a.out_kpad + n] = cvt_e4m3(y - e4m3_to_f32(hi));
-                        if (lane == 0) rec[a.out_terms * a.out_kpad + n / 32] = (uint8_t)(e + 127);
-                    }
-                } else if (n < a.N && c0 + j < rows) {
-                    const int row = row0 + c0 + j;
-                    float v;
-                    if (DUAL) {
-                        const float gv = __uint_as_float(r0[j]) * al0 * ts + bn0;
-                        const float uv = __uint_as_float(r1[j]) * al1 * ts + bn1;
-                        v = (a.act == MOE_ACT_SWIGLUOAI
-                                 ? swigluoai_fast(gv, uv, a.sw_alpha, a.sw_beta, a.sw_limit)
-                                 : act_apply_fast(a.act, gv, uv, a.sa, a.sb, inv_sa, inv_sb)) *
-                            pw;
-                        v *= a.out_scale;
-                    } else {
-                        v = __uint_as_float(r0[j]) * al0 * ts * a.out_scale + pw * bn0;
-                    }
-                    const size_t idx = (size_t)row * a.N + n;
-                    if (OUT == OUT_BF16) reinterpret_cast<__nv_bfloat16*>(a.out)[idx] = __float2bfloat16_rn(v);
-                    else if (OUT == OUT_F16) reinterpret_cast<__half*>(a.out)[idx] = __float2half_rn(v);
-                    else reinterpret_cast<float*>(a.out)[idx] = v;
-                }
+                vals[ci][j] = n < a.N ? epi_gated(a, c, r0[j], r1[j], ts, pw) : 0.0f;
             }
         }
+    }
+    release();
+#pragma unroll
+    for (int ci = 0; ci < NCH; ++ci) {
+        const int c0 = 16 * (h + ci * EW);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c0 + j < rows) epi_store_mx8(a, row0 + c0 + j, n, lane, vals[ci][j]);
+    }
+}
+
+// The token half of a stage gathered by the producer warp: 128 rows of 64 K values (128
+// bytes), row r of the tile from token tok(r), where lane l holds the tokens of rows l + 32 j
+// in tok[j]. Lane 8 rr + c copies chunk c (16 bytes) of rows 4 i + rr, so one warp
+// instruction reads four whole 128-byte row segments; chunk c of row r lands at chunk
+// position c ^ (r % 8), the 128-byte swizzle the MMA reads. Chunks past K are zero-filled.
+__device__ __forceinline__ void gather_stage_rows(uint32_t bb, const __nv_bfloat16* gx, const int (&tok)[4], int K,
+                                                  int kb, int lane) {
+    const int rr = lane >> 3, c = lane & 7;
+    const int k = kb * kTileK + c * 8;
+    const bool kin = k < K;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int row = 4 * i + rr;
+        const int t = __shfl_sync(0xffffffffu, tok[i >> 3], 4 * (i & 7) + rr);
+        cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), kin ? gx + (size_t)t * K + k : gx, kin ? 16u : 0u);
     }
 }
 
@@ -371,14 +461,13 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
             for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
                 int g, nt, row0, rows;
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
-                // this lane's tile rows lane + 32 i; rows past the GEMM's rows read a valid token
+                // the tokens of tile rows lane + 32 i; rows past the GEMM's rows read a valid token
                 // (their products are discarded), ids outside [0, gather_rows) too
-                const __nv_bfloat16* src[4];
+                int tok[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = min(row0 + lane + 32 * i, a.M_alloc - 1);
-                    const int t = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
-                    src[i] = a.gx + (size_t)t * K;
+                    tok[i] = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
                 }
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit))) {
@@ -390,18 +479,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                         tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
                         if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
                     }
-                    const uint32_t bb = smem_u32(opB(s));
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = lane + 32 * i;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const int k = kb * kTileK + c * 8;
-                            // 16 bytes of row `row`, chunk c, at chunk position c ^ (row % 8)
-                            cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), k < K ? src[i] + k : a.gx,
-                                       k < K ? 16u : 0u);
-                        }
-                    }
+                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane);
                     cp_async_arrive_noinc(&ctl->full[s]);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
@@ -512,11 +590,14 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(
-                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, nt, row0, rows, q, lane, h);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS);
+            auto release = [&] {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            };
+            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(a, tb, g, nt, row0, rows, q, lane, h);
+            release();
             if (++b == C::ACC_BUFS) {
                 b = 0;
                 bph ^= 1u;
@@ -648,14 +729,13 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                 decode_tile<BT>(L, ctl, G, NT, g, nt, row0, rows);
                 const int trow = row0 + (int)rank * (pair_mma_n(rows, BT) / 2);
                 const int wrow = (2 * nt + (int)rank) * kTileN;
-                // this lane's rows of the half: lane + 32 i; rows past the GEMM's rows read a
+                // the tokens of the half's rows lane + 32 i; rows past the GEMM's rows read a
                 // valid token (their products are discarded), ids outside [0, gather_rows) too
-                const __nv_bfloat16* src[4];
+                int tok[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = min(trow + lane + 32 * i, a.M_alloc - 1);
-                    const int t = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
-                    src[i] = a.gx + (size_t)t * K;
+                    tok[i] = min(max(a.gather_idx[r], 0), a.gather_rows - 1);
                 }
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[s], ph ^ 1u, abort_flag, a.wait_limit))) {
@@ -667,18 +747,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                         tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
                         if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
                     }
-                    const uint32_t bb = smem_u32(opB(s));
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = lane + 32 * i;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const int k = kb * kTileK + c * 8;
-                            // 16 bytes of row `row`, chunk c, at chunk position c ^ (row % 8)
-                            cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), k < K ? src[i] + k : a.gx,
-                                       k < K ? 16u : 0u);
-                        }
-                    }
+                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane);
                     cp_async_arrive_noinc(&ctl->full[s]);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
@@ -820,12 +889,14 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(
-                a, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS), g, 2 * nt + (int)rank, row0,
-                rows, q, lane, h);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS);
+            auto release = [&] {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
+            };
+            epilogue_tile<BT, DUAL, OUT, 1, false, C::EW>(a, tb, g, 2 * nt + (int)rank, row0, rows, q, lane, h);
+            release();
             if (++b == C::ACC_BUFS) {
                 b = 0;
                 bph ^= 1u;
@@ -1768,16 +1839,22 @@ __global__ void __launch_bounds__(Mx8Cfg<BT, DUAL || WIDE, TWO>::THREADS, 1)
             }
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC_COLS);
+            auto release = [&] {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tempty[b]);
+            };
             if constexpr (WIDE) {  // block 2nt, then block 2nt + 1 (its partials NPART * BT columns on)
                 epilogue_tile<BT, false, OUT, C::NPART, true, C::EW>(a, tb, g, 2 * nt, row0, rows, q, lane, h);
                 epilogue_tile<BT, false, OUT, C::NPART, true, C::EW>(a, tb + C::NPART * BT, g, 2 * nt + 1, row0, rows,
                                                                      q, lane, h);
+                release();
+            } else if constexpr (DUAL && C::ACC_BUFS == 1 && OUT == OUT_MX8) {
+                epilogue_tile_mx8_staged<BT, C::NPART, true, C::EW>(a, tb, g, nt, row0, rows, q, lane, h, release);
             } else {
                 epilogue_tile<BT, DUAL, OUT, C::NPART, true, C::EW>(a, tb, g, nt, row0, rows, q, lane, h);
+                release();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->tempty[b]);
             if (++b == C::ACC_BUFS) {
                 b = 0;
                 bph ^= 1u;
@@ -2181,16 +2258,23 @@ long long wait_limit_cycles() {
     return kWaitLimitCycles;
 }
 
-// The BF16 GEMM runs on CTA pairs on request: MOE_GEMM_PAIRS=1 for any segment size, =2 when
-// segments average more than 96 rows (a pair tile is up to 256 tokens wide) and no token tile
-// was forced. Off by default: the one-SM kernel measured faster on B200.
+// Whether a BF16 GEMM runs on CTA pairs. MOE_GEMM_PAIRS=0: never; 1: always; 2: when the
+// segments average more than 96 rows. Unset: when they average more than 512 rows and no
+// token tile was forced. Long segments fill the pair's 256-token tiles; the pair measured
+// faster than one SM per tile there (the Mixtral-shaped prefill) and not at DeepSeek-shaped
+// segments of about 250 rows.
 bool use_pairs(const GemmProblem& p) {
     const char* env = getenv("MOE_GEMM_PAIRS");
-    if (!env || env[1] != '\0') return false;
-    if (env[0] == '1') return true;
-    if (env[0] != '2' || p.bt || getenv("MOE_TOKEN_TILE")) return false;
+    int mode = 3;
+    if (env) {
+        if (env[0] < '0' || env[0] > '2' || env[1] != '\0') return false;
+        mode = env[0] - '0';
+    }
+    if (mode == 0) return false;
+    if (mode == 1) return true;
+    if (p.bt || getenv("MOE_TOKEN_TILE")) return false;
     const long long segs = std::max<long long>(1, std::min<long long>(p.G, p.M_alloc));
-    return p.M_alloc > 96 * segs;
+    return p.M_alloc > (mode == 2 ? 96 : 512) * segs;
 }
 
 // Whether launch_grouped_gemm can gather this problem's token rows itself (BF16 gate/up with

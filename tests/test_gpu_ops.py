@@ -210,6 +210,7 @@ def test_forward_bf16_fused_gather_one_sm(lib, monkeypatch):
     cfg = W.MoEConfig("gather1", T=600, H=208, I=256, E=8, topk=2, B=3, B_used=2)
     inp = W.gen_inputs(cfg)
     outs = {}
+    monkeypatch.setenv("MOE_GEMM_PAIRS", "0")
     for fg in ("1", "0"):
         monkeypatch.setenv("MOE_FUSED_GATHER", fg)
         outs[fg], _, _, _ = run_layer(lib, cfg, inp)
