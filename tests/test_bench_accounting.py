@@ -48,6 +48,20 @@ def test_tensor_peak_of_each_mma_kind():
     assert bench.tensor_peak_ratio(W.CONFIGS["mxfp4_prefill"])[0] == 1.0  # two fp8 products per MAC
 
 
+def test_tensor_peak_regime_follows_the_clock_record(tmp_path, monkeypatch):
+    # sustained (power-capped) bf16 peak only when the timed region saw the power cap
+    assert bench.tensor_peak_key({"reasons": ["sw_power_cap"]})[0] == "bf16_tflops_sustained"
+    assert bench.tensor_peak_key({"reasons": []})[0] == "bf16_tflops"
+    assert bench.tensor_peak_key({"error": "nvml unavailable"})[0] == "bf16_tflops"
+    # a measured file without the sustained figure keeps its other numbers
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 7000.0, "bf16_tflops": 1700.0}')
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert peaks["hbm_gbs"] == 7000.0 and peaks["bf16_tflops"] == 1700.0
+    assert peaks["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert src.startswith("measured") and "bf16_tflops_sustained" in src
+
+
 def test_launch_counts_and_dtype():
     assert bench.kernel_launches(W.CONFIGS["mixtral_prefill"]) == 8
     assert bench.kernel_launches(W.CONFIGS["nvfp4"]) == 9
