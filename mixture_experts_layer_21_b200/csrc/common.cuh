@@ -159,6 +159,15 @@ MOE_DEV void cp_async16(uint32_t dst_smem, const void* src, uint32_t src_bytes) 
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
                  : "memory");
 }
+// The same with an L2 cache policy (from l2_policy; 0 = none).
+MOE_DEV void cp_async16_p(uint32_t dst_smem, const void* src, uint32_t src_bytes, uint64_t pol) {
+    if (pol)
+        asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst_smem), "l"(src),
+                     "r"(src_bytes), "l"(pol)
+                     : "memory");
+    else
+        cp_async16(dst_smem, src, src_bytes);
+}
 // Arrive on an mbarrier (counted in its expected arrivals) once this thread's cp.asyncs land.
 MOE_DEV void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -436,21 +445,10 @@ MOE_DEV float e4m3_to_f32(uint8_t c) {
 // block takes -127. Clamped to e8m0's [-127, 127].
 MOE_DEV int mx8_block_exp(float amax, bool two) {
     if (!(amax > 0.0f)) return -127;
-    // amax = m * 2^ex with m in [0.5, 1). For a normal amax = (1 + f) 2^(E - 127) that is
-    // ex = E - 126 and m = (1 + f) / 2, so m > 0.875 exactly when f > 0.75, i.e. when the
-    // fraction field exceeds 0x600000; subnormals and infinities take frexpf.
-    const uint32_t bits = __float_as_uint(amax);
-    const int E = (int)(bits >> 23);
     int ex;
-    bool big;
-    if (E > 0 && E < 255) {
-        ex = E - 126;
-        big = (bits & 0x7FFFFFu) > 0x600000u;
-    } else {
-        big = frexpf(amax, &ex) > 0.875f;
-    }
+    const float m = frexpf(amax, &ex);  // amax = m * 2^ex, m in [0.5, 1)
     // hi/lo: 448 * 2^(ex-9) = 0.875 * 2^ex; one term: floor(log2 amax) - 8 = ex - 9
-    const int e = (two && big) ? ex - 8 : ex - 9;
+    const int e = (two && m > 0.875f) ? ex - 8 : ex - 9;
     return max(-127, min(127, e));
 }
 // 2^-e as a normal float for the e of mx8_block_exp (finite inputs give e <= 120).

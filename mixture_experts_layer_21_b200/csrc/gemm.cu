@@ -343,9 +343,13 @@ __device__ __forceinline__ void epilogue_tile_mx8_staged(const GemmArgs& a, uint
 #pragma unroll
     for (int ci = 0; ci < NCH; ++ci) {
         const int c0 = 16 * (h + ci * EW);
+        if (c0 < rows) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (c0 + j < rows) epi_store_mx8(a, row0 + c0 + j, n, lane, vals[ci][j]);
+            for (int j = 0; j < 16; ++j) {
+                if (c0 + j >= rows) break;  // the same in every lane
+                epi_store_mx8(a, row0 + c0 + j, n, lane, vals[ci][j]);
+            }
+        }
     }
 }
 
@@ -355,7 +359,7 @@ __device__ __forceinline__ void epilogue_tile_mx8_staged(const GemmArgs& a, uint
 // instruction reads four whole 128-byte row segments; chunk c of row r lands at chunk
 // position c ^ (r % 8), the 128-byte swizzle the MMA reads. Chunks past K are zero-filled.
 __device__ __forceinline__ void gather_stage_rows(uint32_t bb, const __nv_bfloat16* gx, const int (&tok)[4], int K,
-                                                  int kb, int lane) {
+                                                  int kb, int lane, uint64_t pol) {
     const int rr = lane >> 3, c = lane & 7;
     const int k = kb * kTileK + c * 8;
     const bool kin = k < K;
@@ -363,7 +367,7 @@ __device__ __forceinline__ void gather_stage_rows(uint32_t bb, const __nv_bfloat
     for (int i = 0; i < 32; ++i) {
         const int row = 4 * i + rr;
         const int t = __shfl_sync(0xffffffffu, tok[i >> 3], 4 * (i & 7) + rr);
-        cp_async16(bb + row * 128 + ((c ^ (row & 7)) << 4), kin ? gx + (size_t)t * K + k : gx, kin ? 16u : 0u);
+        cp_async16_p(bb + row * 128 + ((c ^ (row & 7)) << 4), kin ? gx + (size_t)t * K + k : gx, kin ? 16u : 0u, pol);
     }
 }
 
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
 
     if (warp == 0) {
         if (GATHER) {  // ---------------- producer warp: weights by TMA (lane 0), tokens gathered
-            const uint64_t pol_w = l2_policy(a.l2_w);
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BT, DUAL>::THREADS, 1)
                         tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
                         if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, nt * kTileN, g, pol_w);
                     }
-                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane);
+                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane, pol_t);
                     cp_async_arrive_noinc(&ctl->full[s]);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
@@ -719,7 +723,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
 
     if (warp == 0) {
         if (GATHER) {  // ---------------- producer warp: weights by TMA (lane 0), tokens gathered
-            const uint64_t pol_w = l2_policy(a.l2_w);
+            const uint64_t pol_w = l2_policy(a.l2_w), pol_t = l2_policy(a.l2_t);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -747,7 +751,7 @@ __global__ void __launch_bounds__(PairCfg<BT, DUAL>::THREADS, 1)
                         tma_load_3d_p(opA(s, 0), &tm_w0, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
                         if (DUAL) tma_load_3d_p(opA(s, 1), &tm_w1, &ctl->full[s], kb * kTileK, wrow, g, pol_w);
                     }
-                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane);
+                    gather_stage_rows(smem_u32(opB(s)), a.gx, tok, K, kb, lane, pol_t);
                     cp_async_arrive_noinc(&ctl->full[s]);
                     is.mask |= 1u << s;
                     is.par = (is.par & ~(1u << s)) | (ph << s);
@@ -1587,9 +1591,10 @@ struct Mx8Cfg {
     static constexpr int SF_BASE = ACC_BUFS * ACC_COLS;
     static constexpr int STAGES = cmin(cmin(kMaxStages, kSmemBudget / STAGE), (512 - SF_BASE) / SF_SLOT);
     static constexpr int TMEM_COLS = tmem_cols_pow2(SF_BASE + STAGES * SF_SLOT);
-    // Two epilogue warps per TMEM lane quarter: with one accumulator buffer the MMAs wait
-    // for the epilogue, and one warp per quarter takes about as long as the main loop.
-    static constexpr int EW = 2;
+    // Epilogue warps per TMEM lane quarter. With one accumulator buffer the MMAs wait for
+    // the epilogue, whose instruction chains are latency-bound: four warps per quarter
+    // (the MXFP4 prefill gate/up GEMM measured about 1.1 ms with two, 0.8 with four), else two.
+    static constexpr int EW = ACC_BUFS == 1 ? 4 : 2;
     static constexpr int EPI_WARP0 = 1 + NI;
     static constexpr int SCALE_WARP = EPI_WARP0 + 4 * EW;
     static constexpr int THREADS = (SCALE_WARP + 1) * 32;
