@@ -440,6 +440,24 @@ def test_forward_small_matches_oracle(lib, name):
         check_fp4_layer(out, ref, cfg, inp, what=name)
 
 
+@pytest.mark.parametrize("bt", [16, 32, 64, 128])
+@pytest.mark.parametrize("act_quant", [0, 2])
+def test_forward_mxfp4_every_token_tile(lib, bt, act_quant, monkeypatch):
+    # the MXFP4 layer with each token tile forced, hi/lo and W4A8: the 64- and 128-token
+    # gate/up tiles have one accumulator buffer (four epilogue warps per lane quarter, the
+    # staged record epilogue); segments of about 56 rows leave every width ragged, and
+    # I = 320 ends in half a weight block
+    monkeypatch.setenv("MOE_TOKEN_TILE", str(bt))
+    cfg = W.MoEConfig("mx_tiles", T=140, H=192, I=320, E=10, topk=4, act="situ", wfmt="mxfp4",
+                      act_quant=act_quant)
+    inp = W.gen_inputs(cfg)
+    out, ids, _, _ = run_layer(lib, cfg, inp)
+    ref = O.moe_forward(cfg, inp.x, inp.logits.numpy(), inp.replica_src.numpy(), inp.w_gate, inp.w_up,
+                        inp.w_down, keep=True)
+    assert np.array_equal(ids.cpu().numpy(), ref["ids"])
+    check_fp4_layer(out, ref, cfg, inp, what=f"mxfp4 bt{bt} act_quant {act_quant}")
+
+
 def test_forward_bf16_256_token_tiles(lib, monkeypatch):
     # the 256-token gate/up tile (one accumulator buffer, eight epilogue warps) and the
     # per-tile MMA width: segments of about 75 rows use a fraction of each tile
