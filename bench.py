@@ -106,13 +106,13 @@ def tensor_peak_ratio(cfg) -> tuple[float, str]:
     """Tensor peak of the path's MMA kind relative to the measured bf16 one (the nominal
     dense ratios: fp8 2x, fp4 4x bf16)."""
     if cfg.wfmt == "nvfp4" and cfg.act_quant == 1:
-        return 4.0, "= measured bf16 x 4 (kind::mxf4nvf4, the nominal fp4/bf16 ratio)"
+        return 4.0, "bf16 x 4 (kind::mxf4nvf4, the nominal fp4/bf16 ratio)"
     if cfg.wfmt == "mxfp4" and cfg.act_quant == 2:
-        return 2.0, "= measured bf16 x 2 (kind::mxf8f6f4, the nominal fp8/bf16 ratio)"
+        return 2.0, "bf16 x 2 (kind::mxf8f6f4, the nominal fp8/bf16 ratio)"
     if cfg.wfmt == "mxfp4":
-        return 1.0, ("= measured bf16 (kind::mxf8f6f4 at the fp8 rate, two e4m3 products per "
+        return 1.0, ("bf16 x 1 (kind::mxf8f6f4 at the fp8 rate, two e4m3 products per "
                      "multiply-add for the hi/lo activations)")
-    return 1.0, "= measured bf16"
+    return 1.0, "bf16 (kind::f16)"
 
 
 def routing_config(cfg) -> dict:
@@ -497,8 +497,9 @@ def run_ours(args, cfg, rank, world):
     roof.update({"traffic": traffic, "kernel": kname,
                  "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
                  "kernel_ms": fc1_ms,
-                 "peak_source": f"{peak_src}; HBM copy bandwidth; bf16 tensor peak {tensor_regime}, "
-                                f"this path's {tensor_note}"})
+                 "peak_source": f"{peak_src} peaks: HBM {peaks['hbm_gbs']:.0f} GB/s (copy); bf16 tensor "
+                                f"{peaks[tensor_key]:.0f} TFLOP/s ({tensor_regime}); this path's tensor peak "
+                                f"= {tensor_note}"})
     t_layer_roof = max(acc["layer_flops"] / (tensor_peak * 1e12),
                        acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
     tok_s = job_tokens_per_s(world, cfg.T, K, ms_total)
