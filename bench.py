@@ -343,6 +343,35 @@ def kernel_launches(cfg) -> int:
     return n
 
 
+def roofline_records(cfg, acc: dict, fc1_ms: float, clocks: dict, traffic) -> tuple[dict, float]:
+    """The gate/up GEMM's roofline record (its algorithmic FLOPs or bytes over its measured
+    time, against the bound that is larger) and the layer's roofline time in seconds."""
+    peaks, peak_src = load_peaks()
+    tensor_mult, tensor_note = tensor_peak_ratio(cfg)
+    tensor_key, tensor_regime = tensor_peak_key(clocks)
+    tensor_peak = peaks[tensor_key] * tensor_mult
+    t_fc1_tensor = acc["fc1_flops"] / (tensor_peak * 1e12)
+    t_fc1_hbm = acc["fc1_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if t_fc1_tensor >= t_fc1_hbm:
+        ach = acc["fc1_flops"] / (fc1_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": ach / tensor_peak}
+    else:
+        ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    kname = "grouped GEMM gate+up (fused activation" + (", biases)" if cfg.bias else ")")
+    roof.update({"traffic": traffic, "kernel": kname,
+                 "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
+                 "kernel_ms": fc1_ms,
+                 "peak_source": f"{peak_src} peaks: HBM {peaks['hbm_gbs']:.0f} GB/s (copy); bf16 tensor "
+                                f"{peaks[tensor_key]:.0f} TFLOP/s ({tensor_regime}); this path's tensor peak "
+                                f"= {tensor_note}"})
+    t_layer_roof = max(acc["layer_flops"] / (tensor_peak * 1e12),
+                       acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    return roof, t_layer_roof
+
+
 def run_ours(args, cfg, rank, world):
     import mixture_experts_layer_21_b200 as m
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -476,32 +505,9 @@ def run_ours(args, cfg, rank, world):
                "d2h_bytes_per_step": int(o_h[0].numel() * 2),
                "overlap": "double-buffered: H2D and D2H on their own streams overlap the layer"}
 
-    peaks, peak_src = load_peaks()
     clocks = clk.summary()
     ms_step = ms_total / K
-    tensor_mult, tensor_note = tensor_peak_ratio(cfg)
-    tensor_key, tensor_regime = tensor_peak_key(clocks)
-    tensor_peak = peaks[tensor_key] * tensor_mult
-    t_fc1_tensor = acc["fc1_flops"] / (tensor_peak * 1e12)
-    t_fc1_hbm = acc["fc1_bytes"] / (peaks["hbm_gbs"] * 1e9)
-    traffic = profiled_traffic(args.config)
-    if t_fc1_tensor >= t_fc1_hbm:
-        ach = acc["fc1_flops"] / (fc1_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": ach / tensor_peak}
-    else:
-        ach = acc["fc1_bytes"] / (fc1_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"]}
-    kname = "grouped GEMM gate+up (fused activation" + (", biases)" if cfg.bias else ")")
-    roof.update({"traffic": traffic, "kernel": kname,
-                 "algorithmic_flops": acc["fc1_flops"], "algorithmic_bytes": acc["fc1_bytes"],
-                 "kernel_ms": fc1_ms,
-                 "peak_source": f"{peak_src} peaks: HBM {peaks['hbm_gbs']:.0f} GB/s (copy); bf16 tensor "
-                                f"{peaks[tensor_key]:.0f} TFLOP/s ({tensor_regime}); this path's tensor peak "
-                                f"= {tensor_note}"})
-    t_layer_roof = max(acc["layer_flops"] / (tensor_peak * 1e12),
-                       acc["layer_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    roof, t_layer_roof = roofline_records(cfg, acc, fc1_ms, clocks, profiled_traffic(args.config))
     tok_s = job_tokens_per_s(world, cfg.T, K, ms_total)
 
     cpu = None

@@ -62,6 +62,20 @@ def test_tensor_peak_regime_follows_the_clock_record(tmp_path, monkeypatch):
     assert src.startswith("measured") and "bf16_tflops_sustained" in src
 
 
+def test_roofline_records_on_both_bounds():
+    # the record the bench prints for the dominant kernel, built without a GPU
+    for name, clocks, bound in (("deepseek_prefill", {"reasons": ["sw_power_cap"]}, "tensor"),
+                                ("nvfp4", {"reasons": []}, "hbm")):
+        cfg = W.CONFIGS[name]
+        acc = {"fc1_flops": 4.0e12, "fc1_bytes": 5.0e9, "layer_flops": 6.0e12, "layer_bytes": 8.0e9}
+        if bound == "hbm":
+            acc = {"fc1_flops": 4.0e11, "fc1_bytes": 5.0e9, "layer_flops": 6.0e11, "layer_bytes": 8.0e9}
+        roof, t_roof = bench.roofline_records(cfg, acc, 2.0, clocks, None)
+        assert roof["bound"] == bound and roof["frac"] == roof["achieved"] / roof["peak"]
+        assert "sustained" in roof["peak_source"] if clocks["reasons"] else "burst" in roof["peak_source"]
+        assert t_roof > 0 and set(roof) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+
+
 def test_launch_counts_and_dtype():
     assert bench.kernel_launches(W.CONFIGS["mixtral_prefill"]) == 8
     assert bench.kernel_launches(W.CONFIGS["nvfp4"]) == 9
