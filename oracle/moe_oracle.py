@@ -50,11 +50,12 @@ E2M1_MAG = _e2m1_magnitudes()          # [0, .5, 1, 1.5, 2, 3, 4, 6]
 E2M1_MAX = 6.0
 
 
+E2M1_VALUES = np.concatenate([E2M1_MAG, -E2M1_MAG])   # by code: bit 3 is the sign
+
+
 def e2m1_decode(codes) -> np.ndarray:
-    """e2m1 code (0..15) -> value, fp64."""
-    c = np.asarray(codes).astype(np.int64)
-    mag = E2M1_MAG[c & 7]
-    return np.where(c & 8, -mag, mag)
+    """e2m1 code (0..15) -> value, fp64: bit 3 the sign, bits 0-2 the magnitude above."""
+    return E2M1_VALUES[np.asarray(codes).astype(np.uint8) & 15]
 
 
 def unpack_e2m1(packed) -> np.ndarray:
@@ -68,12 +69,20 @@ def unpack_e2m1(packed) -> np.ndarray:
 
 # e4m3 (the "fn" variant): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no inf;
 # exponent 15 with mantissa 7 is NaN, so the largest finite value is 448.
-def e4m3_decode(codes) -> np.ndarray:
+def _e4m3_value(codes) -> np.ndarray:
     c = np.asarray(codes).astype(np.int64)
     s, e, m = (c >> 7) & 1, (c >> 3) & 0xF, c & 7
     mag = np.where(e == 0, m * 2.0 ** -9, 2.0 ** (e - 7.0) * (1.0 + m / 8.0))
     mag = np.where((e == 15) & (m == 7), np.nan, mag)
     return np.where(s == 1, -mag, mag)
+
+
+E4M3_TABLE = _e4m3_value(np.arange(256))   # the value of every code
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """e4m3 code (a byte) -> value, fp64, from the table of all 256 codes."""
+    return E4M3_TABLE[np.asarray(codes).astype(np.uint8)]
 
 
 E4M3_MAX = 448.0
@@ -135,13 +144,12 @@ def weight_rows(ws, g: int) -> np.ndarray:
     if ws.fmt == "bf16":
         return to_f64(ws.data[g])
     q = e2m1_decode(unpack_e2m1(ws.data[g].numpy()))
-    if ws.fmt == "mxfp4":
-        sc = e8m0_decode(ws.scale[g].numpy())
-        return q * np.repeat(sc, 32, axis=-1)
-    if ws.fmt == "nvfp4":
-        sc = e4m3_decode(ws.scale[g].numpy())
-        return q * np.repeat(sc, 16, axis=-1)
-    raise ValueError(ws.fmt)
+    blk = {"mxfp4": 32, "nvfp4": 16}.get(ws.fmt)
+    if blk is None:
+        raise ValueError(ws.fmt)
+    sc = (e8m0_decode if ws.fmt == "mxfp4" else e4m3_decode)(ws.scale[g].numpy())
+    # each scale multiplies its block of blk consecutive values along K
+    return (q.reshape(q.shape[0], -1, blk) * sc[..., None]).reshape(q.shape)
 
 
 def weight_alpha(ws) -> np.ndarray:
